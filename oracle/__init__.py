@@ -1,0 +1,156 @@
+"""fp64 CPU oracle for HHST sparse attention (ctypes wrapper of s2_oracle.c).
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. The library package
+(``head_heterogeneous_block_s2_b200``) never imports it, and the oracle imports
+nothing from the library: the two share no code.
+
+This module does argument marshalling only; every number is computed by the C
+code in ``s2_oracle.c``, which states the definition it follows (masked softmax
+attention under the per-head strided block rule of S2-Attention / HHST,
+"S2-Attention: Hardware-aware context sharding among attention heads",
+Abstract).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "s2_oracle.c")
+_LIB = os.path.join(_HERE, "libs2oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile s2_oracle.c into libs2oracle.so (plain gcc, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    i64, i32, dbl, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
+    lib.s2o_block_active.restype = i32
+    lib.s2o_block_active.argtypes = [i64, i64, i64, i64, i64, i32]
+    lib.s2o_block_mask.restype = None
+    lib.s2o_block_mask.argtypes = [i64, i64, i64, i64, vp, vp]
+    lib.s2o_default_threads.restype = i32
+    lib.s2o_default_threads.argtypes = []
+    lib.s2o_prefill_rows.restype = i32
+    lib.s2o_prefill_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, vp,
+                                     dbl, i64, vp, vp, vp, i32]
+    lib.s2o_decode_items.restype = i32
+    lib.s2o_decode_items.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
+                                     i64, vp, dbl, i64, vp, vp, vp, i32]
+    _lib = lib
+    return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bits(a) -> np.ndarray:
+    """Accept a torch bf16 tensor or a uint16 array of bf16 bits; return uint16 C-contiguous."""
+    if hasattr(a, "detach"):  # torch tensor (oracle stays importable without torch)
+        import torch
+
+        assert a.dtype == torch.bfloat16, a.dtype
+        a = a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+def _dense(H, dense):
+    if dense is None:
+        return None
+    d = np.zeros(H, dtype=np.uint8)
+    for h in dense:
+        d[int(h)] = 1
+    return d
+
+
+def default_threads() -> int:
+    return int(_load().s2o_default_threads())
+
+
+def block_active(h, i, j, S, L, dense=False) -> bool:
+    return bool(_load().s2o_block_active(h, i, j, S, L, int(bool(dense))))
+
+
+def block_mask(H, nb, S, L, dense_heads=None) -> np.ndarray:
+    """uint8 mask [H, nb, nb]: 1 where key block j is visible to query block i of head h."""
+    m = np.zeros((H, nb, nb), dtype=np.uint8)
+    d = _dense(H, dense_heads)
+    _load().s2o_block_mask(H, nb, S, L, _ptr(d), _ptr(m))
+    return m
+
+
+def prefill(q, k, v, B, S, L, scale, dense_heads=None, rows=None, nthreads=0):
+    """Oracle prefill. q, k, v: [batch, H, seq, D] bf16 (torch or uint16 bits).
+
+    rows: None for every row, else linear ids (b*H + h)*seq + q.
+    Returns (out fp64 [n_rows, D], lse fp64 [n_rows]).
+    """
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    batch, H, seq, D = q.shape
+    assert k.shape == q.shape and v.shape == q.shape
+    d = _dense(H, dense_heads)
+    if rows is None:
+        n = batch * H * seq
+        r = None
+    else:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        n = r.size
+    out = np.empty((n, D), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    rc = _load().s2o_prefill_rows(_ptr(q), _ptr(k), _ptr(v), batch, H, seq, D, B, S, L,
+                                  _ptr(d), float(scale), n, _ptr(r), _ptr(out), _ptr(lse),
+                                  int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle prefill rejected its arguments")
+    return out, lse
+
+
+def decode(q, k_cache, v_cache, block_table, ctx_lens, B, S, L, scale,
+           dense_heads=None, items=None, nthreads=0):
+    """Oracle decode over a paged cache.
+
+    q: [batch, H, D]; k_cache, v_cache: [pages, H, page_size, D] (bf16);
+    block_table: int32 [batch, max_pages]; ctx_lens: int32 [batch].
+    items: None for all (s, h), else ids s*H + h. Returns (out [n, D], lse [n]).
+    """
+    q, kc, vc = _bits(q), _bits(k_cache), _bits(v_cache)
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    cl = np.ascontiguousarray(np.asarray(ctx_lens, dtype=np.int32))
+    batch, H, D = q.shape
+    _, H2, page_size, D2 = kc.shape
+    assert H2 == H and D2 == D and vc.shape == kc.shape
+    max_pages = bt.shape[1]
+    d = _dense(H, dense_heads)
+    if items is None:
+        n, it = batch * H, None
+    else:
+        it = np.ascontiguousarray(np.asarray(items, dtype=np.int64))
+        n = it.size
+    out = np.empty((n, D), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    rc = _load().s2o_decode_items(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), _ptr(cl), batch, H, D,
+                                  page_size, max_pages, B, S, L, _ptr(d), float(scale), n,
+                                  _ptr(it), _ptr(out), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle decode rejected its arguments")
+    return out, lse

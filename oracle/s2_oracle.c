@@ -1,0 +1,300 @@
+/*
+ * s2_oracle.c -- plain fp64 CPU oracle for HHST sparse attention.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package's smoke check and the
+ * benchmark's CPU-baseline leg load this file's library. The CUDA library never
+ * calls it, and the two share no code, header, table or helper: this file
+ * includes nothing but the C standard library and pthreads.
+ *
+ * What it computes. "S2-Attention: Hardware-aware context sharding among
+ * attention heads" (OpenReview forum page, Abstract; arXiv 2407.17678 abstract)
+ * describes HHST only in words: attention is sparse, the pattern can differ per
+ * head, each head attends to a different strided subset of the context while
+ * the heads together cover all of it, and sparse heads can be mixed with dense
+ * ones ("hybrid"). The pages give no formula, so the oracle uses this explicit
+ * block rule, with query block i = q / B and key block j = k / B:
+ *
+ *     active(h, i, j) = j <= i and (dense[h] or i - j < L or (j + h) mod S == 0)
+ *
+ * and causality inside the diagonal block (key k visible to query q iff k <= q).
+ * The method reaches exactly (up to rounding order) masked softmax attention, so
+ * the oracle is that definition written out in fp64, on inputs given as bf16
+ * bit patterns (widened exactly to double):
+ *
+ *     s_k  = scale * sum_d Q[q,d] K[k,d]            for every visible key k
+ *     m    = max_k s_k,  den = sum_k exp(s_k - m)
+ *     O[q] = sum_k exp(s_k - m) / den * V[k]
+ *     LSE  = m + log(den)
+ *
+ * Decode is the same definition for one query at position n-1 of a context of
+ * n tokens whose keys and values sit in a paged cache addressed through a block
+ * table (PagedAttention is in the arXiv page's reference list).
+ *
+ * Every loop visits keys in ascending order; nothing is blocked, fused or
+ * reordered beyond the definition.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* bf16 bit pattern -> double: the bf16 value is the top half of an fp32. */
+static double bf16_bits_to_double(uint16_t u)
+{
+    uint32_t bits = ((uint32_t)u) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* The block rule above. Returns 1 when key block j is visible to query block i
+ * of head h, 0 otherwise (including j > i and negative indices). */
+int s2o_block_active(int64_t h, int64_t i, int64_t j, int64_t S, int64_t L, int dense)
+{
+    if (j < 0 || i < 0 || j > i) return 0;
+    if (dense) return 1;
+    if (i - j < L) return 1;
+    return ((j + h) % S) == 0;
+}
+
+/* Full block mask, mask[(h * nb + i) * nb + j] in {0,1}. dense may be NULL. */
+void s2o_block_mask(int64_t H, int64_t nb, int64_t S, int64_t L,
+                    const uint8_t* dense, uint8_t* mask)
+{
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t i = 0; i < nb; ++i)
+            for (int64_t j = 0; j < nb; ++j)
+                mask[(h * nb + i) * nb + j] =
+                    (uint8_t)s2o_block_active(h, i, j, S, L, dense ? dense[h] != 0 : 0);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Work distribution: a pool of pthreads pulls item indices from a counter.   */
+/* ------------------------------------------------------------------------- */
+
+typedef struct {
+    int kind; /* 0 = prefill rows, 1 = decode items */
+    const uint16_t *q, *k, *v;
+    const int32_t *block_table, *ctx_lens;
+    int64_t batch, H, seq, D, B, S, L, page_size, max_pages;
+    const uint8_t* dense;
+    double scale;
+    int64_t n_items;
+    const int64_t* items;
+    double *out, *lse;
+    int64_t next;
+    int failed;
+    pthread_mutex_t lock;
+} job_t;
+
+static int64_t take(job_t* J)
+{
+    pthread_mutex_lock(&J->lock);
+    int64_t r = J->next++;
+    pthread_mutex_unlock(&J->lock);
+    return r;
+}
+
+/* Prefill row r = (b * H + h) * seq + q: keys 0..q of the same (b, h). */
+static void prefill_row(const job_t* J, int64_t r, double* s, double* qd,
+                        double* out, double* lse)
+{
+    const int64_t D = J->D, seq = J->seq;
+    const int64_t q = r % seq;
+    const int64_t bh = r / seq;
+    const int64_t h = bh % J->H;
+    const int64_t i = q / J->B;
+    const int dense = J->dense ? J->dense[h] != 0 : 0;
+    const uint16_t* Q = J->q + r * D;
+    const uint16_t* K = J->k + bh * seq * D;
+    const uint16_t* V = J->v + bh * seq * D;
+
+    for (int64_t d = 0; d < D; ++d) qd[d] = bf16_bits_to_double(Q[d]);
+
+    double m = -INFINITY;
+    for (int64_t k = 0; k <= q; ++k) {
+        if (!s2o_block_active(h, i, k / J->B, J->S, J->L, dense)) continue;
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qd[d] * bf16_bits_to_double(K[k * D + d]);
+        s[k] = J->scale * dot;
+        if (s[k] > m) m = s[k];
+    }
+    double den = 0.0;
+    for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
+    for (int64_t k = 0; k <= q; ++k) {
+        if (!s2o_block_active(h, i, k / J->B, J->S, J->L, dense)) continue;
+        const double p = exp(s[k] - m);
+        den += p;
+        for (int64_t d = 0; d < D; ++d) out[d] += p * bf16_bits_to_double(V[k * D + d]);
+    }
+    for (int64_t d = 0; d < D; ++d) out[d] /= den;
+    *lse = m + log(den);
+}
+
+/* Decode item e = seq_index * H + h: the query of sequence s sits at position
+ * n-1 (n = ctx_lens[s]) and sees keys 0..n-1, token t being row t % page_size
+ * of page block_table[s][t / page_size] in a [pages][H][page_size][D] cache. */
+static int decode_item(const job_t* J, int64_t e, double* s, double* qd,
+                       double* out, double* lse)
+{
+    const int64_t D = J->D, H = J->H, P = J->page_size;
+    const int64_t sq = e / H, h = e % H;
+    const int64_t n = J->ctx_lens[sq];
+    if (n < 1) return -1;
+    const int64_t i = (n - 1) / J->B;
+    const int dense = J->dense ? J->dense[h] != 0 : 0;
+    const uint16_t* Q = J->q + e * D;
+
+    for (int64_t d = 0; d < D; ++d) qd[d] = bf16_bits_to_double(Q[d]);
+
+    double m = -INFINITY;
+    for (int64_t k = 0; k < n; ++k) {
+        if (!s2o_block_active(h, i, k / J->B, J->S, J->L, dense)) continue;
+        const int64_t page = J->block_table[sq * J->max_pages + k / P];
+        if (page < 0) return -1;
+        const uint16_t* Krow = J->k + ((page * H + h) * P + k % P) * D;
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qd[d] * bf16_bits_to_double(Krow[d]);
+        s[k] = J->scale * dot;
+        if (s[k] > m) m = s[k];
+    }
+    double den = 0.0;
+    for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
+    for (int64_t k = 0; k < n; ++k) {
+        if (!s2o_block_active(h, i, k / J->B, J->S, J->L, dense)) continue;
+        const int64_t page = J->block_table[sq * J->max_pages + k / P];
+        const uint16_t* Vrow = J->v + ((page * H + h) * P + k % P) * D;
+        const double p = exp(s[k] - m);
+        den += p;
+        for (int64_t d = 0; d < D; ++d) out[d] += p * bf16_bits_to_double(Vrow[d]);
+    }
+    for (int64_t d = 0; d < D; ++d) out[d] /= den;
+    *lse = m + log(den);
+    return 0;
+}
+
+static void* worker(void* arg)
+{
+    job_t* J = (job_t*)arg;
+    const int64_t span = J->kind == 0 ? J->seq
+                                      : J->max_pages * J->page_size;
+    double* s = (double*)malloc(sizeof(double) * (size_t)(span > 0 ? span : 1));
+    double* qd = (double*)malloc(sizeof(double) * (size_t)J->D);
+    if (!s || !qd) {
+        pthread_mutex_lock(&J->lock);
+        J->failed = 1;
+        pthread_mutex_unlock(&J->lock);
+        free(s);
+        free(qd);
+        return NULL;
+    }
+    for (;;) {
+        const int64_t t = take(J);
+        if (t >= J->n_items) break;
+        const int64_t id = J->items ? J->items[t] : t;
+        double* out = J->out + t * J->D;
+        double* lse = J->lse + t;
+        if (J->kind == 0) {
+            prefill_row(J, id, s, qd, out, lse);
+        } else if (decode_item(J, id, s, qd, out, lse) != 0) {
+            pthread_mutex_lock(&J->lock);
+            J->failed = 1;
+            pthread_mutex_unlock(&J->lock);
+        }
+    }
+    free(s);
+    free(qd);
+    return NULL;
+}
+
+static int run_job(job_t* J, int nthreads)
+{
+    if (nthreads <= 0) {
+        long n = sysconf(_SC_NPROCESSORS_ONLN);
+        nthreads = n > 0 ? (int)n : 1;
+    }
+    if (nthreads > 1024) nthreads = 1024;
+    pthread_mutex_init(&J->lock, NULL);
+    J->next = 0;
+    J->failed = 0;
+    pthread_t tid[1024];
+    int started = 0;
+    for (int t = 1; t < nthreads; ++t)
+        if (pthread_create(&tid[started], NULL, worker, J) == 0) ++started;
+    worker(J);
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    pthread_mutex_destroy(&J->lock);
+    return J->failed ? -1 : 0;
+}
+
+/* Number of threads a call with nthreads <= 0 uses. */
+int s2o_default_threads(void)
+{
+    long n = sysconf(_SC_NPROCESSORS_ONLN);
+    return n > 0 ? (int)n : 1;
+}
+
+/* Prefill oracle on selected rows.
+ * q, k, v: bf16 bits, [batch][H][seq][D] contiguous.
+ * rows: n_rows linear row ids (b * H + h) * seq + q, or NULL for all rows in
+ *       order (then n_rows must be batch * H * seq).
+ * out: [n_rows][D] fp64, lse: [n_rows] fp64. dense: [H] or NULL.
+ * Returns 0, or -1 on a bad argument / allocation failure. */
+int s2o_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                     int64_t batch, int64_t H, int64_t seq, int64_t D,
+                     int64_t B, int64_t S, int64_t L, const uint8_t* dense,
+                     double scale, int64_t n_rows, const int64_t* rows,
+                     double* out, double* lse, int nthreads)
+{
+    if (!q || !k || !v || !out || !lse || batch < 1 || H < 1 || seq < 1 || D < 1 ||
+        B < 1 || S < 1 || L < 1 || n_rows < 0)
+        return -1;
+    if (!rows && n_rows != batch * H * seq) return -1;
+    if (rows)
+        for (int64_t t = 0; t < n_rows; ++t)
+            if (rows[t] < 0 || rows[t] >= batch * H * seq) return -1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.kind = 0;
+    J.q = q; J.k = k; J.v = v;
+    J.batch = batch; J.H = H; J.seq = seq; J.D = D;
+    J.B = B; J.S = S; J.L = L; J.dense = dense; J.scale = scale;
+    J.n_items = n_rows; J.items = rows; J.out = out; J.lse = lse;
+    return run_job(&J, nthreads);
+}
+
+/* Decode oracle on selected (sequence, head) items.
+ * q: bf16 bits [batch][H][D]; k_cache, v_cache: [num_pages][H][page_size][D];
+ * block_table: [batch][max_pages] physical page ids; ctx_lens: [batch], >= 1.
+ * items: n_items ids s * H + h, or NULL for all in order (n_items = batch*H).
+ * out: [n_items][D], lse: [n_items]. Returns 0, or -1 on a bad argument
+ * (including a negative page id inside a context). */
+int s2o_decode_items(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                     const int32_t* block_table, const int32_t* ctx_lens,
+                     int64_t batch, int64_t H, int64_t D, int64_t page_size,
+                     int64_t max_pages, int64_t B, int64_t S, int64_t L,
+                     const uint8_t* dense, double scale, int64_t n_items,
+                     const int64_t* items, double* out, double* lse, int nthreads)
+{
+    if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !out || !lse ||
+        batch < 1 || H < 1 || D < 1 || page_size < 1 || max_pages < 1 || B < 1 ||
+        S < 1 || L < 1 || n_items < 0)
+        return -1;
+    if (!items && n_items != batch * H) return -1;
+    for (int64_t s = 0; s < batch; ++s)
+        if (ctx_lens[s] < 1 || ctx_lens[s] > max_pages * page_size) return -1;
+    if (items)
+        for (int64_t t = 0; t < n_items; ++t)
+            if (items[t] < 0 || items[t] >= batch * H) return -1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.kind = 1;
+    J.q = q; J.k = k_cache; J.v = v_cache;
+    J.block_table = block_table; J.ctx_lens = ctx_lens;
+    J.batch = batch; J.H = H; J.D = D; J.page_size = page_size; J.max_pages = max_pages;
+    J.B = B; J.S = S; J.L = L; J.dense = dense; J.scale = scale;
+    J.n_items = n_items; J.items = items; J.out = out; J.lse = lse;
+    return run_job(&J, nthreads);
+}
