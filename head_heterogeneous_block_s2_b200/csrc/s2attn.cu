@@ -1,0 +1,322 @@
+// s2attn.cu -- C ABI of the HHST sparse-attention library (see include/s2attn.h).
+//
+// Host side of the prefill and decode paths: argument validation, TMA tensor
+// maps (encoded through the driver entry point, so the library does not link
+// libcuda and loads on machines without a GPU), launches, and the device
+// error flags shared by all kernels of this translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "s2attn.h"
+#include "ptx.cuh"
+#include "prefill_sm100.cuh"
+#include "decode.cuh"
+
+namespace {
+
+__device__ uint32_t g_s2_flags;
+
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+constexpr int kMaxDevices = 64;
+struct DevInfo {
+    int checked = 0;  // 0 unknown, 1 sm_100, -1 other
+    int num_sms = 0;
+    uint32_t* flags = nullptr;
+    bool prefill_attr_done[4] = {false, false, false, false};
+    bool decode_attr_done[2] = {false, false};
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Device checks, once per device: compute capability 10.x and the address of
+// the error flags.
+int device_ready(int* dev_out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return S2_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return S2_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevInfo& d = g_dev[dev];
+    if (d.checked == 0) {
+        int major = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return S2_ERR_CUDA;
+        if (major != 10) {
+            d.checked = -1;
+        } else {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_s2_flags) != cudaSuccess) return S2_ERR_CUDA;
+            d.flags = static_cast<uint32_t*>(p);
+            d.num_sms = sms;
+            d.checked = 1;
+        }
+    }
+    if (d.checked != 1) return S2_ERR_UNSUPPORTED;
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return S2_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    *dev_out = dev;
+    return S2_OK;
+}
+
+// 2-D bf16 tensor map over [rows][cols], box [box_rows][64], SWIZZLE_128B.
+int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? S2_OK : S2_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int HD, int BK>
+int launch_prefill(const void* q, const void* k, const void* v, s2::PrefillParams& pp, int dev,
+                   int attr_slot, cudaStream_t stream)
+{
+    using C = s2::PrefillCfg<HD, BK>;
+    const uint64_t rows = (uint64_t)pp.batch * pp.heads * pp.seq;
+    CUtensorMap mq, mk, mv;
+    if (make_map(&mq, q, rows, HD, 128) || make_map(&mk, k, rows, HD, BK) ||
+        make_map(&mv, v, rows, HD, BK))
+        return S2_ERR_CUDA;
+    auto kern = s2::s2_prefill_kernel<HD, BK>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_dev[dev].prefill_attr_done[attr_slot]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::SMEM_ALLOC) != cudaSuccess)
+                return S2_ERR_CUDA;
+            g_dev[dev].prefill_attr_done[attr_slot] = true;
+        }
+    }
+    const uint64_t grid = (uint64_t)pp.batch * pp.heads * pp.nqt;
+    kern<<<(unsigned)grid, 192, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
+    return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
+}
+
+template <int HD>
+int launch_decode(s2::DecodeParams& dp, int dev, cudaStream_t stream)
+{
+    using C = s2::DecodeCfg<HD>;
+    auto kern = s2::s2_decode_split_kernel<HD>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        const int slot = HD == 128 ? 1 : 0;
+        if (!g_dev[dev].decode_attr_done[slot]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+                cudaSuccess)
+                return S2_ERR_CUDA;
+            g_dev[dev].decode_attr_done[slot] = true;
+        }
+    }
+    dim3 grid(dp.num_splits, dp.heads, dp.batch);
+    kern<<<grid, 160, C::SMEM, stream>>>(dp);
+    if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
+    if (dp.num_splits > 1) {
+        s2::s2_decode_combine_kernel<HD><<<(unsigned)(dp.batch * dp.heads), HD, 0, stream>>>(
+            dp.ws_o, dp.ws_ml, dp.num_splits, dp.out, dp.lse);
+        if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
+    }
+    return S2_OK;
+}
+
+constexpr int kMaxSplits = 64;
+
+size_t ws_bytes(int64_t batch, int64_t heads, int64_t head_dim, int64_t splits)
+{
+    if (splits <= 1) return 0;
+    const size_t o = (size_t)(batch * heads * splits * head_dim) * sizeof(float);
+    const size_t o_pad = (o + 255) & ~size_t(255);
+    return o_pad + (size_t)(batch * heads * splits) * sizeof(float2);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* s2_status_string(int status)
+{
+    switch (status) {
+    case S2_OK: return "S2_OK";
+    case S2_ERR_INVALID_ARG: return "S2_ERR_INVALID_ARG";
+    case S2_ERR_UNSUPPORTED: return "S2_ERR_UNSUPPORTED";
+    case S2_ERR_CAPACITY: return "S2_ERR_CAPACITY";
+    case S2_ERR_CUDA: return "S2_ERR_CUDA";
+    case S2_ERR_TIMEOUT: return "S2_ERR_TIMEOUT";
+    case S2_ERR_DEVICE_INDEX: return "S2_ERR_DEVICE_INDEX";
+    default: return "S2_ERR_UNKNOWN";
+    }
+}
+
+const char* s2_version(void) { return "s2attn-b200 0.1 (sm_100a)"; }
+
+int s2_set_wait_timeout_ns(uint64_t ns)
+{
+    g_timeout_ns.store(ns);
+    return S2_OK;
+}
+
+int s2_device_status(int reset, uint32_t* flags_out)
+{
+    int dev = 0;
+    const int rc = device_ready(&dev);
+    if (rc) return rc;
+    uint32_t f = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return S2_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&f, g_s2_flags, sizeof f) != cudaSuccess) return S2_ERR_CUDA;
+    if (reset) {
+        const uint32_t z = 0;
+        if (cudaMemcpyToSymbol(g_s2_flags, &z, sizeof z) != cudaSuccess) return S2_ERR_CUDA;
+    }
+    if (flags_out) *flags_out = f;
+    if (f & s2::kFlagTimeout) return S2_ERR_TIMEOUT;
+    if (f & s2::kFlagIndex) return S2_ERR_DEVICE_INDEX;
+    return S2_OK;
+}
+
+int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int32_t batch, int32_t heads, int32_t seq, int32_t head_dim, float scale,
+                    int32_t block_size, int32_t num_blocks, const int32_t* row_ptr,
+                    const int32_t* col_idx, int64_t nnz, void* stream)
+{
+    if (!q || !k || !v || !o || !row_ptr || !col_idx) return S2_ERR_INVALID_ARG;
+    if (batch < 1 || heads < 1 || seq < 1 || nnz < 1 || !std::isfinite(scale))
+        return S2_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
+    if (block_size != 64 && block_size != 128) return S2_ERR_UNSUPPORTED;
+    if (seq % block_size != 0 || num_blocks != seq / block_size) return S2_ERR_INVALID_ARG;
+    if ((int64_t)batch * heads * seq >= (int64_t)INT32_MAX) return S2_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return S2_ERR_INVALID_ARG;
+    int dev = 0;
+    int rc = device_ready(&dev);
+    if (rc) return rc;
+
+    s2::PrefillParams pp;
+    pp.row_ptr = row_ptr;
+    pp.col_idx = col_idx;
+    pp.nnz = nnz;
+    pp.o = static_cast<uint16_t*>(o);
+    pp.lse = lse;
+    pp.batch = batch;
+    pp.heads = heads;
+    pp.seq = seq;
+    pp.nb = num_blocks;
+    pp.nqt = (seq + 127) / 128;
+    pp.scale_log2 = scale * 1.4426950408889634f;
+    pp.timeout_ns = g_timeout_ns.load();
+    pp.gflags = g_dev[dev].flags;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (head_dim == 128 && block_size == 128) return launch_prefill<128, 128>(q, k, v, pp, dev, 0, st);
+    if (head_dim == 128 && block_size == 64) return launch_prefill<128, 64>(q, k, v, pp, dev, 1, st);
+    if (head_dim == 64 && block_size == 128) return launch_prefill<64, 128>(q, k, v, pp, dev, 2, st);
+    return launch_prefill<64, 64>(q, k, v, pp, dev, 3, st);
+}
+
+int32_t s2_attn_decode_auto_splits(int32_t batch, int32_t heads)
+{
+    if (batch < 1 || heads < 1) return 1;
+    // Aim for about 4 waves of 3 resident CTAs on each of 148 SMs.
+    const int64_t target = 148 * 3 * 4;
+    int64_t sp = (target + (int64_t)batch * heads - 1) / ((int64_t)batch * heads);
+    if (sp < 1) sp = 1;
+    if (sp > 16) sp = 16;
+    return (int32_t)sp;
+}
+
+size_t s2_attn_decode_workspace_size(int32_t batch, int32_t heads, int32_t head_dim,
+                                     int32_t num_splits)
+{
+    if (batch < 1 || heads < 1 || head_dim < 1) return 0;
+    const int32_t sp = num_splits > 0 ? num_splits : s2_attn_decode_auto_splits(batch, heads);
+    return ws_bytes(batch, heads, head_dim, sp);
+}
+
+int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* block_table, const int32_t* ctx_lens, int32_t batch,
+                   int32_t heads, int32_t head_dim, int32_t page_size, int32_t max_pages,
+                   int64_t num_pages, int32_t block_size, int32_t num_blocks,
+                   const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz, float scale,
+                   void* out, float* lse, void* workspace, size_t workspace_bytes,
+                   int32_t num_splits, void* stream)
+{
+    if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !row_ptr || !col_idx || !out)
+        return S2_ERR_INVALID_ARG;
+    if (batch < 1 || heads < 1 || max_pages < 1 || num_pages < 1 || num_blocks < 1 || nnz < 1 ||
+        !std::isfinite(scale) || num_splits > kMaxSplits)
+        return S2_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
+    if (page_size != s2::kPage) return S2_ERR_UNSUPPORTED;
+    if (block_size < page_size || block_size % page_size != 0) return S2_ERR_UNSUPPORTED;
+    if (batch > 65535 || heads > 65535) return S2_ERR_UNSUPPORTED;
+    if (num_pages * heads * page_size * head_dim >= (int64_t)1 << 62) return S2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return S2_ERR_INVALID_ARG;
+    const int32_t sp = num_splits > 0 ? num_splits : s2_attn_decode_auto_splits(batch, heads);
+    const size_t need = ws_bytes(batch, heads, head_dim, sp);
+    if (need > 0) {
+        if (!workspace) return S2_ERR_INVALID_ARG;
+        if (workspace_bytes < need) return S2_ERR_CAPACITY;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return S2_ERR_INVALID_ARG;
+    }
+    int dev = 0;
+    int rc = device_ready(&dev);
+    if (rc) return rc;
+
+    s2::DecodeParams dp;
+    dp.q = static_cast<const uint16_t*>(q);
+    dp.k_cache = static_cast<const uint16_t*>(k_cache);
+    dp.v_cache = static_cast<const uint16_t*>(v_cache);
+    dp.block_table = block_table;
+    dp.ctx_lens = ctx_lens;
+    dp.row_ptr = row_ptr;
+    dp.col_idx = col_idx;
+    dp.nnz = nnz;
+    dp.num_pages = num_pages;
+    dp.batch = batch;
+    dp.heads = heads;
+    dp.max_pages = max_pages;
+    dp.block_size = block_size;
+    dp.nb = num_blocks;
+    dp.num_splits = sp;
+    dp.scale_log2 = scale * 1.4426950408889634f;
+    dp.out = static_cast<uint16_t*>(out);
+    dp.lse = lse;
+    const size_t o_bytes = ((size_t)batch * heads * sp * head_dim * sizeof(float) + 255) & ~size_t(255);
+    dp.ws_o = need ? static_cast<float*>(workspace) : nullptr;
+    dp.ws_ml = need ? reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + o_bytes) : nullptr;
+    dp.timeout_ns = g_timeout_ns.load();
+    dp.gflags = g_dev[dev].flags;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return head_dim == 128 ? launch_decode<128>(dp, dev, st) : launch_decode<64>(dp, dev, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,263 @@
+"""Thin ctypes binding of libs2attn.so (argument marshalling only).
+
+Every step of the attention path runs in the library's CUDA kernels; this
+module checks tensor types, passes raw device pointers and the current torch
+stream, and turns status codes into exceptions. There is no fallback: if the
+library is missing or a call fails, it raises.
+
+Entry points mirror the C ABI in ``include/s2attn.h``:
+``build_layout`` (host), ``prefill``, ``decode``, ``decode_workspace_size``,
+``device_status`` and ``set_wait_timeout_ns``.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libs2attn.so")
+
+S2_OK = 0
+STATUS_NAMES = {0: "S2_OK", 1: "S2_ERR_INVALID_ARG", 2: "S2_ERR_UNSUPPORTED", 3: "S2_ERR_CAPACITY",
+                4: "S2_ERR_CUDA", 5: "S2_ERR_TIMEOUT", 6: "S2_ERR_DEVICE_INDEX"}
+
+EXPORTED = ("s2_status_string", "s2_build_layout", "s2_attn_prefill",
+            "s2_attn_decode_workspace_size", "s2_attn_decode_auto_splits", "s2_attn_decode",
+            "s2_device_status", "s2_set_wait_timeout_ns", "s2_version")
+
+
+class S2Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class _LayoutDesc(ctypes.Structure):
+    _fields_ = [("num_heads", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("vertical_stride", ctypes.c_int32), ("local_blocks", ctypes.c_int32),
+                ("num_blocks", ctypes.c_int32), ("dense_head_mask", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load the CUDA library (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"{path} not found: build it with "
+                      "`python -m head_heterogeneous_block_s2_b200.build`")
+    lib = ctypes.CDLL(path)
+    i32, i64, vp, f32, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+    lib.s2_status_string.restype = ctypes.c_char_p
+    lib.s2_status_string.argtypes = [ctypes.c_int]
+    lib.s2_version.restype = ctypes.c_char_p
+    lib.s2_version.argtypes = []
+    lib.s2_build_layout.restype = ctypes.c_int
+    lib.s2_build_layout.argtypes = [ctypes.POINTER(_LayoutDesc), vp, vp, i64, ctypes.POINTER(i64)]
+    lib.s2_attn_prefill.restype = ctypes.c_int
+    lib.s2_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp, vp,
+                                    i64, vp]
+    lib.s2_attn_decode_workspace_size.restype = sz
+    lib.s2_attn_decode_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.s2_attn_decode_auto_splits.restype = i32
+    lib.s2_attn_decode_auto_splits.argtypes = [i32, i32]
+    lib.s2_attn_decode.restype = ctypes.c_int
+    lib.s2_attn_decode.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64, i32, i32, vp,
+                                   vp, i64, f32, vp, vp, vp, sz, i32, vp]
+    lib.s2_device_status.restype = ctypes.c_int
+    lib.s2_device_status.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)]
+    lib.s2_set_wait_timeout_ns.restype = ctypes.c_int
+    lib.s2_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    _lib = lib
+    return lib
+
+
+def _check(rc: int, what: str):
+    if rc != S2_OK:
+        raise S2Error(rc, what)
+
+
+# ------------------------------------------------------------------ layout
+
+@dataclasses.dataclass
+class Layout:
+    """Per-head compacted key-block lists (CSR) of one HHST layout."""
+    heads: int
+    block_size: int
+    stride: int
+    local: int
+    num_blocks: int
+    dense_heads: Tuple[int, ...]
+    row_ptr: np.ndarray  # int32 [heads * (num_blocks + 1)]
+    col_idx: np.ndarray  # int32 [nnz]
+    d_row_ptr: Optional[torch.Tensor] = None
+    d_col_idx: Optional[torch.Tensor] = None
+
+    @property
+    def nnz(self) -> int:
+        return int(self.col_idx.size)
+
+    def row(self, h: int, i: int) -> np.ndarray:
+        base = h * (self.num_blocks + 1)
+        return self.col_idx[self.row_ptr[base + i]:self.row_ptr[base + i + 1]]
+
+    def to(self, device) -> "Layout":
+        self.d_row_ptr = torch.from_numpy(self.row_ptr).to(device)
+        self.d_col_idx = torch.from_numpy(self.col_idx).to(device)
+        return self
+
+
+def _desc(heads, block_size, stride, local, num_blocks, dense_heads):
+    mask = None
+    keep = None
+    if dense_heads:
+        keep = (ctypes.c_uint8 * heads)()
+        for h in dense_heads:
+            keep[int(h)] = 1
+        mask = ctypes.cast(keep, ctypes.c_void_p)
+    d = _LayoutDesc(heads, block_size, stride, local, num_blocks, mask)
+    return d, keep
+
+
+def layout_nnz(heads, block_size, stride, local, num_blocks, dense_heads=()) -> int:
+    d, _keep = _desc(heads, block_size, stride, local, num_blocks, dense_heads)
+    nnz = ctypes.c_int64(0)
+    _check(load().s2_build_layout(ctypes.byref(d), None, None, 0, ctypes.byref(nnz)),
+           "s2_build_layout")
+    return nnz.value
+
+
+def build_layout(heads: int, block_size: int, stride: int, local: int, num_blocks: int,
+                 dense_heads: Sequence[int] = (), device=None) -> Layout:
+    """Run s2_build_layout (host) and optionally copy the arrays to ``device``."""
+    lib = load()
+    d, _keep = _desc(heads, block_size, stride, local, num_blocks, dense_heads)
+    nnz = ctypes.c_int64(0)
+    _check(lib.s2_build_layout(ctypes.byref(d), None, None, 0, ctypes.byref(nnz)), "s2_build_layout")
+    row_ptr = np.zeros(heads * (num_blocks + 1), dtype=np.int32)
+    col_idx = np.zeros(max(1, nnz.value), dtype=np.int32)
+    _check(lib.s2_build_layout(ctypes.byref(d), row_ptr.ctypes.data, col_idx.ctypes.data,
+                               col_idx.size, ctypes.byref(nnz)), "s2_build_layout")
+    lay = Layout(heads, block_size, stride, local, num_blocks, tuple(int(h) for h in dense_heads),
+                 row_ptr, col_idx[:nnz.value].copy())
+    if device is not None:
+        lay.to(device)
+    return lay
+
+
+# ------------------------------------------------------------------ kernels
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: Layout,
+            scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+            lse: Optional[torch.Tensor] = None, want_lse: bool = False):
+    """s2_attn_prefill on [batch, heads, seq, head_dim] bf16 CUDA tensors.
+
+    Returns out, or (out, lse) when ``want_lse`` or ``lse`` is given."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    batch, heads, seq, hd = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v shapes differ")
+    if layout.d_row_ptr is None:
+        layout.to(q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out")
+    if lse is None and want_lse:
+        lse = torch.empty((batch, heads, seq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    rc = load().s2_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), batch, heads, seq,
+                                hd, sc, layout.block_size, layout.num_blocks,
+                                _ptr(layout.d_row_ptr), _ptr(layout.d_col_idx), layout.nnz,
+                                _stream(q.device))
+    _check(rc, "s2_attn_prefill")
+    return (out, lse) if lse is not None else out
+
+
+def decode_auto_splits(batch: int, heads: int) -> int:
+    return int(load().s2_attn_decode_auto_splits(batch, heads))
+
+
+def decode_workspace_size(batch: int, heads: int, head_dim: int, num_splits: int = 0) -> int:
+    return int(load().s2_attn_decode_workspace_size(batch, heads, head_dim, num_splits))
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+           block_table: torch.Tensor, ctx_lens: torch.Tensor, layout: Layout,
+           scale: Optional[float] = None, num_splits: int = 0,
+           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+           want_lse: bool = False, workspace: Optional[torch.Tensor] = None):
+    """s2_attn_decode: q [batch, heads, D]; caches [pages, heads, 16, D];
+    block_table int32 [batch, max_pages]; ctx_lens int32 [batch] (all CUDA)."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n)
+    _need(block_table, "block_table", torch.int32)
+    _need(ctx_lens, "ctx_lens", torch.int32)
+    batch, heads, hd = q.shape
+    num_pages, h2, page_size, hd2 = k_cache.shape
+    if h2 != heads or hd2 != hd or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape does not match q")
+    if layout.d_row_ptr is None:
+        layout.to(q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out")
+    if lse is None and want_lse:
+        lse = torch.empty((batch, heads), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+    ws_bytes = decode_workspace_size(batch, heads, hd, num_splits)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    rc = load().s2_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                               _ptr(ctx_lens), batch, heads, hd, page_size, block_table.shape[1],
+                               num_pages, layout.block_size, layout.num_blocks,
+                               _ptr(layout.d_row_ptr), _ptr(layout.d_col_idx), layout.nnz, sc,
+                               _ptr(out), _ptr(lse), _ptr(workspace), ws_len, num_splits,
+                               _stream(q.device))
+    _check(rc, "s2_attn_decode")
+    return (out, lse) if lse is not None else out
+
+
+def device_status(reset: bool = True) -> Tuple[int, int]:
+    """(status, raw flags) after synchronising the current device."""
+    flags = ctypes.c_uint32(0)
+    rc = load().s2_device_status(1 if reset else 0, ctypes.byref(flags))
+    return rc, flags.value
+
+
+def set_wait_timeout_ns(ns: int):
+    _check(load().s2_set_wait_timeout_ns(int(ns)), "s2_set_wait_timeout_ns")
+
+
+def version() -> str:
+    return load().s2_version().decode()

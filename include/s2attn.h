@@ -1,0 +1,187 @@
+/*
+ * s2attn.h -- C ABI of the B200 (sm_100a) HHST sparse-attention library.
+ *
+ * The operation. "S2-Attention: Hardware-aware context sharding among attention
+ * heads" (OpenReview forum page, Abstract, and the arXiv 2407.17678 abstract)
+ * introduces the Head-Heterogenous Strided Transformer (HHST): attention is
+ * restricted per head to a strided subset of the context plus a local window,
+ * different heads take different subsets so that together they cover all of
+ * it, and dense heads may be mixed in ("hybrid"). The pages state the pattern
+ * only in words; this library uses the explicit block rule
+ *
+ *     key block j is active for (head h, query block i)  iff  j <= i and
+ *     (dense[h]  or  i - j < L  or  (j + h) mod S == 0)
+ *
+ * with block size B (query block i = q / B, key block j = k / B), vertical
+ * stride S and L local blocks, plus token-level causality (k <= q) inside the
+ * diagonal block. The result is exact softmax attention under that mask:
+ * O[q] = sum_k softmax_k(scale * Q[q].K[k]) V[k] over the visible keys k.
+ *
+ * Conventions for every entry point:
+ *  - Returns an int status (S2_OK = 0, else one of the S2_ERR_* codes). No C++
+ *    exception crosses the ABI. A call that returns an error launches nothing.
+ *  - The caller owns every buffer. The library never allocates, frees or
+ *    synchronises device memory (s2_device_status is the one synchronous call).
+ *  - Device pointers must stay valid until the work queued on `stream` ends.
+ *    `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream). Launches are asynchronous.
+ *  - Tensors are bf16 (IEEE bfloat16 bit patterns in uint16 storage), dense and
+ *    row-major with the innermost dimension last, 16-byte aligned.
+ *  - Device waits inside the kernels are bounded. A wait that runs out sets a
+ *    device flag that s2_device_status reports as S2_ERR_TIMEOUT. While that
+ *    flag is set, any kernel wait that is not already satisfied gives up at
+ *    once (so one stuck CTA does not stall the rest); s2_device_status(1, ...)
+ *    clears it.
+ */
+#ifndef S2ATTN_H
+#define S2ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    S2_OK = 0,
+    S2_ERR_INVALID_ARG = 1, /* a null pointer, a bad size, or a malformed layout */
+    S2_ERR_UNSUPPORTED = 2, /* head_dim, block size or page size outside the built set;
+                               no sm_100 device */
+    S2_ERR_CAPACITY = 3,    /* an output array or workspace is too small */
+    S2_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed */
+    S2_ERR_TIMEOUT = 5,     /* a bounded device wait ran out (s2_device_status) */
+    S2_ERR_DEVICE_INDEX = 6 /* a kernel met an index outside its buffers and skipped it
+                               (s2_device_status) */
+};
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* s2_status_string(int status);
+
+/* ------------------------------------------------------------------------ */
+/* Layout builder (host only)                                                */
+/* ------------------------------------------------------------------------ */
+
+/* Parameters of one HHST layout (the block rule in the file header). */
+typedef struct s2_layout_desc {
+    int32_t num_heads;       /* H >= 1 */
+    int32_t block_size;      /* B >= 1 tokens per query/key block */
+    int32_t vertical_stride; /* S >= 1 */
+    int32_t local_blocks;    /* L >= 1 (so every row holds its diagonal block) */
+    int32_t num_blocks;      /* nb >= 1 query/key blocks (ceil(seq / B)) */
+    const uint8_t* dense_head_mask; /* host, [num_heads], nonzero = dense causal head;
+                                       NULL = no dense heads */
+} s2_layout_desc;
+
+/*
+ * Build the per-head compacted key-block index lists (CSR) of a layout.
+ *
+ * Two-call protocol: with col_idx == NULL only *nnz_out is set (row_ptr is
+ * still filled when non-NULL). Otherwise:
+ *   row_ptr [H * (nb + 1)] (host, written): row_ptr[h*(nb+1) + i] is the offset
+ *     into col_idx of the list for (head h, query block i); the list ends at
+ *     row_ptr[h*(nb+1) + i + 1]. Offsets are global across heads, so
+ *     row_ptr[h*(nb+1) + nb] == row_ptr[(h+1)*(nb+1)] and row_ptr[0] == 0.
+ *   col_idx [col_idx_cap] (host, written): active key blocks j, ascending within
+ *     each list, so the diagonal block i is always last.
+ *   *nnz_out = total entries. S2_ERR_CAPACITY when col_idx_cap < nnz.
+ * Cost O(H * nb^2) rule evaluations; call once per layout and copy the arrays
+ * to the device for the kernels.
+ */
+int s2_build_layout(const s2_layout_desc* desc, int32_t* row_ptr, int32_t* col_idx,
+                    int64_t col_idx_cap, int64_t* nnz_out);
+
+/* ------------------------------------------------------------------------ */
+/* Prefill: block-sparse causal attention over whole sequences               */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * O = HHST-masked softmax(scale * Q K^T) V for every query row.
+ *
+ *   q, k, v   device bf16 [batch][heads][seq][head_dim] (read).
+ *   o         device bf16 [batch][heads][seq][head_dim] (written).
+ *   lse       device fp32 [batch][heads][seq] or NULL: natural-log
+ *             log-sum-exp of the scaled visible logits of each row (written).
+ *   head_dim  64 or 128.  block_size 64 or 128.  seq % block_size == 0.
+ *   num_blocks == seq / block_size.
+ *   row_ptr, col_idx, nnz: the layout of s2_build_layout for (heads,
+ *             block_size, num_blocks), copied to device memory (read).
+ *   scale     multiplier of the logits (1/sqrt(head_dim) in the usual case).
+ * Runs tcgen05 tensor-core tiles of 128 query rows; only the listed key blocks
+ * are visited and causality is applied inside the diagonal block only.
+ */
+int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int32_t batch, int32_t heads, int32_t seq, int32_t head_dim,
+                    float scale, int32_t block_size, int32_t num_blocks,
+                    const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz,
+                    void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode: one query token per sequence over a paged KV cache               */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of device workspace s2_attn_decode needs for this shape and split
+ * count (num_splits <= 0 means the automatic choice for this shape). */
+size_t s2_attn_decode_workspace_size(int32_t batch, int32_t heads, int32_t head_dim,
+                                     int32_t num_splits);
+
+/* The split count s2_attn_decode uses when given num_splits <= 0. */
+int32_t s2_attn_decode_auto_splits(int32_t batch, int32_t heads);
+
+/*
+ * Split-KV decode: for each sequence s and head h, the query at position
+ * n-1 (n = ctx_lens[s]) attends to keys 0..n-1 of its own context under the
+ * same block rule (query block i = (n-1) / block_size).
+ *
+ *   q            device bf16 [batch][heads][head_dim] (read).
+ *   k_cache,     device bf16 [num_pages][heads][page_size][head_dim] (read):
+ *   v_cache      token t of sequence s is row t % page_size of physical page
+ *                block_table[s][t / page_size].
+ *   block_table  device int32 [batch][max_pages] (read); entries past a
+ *                sequence's last page are ignored (-1 by convention).
+ *   ctx_lens     device int32 [batch] (read), 1 <= n <= min(max_pages *
+ *                page_size, num_blocks * block_size).
+ *   page_size 16.  head_dim 64 or 128.  block_size a multiple of page_size.
+ *   row_ptr, col_idx, nnz: device layout for (heads, block_size, num_blocks).
+ *   out          device bf16 [batch][heads][head_dim] (written).
+ *   lse          device fp32 [batch][heads] or NULL (written).
+ *   workspace    device, >= s2_attn_decode_workspace_size(...) bytes, 256-byte
+ *                aligned; holds per-split partial results (scratch, clobbered).
+ * A ctx_lens entry out of range, or a block-table entry outside [0, num_pages)
+ * inside a context, is skipped by the kernel and reported by s2_device_status
+ * as S2_ERR_DEVICE_INDEX.
+ */
+int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* block_table, const int32_t* ctx_lens,
+                   int32_t batch, int32_t heads, int32_t head_dim, int32_t page_size,
+                   int32_t max_pages, int64_t num_pages, int32_t block_size,
+                   int32_t num_blocks, const int32_t* row_ptr, const int32_t* col_idx,
+                   int64_t nnz, float scale, void* out, float* lse,
+                   void* workspace, size_t workspace_bytes, int32_t num_splits,
+                   void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Device status and limits                                                  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Synchronise the current device and report the kernels' error flags:
+ * S2_OK, S2_ERR_TIMEOUT (a bounded wait ran out) or S2_ERR_DEVICE_INDEX (an
+ * index was out of range and skipped). *flags_out (may be NULL) receives the
+ * raw bit set (1 = timeout, 2 = index). reset != 0 clears the flags.
+ */
+int s2_device_status(int reset, uint32_t* flags_out);
+
+/* Bound, in nanoseconds, of every device wait in kernels launched after this
+ * call (process-wide; default 2e9). 0 makes any wait that is not already
+ * satisfied give up at once, which tests use to exercise the timeout path. */
+int s2_set_wait_timeout_ns(uint64_t ns);
+
+/* Library version string. */
+const char* s2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S2ATTN_H */

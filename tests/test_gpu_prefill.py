@@ -1,0 +1,122 @@
+"""Prefill parity: the sm_100a kernel (through the C ABI) against the fp64 oracle.
+
+Small cases compare every row; the full-size workloads compare a seeded sample
+of rows per head (first, last and random query blocks, and the planted rows)
+in the exact launch configuration the benchmark uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import parity
+from head_heterogeneous_block_s2_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def run_prefill(s2, w, q, k, v):
+    lay = s2.build_layout(w.heads, w.block, w.stride, w.local, w.num_blocks, w.dense_heads,
+                          device=q.device)
+    out, lse = s2.prefill(q, k, v, lay, scale=w.scale, want_lse=True)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def check_all_rows(s2, w, q=None, k=None, v=None):
+    if q is None:
+        q, k, v = synth.prefill_inputs(w)
+    out, lse = run_prefill(s2, w, q.cuda(), k.cuda(), v.cuda())
+    ref, ref_lse = oracle.prefill(q, k, v, w.block, w.stride, w.local, w.scale, w.dense_heads)
+    parity(out.reshape(-1, w.head_dim), ref)
+    parity(lse.reshape(-1), ref_lse, max_tol=1e-3, mean_tol=1e-4)
+
+
+def test_tiny_workload_all_rows(s2gpu):
+    check_all_rows(s2gpu, synth.TINY)
+
+
+@pytest.mark.parametrize("hd", [64, 128])
+@pytest.mark.parametrize("bk", [64, 128])
+@pytest.mark.parametrize("S,L,dense", [(4, 1, ()), (3, 2, (1,)), (1, 1, ())])
+def test_small_shapes_all_rows(s2gpu, hd, bk, S, L, dense):
+    # 3 heads, 2 batches; seq = 9 blocks of 64 (a ragged last 128-row tile) or 5 of 128
+    seq = 9 * 64 if bk == 64 else 5 * 128
+    w = synth.PrefillWorkload("t", 2, 3, hd, seq, bk, S, L, dense_heads=dense, seed=21)
+    check_all_rows(s2gpu, w)
+
+
+def test_stride_one_matches_causal_sdpa(s2gpu):
+    w = synth.PrefillWorkload("t", 1, 4, 128, 1024, 128, 1, 1, seed=3)
+    q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
+    out, _ = run_prefill(s2gpu, w, q, k, v)
+    ref = torch.nn.functional.scaled_dot_product_attention(q.float(), k.float(), v.float(),
+                                                           is_causal=True)
+    assert (out.float() - ref).abs().max().item() < 2e-2
+
+
+def test_scaled_keys_and_large_logits(s2gpu):
+    # per-head K scales as in the 1.3B-shaped workload, at a small size
+    w = synth.PREFILL_1P3B.with_(batch=1, heads=4, seq=2048)
+    check_all_rows(s2gpu, w)
+    # sharper softmax: logits several times larger than unit scale
+    w2 = synth.PrefillWorkload("t", 1, 2, 128, 1024, 128, 4, 2, seed=5)
+    q, k, v = synth.prefill_inputs(w2)
+    check_all_rows(s2gpu, w2.with_(), (q.float() * 3).to(torch.bfloat16), k, v)
+
+
+def test_repeated_calls_are_deterministic(s2gpu):
+    w = synth.TINY
+    q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
+    a, _ = run_prefill(s2gpu, w, q, k, v)
+    b, _ = run_prefill(s2gpu, w, q, k, v)
+    assert torch.equal(a, b)
+
+
+def sample_rows(w, seed, blocks_random=6, per_block=16):
+    rng = np.random.default_rng(seed)
+    rows = []
+    nb = w.num_blocks
+    for b in range(w.batch):
+        for h in range(w.heads):
+            blocks = {0, nb - 1} | set(int(x) for x in rng.choice(nb, blocks_random, replace=False))
+            for i in sorted(blocks):
+                toks = {i * w.block, i * w.block + w.block - 1} | set(
+                    int(x) for x in i * w.block + rng.choice(w.block, per_block - 2, replace=False))
+                rows += [(b * w.heads + h) * w.seq + t for t in sorted(toks)]
+    return np.array(rows, dtype=np.int64)
+
+
+def planted_positions(w, seed):
+    """For every head, a token in a strided key block (<= nb/2) that the last
+    query block sees, chosen with the oracle's rule."""
+    rng = np.random.default_rng(seed)
+    nb, last = w.num_blocks, w.num_blocks - 1
+    pos = {}
+    for h in range(w.heads):
+        cands = [j for j in range(nb // 2 + 1)
+                 if oracle.block_active(h, last, j, w.stride, w.local) and last - j >= w.local]
+        j = int(rng.choice(cands))
+        pos[h] = j * w.block + int(rng.integers(w.block))
+    return pos
+
+
+@pytest.mark.parametrize("name", ["prefill_1p3b", "prefill_7b_hybrid", "prefill_long_131k"])
+def test_full_size_workload_sampled_rows(s2gpu, name):
+    w = synth.PREFILL_WORKLOADS[name]
+    plant = planted_positions(w, 7) if w.planted else None
+    q, k, v = synth.prefill_inputs(w, device="cuda", plant_positions=plant)
+    out, lse = run_prefill(s2gpu, w, q, k, v)
+    rows = sample_rows(w, seed=w.seed + 100)
+    qh, kh, vh = q.cpu(), k.cpu(), v.cpu()
+    ref, ref_lse = oracle.prefill(qh, kh, vh, w.block, w.stride, w.local, w.scale, w.dense_heads,
+                                  rows=rows)
+    got = out.reshape(-1, w.head_dim)[torch.from_numpy(rows).cuda()]
+    parity(got, ref)
+    parity(lse.reshape(-1)[torch.from_numpy(rows).cuda()], ref_lse, max_tol=1e-3, mean_tol=1e-4)
+    assert torch.isfinite(out).all()
+    if plant:
+        # the last query row of each head retrieves the planted value row
+        for h, t in plant.items():
+            o_last = out[0, h, w.seq - 1].double().cpu()
+            assert (o_last - v[0, h, t].double().cpu()).abs().max().item() < 2e-2
