@@ -1,0 +1,526 @@
+#!/usr/bin/env python3
+"""Benchmark of the HHST sparse-attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  * prefill (block-sparse attention, tcgen05 kernel) over the 1.3B-shaped
+    layer batch: batch 4, 16 heads, head_dim 128, seq 8192, B 64, S 8, L 2,
+    per-head K scale U(0.5, 2);
+  * decode (split-KV paged kernel + combine) over 64 sequences, 32 heads,
+    head_dim 128, contexts U[4096, 32768], 16-token pages, permuted block table,
+    B 128, S 16, L 4.
+The layouts are built once (host, per layout) before timing.
+
+Headline: prefill effective TFLOP/s (4 * head_dim per visible (query, key)
+pair; the dense work the pattern skips is not counted), from CUDA events around
+the prefill launches inside the timed steps. The decode part reports active
+K+V GB/s and tokens/s in "decode". Multi-GPU: one process per GPU, each
+processing its own batch (weak scaling, no collective on the data path);
+time = max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HHST sparse attn fwd effective TFLOP/s & % bf16 TC peak; decode KV GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------- work counts
+
+def prefill_flops(lay, w) -> int:
+    """Algorithmic FLOPs: 4*D per visible (q, k) pair. A non-diagonal active
+    block holds B*B pairs, a diagonal block B*(B+1)/2."""
+    nnz = int(lay.col_idx.size)
+    rows = lay.heads * lay.num_blocks  # every row holds exactly one diagonal block
+    B = w.block
+    pairs = (nnz - rows) * B * B + rows * B * (B + 1) // 2
+    return 4 * w.head_dim * pairs * w.batch
+
+
+def prefill_issued_flops(lay, w) -> int:
+    return 4 * w.head_dim * w.block * w.block * int(lay.col_idx.size) * w.batch
+
+
+def decode_counts(lay, w, ctx_lens):
+    """(active tokens over all (seq, head), pages touched) for the batch."""
+    tokens = pages = 0
+    B = w.block
+    for n in ctx_lens:
+        n = int(n)
+        i = (n - 1) // B
+        for h in range(w.heads):
+            base = h * (lay.num_blocks + 1)
+            for j in lay.col_idx[lay.row_ptr[base + i]:lay.row_ptr[base + i + 1]]:
+                t0, t1 = int(j) * B, min((int(j) + 1) * B, n)
+                tokens += t1 - t0
+                pages += -(-(t1 - t0) // 16)
+    return tokens, pages
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "head_heterogeneous_block_s2_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".cpp")):
+            h.update(fn.encode())
+            h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("source_sha") != source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML (read-only)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report nothing rather than guess
+            log(f"clock sampling unavailable: {e}")
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((time.time(), mhz, rs, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        loaded = [s for s in self.samples if not (s[2] & 0x1)] or self.samples
+        reasons = set()
+        for _, _, rs, _ in loaded:
+            for bit, name in self.REASONS.items():
+                if rs & bit and bit != 0x1:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in loaded), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, dist):
+    import torch
+
+    from head_heterogeneous_block_s2_b200 import s2attn, synth
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    s2attn.load()
+    wp = synth.PREFILL_WORKLOADS[args.prefill]
+    wd = synth.DECODE_WORKLOADS[args.decode] if args.decode != "none" else None
+    if wd is not None and args.decode_batch > 0:
+        wd = wd.with_(batch=args.decode_batch)
+
+    # setup (untimed): inputs resident in HBM, layouts built once per layout
+    t0 = time.time()
+    q, k, v = synth.prefill_inputs(wp, device=dev)
+    lay_p = s2attn.build_layout(wp.heads, wp.block, wp.stride, wp.local, wp.num_blocks,
+                                wp.dense_heads, device=dev)
+    layout_ms = None
+    t1 = time.time()
+    _ = s2attn.build_layout(wp.heads, wp.block, wp.stride, wp.local, wp.num_blocks, wp.dense_heads)
+    layout_ms = (time.time() - t1) * 1e3
+    out = torch.empty_like(q)
+    flops = prefill_flops(lay_p, wp)
+    issued = prefill_issued_flops(lay_p, wp)
+    if wd is not None:
+        d = synth.decode_inputs(wd, device=dev)
+        nb_d = -(-wd.ctx_max // wd.block)
+        lay_d = s2attn.build_layout(wd.heads, wd.block, wd.stride, wd.local, nb_d, wd.dense_heads,
+                                    device=dev)
+        splits = args.splits if args.splits > 0 else s2attn.decode_auto_splits(wd.batch, wd.heads)
+        ws_n = s2attn.decode_workspace_size(wd.batch, wd.heads, wd.head_dim, splits)
+        ws = torch.empty(max(ws_n, 256), dtype=torch.uint8, device=dev)
+        dout = torch.empty_like(d.q)
+        ctx_host = d.ctx_lens.cpu().numpy()
+        tokens, pages = decode_counts(lay_d, wd, ctx_host)
+        kv_bytes = tokens * wd.head_dim * 2 * 2
+        kv_page_bytes = pages * 16 * wd.head_dim * 2 * 2
+    torch.cuda.synchronize()
+    log(f"[rank {rank}] setup {time.time() - t0:.1f}s; prefill {flops / 1e9:.1f} GFLOP/step"
+        + (f"; decode {kv_bytes / 1e9:.3f} GB active KV, splits {splits}" if wd else ""))
+
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        s2attn.prefill(q, k, v, lay_p, scale=wp.scale, out=out)
+        if evs:
+            evs[1].record(stream)
+        if wd is not None:
+            s2attn.decode(d.q, d.k_cache, d.v_cache, d.block_table, d.ctx_lens, lay_d,
+                          scale=wd.scale, num_splits=splits, out=dout, workspace=ws)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rc, flags = s2attn.device_status(reset=True)
+    if rc != 0:
+        raise RuntimeError(f"device flags {flags:#x} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    sampler.stop()
+    total_ms = start.elapsed_time(end)
+    pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs) if wd else 0.0
+    rc, flags = s2attn.device_status(reset=True)
+    if rc != 0:
+        raise RuntimeError(f"device flags {flags:#x} after timing")
+
+    # ---------------- end to end through the public API with host buffers
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, args.e2e_steps))
+    hq = q.cpu().pin_memory()
+    hk = k.cpu().pin_memory()
+    hv = v.cpu().pin_memory()
+    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    gq, gk, gv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = out.numel() * out.element_size()
+    if wd is not None:
+        hdq = d.q.cpu().pin_memory()
+        hbt = d.block_table.cpu().pin_memory()
+        hcl = d.ctx_lens.cpu().pin_memory()
+        hdout = torch.empty(d.q.shape, dtype=d.q.dtype).pin_memory()
+        gdq, gbt, gcl = torch.empty_like(d.q), torch.empty_like(d.block_table), torch.empty_like(d.ctx_lens)
+        h2d += sum(t.numel() * t.element_size() for t in (hdq, hbt, hcl))
+        d2h += hdout.numel() * hdout.element_size()
+
+    def e2e_step(ev):
+        ev[0].record(stream)
+        gq.copy_(hq, non_blocking=True)
+        gk.copy_(hk, non_blocking=True)
+        gv.copy_(hv, non_blocking=True)
+        s2attn.prefill(gq, gk, gv, lay_p, scale=wp.scale, out=out)
+        hout.copy_(out, non_blocking=True)
+        ev[1].record(stream)
+        if wd is not None:
+            gdq.copy_(hdq, non_blocking=True)
+            gbt.copy_(hbt, non_blocking=True)
+            gcl.copy_(hcl, non_blocking=True)
+            s2attn.decode(gdq, d.k_cache, d.v_cache, gbt, gcl, lay_d, scale=wd.scale,
+                          num_splits=splits, out=dout, workspace=ws)
+            hdout.copy_(dout, non_blocking=True)
+        ev[2].record(stream)
+
+    e2e_pre_ms = e2e_dec_ms = 0.0
+    if e2e_steps:
+        warm = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e2e_step(warm)
+        torch.cuda.synchronize()
+        eevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(e2e_steps)]
+        if dist:
+            dist.barrier()
+        for i in range(e2e_steps):
+            e2e_step(eevs[i])
+        torch.cuda.synchronize()
+        e2e_pre_ms = sum(e[0].elapsed_time(e[1]) for e in eevs)
+        e2e_dec_ms = sum(e[1].elapsed_time(e[2]) for e in eevs) if wd else 0.0
+        assert torch.equal(hout, out.cpu()), "e2e output differs from the device output"
+
+    # ---------------- max over ranks
+    vals = [total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms]
+    if dist:
+        import torch.distributed as tdist
+
+        t = torch.tensor(vals, dtype=torch.float64, device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        vals = t.tolist()
+    total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms = vals
+    clocks = sampler.summary()
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    K = args.steps
+    tc_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    pre_tflops = world * flops * K / (pre_ms * 1e-3) / 1e12
+    per_launch_tflops = flops / (pre_ms / K * 1e-3) / 1e12
+    launches = K * (1 + ((1 + (1 if splits > 1 else 0)) if wd else 0))
+    splits = splits if wd else 0
+    line = {
+        "metric": METRIC,
+        "value": round(pre_tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, torch generator on device)",
+        "config": {
+            "workload": f"{wp.name}+{wd.name}" if wd else wp.name,
+            "prefill": {"batch": wp.batch, "heads": wp.heads, "head_dim": wp.head_dim,
+                        "seq": wp.seq, "block": wp.block, "stride": wp.stride,
+                        "local": wp.local, "dense_heads": list(wp.dense_heads),
+                        "algorithmic_gflop_per_step": round(flops / 1e9, 3),
+                        "issued_gflop_per_step": round(issued / 1e9, 3),
+                        "ms_per_step": round(pre_ms / K, 4)},
+            "layout_build_ms_host": round(layout_ms, 3),
+            "l2": "inputs larger than L2 (prefill Q+K+V 403 MB; decode active KV > 1.7 GB)",
+            "parallelism": f"replicas x{world} (no data-path collective)",
+        },
+        "roofline": {
+            "kernel": "s2_prefill_kernel<128,64>",
+            "bound": "tensor",
+            "achieved": round(per_launch_tflops, 2),
+            "peak": tc_peak,
+            "unit": "TFLOP/s",
+            "frac": round(per_launch_tflops / tc_peak, 4),
+            "traffic": load_traffic("s2_prefill_kernel", wp.name),
+            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long loop)",
+        },
+        "e2e": None if not e2e_steps else {
+            "value": round(world * flops * e2e_steps / (e2e_pre_ms * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "steps": e2e_steps,
+            "what": "s2attn.prefill/decode with Q/K/V (and decode q, block table, context lengths) "
+                    "copied from pinned host memory and outputs read back each step; "
+                    "the KV cache stays resident",
+        },
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if wd is not None:
+        dec_gbs = world * kv_bytes * K / (dec_ms * 1e-3) / 1e9
+        per_launch_gbs = kv_bytes / (dec_ms / K * 1e-3) / 1e9
+        hbm = float(peaks["hbm_gbs"])
+        line["decode"] = {
+            "value": round(dec_gbs, 1), "unit": "GB/s",
+            "tokens_per_s": round(world * wd.batch * K / (dec_ms * 1e-3), 1),
+            "ms_per_step": round(dec_ms / K, 4),
+            "active_kv_bytes_per_step": kv_bytes,
+            "page_granular_kv_bytes_per_step": kv_page_bytes,
+            "num_splits": splits,
+            "config": {"batch": wd.batch, "heads": wd.heads, "head_dim": wd.head_dim,
+                       "ctx": [wd.ctx_min, wd.ctx_max], "page": wd.page_size,
+                       "block": wd.block, "stride": wd.stride, "local": wd.local},
+            "roofline": {"kernel": "s2_decode_split_kernel<128>" + (" + combine" if splits > 1 else ""),
+                         "bound": "hbm", "achieved": round(per_launch_gbs, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(per_launch_gbs / hbm, 4),
+                         "traffic": load_traffic("s2_decode_split_kernel", wd.name),
+                         "peak_source": f"{peak_src} hbm_gbs"},
+            "e2e": None if not e2e_steps else {
+                "value": round(world * kv_bytes * e2e_steps / (e2e_dec_ms * 1e-3) / 1e9, 1),
+                "unit": "GB/s"},
+        }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wp, args.cpu_seconds)
+    return line
+
+
+# ---------------------------------------------------------------- oracle arm
+
+def oracle_sample(wp, n_rows, seed, q=None, k=None, v=None):
+    """Time the fp64 oracle on n_rows seeded random rows of the prefill workload.
+    Returns (seconds, algorithmic flops of those rows, threads)."""
+    import oracle
+    from head_heterogeneous_block_s2_b200 import synth
+
+    if q is None:
+        q, k, v = synth.prefill_inputs(wp)
+    rng = np.random.default_rng(seed)
+    total = wp.batch * wp.heads * wp.seq
+    rows = np.sort(rng.choice(total, n_rows, replace=False)).astype(np.int64)
+    # visible keys of each sampled row (the work the definition does)
+    mask = oracle.block_mask(wp.heads, wp.num_blocks, wp.stride, wp.local, wp.dense_heads)
+    t = rows % wp.seq
+    h = (rows // wp.seq) % wp.heads
+    i = t // wp.block
+    full = mask[h, i, :].astype(np.int64)  # active blocks of each row
+    nfull = full.sum(1) - 1  # blocks before the diagonal
+    keys = nfull * wp.block + (t % wp.block) + 1
+    flops = int(4 * wp.head_dim * keys.sum())
+    t0 = time.perf_counter()
+    oracle.prefill(q, k, v, wp.block, wp.stride, wp.local, wp.scale, wp.dense_heads, rows=rows)
+    dt = time.perf_counter() - t0
+    return dt, flops, oracle.default_threads(), (q, k, v)
+
+
+def cpu_baseline(wp, seconds):
+    """The oracle as it stands, on the host cores, over a bounded row sample
+    calibrated to take about `seconds`."""
+    dt, fl, th, qkv = oracle_sample(wp, 512, 1)
+    n = int(min(wp.batch * wp.heads * wp.seq, max(512, 512 * seconds / max(dt, 1e-3))))
+    dt, fl, th, _ = oracle_sample(wp, n, 2, *qkv)
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": th, "kind": "oracle",
+            "sample": f"{n} seeded random query rows of {wp.name} "
+                      f"({n / (wp.batch * wp.heads * wp.seq):.2%} of the batch), fp64, "
+                      f"{dt:.1f} s on {th} threads"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    from head_heterogeneous_block_s2_b200 import synth
+
+    wp = synth.PREFILL_WORKLOADS[args.prefill]
+    # calibrate rows per step so the whole run takes about args.ref_seconds
+    dt, fl, th, qkv = oracle_sample(wp, 256, 1)
+    per_step_s = args.ref_seconds / max(1, args.steps + args.warmup)
+    n = int(max(16, min(wp.batch * wp.heads * wp.seq, 256 * per_step_s / max(dt, 1e-4))))
+    for i in range(args.warmup):
+        oracle_sample(wp, n, 100 + i, *qkv)
+    tot_t = tot_f = 0.0
+    for i in range(args.steps):
+        dt, fl, th, _ = oracle_sample(wp, n, 1000 + i, *qkv)
+        tot_t += dt
+        tot_f += fl
+    val = tot_f / tot_t / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wp.name, "rows_per_step": n},
+        "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": th, "kind": "oracle",
+                         "sample": f"{n} seeded random query rows of {wp.name} per step"},
+        "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--prefill", default="prefill_1p3b",
+                    choices=["tiny", "prefill_1p3b", "prefill_7b_hybrid", "prefill_long_131k"])
+    ap.add_argument("--decode", default="decode_paged", choices=["decode_paged", "none"])
+    ap.add_argument("--splits", type=int, default=0, help="decode splits (0 = automatic)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="override the decode batch (small cases for profiling only)")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling only)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank)
+        else:
+            line = run_ours(args, rank, world, dist)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
