@@ -320,3 +320,61 @@ int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- decode without allocation
+//
+// s2_attn_decode_noalloc: the same split-KV decode, but its split partials go
+// to a scratch array that lives in this library's own device image instead of
+// a caller-supplied workspace. Meant for callers that cannot allocate device
+// memory themselves (see the header). The array is a file-scope device
+// variable: every GPU that loads the library holds S2_NOALLOC_SCRATCH_BYTES of
+// it until the process exits, and all calls share it.
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[S2_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch per device. In host code the symbol
+// name is only a host-side stand-in, so the real address is looked up once
+// per device (with that device current) and passed to the kernels.
+void* g_noalloc_addr[kMaxDevices] = {};
+
+int noalloc_scratch(int dev, void** out)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return S2_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return S2_OK;
+}
+
+}  // namespace
+
+extern "C" int s2_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_table, const int32_t* ctx_lens,
+                                      int32_t batch, int32_t heads, int32_t head_dim,
+                                      int32_t page_size, int32_t max_pages, int64_t num_pages,
+                                      int32_t block_size, int32_t num_blocks,
+                                      const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz,
+                                      float scale, void* out, float* lse, int32_t num_splits,
+                                      void* stream)
+{
+    if (batch < 1 || heads < 1 || num_splits > kMaxSplits) return S2_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
+    const int32_t sp = num_splits > 0 ? num_splits : s2_attn_decode_auto_splits(batch, heads);
+    if (ws_bytes(batch, heads, head_dim, sp) > S2_NOALLOC_SCRATCH_BYTES) return S2_ERR_CAPACITY;
+    int dev = 0;
+    int rc = device_ready(&dev);
+    if (rc) return rc;
+    void* scratch = nullptr;
+    rc = noalloc_scratch(dev, &scratch);
+    if (rc) return rc;
+    // Nothing in the scratch has to start at zero: the split kernel writes
+    // every partial (max, sum, output) that the combine kernel then reads.
+    return s2_attn_decode(q, k_cache, v_cache, block_table, ctx_lens, batch, heads, head_dim,
+                          page_size, max_pages, num_pages, block_size, num_blocks, row_ptr,
+                          col_idx, nnz, scale, out, lse, scratch, S2_NOALLOC_SCRATCH_BYTES, sp,
+                          stream);
+}

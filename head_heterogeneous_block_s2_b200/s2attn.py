@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "S2_OK", 1: "S2_ERR_INVALID_ARG", 2: "S2_ERR_UNSUPPORTED", 3:
 
 EXPORTED = ("s2_status_string", "s2_build_layout", "s2_attn_prefill",
             "s2_attn_decode_workspace_size", "s2_attn_decode_auto_splits", "s2_attn_decode",
-            "s2_device_status", "s2_set_wait_timeout_ns", "s2_version")
+            "s2_device_status", "s2_set_wait_timeout_ns", "s2_version", "s2_attn_decode_noalloc")
 
 
 class S2Error(RuntimeError):
@@ -72,6 +72,9 @@ def load(path: str = LIB_PATH):
     lib.s2_attn_decode.restype = ctypes.c_int
     lib.s2_attn_decode.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64, i32, i32, vp,
                                    vp, i64, f32, vp, vp, vp, sz, i32, vp]
+    lib.s2_attn_decode_noalloc.restype = ctypes.c_int
+    lib.s2_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i64, i32,
+                                           i32, vp, vp, i64, f32, vp, vp, i32, vp]
     lib.s2_device_status.restype = ctypes.c_int
     lib.s2_device_status.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)]
     lib.s2_set_wait_timeout_ns.restype = ctypes.c_int
@@ -245,6 +248,49 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                                _ptr(out), _ptr(lse), _ptr(workspace), ws_len, num_splits,
                                _stream(q.device))
     _check(rc, "s2_attn_decode")
+    return (out, lse) if lse is not None else out
+
+
+# Size of the library's built-in decode scratch (S2_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   block_table: torch.Tensor, ctx_lens: torch.Tensor, layout: Layout,
+                   scale: Optional[float] = None, num_splits: int = 0,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   want_lse: bool = False):
+    """s2_attn_decode_noalloc: decode for callers that cannot allocate device
+    memory. The split partials go to the library's own built-in scratch, so no
+    workspace is passed; ``out`` (and ``lse``) must be supplied by a caller
+    that cannot allocate (they are only created here for convenience). Calls
+    share that scratch, so calls that may overlap on the GPU must be ordered
+    by the caller."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n)
+    _need(block_table, "block_table", torch.int32)
+    _need(ctx_lens, "ctx_lens", torch.int32)
+    batch, heads, hd = q.shape
+    num_pages, h2, page_size, hd2 = k_cache.shape
+    if h2 != heads or hd2 != hd or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape does not match q")
+    if layout.d_row_ptr is None:
+        layout.to(q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out")
+    if lse is None and want_lse:
+        lse = torch.empty((batch, heads), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    rc = load().s2_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                       _ptr(ctx_lens), batch, heads, hd, page_size,
+                                       block_table.shape[1], num_pages, layout.block_size,
+                                       layout.num_blocks, _ptr(layout.d_row_ptr),
+                                       _ptr(layout.d_col_idx), layout.nnz, sc, _ptr(out), _ptr(lse),
+                                       num_splits, _stream(q.device))
+    _check(rc, "s2_attn_decode_noalloc")
     return (out, lse) if lse is not None else out
 
 

@@ -160,6 +160,39 @@ int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                    void* workspace, size_t workspace_bytes, int32_t num_splits,
                    void* stream);
 
+/*
+ * Decode that allocates nothing: s2_attn_decode with the split partials kept
+ * in a scratch array inside the library instead of a caller workspace.
+ *
+ * This entry point has no counterpart in the paper; it exists for callers that
+ * cannot call cudaMalloc: plug-ins whose host framework owns every device
+ * allocation and gives them none, C programs that link this library without a
+ * device allocator of their own, and latency-critical loops that must not
+ * allocate or free because cudaMalloc and cudaFree can synchronise the device.
+ *
+ * Arguments, layouts and results are those of s2_attn_decode, without
+ * workspace and workspace_bytes. The scratch is a file-scope device array of
+ * S2_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU loading the library holds
+ * until the process exits. A shape whose partials need more than that
+ * (s2_attn_decode_workspace_size(batch, heads, head_dim, num_splits) >
+ * S2_NOALLOC_SCRATCH_BYTES) is rejected with S2_ERR_CAPACITY before anything
+ * runs. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture. All calls share the one array, which keeps the
+ * last call's contents (nothing in it has to start at zero): calls that can
+ * overlap on the GPU, on different streams, race on it and must be ordered by
+ * the caller. The function calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ */
+#define S2_NOALLOC_SCRATCH_BYTES (8u << 20)
+int s2_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_table, const int32_t* ctx_lens,
+                           int32_t batch, int32_t heads, int32_t head_dim, int32_t page_size,
+                           int32_t max_pages, int64_t num_pages, int32_t block_size,
+                           int32_t num_blocks, const int32_t* row_ptr, const int32_t* col_idx,
+                           int64_t nnz, float scale, void* out, float* lse,
+                           int32_t num_splits, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Device status and limits                                                  */
 /* ------------------------------------------------------------------------ */
