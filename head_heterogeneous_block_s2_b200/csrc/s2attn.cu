@@ -17,6 +17,7 @@
 #include "ptx.cuh"
 #include "prefill_sm100.cuh"
 #include "decode.cuh"
+#include "prefill_pair_sm100.cuh"
 
 namespace {
 
@@ -99,24 +100,25 @@ template <int HD, int BK>
 int launch_prefill(const void* q, const void* k, const void* v, s2::PrefillParams& pp, int dev,
                    int attr_slot, cudaStream_t stream)
 {
-    using C = s2::PrefillCfg<HD, BK>;
+    using C = s2::PairCfg<HD, BK>;
     const uint64_t rows = (uint64_t)pp.batch * pp.heads * pp.seq;
     CUtensorMap mq, mk, mv;
     if (make_map(&mq, q, rows, HD, 128) || make_map(&mk, k, rows, HD, BK) ||
         make_map(&mv, v, rows, HD, BK))
         return S2_ERR_CUDA;
-    auto kern = s2::s2_prefill_kernel<HD, BK>;
+    auto kern = s2::s2_prefill_pair_kernel<HD, BK>;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!g_dev[dev].prefill_attr_done[attr_slot]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      C::SMEM_ALLOC) != cudaSuccess)
                 return S2_ERR_CUDA;
+
             g_dev[dev].prefill_attr_done[attr_slot] = true;
         }
     }
-    const uint64_t grid = (uint64_t)pp.batch * pp.heads * pp.nqt;
-    kern<<<(unsigned)grid, 192, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
+    const uint64_t grid = (uint64_t)pp.batch * pp.heads * ((pp.nqt + 1) / 2);
+    kern<<<(unsigned)grid, 384, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
