@@ -8,9 +8,16 @@
 // ones, so the CTA walks the union of their key-block lists, loads each key
 // block once, and runs each tile's MMAs only on the blocks that tile sees.
 //
+// The kernel is persistent: one CTA per SM walks a static share of the work
+// items (tile pairs, heaviest query blocks first), so the next item's loads
+// and S MMAs overlap the current item's last blocks and epilogue.
+//
 // CTA = 12 warps:
-//   warp 0      TMA producer: Q of both tiles once, then K and V of each union
-//               block into an ST-stage ring (SWIZZLE_128B, 64-column panels).
+//   warp 0      K/V producer: K and V of each union block, item after item,
+//               into an ST-stage ring (TMA, SWIZZLE_128B, 64-column panels).
+//   warp 2      Q producer: Q of both tiles of each item once the previous
+//               item's S MMAs are done with the Q buffer; prefetches the next
+//               item's Q into L2.
 //   warp 1      owns TMEM; one thread issues tcgen05.mma:
 //               S_t = Q_t K^T (A and B from shared memory) into TMEM, and
 //               O_t += P_t V with P_t read from TMEM (A operand) and V from
@@ -21,7 +28,7 @@
 //               reaches its own block), keeps a running max and sum in the
 //               log2 domain, writes P (bf16 pairs) over the S columns in TMEM,
 //               and at the end normalises O and stores it with the LSE.
-//   warps 2, 3  idle (no work; they only take part in block-wide barriers).
+//   warp 3      idle (no work; it only takes part in block-wide barriers).
 // The two softmax warpgroups ping-pong: while one computes exponentials for
 // its tile, the tensor core runs the other tile's MMAs.
 //
@@ -30,6 +37,9 @@
 //    all earlier ones. S_t(next) is issued after PV_t(current), so when the
 //    softmax sees S_t(next) complete, PV_t(current) has finished: P_t's TMEM
 //    columns (aliased on S_t) are free and O_t is stable for a rescale.
+//  * A tile's first P of the next item is published only after its warpgroup
+//    has read O out of TMEM (tcgen05.wait::ld) for the previous item, so the
+//    next item's first PV (which overwrites O) cannot race the epilogue.
 //  * The running-max reference only moves when the max grows by more than
 //    2^8 (kRescaleLog2), so O rescales are rare; P values stay <= 256.
 // Every role walks the union list itself from the CSR arrays, so no shared
@@ -53,22 +63,37 @@ struct PairCfg {
     static constexpr int ROWS = (BK == 128) ? 2 : 4;       // query blocks per CTA
     static constexpr uint32_t QBYTES = M * HD * 2;         // one tile's Q
     static constexpr uint32_t KVBYTES = BK * HD * 2;       // one K (or V) block
-    static constexpr int ST = (2 * QBYTES + 4 * 2 * KVBYTES <= 200 * 1024) ? 4 : 2;
+    static constexpr int LIST_CAP = 2048;                  // union entries per item (>= nb)
+    static constexpr uint32_t LIST_BYTES = 2 * LIST_CAP * 4;  // double-buffered
+    static constexpr int ST = (2 * QBYTES + 4 * 2 * KVBYTES + LIST_BYTES <= 220 * 1024) ? 4 : 2;
+    static constexpr int PREFETCH = 4;                     // K/V blocks prefetched into L2 ahead
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = OFF_Q + 2 * QBYTES;
     static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;
-    static constexpr uint32_t OFF_BAR = OFF_V + ST * KVBYTES;
-    // barriers: q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain
-    static constexpr int NBAR = 1 + 3 * ST + 6 + 1;
+    static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
+    static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
+    // barriers: q_full, q_empty, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2],
+    // pv_done[2], drain, list_full[2], list_empty[2]
+    static constexpr int NBAR = 2 + 3 * ST + 6 + 1 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 16;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
     static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD) <= 256 ? 256 : 512;
+    // list_empty arrivals per item: K/V producer, MMA issuer, 8 softmax warps
+    static constexpr uint32_t LIST_CONSUMERS = 10;
     __host__ __device__ static constexpr uint32_t colS(int t) { return (uint32_t)(t * BK); }
     __host__ __device__ static constexpr uint32_t colO(int t) { return (uint32_t)(2 * BK + t * HD); }
     static_assert(2 * BK + 2 * HD <= 512, "TMEM budget");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
+
+// Union-list entry: key block j (bits 0..23), row tags (bits 24..27), last flag (bit 31).
+__device__ __forceinline__ uint32_t list_pack(int j, int bits, bool last)
+{
+    return (uint32_t)j | ((uint32_t)bits << 24) | (last ? 0x80000000u : 0u);
+}
+__device__ __forceinline__ int list_j(uint32_t e) { return (int)(e & 0xFFFFFFu); }
+__device__ __forceinline__ int list_bits(uint32_t e) { return (int)((e >> 24) & 0xFu); }
 
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -141,6 +166,29 @@ __device__ __forceinline__ bool tile_sees(int bits, int t)
     return BK == 128 ? ((bits >> t) & 1) != 0 : ((bits >> (2 * t)) & 3) != 0;
 }
 
+// One work item: a pair of adjacent 128-row query tiles of one (batch, head).
+struct PairItem {
+    int qt0, qb0, rp;
+    bool tile1;
+    int64_t row_base;
+};
+
+template <int BK>
+__device__ __forceinline__ PairItem pair_item(const PrefillParams& p, int w)
+{
+    const int npairs = (p.nqt + 1) >> 1;
+    const int BH = p.batch * p.heads;
+    const int pr = npairs - 1 - w / BH;  // heaviest pairs first
+    const int bh = w % BH;
+    PairItem it;
+    it.qt0 = 2 * pr;
+    it.tile1 = it.qt0 + 1 < p.nqt;
+    it.qb0 = (BK == 128) ? it.qt0 : 2 * it.qt0;
+    it.rp = (bh % p.heads) * (p.nb + 1);
+    it.row_base = (int64_t)bh * p.seq;
+    return it;
+}
+
 template <int HD, int BK>
 __global__ void __launch_bounds__(384, 1)
 s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -152,31 +200,28 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                                                ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    // Heaviest pairs (largest query blocks) first.
-    const int npairs = (p.nqt + 1) >> 1;
-    const int BH = p.batch * p.heads;
-    const int pr = npairs - 1 - (int)(blockIdx.x / BH);
-    const int bh = (int)(blockIdx.x % BH);
-    const int h = bh % p.heads;
-    const int qt0 = 2 * pr;                        // first query tile
-    const bool tile1 = qt0 + 1 < p.nqt;            // second tile exists
-    const int qb0 = (BK == 128) ? qt0 : 2 * qt0;   // first query block
-    const int64_t row_base = (int64_t)bh * p.seq;
+    const int num_items = p.batch * p.heads * ((p.nqt + 1) >> 1);
 
     const uint32_t bar_q = sb + C::OFF_BAR;
-    auto bar_kf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
-    auto bar_vf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + C::ST + s); };
-    auto bar_ke = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + 2 * C::ST + s); };
-    auto bar_sf = [&](int t) { return sb + C::OFF_BAR + 8u * (1 + 3 * C::ST + t); };
-    auto bar_pf = [&](int t) { return sb + C::OFF_BAR + 8u * (3 + 3 * C::ST + t); };
-    auto bar_pv = [&](int t) { return sb + C::OFF_BAR + 8u * (5 + 3 * C::ST + t); };
-    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (7 + 3 * C::ST);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-    volatile int* abort_cta = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    const uint32_t bar_qe = sb + C::OFF_BAR + 8u;
+    auto bar_kf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + s); };
+    auto bar_vf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + C::ST + s); };
+    auto bar_ke = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + 2 * C::ST + s); };
+    auto bar_sf = [&](int t) { return sb + C::OFF_BAR + 8u * (2 + 3 * C::ST + t); };
+    auto bar_pf = [&](int t) { return sb + C::OFF_BAR + 8u * (4 + 3 * C::ST + t); };
+    auto bar_pv = [&](int t) { return sb + C::OFF_BAR + 8u * (6 + 3 * C::ST + t); };
+    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (8 + 3 * C::ST);
+    auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (9 + 3 * C::ST + b); };
+    auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (11 + 3 * C::ST + b); };
+    const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
+    int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2..3] list lengths
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
+    volatile int* abort_cta = misc + 1;
+    volatile int* list_len = misc + 2;
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
+        mbar_init(bar_qe, 1);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_kf(s), 1);
             mbar_init(bar_vf(s), 1);
@@ -186,6 +231,8 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             mbar_init(bar_sf(t), 1);
             mbar_init(bar_pf(t), 128);
             mbar_init(bar_pv(t), 1);
+            mbar_init(bar_lf(t), 1);
+            mbar_init(bar_le(t), C::LIST_CONSUMERS);
         }
         mbar_init(bar_dr, 1);
         *abort_cta = 0;
@@ -201,30 +248,87 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     const uint32_t tmem = *tmem_slot;
     const WaitCtl ctl{p.timeout_ns, p.gflags, abort_cta};
     constexpr uint64_t kDrainNs = 200000000ull;
-    const int rp = h * (p.nb + 1);
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 2) {
+        // ------------------------------------------------------------ list builder + Q producer
         if (lane == 0) {
-            UnionWalk<C::ROWS> it;
-            const bool ok = it.init(p.row_ptr, rp, qb0, p.nb, p.nnz);
-            if (!ok) atomicOr(p.gflags, kFlagIndex);
-            int n = 0;
-            if (ok) {
-                mbar_arrive_expect_tx(bar_q, (tile1 ? 2 : 1) * C::QBYTES);
-                for (int t = 0; t < (tile1 ? 2 : 1); ++t)
+            int k = 0;
+            uint32_t* wlist = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
+            for (int w = blockIdx.x; w < num_items; w += gridDim.x, ++k) {
+                const PairItem I = pair_item<BK>(p, w);
+                const int b = k & 1;
+                // union list of this item into buffer b (free once item k-2 is consumed)
+                if (!mbar_wait(bar_le(b), ((k >> 1) & 1) ^ 1, ctl)) break;
+                UnionWalk<C::ROWS> it;
+                int len = 0;
+                if (it.init(p.row_ptr, I.rp, I.qb0, p.nb, p.nnz)) {
+                    for (;;) {
+                        int j, bits;
+                        bool last, bad;
+                        it.next(p.col_idx, j, bits, last, bad);
+                        if (bad) atomicOr(p.gflags, kFlagIndex);
+                        if (len == C::LIST_CAP - 1 && !last) {  // cannot happen when nb <= LIST_CAP
+                            atomicOr(p.gflags, kFlagIndex);
+                            last = true;
+                        }
+                        wlist[b * C::LIST_CAP + len++] = list_pack(j, bits, last);
+                        if (last) break;
+                    }
+                } else {
+                    atomicOr(p.gflags, kFlagIndex);
+                }
+                list_len[b] = len;
+                mbar_arrive(bar_lf(b));
+                // Q of both tiles, once the previous item's S MMAs are done with the buffer
+                if (!mbar_wait(bar_qe, (k & 1) ^ 1, ctl)) break;
+                mbar_arrive_expect_tx(bar_q, (I.tile1 ? 2 : 1) * C::QBYTES);
+                for (int t = 0; t < (I.tile1 ? 2 : 1); ++t)
 #pragma unroll
                     for (int pn = 0; pn < HD / 64; ++pn)
                         tma_load_2d(sb + C::OFF_Q + t * C::QBYTES + pn * (C::M * 128), &tmQ, pn * 64,
-                                    (int32_t)(row_base + (qt0 + t) * C::M), bar_q);
-                for (;;) {
-                    int j, bits;
-                    bool last, bad;
-                    it.next(p.col_idx, j, bits, last, bad);
-                    if (bad) atomicOr(p.gflags, kFlagIndex);
+                                    (int32_t)(I.row_base + (I.qt0 + t) * C::M), bar_q);
+                if (w + (int)gridDim.x < num_items) {  // next item's Q into L2
+                    const PairItem J = pair_item<BK>(p, w + gridDim.x);
+                    for (int t = 0; t < (J.tile1 ? 2 : 1); ++t)
+                        for (int pn = 0; pn < HD / 64; ++pn)
+                            tma_prefetch_2d(&tmQ, pn * 64, (int32_t)(J.row_base + (J.qt0 + t) * C::M));
+                }
+            }
+            if (*abort_cta && k > 0) mbar_drain(bar_q, (k - 1) & 1, kDrainNs);
+        }
+        __syncwarp();
+    } else if (warp == 0) {
+        // ------------------------------------------------------------ K/V producer
+        if (lane == 0) {
+            int n = 0, k = 0;
+            bool stop = false;
+            for (int w = blockIdx.x; w < num_items && !stop; w += gridDim.x, ++k) {
+                const PairItem I = pair_item<BK>(p, w);
+                const int b = k & 1;
+                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                const uint32_t* L = list + b * C::LIST_CAP;
+                const int len = list_len[b];
+                for (int e = 0; e < C::PREFETCH && e < len; ++e) {
+                    const int32_t row = (int32_t)(I.row_base + (int64_t)list_j(L[e]) * BK);
+                    for (int pn = 0; pn < HD / 64; ++pn) {
+                        tma_prefetch_2d(&tmK, pn * 64, row);
+                        tma_prefetch_2d(&tmV, pn * 64, row);
+                    }
+                }
+                for (int e = 0; e < len; ++e, ++n) {
+                    if (e + C::PREFETCH < len) {
+                        const int32_t row = (int32_t)(I.row_base + (int64_t)list_j(L[e + C::PREFETCH]) * BK);
+                        for (int pn = 0; pn < HD / 64; ++pn) {
+                            tma_prefetch_2d(&tmK, pn * 64, row);
+                            tma_prefetch_2d(&tmV, pn * 64, row);
+                        }
+                    }
                     const int st = n % C::ST;
-                    if (!mbar_wait(bar_ke(st), ((n / C::ST) & 1) ^ 1, ctl)) break;
-                    const int32_t krow = (int32_t)(row_base + (int64_t)j * BK);
+                    if (!mbar_wait(bar_ke(st), ((n / C::ST) & 1) ^ 1, ctl)) {
+                        stop = true;
+                        break;
+                    }
+                    const int32_t krow = (int32_t)(I.row_base + (int64_t)list_j(L[e]) * BK);
                     mbar_arrive_expect_tx(bar_kf(st), C::KVBYTES);
 #pragma unroll
                     for (int pn = 0; pn < HD / 64; ++pn)
@@ -235,73 +339,80 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     for (int pn = 0; pn < HD / 64; ++pn)
                         tma_load_2d(sb + C::OFF_V + st * C::KVBYTES + pn * (BK * 128), &tmV, pn * 64,
                                     krow, bar_vf(st));
-                    ++n;
-                    if (last) break;
                 }
+                if (!stop) mbar_arrive(bar_le(b));
             }
-            if (*abort_cta && ok) {  // let this CTA's own loads land before exit
-                mbar_drain(bar_q, 0, kDrainNs);
+            if (*abort_cta)  // let this CTA's own loads land before exit
                 for (int m = (n > C::ST ? n - C::ST : 0); m < n; ++m) {
                     mbar_drain(bar_kf(m % C::ST), (m / C::ST) & 1, kDrainNs);
                     mbar_drain(bar_vf(m % C::ST), (m / C::ST) & 1, kDrainNs);
                 }
-            }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            UnionWalk<C::ROWS> it;
-            const bool ok = it.init(p.row_ptr, rp, qb0, p.nb, p.nnz);
             constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);
             constexpr uint32_t idesc_o = umma_idesc(128, HD, 0, 1);
-            bool issued = false;
-            int pvc[2] = {0, 0};
+            bool issued = false, fail = false;
+            int pvc[2] = {0, 0};   // PV MMAs issued per tile (all items)
+            bool first_pv[2] = {true, true};
+            int n = 0;             // union elements consumed (all items)
             auto issue_s = [&](int t, int st) {
                 const uint32_t d = tmem + C::colS(t);
+                const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
+                const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t a = sb + C::OFF_Q + t * C::QBYTES + (kk >> 2) * (C::M * 128) + (kk & 3) * 32;
-                    const uint32_t b = sb + C::OFF_K + st * C::KVBYTES + (kk >> 2) * (BK * 128) + (kk & 3) * 32;
-                    umma_bf16_ss(d, umma_sdesc(a, 16, 1024), umma_sdesc(b, 16, 1024), idesc_s,
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_bf16_ss(d, dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
+                                 dk + (((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4), idesc_s,
                                  kk > 0 ? 1u : 0u);
-                }
                 umma_commit(bar_sf(t));
                 issued = true;
             };
             auto issue_pv = [&](int t, int st) {
+                const uint64_t dv = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, BK * 128, 1024);
+                const uint32_t acc0 = first_pv[t] ? 0u : 1u;
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk) {
-                    const uint32_t b = sb + C::OFF_V + st * C::KVBYTES + kk * (16 * 128);
-                    umma_bf16_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8,
-                                 umma_sdesc(b, BK * 128, 1024), idesc_o,
-                                 (pvc[t] > 0 || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    umma_bf16_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, dv + ((kk * 2048) >> 4),
+                                 idesc_o, kk > 0 ? 1u : acc0);
                 umma_commit(bar_pv(t));
                 ++pvc[t];
+                first_pv[t] = false;
             };
-            do {
-                if (!ok) break;
-                int j, bits, nbits;
-                bool last, nlast, bad;
-                it.next(p.col_idx, j, bits, last, bad);
-                if (!mbar_wait(bar_q, 0, ctl)) break;
-                if (!mbar_wait(bar_kf(0), 0, ctl)) break;
+            int k = 0;
+            for (int w = blockIdx.x; w < num_items && !fail; w += gridDim.x, ++k) {
+                const int b = k & 1;
+                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                const uint32_t* L = list + b * C::LIST_CAP;
+                const int len = list_len[b];
+                if (!mbar_wait(bar_q, k & 1, ctl)) break;
+                if (len == 0) {
+                    umma_commit(bar_qe);
+                    mbar_arrive(bar_le(b));
+                    continue;
+                }
+                first_pv[0] = first_pv[1] = true;
+                uint32_t cur = L[0];
+                if (!mbar_wait(bar_kf(n % C::ST), (n / C::ST) & 1, ctl)) break;
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t)
-                    if (tile_sees<BK>(bits, t)) issue_s(t, 0);
-                bool fail = false;
-                for (int n = 0;; ++n) {
+                    if (tile_sees<BK>(list_bits(cur), t)) issue_s(t, n % C::ST);
+                for (int e = 0;; ++e, ++n) {
+                    const bool last = e + 1 == len;
+                    const uint32_t nxt = last ? 0u : L[e + 1];
+                    const int bits = list_bits(cur), nbits = list_bits(nxt);
                     const int st = n % C::ST;
                     const int st1 = (n + 1) % C::ST;
-                    nbits = 0;
-                    nlast = true;
-                    if (!last) it.next(p.col_idx, j, nbits, nlast, bad);
+                    if (last) umma_commit(bar_qe);  // no more S MMAs of this item read Q
                     bool v_ready = false, k_next_ready = false;
                     if (bits == 0) {  // malformed entry no tile sees: let its loads land first
                         if (!mbar_wait(bar_kf(st), (n / C::ST) & 1, ctl) ||
-                            !mbar_wait(bar_vf(st), (n / C::ST) & 1, ctl))
+                            !mbar_wait(bar_vf(st), (n / C::ST) & 1, ctl)) {
+                            fail = true;
                             break;
+                        }
                     }
                     const int last_t = tile_sees<BK>(bits, 1) ? 1 : (tile_sees<BK>(bits, 0) ? 0 : 1);
                     for (int t = 0; t < 2 && !fail; ++t) {
@@ -324,11 +435,15 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                             issue_s(t, st1);
                         }
                     }
-                    if (fail || last) break;
-                    bits = nbits;
-                    last = nlast;
+                    if (fail) break;
+                    if (last) {
+                        ++n;
+                        break;
+                    }
+                    cur = nxt;
                 }
-            } while (0);
+                if (!fail) mbar_arrive(bar_le(b));
+            }
             if (*abort_cta && issued) {
                 umma_commit(bar_dr);
                 mbar_drain(bar_dr, 0, kDrainNs);
@@ -340,57 +455,81 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const int t = (warp - 4) >> 2;              // tile of this warpgroup
         const int quad = warp & 3;                  // TMEM lane quadrant
         const int r = quad * 32 + lane;             // row within the tile
-        const int qpos = (qt0 + t) * C::M + r;      // query position
-        const int rowbit = (BK == 128) ? t : 2 * t + (r >> 6);
-        const bool active = (t == 0) || tile1;
-        const bool row_valid = active && qpos < p.seq && (qb0 + rowbit) < p.nb;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        float m_used = -1e30f, l = 0.f;
-        int cnt = 0;
-        bool done = false;
-        UnionWalk<C::ROWS> it;
-        const bool ok = it.init(p.row_ptr, rp, qb0, p.nb, p.nnz);
-        if (ok && active) {
-            for (;;) {
-                int j, bits;
-                bool last, bad;
-                it.next(p.col_idx, j, bits, last, bad);
-                if (tile_sees<BK>(bits, t)) {
-                    bool w = mbar_wait(bar_sf(t), cnt & 1, ctl);
-                    if (!__all_sync(0xffffffffu, w)) break;
+        const float sc = p.scale_log2;              // > 0
+        int cnt = 0;                                // S_t blocks processed (all items)
+        bool fail = false;
+        int k = 0;
+        for (int w = blockIdx.x; w < num_items && !fail; w += gridDim.x, ++k) {
+            const PairItem I = pair_item<BK>(p, w);
+            const int qpos = (I.qt0 + t) * C::M + r;
+            const int rowbit = (BK == 128) ? t : 2 * t + (r >> 6);
+            const bool active = (t == 0) || I.tile1;
+            const bool row_valid = active && qpos < p.seq && (I.qb0 + rowbit) < p.nb;
+            const int b = k & 1;
+            bool wl = mbar_wait(bar_lf(b), (k >> 1) & 1, ctl);
+            if (!__all_sync(0xffffffffu, wl)) break;
+            const uint32_t* L = list + b * C::LIST_CAP;
+            const int len = list_len[b];
+            float m_used = -1e30f, l = 0.f;
+            int cnt_item = 0;
+            if (active) {
+                for (int e = 0; e < len; ++e) {
+                    const uint32_t ent = L[e];
+                    const int bits = list_bits(ent);
+                    if (!tile_sees<BK>(bits, t)) continue;
+                    bool wt = mbar_wait(bar_sf(t), cnt & 1, ctl);
+                    if (!__all_sync(0xffffffffu, wt)) {
+                        fail = true;
+                        break;
+                    }
                     tc_fence_after();
-                    uint32_t sr[BK];
+                    uint32_t sr[BK];  // S row; packed P overwrites its front as it is consumed
 #pragma unroll
                     for (int c = 0; c < BK / 32; ++c)
                         tmem_ld32(tl + C::colS(t) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
                     tmem_wait_ld();
                     const bool vis = (bits >> rowbit) & 1;
-                    const int lim = qpos - j * BK;  // key column c visible iff c <= lim
-                    float mt = -INFINITY;
+                    const int lim = qpos - list_j(ent) * BK;  // key column c visible iff c <= lim
+                    if (!__all_sync(0xffffffffu, vis && lim >= BK - 1)) {
 #pragma unroll
-                    for (int c = 0; c < BK; ++c) {
-                        const float x = (vis && c <= lim) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-                        sr[c] = __float_as_uint(x);
-                        mt = fmaxf(mt, x);
+                        for (int c = 0; c < BK; ++c)
+                            if (!(vis && c <= lim)) sr[c] = 0xff800000u;  // -inf
                     }
+                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int c = 0; c < BK; c += 4) {
+                        mx[0] = fmaxf(mx[0], __uint_as_float(sr[c]));
+                        mx[1] = fmaxf(mx[1], __uint_as_float(sr[c + 1]));
+                        mx[2] = fmaxf(mx[2], __uint_as_float(sr[c + 2]));
+                        mx[3] = fmaxf(mx[3], __uint_as_float(sr[c + 3]));
+                    }
+                    const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sc;
                     const float m_cand = fmaxf(m_used, mt);
                     const bool move = m_cand - m_used > kRescaleLog2;
                     const float alpha = move ? ex2(m_used - m_cand) : 1.0f;
                     if (move) m_used = m_cand;
-                    float rs = 0.f;
+                    const float neg_m = -m_used;
+                    float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int c = 0; c < BK / 2; ++c) {
-                        const float p0 = ex2(__uint_as_float(sr[2 * c]) - m_used);
-                        const float p1 = ex2(__uint_as_float(sr[2 * c + 1]) - m_used);
-                        rs += p0 + p1;
-                        sr[c] = pack_bf16x2(p0, p1);
+                    for (int c = 0; c < BK; c += 4) {
+                        const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sc, neg_m));
+                        const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sc, neg_m));
+                        const float p2 = ex2(fmaf(__uint_as_float(sr[c + 2]), sc, neg_m));
+                        const float p3 = ex2(fmaf(__uint_as_float(sr[c + 3]), sc, neg_m));
+                        rs[0] += p0;
+                        rs[1] += p1;
+                        rs[2] += p2;
+                        rs[3] += p3;
+                        sr[c / 2] = pack_bf16x2(p0, p1);  // slots c/2, c/2+1 <= c+1: already read
+                        sr[c / 2 + 1] = pack_bf16x2(p2, p3);
                     }
-                    l = l * alpha + rs;
+                    l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
                     // P (bf16 pairs) over the first BK/2 columns of S_t.
 #pragma unroll
                     for (int c = 0; c < BK / 64; ++c)
                         tmem_st32(tl + C::colS(t) + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&sr[32 * c]));
-                    if (cnt > 0 && __any_sync(0xffffffffu, move)) {
+                    if (cnt_item > 0 && __any_sync(0xffffffffu, move)) {
                         // O_t is stable: S_t of this block completed after PV_t of the last one.
 #pragma unroll
                         for (int c = 0; c < HD / 32; ++c) {
@@ -398,7 +537,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                             tmem_ld32(tl + C::colO(t) + 32 * c, o);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            for (int e2 = 0; e2 < 32; ++e2) o[e2] = __float_as_uint(__uint_as_float(o[e2]) * alpha);
                             tmem_st32(tl + C::colO(t) + 32 * c, o);
                         }
                     }
@@ -406,19 +545,18 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     tc_fence_before();
                     mbar_arrive(bar_pf(t));
                     ++cnt;
-                }
-                if (last) {
-                    done = true;
-                    break;
+                    ++cnt_item;
                 }
             }
-        }
-        if (done && cnt > 0) {
-            const bool w = mbar_wait(bar_pv(t), (cnt - 1) & 1, ctl);
-            if (__all_sync(0xffffffffu, w)) {
+            if (fail) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_le(b));
+            if (cnt_item > 0) {
+                const bool wt = mbar_wait(bar_pv(t), (cnt - 1) & 1, ctl);
+                if (!__all_sync(0xffffffffu, wt)) break;
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.0f / l : 0.f;
-                uint16_t* orow = p.o + (row_base + qpos) * HD;
+                uint16_t* orow = p.o + (I.row_base + qpos) * HD;
 #pragma unroll
                 for (int c = 0; c < HD / 32; ++c) {
                     uint32_t o[32];
@@ -426,23 +564,23 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     tmem_wait_ld();
                     if (row_valid) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
+                        for (int e2 = 0; e2 < 32; e2 += 8) {
                             uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv, __uint_as_float(o[e + 1]) * inv);
-                            v.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-                            v.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-                            v.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
-                            *reinterpret_cast<uint4*>(orow + 32 * c + e) = v;
+                            v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * inv, __uint_as_float(o[e2 + 1]) * inv);
+                            v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * inv, __uint_as_float(o[e2 + 3]) * inv);
+                            v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * inv, __uint_as_float(o[e2 + 5]) * inv);
+                            v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * inv, __uint_as_float(o[e2 + 7]) * inv);
+                            *reinterpret_cast<uint4*>(orow + 32 * c + e2) = v;
                         }
                     }
                 }
                 if (row_valid && p.lse)
-                    p.lse[row_base + qpos] = l > 0.f ? (m_used + lg2(l)) * 0.69314718055994531f : -INFINITY;
+                    p.lse[I.row_base + qpos] = l > 0.f ? (m_used + lg2(l)) * 0.69314718055994531f : -INFINITY;
+            } else if (row_valid && len == 0) {
+                uint16_t* orow = p.o + (I.row_base + qpos) * HD;
+                for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
+                if (p.lse) p.lse[I.row_base + qpos] = -INFINITY;
             }
-        } else if (row_valid && !ok) {
-            uint16_t* orow = p.o + (row_base + qpos) * HD;
-            for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
-            if (p.lse) p.lse[row_base + qpos] = -INFINITY;
         }
         tc_fence_before();
     }

@@ -117,7 +117,10 @@ int launch_prefill(const void* q, const void* k, const void* v, s2::PrefillParam
             g_dev[dev].prefill_attr_done[attr_slot] = true;
         }
     }
-    const uint64_t grid = (uint64_t)pp.batch * pp.heads * ((pp.nqt + 1) / 2);
+    // Persistent: one CTA per SM (one fits by shared memory), each walking a
+    // static share of the tile pairs.
+    const uint64_t items = (uint64_t)pp.batch * pp.heads * ((pp.nqt + 1) / 2);
+    const uint64_t grid = items < (uint64_t)g_dev[dev].num_sms ? items : (uint64_t)g_dev[dev].num_sms;
     kern<<<(unsigned)grid, 384, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
@@ -208,10 +211,11 @@ int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float*
                     const int32_t* col_idx, int64_t nnz, void* stream)
 {
     if (!q || !k || !v || !o || !row_ptr || !col_idx) return S2_ERR_INVALID_ARG;
-    if (batch < 1 || heads < 1 || seq < 1 || nnz < 1 || !std::isfinite(scale))
+    if (batch < 1 || heads < 1 || seq < 1 || nnz < 1 || !std::isfinite(scale) || !(scale > 0.f))
         return S2_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
     if (block_size != 64 && block_size != 128) return S2_ERR_UNSUPPORTED;
+    if (num_blocks > 2048) return S2_ERR_UNSUPPORTED;  // union lists are staged in shared memory
     if (seq % block_size != 0 || num_blocks != seq / block_size) return S2_ERR_INVALID_ARG;
     if ((int64_t)batch * heads * seq >= (int64_t)INT32_MAX) return S2_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
