@@ -3,32 +3,41 @@
 // S2-Attention ("S2-Attention: Hardware-aware context sharding among attention
 // heads", Abstract) needs a FlashAttention-style kernel for sparsity to pay off;
 // HHST shards the context across heads at block granularity, so the block is
-// the tile here. One CTA owns two adjacent 128-row query tiles of one
-// (batch, head). Adjacent tiles share their strided key blocks and most local
-// ones, so the CTA walks the union of their key-block lists, loads each key
-// block once, and runs each tile's MMAs only on the blocks that tile sees.
+// the tile here. One work item is a pair of adjacent 128-row query tiles of
+// one (batch, head). Adjacent tiles share their strided key blocks and most
+// local ones, so the CTA walks the union of their key-block lists, loads each
+// key block once, and runs each tile's MMAs only on the blocks that tile sees.
+//
+// Key blocks are consumed in groups of G blocks (one S MMA of N = G * B keys
+// and one softmax pass per group). K is stored panel-major across the stage
+// ring so that G adjacent stages form one G*B-row K operand, and union lists
+// are padded to a multiple of G with a fully masked entry. G = 2 for B = 64
+// (N = 128 MMAs) was measured and lost to the extra masked work it issues
+// (a tile computes both blocks of a group if it sees either), so G = 1.
 //
 // The kernel is persistent: one CTA per SM walks a static share of the work
-// items (tile pairs, heaviest query blocks first), so the next item's loads
-// and S MMAs overlap the current item's last blocks and epilogue.
+// items (heaviest query blocks first), so the next item's loads and S MMAs
+// overlap the current item's last groups and epilogue.
 //
 // CTA = 12 warps:
+//   warp 2      list builder and Q producer: writes each item's union list
+//               into a double-buffered shared-memory list, loads the item's Q
+//               tiles once the previous item's S MMAs release the buffer, and
+//               prefetches the next item's Q into L2.
 //   warp 0      K/V producer: K and V of each union block, item after item,
-//               into an ST-stage ring (TMA, SWIZZLE_128B, 64-column panels).
-//   warp 2      Q producer: Q of both tiles of each item once the previous
-//               item's S MMAs are done with the Q buffer; prefetches the next
-//               item's Q into L2.
+//               into an ST-stage ring (TMA, SWIZZLE_128B, 64-column panels),
+//               prefetching blocks into L2 a few entries ahead.
 //   warp 1      owns TMEM; one thread issues tcgen05.mma:
 //               S_t = Q_t K^T (A and B from shared memory) into TMEM, and
 //               O_t += P_t V with P_t read from TMEM (A operand) and V from
 //               shared memory (MN-major B operand).
 //   warps 4..7  softmax of tile 0, warps 8..11 softmax of tile 1: thread = one
-//               query row = one TMEM lane. Loads its S row, masks (union tag
-//               bit of its query block; token causality where the key block
-//               reaches its own block), keeps a running max and sum in the
-//               log2 domain, writes P (bf16 pairs) over the S columns in TMEM,
-//               and at the end normalises O and stores it with the LSE.
-//   warp 3      idle (no work; it only takes part in block-wide barriers).
+//               query row = one TMEM lane. Loads its S row of a group, masks
+//               (union tag bit of its query block; token causality where the
+//               key block reaches its own block), keeps a running max and sum
+//               in the log2 domain, writes P (bf16 pairs) over the S columns
+//               in TMEM, and at the end normalises O and stores it with the LSE.
+//   warp 3      idle (it only takes part in block-wide barriers).
 // The two softmax warpgroups ping-pong: while one computes exponentials for
 // its tile, the tensor core runs the other tile's MMAs.
 //
@@ -42,8 +51,6 @@
 //    next item's first PV (which overwrites O) cannot race the epilogue.
 //  * The running-max reference only moves when the max grows by more than
 //    2^8 (kRescaleLog2), so O rescales are rare; P values stay <= 256.
-// Every role walks the union list itself from the CSR arrays, so no shared
-// per-stage record can be overwritten under a warpgroup that lags behind.
 // Every wait is bounded; on a timeout the CTA drains its own copies and MMAs,
 // frees TMEM and exits with the device timeout flag set.
 #pragma once
@@ -57,19 +64,30 @@
 
 namespace s2 {
 
+// Warp-wide bounded wait (every lane polls: measured faster than one lane
+// polling and broadcasting).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl)
+{
+    const bool ok = mbar_wait(bar, parity, ctl);
+    return __all_sync(0xffffffffu, ok);
+}
+
 template <int HD, int BK>
 struct PairCfg {
     static constexpr int M = 128;                          // rows per tile
-    static constexpr int ROWS = (BK == 128) ? 2 : 4;       // query blocks per CTA
+    static constexpr int ROWS = (BK == 128) ? 2 : 4;       // query blocks per item
+    static constexpr int G = 1;                            // key blocks per group (see below)
+    static constexpr int NK = BK * G;                      // keys per group = S columns
     static constexpr uint32_t QBYTES = M * HD * 2;         // one tile's Q
     static constexpr uint32_t KVBYTES = BK * HD * 2;       // one K (or V) block
-    static constexpr int LIST_CAP = 2048;                  // union entries per item (>= nb)
+    static constexpr int LIST_CAP = 2048;                  // union entries per item (>= nb + 1)
     static constexpr uint32_t LIST_BYTES = 2 * LIST_CAP * 4;  // double-buffered
     static constexpr int ST = (2 * QBYTES + 4 * 2 * KVBYTES + LIST_BYTES <= 220 * 1024) ? 4 : 2;
     static constexpr int PREFETCH = 4;                     // K/V blocks prefetched into L2 ahead
+    static constexpr uint32_t KPANEL = ST * BK * 128;      // bytes of one 64-column K panel, all stages
     static constexpr uint32_t OFF_Q = 0;
-    static constexpr uint32_t OFF_K = OFF_Q + 2 * QBYTES;
-    static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;
+    static constexpr uint32_t OFF_K = OFF_Q + 2 * QBYTES;  // [panel][stage][BK rows x 128 B]
+    static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;  // [stage][panel][BK rows x 128 B]
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
     static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
     // barriers: q_full, q_empty, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2],
@@ -78,28 +96,26 @@ struct PairCfg {
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 16;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
-    static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD) <= 256 ? 256 : 512;
+    static constexpr uint32_t TMEM_COLS = (2 * NK + 2 * HD) <= 256 ? 256 : 512;
     // list_empty arrivals per item: K/V producer, MMA issuer, 8 softmax warps
     static constexpr uint32_t LIST_CONSUMERS = 10;
-    __host__ __device__ static constexpr uint32_t colS(int t) { return (uint32_t)(t * BK); }
-    __host__ __device__ static constexpr uint32_t colO(int t) { return (uint32_t)(2 * BK + t * HD); }
-    static_assert(2 * BK + 2 * HD <= 512, "TMEM budget");
+    __host__ __device__ static constexpr uint32_t colS(int t) { return (uint32_t)(t * NK); }
+    __host__ __device__ static constexpr uint32_t colO(int t) { return (uint32_t)(2 * NK + t * HD); }
+    static_assert(2 * NK + 2 * HD <= 512, "TMEM budget");
+    static_assert(ST % G == 0, "groups must not wrap the stage ring");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-// Union-list entry: key block j (bits 0..23), row tags (bits 24..27), last flag (bit 31).
-__device__ __forceinline__ uint32_t list_pack(int j, int bits, bool last)
-{
-    return (uint32_t)j | ((uint32_t)bits << 24) | (last ? 0x80000000u : 0u);
-}
+constexpr float kRescaleLog2 = 8.0f;
+
+// Union-list entry: key block j (bits 0..23), row tags (bits 24..27).
+__device__ __forceinline__ uint32_t list_pack(int j, int bits) { return (uint32_t)j | ((uint32_t)bits << 24); }
 __device__ __forceinline__ int list_j(uint32_t e) { return (int)(e & 0xFFFFFFu); }
 __device__ __forceinline__ int list_bits(uint32_t e) { return (int)((e >> 24) & 0xFu); }
 
-constexpr float kRescaleLog2 = 8.0f;
-
 // Walks the ascending union of up to ROWS compacted lists (query blocks
 // qb0 .. qb0+ROWS-1 of one head) and tags each key block with the rows that
-// list it. Every role runs its own copy; all copies see the same sequence.
+// list it.
 template <int ROWS>
 struct UnionWalk {
     int a[ROWS], e[ROWS];
@@ -195,6 +211,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                        const __grid_constant__ CUtensorMap tmV, const PrefillParams p)
 {
     using C = PairCfg<HD, BK>;
+    constexpr int G = C::G;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -267,13 +284,14 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         bool last, bad;
                         it.next(p.col_idx, j, bits, last, bad);
                         if (bad) atomicOr(p.gflags, kFlagIndex);
-                        if (len == C::LIST_CAP - 1 && !last) {  // cannot happen when nb <= LIST_CAP
+                        if (len >= C::LIST_CAP - G) {  // cannot happen when nb <= LIST_CAP - G
                             atomicOr(p.gflags, kFlagIndex);
                             last = true;
                         }
-                        wlist[b * C::LIST_CAP + len++] = list_pack(j, bits, last);
+                        wlist[b * C::LIST_CAP + len++] = list_pack(j, bits);
                         if (last) break;
                     }
+                    while (len % G) wlist[b * C::LIST_CAP + len++] = list_pack(0, 0);  // masked pad
                 } else {
                     atomicOr(p.gflags, kFlagIndex);
                 }
@@ -332,8 +350,8 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     mbar_arrive_expect_tx(bar_kf(st), C::KVBYTES);
 #pragma unroll
                     for (int pn = 0; pn < HD / 64; ++pn)
-                        tma_load_2d(sb + C::OFF_K + st * C::KVBYTES + pn * (BK * 128), &tmK, pn * 64,
-                                    krow, bar_kf(st));
+                        tma_load_2d(sb + C::OFF_K + pn * C::KPANEL + st * (BK * 128), &tmK, pn * 64, krow,
+                                    bar_kf(st));
                     mbar_arrive_expect_tx(bar_vf(st), C::KVBYTES);
 #pragma unroll
                     for (int pn = 0; pn < HD / 64; ++pn)
@@ -352,31 +370,36 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);
+            constexpr uint32_t idesc_s = umma_idesc(128, C::NK, 0, 0);
             constexpr uint32_t idesc_o = umma_idesc(128, HD, 0, 1);
+            constexpr int KSTEPS_BLK = BK / 16;  // PV k-steps per key block
             bool issued = false, fail = false;
-            int pvc[2] = {0, 0};   // PV MMAs issued per tile (all items)
+            int pvc[2] = {0, 0};  // PV groups issued per tile (all items)
             bool first_pv[2] = {true, true};
-            int n = 0;             // union elements consumed (all items)
+            int n = 0;            // union elements consumed (all items); a multiple of G
+            // S_t = Q_t K^T over the G blocks of the group starting at stage st (N = 128).
             auto issue_s = [&](int t, int st) {
-                const uint32_t d = tmem + C::colS(t);
                 const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
-                const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
+                const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * (BK * 128), 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk)
-                    umma_bf16_ss(d, dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
-                                 dk + (((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4), idesc_s,
+                    umma_bf16_ss(tmem + C::colS(t), dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
+                                 dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4), idesc_s,
                                  kk > 0 ? 1u : 0u);
                 umma_commit(bar_sf(t));
                 issued = true;
             };
+            // O_t += P_t V over the group's G blocks (stages st .. st+G-1).
             auto issue_pv = [&](int t, int st) {
-                const uint64_t dv = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, BK * 128, 1024);
                 const uint32_t acc0 = first_pv[t] ? 0u : 1u;
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    umma_bf16_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, dv + ((kk * 2048) >> 4),
-                                 idesc_o, kk > 0 ? 1u : acc0);
+                for (int kk = 0; kk < C::NK / 16; ++kk) {
+                    const int s = st + kk / KSTEPS_BLK;
+                    const uint64_t dv = umma_sdesc(sb + C::OFF_V + s * C::KVBYTES + (kk % KSTEPS_BLK) * 2048,
+                                                   BK * 128, 1024);
+                    umma_bf16_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, dv, idesc_o,
+                                 kk > 0 ? 1u : acc0);
+                }
                 umma_commit(bar_pv(t));
                 ++pvc[t];
                 first_pv[t] = false;
@@ -393,23 +416,38 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     mbar_arrive(bar_le(b));
                     continue;
                 }
+                const int ngroups = len / G;
                 first_pv[0] = first_pv[1] = true;
-                uint32_t cur = L[0];
-                if (!mbar_wait(bar_kf(n % C::ST), (n / C::ST) & 1, ctl)) break;
+                auto gbits = [&](int g) {
+                    int bits = 0;
+#pragma unroll
+                    for (int i = 0; i < G; ++i) bits |= list_bits(L[g * G + i]);
+                    return bits;
+                };
+                auto wait_k = [&](int n0) {
+                    for (int i = 0; i < G; ++i)
+                        if (!mbar_wait(bar_kf((n0 + i) % C::ST), ((n0 + i) / C::ST) & 1, ctl)) return false;
+                    return true;
+                };
+                auto wait_v = [&](int n0) {
+                    for (int i = 0; i < G; ++i)
+                        if (!mbar_wait(bar_vf((n0 + i) % C::ST), ((n0 + i) / C::ST) & 1, ctl)) return false;
+                    return true;
+                };
+                int bits = gbits(0);
+                if (!wait_k(n)) break;
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t)
-                    if (tile_sees<BK>(list_bits(cur), t)) issue_s(t, n % C::ST);
-                for (int e = 0;; ++e, ++n) {
-                    const bool last = e + 1 == len;
-                    const uint32_t nxt = last ? 0u : L[e + 1];
-                    const int bits = list_bits(cur), nbits = list_bits(nxt);
+                    if (tile_sees<BK>(bits, t)) issue_s(t, n % C::ST);
+                for (int g = 0;; ++g, n += G) {
+                    const bool last = g + 1 == ngroups;
+                    const int nbits = last ? 0 : gbits(g + 1);
                     const int st = n % C::ST;
-                    const int st1 = (n + 1) % C::ST;
+                    const int st1 = (n + G) % C::ST;
                     if (last) umma_commit(bar_qe);  // no more S MMAs of this item read Q
                     bool v_ready = false, k_next_ready = false;
-                    if (bits == 0) {  // malformed entry no tile sees: let its loads land first
-                        if (!mbar_wait(bar_kf(st), (n / C::ST) & 1, ctl) ||
-                            !mbar_wait(bar_vf(st), (n / C::ST) & 1, ctl)) {
+                    if (bits == 0) {  // malformed group no tile sees: let its loads land first
+                        if (!wait_k(n) || !wait_v(n)) {
                             fail = true;
                             break;
                         }
@@ -419,16 +457,17 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         if (tile_sees<BK>(bits, t)) {
                             if (!mbar_wait(bar_pf(t), pvc[t] & 1, ctl)) { fail = true; break; }
                             if (!v_ready) {
-                                if (!mbar_wait(bar_vf(st), (n / C::ST) & 1, ctl)) { fail = true; break; }
+                                if (!wait_v(n)) { fail = true; break; }
                                 v_ready = true;
                             }
                             tc_fence_after();
                             issue_pv(t, st);
                         }
-                        if (t == last_t) umma_commit(bar_ke(st));
+                        if (t == last_t)
+                            for (int i = 0; i < G; ++i) umma_commit(bar_ke(st + i));
                         if (!last && tile_sees<BK>(nbits, t)) {
                             if (!k_next_ready) {
-                                if (!mbar_wait(bar_kf(st1), ((n + 1) / C::ST) & 1, ctl)) { fail = true; break; }
+                                if (!wait_k(n + G)) { fail = true; break; }
                                 k_next_ready = true;
                                 tc_fence_after();
                             }
@@ -437,10 +476,10 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     }
                     if (fail) break;
                     if (last) {
-                        ++n;
+                        n += G;
                         break;
                     }
-                    cur = nxt;
+                    bits = nbits;
                 }
                 if (!fail) mbar_arrive(bar_le(b));
             }
@@ -457,7 +496,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const int r = quad * 32 + lane;             // row within the tile
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const float sc = p.scale_log2;              // > 0
-        int cnt = 0;                                // S_t blocks processed (all items)
+        int cnt = 0;                                // S_t groups processed (all items)
         bool fail = false;
         int k = 0;
         for (int w = blockIdx.x; w < num_items && !fail; w += gridDim.x, ++k) {
@@ -467,44 +506,54 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             const bool active = (t == 0) || I.tile1;
             const bool row_valid = active && qpos < p.seq && (I.qb0 + rowbit) < p.nb;
             const int b = k & 1;
-            bool wl = mbar_wait(bar_lf(b), (k >> 1) & 1, ctl);
-            if (!__all_sync(0xffffffffu, wl)) break;
+            if (!warp_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
             const uint32_t* L = list + b * C::LIST_CAP;
             const int len = list_len[b];
             float m_used = -1e30f, l = 0.f;
             int cnt_item = 0;
             if (active) {
-                for (int e = 0; e < len; ++e) {
-                    const uint32_t ent = L[e];
-                    const int bits = list_bits(ent);
+                for (int g = 0; g < len / G; ++g) {
+                    uint32_t ent[G];
+                    int bits = 0;
+#pragma unroll
+                    for (int i = 0; i < G; ++i) {
+                        ent[i] = L[g * G + i];
+                        bits |= list_bits(ent[i]);
+                    }
                     if (!tile_sees<BK>(bits, t)) continue;
-                    bool wt = mbar_wait(bar_sf(t), cnt & 1, ctl);
-                    if (!__all_sync(0xffffffffu, wt)) {
+                    if (!warp_wait(bar_sf(t), cnt & 1, ctl)) {
                         fail = true;
                         break;
                     }
                     tc_fence_after();
-                    uint32_t sr[BK];  // S row; packed P overwrites its front as it is consumed
+                    uint32_t sr[C::NK];  // S row; packed P overwrites its front as it is consumed
 #pragma unroll
-                    for (int c = 0; c < BK / 32; ++c)
+                    for (int c = 0; c < C::NK / 32; ++c)
                         tmem_ld32(tl + C::colS(t) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
                     tmem_wait_ld();
-                    const bool vis = (bits >> rowbit) & 1;
-                    const int lim = qpos - list_j(ent) * BK;  // key column c visible iff c <= lim
-                    if (!__all_sync(0xffffffffu, vis && lim >= BK - 1)) {
+                    bool vis[G];
+                    int lim[G];  // key column c of block i visible iff vis[i] && c <= lim[i]
+                    bool full = true;
 #pragma unroll
-                        for (int c = 0; c < BK; ++c)
-                            if (!(vis && c <= lim)) sr[c] = 0xff800000u;  // -inf
+                    for (int i = 0; i < G; ++i) {
+                        vis[i] = (list_bits(ent[i]) >> rowbit) & 1;
+                        lim[i] = qpos - list_j(ent[i]) * BK;
+                        full = full && vis[i] && lim[i] >= BK - 1;
+                    }
+                    if (!__all_sync(0xffffffffu, full)) {
+#pragma unroll
+                        for (int c = 0; c < C::NK; ++c)
+                            if (!(vis[c / BK] && (c % BK) <= lim[c / BK])) sr[c] = 0xff800000u;  // -inf
                     }
                     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                    for (int c = 0; c < BK; c += 4) {
-                        mx[0] = fmaxf(mx[0], __uint_as_float(sr[c]));
-                        mx[1] = fmaxf(mx[1], __uint_as_float(sr[c + 1]));
-                        mx[2] = fmaxf(mx[2], __uint_as_float(sr[c + 2]));
-                        mx[3] = fmaxf(mx[3], __uint_as_float(sr[c + 3]));
+                    for (int c = 0; c < C::NK; c += 8) {
+                        mx[0] = fmax3(mx[0], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                        mx[1] = fmax3(mx[1], __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+                        mx[2] = fmax3(mx[2], __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+                        mx[3] = fmax3(mx[3], __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
                     }
-                    const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sc;
+                    const float mt = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
                     const float m_cand = fmaxf(m_used, mt);
                     const bool move = m_cand - m_used > kRescaleLog2;
                     const float alpha = move ? ex2(m_used - m_cand) : 1.0f;
@@ -512,25 +561,21 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     const float neg_m = -m_used;
                     float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int c = 0; c < BK; c += 4) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sc, neg_m));
-                        const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sc, neg_m));
-                        const float p2 = ex2(fmaf(__uint_as_float(sr[c + 2]), sc, neg_m));
-                        const float p3 = ex2(fmaf(__uint_as_float(sr[c + 3]), sc, neg_m));
-                        rs[0] += p0;
-                        rs[1] += p1;
-                        rs[2] += p2;
-                        rs[3] += p3;
-                        sr[c / 2] = pack_bf16x2(p0, p1);  // slots c/2, c/2+1 <= c+1: already read
-                        sr[c / 2 + 1] = pack_bf16x2(p2, p3);
+                    for (int q = 0; q < C::NK / 2; ++q) {  // column pair (2q, 2q+1)
+                        const float p0 = ex2(fmaf(__uint_as_float(sr[2 * q]), sc, neg_m));
+                        const float p1 = ex2(fmaf(__uint_as_float(sr[2 * q + 1]), sc, neg_m));
+                        rs[(2 * q) & 3] += p0;
+                        rs[(2 * q + 1) & 3] += p1;
+                        sr[q] = pack_bf16x2(p0, p1);  // slot q <= 2q: already read
                     }
                     l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
-                    // P (bf16 pairs) over the first BK/2 columns of S_t.
+                    // P (bf16 pairs) over the first NK/2 columns of S_t.
 #pragma unroll
-                    for (int c = 0; c < BK / 64; ++c)
+                    for (int c = 0; c < C::NK / 64; ++c)
                         tmem_st32(tl + C::colS(t) + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&sr[32 * c]));
+                    static_assert(C::NK % 64 == 0, "P stored in 32-column chunks");
                     if (cnt_item > 0 && __any_sync(0xffffffffu, move)) {
-                        // O_t is stable: S_t of this block completed after PV_t of the last one.
+                        // O_t is stable: S_t of this group completed after PV_t of the last one.
 #pragma unroll
                         for (int c = 0; c < HD / 32; ++c) {
                             uint32_t o[32];
@@ -552,8 +597,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_le(b));
             if (cnt_item > 0) {
-                const bool wt = mbar_wait(bar_pv(t), (cnt - 1) & 1, ctl);
-                if (!__all_sync(0xffffffffu, wt)) break;
+                if (!warp_wait(bar_pv(t), (cnt - 1) & 1, ctl)) break;
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.0f / l : 0.f;
                 uint16_t* orow = p.o + (I.row_base + qpos) * HD;

@@ -249,6 +249,14 @@ __device__ __forceinline__ float lg2(float x)
     return y;
 }
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Two floats -> packed bf16x2 (round to nearest even), low half = a.
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
 {

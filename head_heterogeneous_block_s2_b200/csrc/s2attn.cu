@@ -215,7 +215,7 @@ int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float*
         return S2_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
     if (block_size != 64 && block_size != 128) return S2_ERR_UNSUPPORTED;
-    if (num_blocks > 2048) return S2_ERR_UNSUPPORTED;  // union lists are staged in shared memory
+    if (num_blocks > 2046) return S2_ERR_UNSUPPORTED;  // union lists are staged in shared memory
     if (seq % block_size != 0 || num_blocks != seq / block_size) return S2_ERR_INVALID_ARG;
     if ((int64_t)batch * heads * seq >= (int64_t)INT32_MAX) return S2_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
