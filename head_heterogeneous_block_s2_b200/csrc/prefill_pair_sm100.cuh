@@ -620,7 +620,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
                 if (row_valid && p.lse)
                     p.lse[I.row_base + qpos] = l > 0.f ? (m_used + lg2(l)) * 0.69314718055994531f : -INFINITY;
-            } else if (row_valid && len == 0) {
+            } else if (row_valid) {  // malformed layout: the row saw no key block
                 uint16_t* orow = p.o + (I.row_base + qpos) * HD;
                 for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
                 if (p.lse) p.lse[I.row_base + qpos] = -INFINITY;

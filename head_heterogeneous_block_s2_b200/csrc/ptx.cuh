@@ -60,6 +60,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking probe of the phase (no hardware suspend).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Shared state for bounded waits: the kernel-wide give-up time and a flag in
 // shared memory that tells every role of the CTA to stop.
 struct WaitCtl {
@@ -73,6 +87,12 @@ struct WaitCtl {
 // sets the device timeout flag and the CTA abort flag.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl)
 {
+    if (ctl.timeout_ns == 0) {  // a zero limit: succeed only if the phase is already complete
+        if (mbar_test_wait(bar, parity)) return true;
+        atomicOr(ctl.gflags, kFlagTimeout);
+        *ctl.abort_cta = 1;
+        return false;
+    }
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0;; ++it) {

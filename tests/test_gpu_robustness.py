@@ -1,0 +1,102 @@
+"""Failure detection without a GPU fault.
+
+* Every device wait is bounded: with the limit forced to 0, any wait that is
+  not already satisfied gives up, the kernel sets the device timeout flag,
+  drains its own copies and MMAs, frees TMEM and returns. The context must stay
+  usable: after clearing the flag, the same call gives correct results.
+* Malformed layouts (out-of-range or non-causal key blocks, broken row
+  offsets) are skipped and reported as S2_ERR_DEVICE_INDEX, never faulted.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import parity
+from head_heterogeneous_block_s2_b200 import s2attn, synth
+
+pytestmark = pytest.mark.gpu
+
+S2_ERR_TIMEOUT, S2_ERR_DEVICE_INDEX = 5, 6
+
+
+def tiny():
+    w = synth.TINY
+    q, k, v = synth.prefill_inputs(w)
+    lay = s2attn.build_layout(w.heads, w.block, w.stride, w.local, w.num_blocks, device="cuda")
+    return w, q, k, v, lay
+
+
+def test_prefill_wait_timeout_is_reported_and_recoverable(s2gpu):
+    w, q, k, v, lay = tiny()
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    s2gpu.set_wait_timeout_ns(0)
+    try:
+        s2gpu.prefill(qc, kc, vc, lay, scale=w.scale)
+        rc, flags = s2gpu.device_status(reset=True)
+    finally:
+        s2gpu.set_wait_timeout_ns(500_000_000)
+    assert rc == S2_ERR_TIMEOUT and flags & 1
+    out = s2gpu.prefill(qc, kc, vc, lay, scale=w.scale)
+    torch.cuda.synchronize()
+    ref, _ = oracle.prefill(q, k, v, w.block, w.stride, w.local, w.scale)
+    parity(out.reshape(-1, w.head_dim), ref)
+
+
+def test_decode_wait_timeout_is_reported_and_recoverable(s2gpu):
+    # dense heads and one split: each CTA streams ~125 pages through its 8-stage
+    # ring, so the producer must wait for stages to be released
+    dense = tuple(range(8))
+    wd = synth.DecodeWorkload("t", 4, 8, 128, 1, 2000, 16, 128, 4, 2, dense_heads=dense, seed=3)
+    d = synth.decode_inputs(wd, ctx_lens=[1900, 1950, 1990, 2000])
+    lay = s2gpu.build_layout(wd.heads, wd.block, wd.stride, wd.local, wd.num_blocks, dense, device="cuda")
+    args = (d.q.cuda(), d.k_cache.cuda(), d.v_cache.cuda(), d.block_table.cuda(), d.ctx_lens.cuda(), lay)
+    s2gpu.set_wait_timeout_ns(0)
+    try:
+        s2gpu.decode(*args, scale=wd.scale, num_splits=1)
+        rc, flags = s2gpu.device_status(reset=True)
+    finally:
+        s2gpu.set_wait_timeout_ns(500_000_000)
+    assert rc == S2_ERR_TIMEOUT and flags & 1
+    out = s2gpu.decode(*args, scale=wd.scale, num_splits=1)
+    ref, _ = oracle.decode(d.q, d.k_cache, d.v_cache, d.block_table.numpy(), d.ctx_lens.numpy(),
+                           wd.block, wd.stride, wd.local, wd.scale, dense)
+    parity(out.reshape(-1, wd.head_dim), ref)
+
+
+@pytest.mark.parametrize("corrupt", ["future_block", "huge_block", "negative_block", "bad_row_ptr"])
+def test_malformed_prefill_layout_is_flagged_not_faulted(s2gpu, corrupt):
+    w, q, k, v, lay = tiny()
+    row_ptr, col_idx = lay.row_ptr.copy(), lay.col_idx.copy()
+    if corrupt == "future_block":
+        col_idx[row_ptr[2]] = 7  # head 0, query block 2 lists key block 7 > 2
+    elif corrupt == "huge_block":
+        col_idx[5] = 1 << 20
+    elif corrupt == "negative_block":
+        col_idx[3] = -4
+    else:
+        row_ptr[4] = row_ptr[5] + 3  # offsets out of order
+    bad = s2attn.Layout(lay.heads, lay.block_size, lay.stride, lay.local, lay.num_blocks, (),
+                        row_ptr, col_idx).to("cuda")
+    out = s2gpu.prefill(q.cuda(), k.cuda(), v.cuda(), bad, scale=w.scale)
+    rc, flags = s2gpu.device_status(reset=True)
+    assert rc == S2_ERR_DEVICE_INDEX and flags == 2
+    assert torch.isfinite(out.float()).all()
+    # the library still works with the good layout
+    good = s2gpu.prefill(q.cuda(), k.cuda(), v.cuda(), lay, scale=w.scale)
+    torch.cuda.synchronize()
+    ref, _ = oracle.prefill(q, k, v, w.block, w.stride, w.local, w.scale)
+    parity(good.reshape(-1, w.head_dim), ref)
+
+
+def test_bad_context_length_is_flagged(s2gpu):
+    wd = synth.DecodeWorkload("t", 3, 4, 128, 1, 512, 16, 128, 4, 1, seed=2)
+    d = synth.decode_inputs(wd, ctx_lens=[10, 200, 512])
+    lay = s2gpu.build_layout(wd.heads, wd.block, wd.stride, wd.local, wd.num_blocks, device="cuda")
+    cl = d.ctx_lens.clone()
+    cl[1] = 100000  # beyond the block table and the layout
+    out = s2gpu.decode(d.q.cuda(), d.k_cache.cuda(), d.v_cache.cuda(), d.block_table.cuda(), cl.cuda(),
+                       lay, scale=wd.scale, num_splits=1)
+    rc, flags = s2gpu.device_status(reset=True)
+    assert rc == S2_ERR_DEVICE_INDEX and flags == 2
+    assert torch.isfinite(out.float()).all()
