@@ -15,12 +15,14 @@
 // (N = 128 MMAs) was measured and lost to the extra masked work it issues
 // (a tile computes both blocks of a group if it sees either), so G = 1.
 //
-// The kernel is persistent: one CTA per SM walks a static share of the work
-// items (heaviest query blocks first), so the next item's loads and S MMAs
-// overlap the current item's last groups and epilogue.
+// The kernel is persistent: one CTA per SM takes work items from a device
+// counter (its first item is its block index), so the next item's loads and
+// S MMAs overlap the current item's last groups and epilogue and the load
+// balances itself (item order: see pair_item).
 //
 // CTA = 12 warps:
-//   warp 2      list builder and Q producer: writes each item's union list
+//   warp 2      scheduler, list builder and Q producer: takes the next item
+//               from the work counter, writes the item's union list and index
 //               into a double-buffered shared-memory list, loads the item's Q
 //               tiles once the previous item's S MMAs release the buffer, and
 //               prefetches the next item's Q into L2.
@@ -94,7 +96,7 @@ struct PairCfg {
     // pv_done[2], drain, list_full[2], list_empty[2]
     static constexpr int NBAR = 2 + 3 * ST + 6 + 1 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
-    static constexpr uint32_t SMEM = OFF_MISC + 16;
+    static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
     static constexpr uint32_t TMEM_COLS = (2 * NK + 2 * HD) <= 256 ? 256 : 512;
     // list_empty arrivals per item: K/V producer, MMA issuer, 8 softmax warps
@@ -182,6 +184,11 @@ __device__ __forceinline__ bool tile_sees(int bits, int t)
     return BK == 128 ? ((bits >> t) & 1) != 0 : ((bits >> (2 * t)) & 3) != 0;
 }
 
+// Item order switch: head-major from this many tile pairs per head (measured:
+// 32 pairs per head ran 5% faster in global heaviest-first order, 128 and 512
+// pairs per head 11% faster head-major).
+constexpr int kHeadMajorPairs = 64;
+
 // One work item: a pair of adjacent 128-row query tiles of one (batch, head).
 struct PairItem {
     int qt0, qb0, rp;
@@ -192,10 +199,15 @@ struct PairItem {
 template <int BK>
 __device__ __forceinline__ PairItem pair_item(const PrefillParams& p, int w)
 {
+    // Long sequences (many pairs per head): head by head, heaviest pairs first
+    // within a head, so CTAs running together share one head's strided key
+    // blocks in L2. Short ones: heaviest pairs of all heads first (the K/V of
+    // every head is small, and a global heaviest-first order balances better).
     const int npairs = (p.nqt + 1) >> 1;
     const int BH = p.batch * p.heads;
-    const int pr = npairs - 1 - w / BH;  // heaviest pairs first
-    const int bh = w % BH;
+    const bool head_major = npairs >= kHeadMajorPairs;
+    const int pr = npairs - 1 - (head_major ? w % npairs : w / BH);
+    const int bh = head_major ? w / npairs : w % BH;
     PairItem it;
     it.qt0 = 2 * pr;
     it.tile1 = it.qt0 + 1 < p.nqt;
@@ -231,10 +243,12 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (9 + 3 * C::ST + b); };
     auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (11 + 3 * C::ST + b); };
     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
-    int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2..3] list lengths
+    // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
+    int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
     volatile int* abort_cta = misc + 1;
     volatile int* list_len = misc + 2;
+    volatile int* list_item = misc + 4;
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -271,11 +285,19 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         if (lane == 0) {
             int k = 0;
             uint32_t* wlist = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
-            for (int w = blockIdx.x; w < num_items; w += gridDim.x, ++k) {
-                const PairItem I = pair_item<BK>(p, w);
+            int w = blockIdx.x;  // first item static, the rest from the work counter
+            for (;; ++k) {
                 const int b = k & 1;
                 // union list of this item into buffer b (free once item k-2 is consumed)
                 if (!mbar_wait(bar_le(b), ((k >> 1) & 1) ^ 1, ctl)) break;
+                if (w >= num_items) {  // tell every role there is no more work
+                    list_item[b] = -1;
+                    list_len[b] = 0;
+                    mbar_arrive(bar_lf(b));
+                    break;
+                }
+                const int w_next = (int)gridDim.x + atomicAdd(p.sched, 1);
+                const PairItem I = pair_item<BK>(p, w);
                 UnionWalk<C::ROWS> it;
                 int len = 0;
                 if (it.init(p.row_ptr, I.rp, I.qb0, p.nb, p.nnz)) {
@@ -296,6 +318,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     atomicOr(p.gflags, kFlagIndex);
                 }
                 list_len[b] = len;
+                list_item[b] = w;
                 mbar_arrive(bar_lf(b));
                 // Q of both tiles, once the previous item's S MMAs are done with the buffer
                 if (!mbar_wait(bar_qe, (k & 1) ^ 1, ctl)) break;
@@ -305,12 +328,13 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     for (int pn = 0; pn < HD / 64; ++pn)
                         tma_load_2d(sb + C::OFF_Q + t * C::QBYTES + pn * (C::M * 128), &tmQ, pn * 64,
                                     (int32_t)(I.row_base + (I.qt0 + t) * C::M), bar_q);
-                if (w + (int)gridDim.x < num_items) {  // next item's Q into L2
-                    const PairItem J = pair_item<BK>(p, w + gridDim.x);
+                if (w_next < num_items) {  // next item's Q into L2
+                    const PairItem J = pair_item<BK>(p, w_next);
                     for (int t = 0; t < (J.tile1 ? 2 : 1); ++t)
                         for (int pn = 0; pn < HD / 64; ++pn)
                             tma_prefetch_2d(&tmQ, pn * 64, (int32_t)(J.row_base + (J.qt0 + t) * C::M));
                 }
+                w = w_next;
             }
             if (*abort_cta && k > 0) mbar_drain(bar_q, (k - 1) & 1, kDrainNs);
         }
@@ -320,10 +344,12 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         if (lane == 0) {
             int n = 0, k = 0;
             bool stop = false;
-            for (int w = blockIdx.x; w < num_items && !stop; w += gridDim.x, ++k) {
-                const PairItem I = pair_item<BK>(p, w);
+            for (; !stop; ++k) {
                 const int b = k & 1;
                 if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                const int w = list_item[b];
+                if (w < 0) break;
+                const PairItem I = pair_item<BK>(p, w);
                 const uint32_t* L = list + b * C::LIST_CAP;
                 const int len = list_len[b];
                 for (int e = 0; e < C::PREFETCH && e < len; ++e) {
@@ -405,9 +431,10 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 first_pv[t] = false;
             };
             int k = 0;
-            for (int w = blockIdx.x; w < num_items && !fail; w += gridDim.x, ++k) {
+            for (; !fail; ++k) {
                 const int b = k & 1;
                 if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                if (list_item[b] < 0) break;
                 const uint32_t* L = list + b * C::LIST_CAP;
                 const int len = list_len[b];
                 if (!mbar_wait(bar_q, k & 1, ctl)) break;
@@ -499,14 +526,16 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         int cnt = 0;                                // S_t groups processed (all items)
         bool fail = false;
         int k = 0;
-        for (int w = blockIdx.x; w < num_items && !fail; w += gridDim.x, ++k) {
+        for (; !fail; ++k) {
+            const int b = k & 1;
+            if (!warp_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+            const int w = list_item[b];
+            if (w < 0) break;
             const PairItem I = pair_item<BK>(p, w);
             const int qpos = (I.qt0 + t) * C::M + r;
             const int rowbit = (BK == 128) ? t : 2 * t + (r >> 6);
             const bool active = (t == 0) || I.tile1;
             const bool row_valid = active && qpos < p.seq && (I.qb0 + rowbit) < p.nb;
-            const int b = k & 1;
-            if (!warp_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
             const uint32_t* L = list + b * C::LIST_CAP;
             const int len = list_len[b];
             float m_used = -1e30f, l = 0.f;
@@ -633,6 +662,16 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    if (threadIdx.x == 0) {
+        // The last CTA to finish resets the counter for the next launch on this slot
+        // (every CTA has stopped taking items by now).
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+            atomicExch(p.sched, 0);
+            atomicExch(p.sched + 1, 0);
+            __threadfence();
+        }
     }
 }
 

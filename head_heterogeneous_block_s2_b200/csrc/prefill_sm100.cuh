@@ -45,6 +45,7 @@ struct PrefillParams {
     float scale_log2;  // scale * log2(e)
     uint64_t timeout_ns;
     uint32_t* gflags;
+    int* sched;  // pair kernel work counter {next item, CTAs done}, zero at launch
 };
 
 template <int HD, int BK>

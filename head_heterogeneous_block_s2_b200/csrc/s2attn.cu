@@ -23,6 +23,13 @@ namespace {
 
 __device__ uint32_t g_s2_flags;
 
+// Work counters of the persistent prefill kernel: {next item, CTAs done} per
+// slot. Each launch takes the next slot in turn; the kernel's last CTA resets
+// its slot, so a slot is free again once its launch has finished.
+constexpr int kSchedSlots = 64;
+__device__ int g_s2_sched[2 * kSchedSlots];
+std::atomic<uint32_t> g_launch_seq{0};
+
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 
 constexpr int kMaxDevices = 64;
@@ -30,6 +37,7 @@ struct DevInfo {
     int checked = 0;  // 0 unknown, 1 sm_100, -1 other
     int num_sms = 0;
     uint32_t* flags = nullptr;
+    int* sched = nullptr;
     bool prefill_attr_done[4] = {false, false, false, false};
     bool decode_attr_done[2] = {false, false};
 };
@@ -62,6 +70,9 @@ int device_ready(int* dev_out)
             void* p = nullptr;
             if (cudaGetSymbolAddress(&p, g_s2_flags) != cudaSuccess) return S2_ERR_CUDA;
             d.flags = static_cast<uint32_t*>(p);
+            void* q = nullptr;
+            if (cudaGetSymbolAddress(&q, g_s2_sched) != cudaSuccess) return S2_ERR_CUDA;
+            d.sched = static_cast<int*>(q);
             d.num_sms = sms;
             d.checked = 1;
         }
@@ -239,6 +250,7 @@ int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float*
     pp.scale_log2 = scale * 1.4426950408889634f;
     pp.timeout_ns = g_timeout_ns.load();
     pp.gflags = g_dev[dev].flags;
+    pp.sched = g_dev[dev].sched + 2 * (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 128 && block_size == 128) return launch_prefill<128, 128>(q, k, v, pp, dev, 0, st);
     if (head_dim == 128 && block_size == 64) return launch_prefill<128, 64>(q, k, v, pp, dev, 1, st);
