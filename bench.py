@@ -355,13 +355,13 @@ def run_ours(args, rank, world, dist):
             "parallelism": f"replicas x{world} (no data-path collective)",
         },
         "roofline": {
-            "kernel": "s2_prefill_kernel<128,64>",
+            "kernel": f"s2_prefill_pair_kernel<{wp.head_dim},{wp.block}>",
             "bound": "tensor",
             "achieved": round(per_launch_tflops, 2),
             "peak": tc_peak,
             "unit": "TFLOP/s",
             "frac": round(per_launch_tflops / tc_peak, 4),
-            "traffic": load_traffic("s2_prefill_kernel", wp.name),
+            "traffic": load_traffic("s2_prefill_pair_kernel", wp.name),
             "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long loop)",
         },
         "e2e": None if not e2e_steps else {

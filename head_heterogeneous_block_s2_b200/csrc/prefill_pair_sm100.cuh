@@ -62,7 +62,7 @@
 #include <cuda.h>
 
 #include "ptx.cuh"
-#include "prefill_sm100.cuh"  // PrefillParams, umma_sdesc, umma_idesc
+#include "umma.cuh"  // PrefillParams, umma_sdesc, umma_idesc
 
 namespace s2 {
 

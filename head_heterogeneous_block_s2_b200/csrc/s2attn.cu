@@ -15,7 +15,6 @@
 
 #include "s2attn.h"
 #include "ptx.cuh"
-#include "prefill_sm100.cuh"
 #include "decode.cuh"
 #include "prefill_pair_sm100.cuh"
 
