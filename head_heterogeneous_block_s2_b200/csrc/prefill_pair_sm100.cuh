@@ -27,8 +27,7 @@
 //               tiles once the previous item's S MMAs release the buffer, and
 //               prefetches the next item's Q into L2.
 //   warp 0      K/V producer: K and V of each union block, item after item,
-//               into an ST-stage ring (TMA, SWIZZLE_128B, 64-column panels),
-//               prefetching blocks into L2 a few entries ahead.
+//               into an ST-stage ring (TMA, SWIZZLE_128B, 64-column panels).
 //   warp 1      owns TMEM; one thread issues tcgen05.mma:
 //               S_t = Q_t K^T (A and B from shared memory) into TMEM, and
 //               O_t += P_t V with P_t read from TMEM (A operand) and V from
@@ -85,7 +84,6 @@ struct PairCfg {
     static constexpr int LIST_CAP = 2048;                  // union entries per item (>= nb + 1)
     static constexpr uint32_t LIST_BYTES = 2 * LIST_CAP * 4;  // double-buffered
     static constexpr int ST = (2 * QBYTES + 4 * 2 * KVBYTES + LIST_BYTES <= 220 * 1024) ? 4 : 2;
-    static constexpr int PREFETCH = 4;                     // K/V blocks prefetched into L2 ahead
     static constexpr uint32_t KPANEL = ST * BK * 128;      // bytes of one 64-column K panel, all stages
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = OFF_Q + 2 * QBYTES;  // [panel][stage][BK rows x 128 B]
@@ -352,21 +350,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 const PairItem I = pair_item<BK>(p, w);
                 const uint32_t* L = list + b * C::LIST_CAP;
                 const int len = list_len[b];
-                for (int e = 0; e < C::PREFETCH && e < len; ++e) {
-                    const int32_t row = (int32_t)(I.row_base + (int64_t)list_j(L[e]) * BK);
-                    for (int pn = 0; pn < HD / 64; ++pn) {
-                        tma_prefetch_2d(&tmK, pn * 64, row);
-                        tma_prefetch_2d(&tmV, pn * 64, row);
-                    }
-                }
                 for (int e = 0; e < len; ++e, ++n) {
-                    if (e + C::PREFETCH < len) {
-                        const int32_t row = (int32_t)(I.row_base + (int64_t)list_j(L[e + C::PREFETCH]) * BK);
-                        for (int pn = 0; pn < HD / 64; ++pn) {
-                            tma_prefetch_2d(&tmK, pn * 64, row);
-                            tma_prefetch_2d(&tmV, pn * 64, row);
-                        }
-                    }
                     const int st = n % C::ST;
                     if (!mbar_wait(bar_ke(st), ((n / C::ST) & 1) ^ 1, ctl)) {
                         stop = true;
