@@ -54,6 +54,16 @@ def _load():
     lib.s2o_decode_items.restype = i32
     lib.s2o_decode_items.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
                                      i64, vp, dbl, i64, vp, vp, vp, i32]
+    lib.s2o_range_block_active.restype = i32
+    lib.s2o_range_block_active.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp]
+    lib.s2o_range_block_mask.restype = None
+    lib.s2o_range_block_mask.argtypes = [i64, i64, vp, vp, vp, vp, vp, vp]
+    lib.s2o_prefill_rows_mask.restype = i32
+    lib.s2o_prefill_rows_mask.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, vp,
+                                          dbl, i64, vp, vp, vp, i32]
+    lib.s2o_decode_items_mask.restype = i32
+    lib.s2o_decode_items_mask.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
+                                          i64, vp, dbl, i64, vp, vp, vp, i32]
     _lib = lib
     return lib
 
@@ -153,4 +163,87 @@ def decode(q, k_cache, v_cache, block_table, ctx_lens, B, S, L, scale,
                                   _ptr(it), _ptr(out), _ptr(lse), int(nthreads))
     if rc != 0:
         raise ValueError("oracle decode rejected its arguments")
+    return out, lse
+
+
+def _flat_ranges(ranges):
+    """Per-head lists of (end_block, S, L, dense) -> CSR arrays for the C code."""
+    ptr = [0]
+    end, S, L, dense = [], [], [], []
+    for head in ranges:
+        for (e, s_, l_, d_) in head:
+            end.append(int(e)); S.append(int(s_)); L.append(int(l_)); dense.append(int(bool(d_)))
+        ptr.append(len(end))
+    a = lambda x, t: np.ascontiguousarray(np.asarray(x, dtype=t))
+    return a(ptr, np.int64), a(end, np.int64), a(S, np.int64), a(L, np.int64), a(dense, np.uint8)
+
+
+def range_block_active(h, i, j, head_ranges) -> bool:
+    """Per-context-range rule for head h; head_ranges = [(end_block, S, L, dense), ...]."""
+    _ptr_, end, S, L, dense = _flat_ranges([head_ranges])
+    return bool(_load().s2o_range_block_active(h, i, j, len(head_ranges), _ptr(end), _ptr(S),
+                                               _ptr(L), _ptr(dense)))
+
+
+def range_block_mask(nb, ranges) -> np.ndarray:
+    """uint8 mask [H, nb, nb] of per-head context ranges (ranges[h] = [(end, S, L, dense), ...])."""
+    H = len(ranges)
+    ptr, end, S, L, dense = _flat_ranges(ranges)
+    m = np.zeros((H, nb, nb), dtype=np.uint8)
+    _load().s2o_range_block_mask(H, nb, _ptr(ptr), _ptr(end), _ptr(S), _ptr(L), _ptr(dense),
+                                 _ptr(m))
+    return m
+
+
+def prefill_mask(q, k, v, B, bmask, scale, rows=None, nthreads=0):
+    """Oracle prefill under a block mask [H, nbm, nbm] (uint8).
+
+    q: [batch, H, seq, D]; k, v: [batch, Hkv, seq, D] with Hkv dividing H.
+    Rows that see no key come back as zeros with LSE -inf.
+    """
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    batch, H, seq, D = q.shape
+    Hkv = k.shape[1]
+    assert k.shape == (batch, Hkv, seq, D) and v.shape == k.shape
+    bm = np.ascontiguousarray(np.asarray(bmask, dtype=np.uint8))
+    assert bm.ndim == 3 and bm.shape[0] == H and bm.shape[1] == bm.shape[2]
+    if rows is None:
+        n, r = batch * H * seq, None
+    else:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        n = r.size
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    rc = _load().s2o_prefill_rows_mask(_ptr(q), _ptr(k), _ptr(v), batch, H, Hkv, seq, D, B,
+                                       bm.shape[1], _ptr(bm), float(scale), n, _ptr(r),
+                                       _ptr(out), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle prefill_mask rejected its arguments")
+    return out, lse
+
+
+def decode_mask(q, k_cache, v_cache, block_table, ctx_lens, B, bmask, scale, items=None,
+                nthreads=0):
+    """Oracle decode under a block mask [H, nbm, nbm]; caches [pages, Hkv, page_size, D]."""
+    q, kc, vc = _bits(q), _bits(k_cache), _bits(v_cache)
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    cl = np.ascontiguousarray(np.asarray(ctx_lens, dtype=np.int32))
+    batch, H, D = q.shape
+    _, Hkv, page_size, D2 = kc.shape
+    assert D2 == D and vc.shape == kc.shape
+    bm = np.ascontiguousarray(np.asarray(bmask, dtype=np.uint8))
+    assert bm.ndim == 3 and bm.shape[0] == H and bm.shape[1] == bm.shape[2]
+    if items is None:
+        n, it = batch * H, None
+    else:
+        it = np.ascontiguousarray(np.asarray(items, dtype=np.int64))
+        n = it.size
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    rc = _load().s2o_decode_items_mask(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), _ptr(cl), batch, H,
+                                       Hkv, D, page_size, bt.shape[1], B, bm.shape[1], _ptr(bm),
+                                       float(scale), n, _ptr(it), _ptr(out), _ptr(lse),
+                                       int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle decode_mask rejected its arguments")
     return out, lse

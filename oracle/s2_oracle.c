@@ -30,6 +30,20 @@
  * n tokens whose keys and values sit in a paged cache addressed through a block
  * table (PagedAttention is in the arXiv page's reference list).
  *
+ * Two generalisations follow the same definition with another block rule.
+ * (1) Per-context-range patterns: the arXiv abstract says the patterns can be
+ * customised per head and per context range. Here a head's key-block axis is
+ * cut into consecutive ranges, each with its own (S, L, dense), and key block j
+ * takes the parameters of the range that holds it (s2o_range_block_active).
+ * (2) Any per-head block mask, given as [H][nb][nb] bytes (the *_mask entry
+ * points), with the same token-level causality inside the diagonal block.
+ * The *_mask entry points also take a number of key/value heads Hkv dividing H:
+ * query head h reads key/value head h / (H / Hkv) (grouped-query attention; the
+ * pages do not mention it; Hkv = H is plain multi-head attention).
+ * A query that sees no key at all (possible only under a given mask) gets a
+ * zero output row and LSE = -inf: the softmax over an empty set is undefined,
+ * and zero is the value whose weight in any later merge is nil.
+ *
  * Every loop visits keys in ascending order; nothing is blocked, fused or
  * reordered beyond the definition.
  */
@@ -70,6 +84,39 @@ void s2o_block_mask(int64_t H, int64_t nb, int64_t S, int64_t L,
                     (uint8_t)s2o_block_active(h, i, j, S, L, dense ? dense[h] != 0 : 0);
 }
 
+/* Per-context-range rule for one head. The head's ranges r = 0..nr-1 cover key
+ * blocks [end[r-1], end[r]) (end[-1] = 0), ends strictly ascending. Key block j
+ * uses the parameters of its range: visible iff j <= i and (dense[r] or
+ * i - j < L[r] or (S[r] > 0 and (j + h) mod S[r] == 0)). S[r] = 0 means the
+ * range has no strided blocks. Blocks past the last range are not visible. */
+int s2o_range_block_active(int64_t h, int64_t i, int64_t j, int64_t nr, const int64_t* end,
+                           const int64_t* S, const int64_t* L, const uint8_t* dense)
+{
+    if (j < 0 || i < 0 || j > i) return 0;
+    for (int64_t r = 0; r < nr; ++r) {
+        if (j >= end[r]) continue;
+        if (dense[r]) return 1;
+        if (i - j < L[r]) return 1;
+        return S[r] > 0 && ((j + h) % S[r]) == 0;
+    }
+    return 0;
+}
+
+/* Block mask [H][nb][nb] of per-head context ranges: head h owns ranges
+ * range_ptr[h] .. range_ptr[h+1]-1 of the flat arrays end/S/L/dense. */
+void s2o_range_block_mask(int64_t H, int64_t nb, const int64_t* range_ptr, const int64_t* end,
+                          const int64_t* S, const int64_t* L, const uint8_t* dense,
+                          uint8_t* mask)
+{
+    for (int64_t h = 0; h < H; ++h) {
+        const int64_t r0 = range_ptr[h], nr = range_ptr[h + 1] - r0;
+        for (int64_t i = 0; i < nb; ++i)
+            for (int64_t j = 0; j < nb; ++j)
+                mask[(h * nb + i) * nb + j] = (uint8_t)s2o_range_block_active(
+                    h, i, j, nr, end + r0, S + r0, L + r0, dense + r0);
+    }
+}
+
 /* ------------------------------------------------------------------------- */
 /* Work distribution: a pool of pthreads pulls item indices from a counter.   */
 /* ------------------------------------------------------------------------- */
@@ -80,6 +127,8 @@ typedef struct {
     const int32_t *block_table, *ctx_lens;
     int64_t batch, H, seq, D, B, S, L, page_size, max_pages;
     const uint8_t* dense;
+    const uint8_t* bmask; /* NULL: the block rule above; else [H][nbm][nbm] */
+    int64_t nbm, Hkv;     /* mask side; key/value heads (query head h reads h / (H / Hkv)) */
     double scale;
     int64_t n_items;
     const int64_t* items;
@@ -97,7 +146,15 @@ static int64_t take(job_t* J)
     return r;
 }
 
-/* Prefill row r = (b * H + h) * seq + q: keys 0..q of the same (b, h). */
+/* Is key block j visible to query block i of head h under this job's rule? */
+static int visible(const job_t* J, int64_t h, int64_t i, int64_t j, int dense)
+{
+    if (J->bmask) return j <= i && j < J->nbm && i < J->nbm && J->bmask[(h * J->nbm + i) * J->nbm + j] != 0;
+    return s2o_block_active(h, i, j, J->S, J->L, dense);
+}
+
+/* Prefill row r = (b * H + h) * seq + q: keys 0..q of the same batch entry, read
+ * from key/value head h / (H / Hkv). */
 static void prefill_row(const job_t* J, int64_t r, double* s, double* qd,
                         double* out, double* lse)
 {
@@ -107,15 +164,16 @@ static void prefill_row(const job_t* J, int64_t r, double* s, double* qd,
     const int64_t h = bh % J->H;
     const int64_t i = q / J->B;
     const int dense = J->dense ? J->dense[h] != 0 : 0;
+    const int64_t kvh = (bh / J->H) * J->Hkv + h / (J->H / J->Hkv);
     const uint16_t* Q = J->q + r * D;
-    const uint16_t* K = J->k + bh * seq * D;
-    const uint16_t* V = J->v + bh * seq * D;
+    const uint16_t* K = J->k + kvh * seq * D;
+    const uint16_t* V = J->v + kvh * seq * D;
 
     for (int64_t d = 0; d < D; ++d) qd[d] = bf16_bits_to_double(Q[d]);
 
     double m = -INFINITY;
     for (int64_t k = 0; k <= q; ++k) {
-        if (!s2o_block_active(h, i, k / J->B, J->S, J->L, dense)) continue;
+        if (!visible(J, h, i, k / J->B, dense)) continue;
         double dot = 0.0;
         for (int64_t d = 0; d < D; ++d) dot += qd[d] * bf16_bits_to_double(K[k * D + d]);
         s[k] = J->scale * dot;
@@ -124,10 +182,14 @@ static void prefill_row(const job_t* J, int64_t r, double* s, double* qd,
     double den = 0.0;
     for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
     for (int64_t k = 0; k <= q; ++k) {
-        if (!s2o_block_active(h, i, k / J->B, J->S, J->L, dense)) continue;
+        if (!visible(J, h, i, k / J->B, dense)) continue;
         const double p = exp(s[k] - m);
         den += p;
         for (int64_t d = 0; d < D; ++d) out[d] += p * bf16_bits_to_double(V[k * D + d]);
+    }
+    if (den == 0.0) { /* no visible key */
+        *lse = -INFINITY;
+        return;
     }
     for (int64_t d = 0; d < D; ++d) out[d] /= den;
     *lse = m + log(den);
@@ -135,7 +197,8 @@ static void prefill_row(const job_t* J, int64_t r, double* s, double* qd,
 
 /* Decode item e = seq_index * H + h: the query of sequence s sits at position
  * n-1 (n = ctx_lens[s]) and sees keys 0..n-1, token t being row t % page_size
- * of page block_table[s][t / page_size] in a [pages][H][page_size][D] cache. */
+ * of page block_table[s][t / page_size] in a [pages][Hkv][page_size][D] cache,
+ * key/value head h / (H / Hkv). */
 static int decode_item(const job_t* J, int64_t e, double* s, double* qd,
                        double* out, double* lse)
 {
@@ -145,16 +208,17 @@ static int decode_item(const job_t* J, int64_t e, double* s, double* qd,
     if (n < 1) return -1;
     const int64_t i = (n - 1) / J->B;
     const int dense = J->dense ? J->dense[h] != 0 : 0;
+    const int64_t Hkv = J->Hkv, kvh = h / (H / Hkv);
     const uint16_t* Q = J->q + e * D;
 
     for (int64_t d = 0; d < D; ++d) qd[d] = bf16_bits_to_double(Q[d]);
 
     double m = -INFINITY;
     for (int64_t k = 0; k < n; ++k) {
-        if (!s2o_block_active(h, i, k / J->B, J->S, J->L, dense)) continue;
+        if (!visible(J, h, i, k / J->B, dense)) continue;
         const int64_t page = J->block_table[sq * J->max_pages + k / P];
         if (page < 0) return -1;
-        const uint16_t* Krow = J->k + ((page * H + h) * P + k % P) * D;
+        const uint16_t* Krow = J->k + ((page * Hkv + kvh) * P + k % P) * D;
         double dot = 0.0;
         for (int64_t d = 0; d < D; ++d) dot += qd[d] * bf16_bits_to_double(Krow[d]);
         s[k] = J->scale * dot;
@@ -163,12 +227,16 @@ static int decode_item(const job_t* J, int64_t e, double* s, double* qd,
     double den = 0.0;
     for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
     for (int64_t k = 0; k < n; ++k) {
-        if (!s2o_block_active(h, i, k / J->B, J->S, J->L, dense)) continue;
+        if (!visible(J, h, i, k / J->B, dense)) continue;
         const int64_t page = J->block_table[sq * J->max_pages + k / P];
-        const uint16_t* Vrow = J->v + ((page * H + h) * P + k % P) * D;
+        const uint16_t* Vrow = J->v + ((page * Hkv + kvh) * P + k % P) * D;
         const double p = exp(s[k] - m);
         den += p;
         for (int64_t d = 0; d < D; ++d) out[d] += p * bf16_bits_to_double(Vrow[d]);
+    }
+    if (den == 0.0) { /* no visible key */
+        *lse = -INFINITY;
+        return 0;
     }
     for (int64_t d = 0; d < D; ++d) out[d] /= den;
     *lse = m + log(den);
@@ -260,7 +328,33 @@ int s2o_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     J.kind = 0;
     J.q = q; J.k = k; J.v = v;
     J.batch = batch; J.H = H; J.seq = seq; J.D = D;
-    J.B = B; J.S = S; J.L = L; J.dense = dense; J.scale = scale;
+    J.B = B; J.S = S; J.L = L; J.dense = dense; J.scale = scale; J.Hkv = H;
+    J.n_items = n_rows; J.items = rows; J.out = out; J.lse = lse;
+    return run_job(&J, nthreads);
+}
+
+/* Prefill oracle under a given block mask [H][nbm][nbm] (nbm >= ceil(seq / B);
+ * entries with j > i are ignored) and Hkv key/value heads: k, v are
+ * [batch][Hkv][seq][D]. Other arguments as s2o_prefill_rows. */
+int s2o_prefill_rows_mask(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                          int64_t batch, int64_t H, int64_t Hkv, int64_t seq, int64_t D,
+                          int64_t B, int64_t nbm, const uint8_t* bmask, double scale,
+                          int64_t n_rows, const int64_t* rows, double* out, double* lse,
+                          int nthreads)
+{
+    if (!q || !k || !v || !out || !lse || !bmask || batch < 1 || H < 1 || Hkv < 1 ||
+        H % Hkv != 0 || seq < 1 || D < 1 || B < 1 || nbm < (seq + B - 1) / B || n_rows < 0)
+        return -1;
+    if (!rows && n_rows != batch * H * seq) return -1;
+    if (rows)
+        for (int64_t t = 0; t < n_rows; ++t)
+            if (rows[t] < 0 || rows[t] >= batch * H * seq) return -1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.kind = 0;
+    J.q = q; J.k = k; J.v = v;
+    J.batch = batch; J.H = H; J.seq = seq; J.D = D; J.B = B; J.Hkv = Hkv;
+    J.bmask = bmask; J.nbm = nbm; J.scale = scale;
     J.n_items = n_rows; J.items = rows; J.out = out; J.lse = lse;
     return run_job(&J, nthreads);
 }
@@ -294,7 +388,40 @@ int s2o_decode_items(const uint16_t* q, const uint16_t* k_cache, const uint16_t*
     J.q = q; J.k = k_cache; J.v = v_cache;
     J.block_table = block_table; J.ctx_lens = ctx_lens;
     J.batch = batch; J.H = H; J.D = D; J.page_size = page_size; J.max_pages = max_pages;
-    J.B = B; J.S = S; J.L = L; J.dense = dense; J.scale = scale;
+    J.B = B; J.S = S; J.L = L; J.dense = dense; J.scale = scale; J.Hkv = H;
+    J.n_items = n_items; J.items = items; J.out = out; J.lse = lse;
+    return run_job(&J, nthreads);
+}
+
+/* Decode oracle under a given block mask [H][nbm][nbm] (nbm >= the block count
+ * of the longest context) and Hkv key/value heads: the caches are
+ * [num_pages][Hkv][page_size][D]. Other arguments as s2o_decode_items. */
+int s2o_decode_items_mask(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                          const int32_t* block_table, const int32_t* ctx_lens,
+                          int64_t batch, int64_t H, int64_t Hkv, int64_t D, int64_t page_size,
+                          int64_t max_pages, int64_t B, int64_t nbm, const uint8_t* bmask,
+                          double scale, int64_t n_items, const int64_t* items, double* out,
+                          double* lse, int nthreads)
+{
+    if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !out || !lse || !bmask ||
+        batch < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || D < 1 || page_size < 1 ||
+        max_pages < 1 || B < 1 || nbm < 1 || n_items < 0)
+        return -1;
+    if (!items && n_items != batch * H) return -1;
+    for (int64_t s = 0; s < batch; ++s)
+        if (ctx_lens[s] < 1 || ctx_lens[s] > max_pages * page_size ||
+            (ctx_lens[s] - 1) / B >= nbm)
+            return -1;
+    if (items)
+        for (int64_t t = 0; t < n_items; ++t)
+            if (items[t] < 0 || items[t] >= batch * H) return -1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.kind = 1;
+    J.q = q; J.k = k_cache; J.v = v_cache;
+    J.block_table = block_table; J.ctx_lens = ctx_lens;
+    J.batch = batch; J.H = H; J.Hkv = Hkv; J.D = D; J.page_size = page_size;
+    J.max_pages = max_pages; J.B = B; J.bmask = bmask; J.nbm = nbm; J.scale = scale;
     J.n_items = n_items; J.items = items; J.out = out; J.lse = lse;
     return run_job(&J, nthreads);
 }
