@@ -1,4 +1,4 @@
-// layout.cpp -- host builder of the HHST per-head compacted key-block lists.
+// layout.cpp -- host builders of the per-head compacted key-block lists (CSR).
 //
 // HHST ("S2-Attention: Hardware-aware context sharding among attention heads",
 // Abstract) gives each head its own strided share of the context plus a local
@@ -77,4 +77,152 @@ extern "C" int s2_build_layout(const s2_layout_desc* d, int32_t* row_ptr, int32_
             row_fill(h, i, S, L, dense, col_idx + row_ptr[h * (nb + 1) + i]);
     }
     return S2_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Per-context-range layouts. The arXiv abstract of S2-Attention says patterns
+// can be customised per head and per context range; here a head's key-block
+// axis is cut into consecutive ranges with their own (S, L, dense), and key
+// block j follows the range that holds it. Enumeration per (h, i) walks the
+// ranges left to right and, inside each, emits the strided blocks below the
+// local window and then the window itself, so lists come out ascending.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+// Visit the active blocks of row (h, i) under one range [a, b): dense, or the
+// strided j = -h (mod S) below the window, then the window i-L+1 .. i.
+template <class F>
+void range_row(int64_t h, int64_t i, int64_t a, int64_t b, const s2_context_range& r, F&& emit)
+{
+    const int64_t hi = b < i + 1 ? b : i + 1;  // exclusive
+    if (a >= hi) return;
+    if (r.dense) {
+        for (int64_t j = a; j < hi; ++j) emit(j);
+        return;
+    }
+    const int64_t L = r.local_blocks, S = r.vertical_stride;
+    int64_t lo = i - L + 1;  // first block of the local window
+    if (lo < a) lo = a;
+    if (lo > hi) lo = hi;
+    if (S > 0) {
+        const int64_t j0 = a + ((S - (a + h) % S) % S);  // first j >= a with (j + h) % S == 0
+        for (int64_t j = j0; j < lo; j += S) emit(j);
+    }
+    for (int64_t j = lo; j < hi; ++j) emit(j);
+}
+
+int64_t range_row_count(int64_t h, int64_t i, int64_t a, int64_t b, const s2_context_range& r)
+{
+    const int64_t hi = b < i + 1 ? b : i + 1;
+    if (a >= hi) return 0;
+    if (r.dense) return hi - a;
+    const int64_t L = r.local_blocks, S = r.vertical_stride;
+    int64_t lo = i - L + 1;
+    if (lo < a) lo = a;
+    if (lo > hi) lo = hi;
+    int64_t n = hi - lo;
+    if (S > 0) {
+        const int64_t j0 = a + ((S - (a + h) % S) % S);
+        if (j0 < lo) n += (lo - 1 - j0) / S + 1;
+    }
+    return n;
+}
+
+// Shared second half of the builders: row offsets from per-row counts, then
+// the lists. count(h, i) and fill(h, i, out) describe one row.
+template <class Count, class Fill>
+int emit_csr(int64_t H, int64_t nb, Count&& count, Fill&& fill, int32_t* row_ptr,
+             int32_t* col_idx, int64_t col_idx_cap, int64_t* nnz_out)
+{
+    int64_t nnz = 0;
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t i = 0; i < nb; ++i) nnz += count(h, i);
+    *nnz_out = nnz;
+    if (nnz > INT32_MAX) return S2_ERR_CAPACITY;
+    if (!row_ptr) return S2_OK;
+    int64_t off = 0;
+    for (int64_t h = 0; h < H; ++h) {
+        for (int64_t i = 0; i < nb; ++i) {
+            row_ptr[h * (nb + 1) + i] = (int32_t)off;
+            off += count(h, i);
+        }
+        row_ptr[h * (nb + 1) + nb] = (int32_t)off;
+    }
+    if (!col_idx) return S2_OK;
+    if (col_idx_cap < nnz) return S2_ERR_CAPACITY;
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t i = 0; i < nb; ++i) fill(h, i, col_idx + row_ptr[h * (nb + 1) + i]);
+    return S2_OK;
+}
+
+}  // namespace
+
+extern "C" int s2_build_layout_ranges(int32_t num_heads, int32_t num_blocks,
+                                      const int32_t* range_ptr, const s2_context_range* ranges,
+                                      int32_t* row_ptr, int32_t* col_idx, int64_t col_idx_cap,
+                                      int64_t* nnz_out)
+{
+    if (!range_ptr || !ranges || !nnz_out || num_heads < 1 || num_blocks < 1)
+        return S2_ERR_INVALID_ARG;
+    if (col_idx && !row_ptr) return S2_ERR_INVALID_ARG;
+    const int64_t H = num_heads, nb = num_blocks;
+    if (range_ptr[0] != 0) return S2_ERR_INVALID_ARG;
+    for (int64_t h = 0; h < H; ++h) {
+        const int32_t r0 = range_ptr[h], r1 = range_ptr[h + 1];
+        if (r1 <= r0) return S2_ERR_INVALID_ARG;
+        int64_t prev = 0;
+        for (int32_t r = r0; r < r1; ++r) {
+            const s2_context_range& c = ranges[r];
+            if (c.end_block <= prev || c.vertical_stride < 0 || c.local_blocks < 0)
+                return S2_ERR_INVALID_ARG;
+            prev = c.end_block;
+        }
+        if (prev != nb) return S2_ERR_INVALID_ARG;
+    }
+    auto count = [&](int64_t h, int64_t i) {
+        int64_t n = 0, a = 0;
+        for (int32_t r = range_ptr[h]; r < range_ptr[h + 1] && a <= i; ++r) {
+            n += range_row_count(h, i, a, ranges[r].end_block, ranges[r]);
+            a = ranges[r].end_block;
+        }
+        return n;
+    };
+    auto fill = [&](int64_t h, int64_t i, int32_t* out) {
+        int64_t n = 0, a = 0;
+        for (int32_t r = range_ptr[h]; r < range_ptr[h + 1] && a <= i; ++r) {
+            range_row(h, i, a, ranges[r].end_block, ranges[r],
+                      [&](int64_t j) { out[n++] = (int32_t)j; });
+            a = ranges[r].end_block;
+        }
+    };
+    return emit_csr(H, nb, count, fill, row_ptr, col_idx, col_idx_cap, nnz_out);
+}
+
+extern "C" int s2_build_layout_mask(int32_t num_heads, int32_t num_blocks,
+                                    const uint8_t* block_mask, int32_t* row_ptr, int32_t* col_idx,
+                                    int64_t col_idx_cap, int64_t* nnz_out)
+{
+    if (!block_mask || !nnz_out || num_heads < 1 || num_blocks < 1) return S2_ERR_INVALID_ARG;
+    if (col_idx && !row_ptr) return S2_ERR_INVALID_ARG;
+    const int64_t H = num_heads, nb = num_blocks;
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t i = 0; i < nb; ++i) {
+            const uint8_t* m = block_mask + (h * nb + i) * nb;
+            for (int64_t j = i + 1; j < nb; ++j)
+                if (m[j]) return S2_ERR_INVALID_ARG;  // above the diagonal
+        }
+    auto count = [&](int64_t h, int64_t i) {
+        const uint8_t* m = block_mask + (h * nb + i) * nb;
+        int64_t n = 0;
+        for (int64_t j = 0; j <= i; ++j) n += m[j] != 0;
+        return n;
+    };
+    auto fill = [&](int64_t h, int64_t i, int32_t* out) {
+        const uint8_t* m = block_mask + (h * nb + i) * nb;
+        int64_t n = 0;
+        for (int64_t j = 0; j <= i; ++j)
+            if (m[j]) out[n++] = (int32_t)j;
+    };
+    return emit_csr(H, nb, count, fill, row_ptr, col_idx, col_idx_cap, nnz_out);
 }

@@ -121,10 +121,13 @@ struct UnionWalk {
     int a[ROWS], e[ROWS];
     int imax;
 
+    // Returns false for offsets outside [0, nnz]; `any` tells whether a list is non-empty.
+    bool any;
+
     __device__ __forceinline__ bool init(const int32_t* row_ptr, int rp, int qb0, int nb, int64_t nnz)
     {
         bool ok = true;
-        bool any = false;
+        any = false;
         imax = -1;
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
@@ -141,8 +144,9 @@ struct UnionWalk {
         if (!ok) {
 #pragma unroll
             for (int r = 0; r < ROWS; ++r) a[r] = e[r] = 0;
+            any = false;
         }
-        return ok && any;
+        return ok;
     }
 
     // Next union element: key block j, row tag bits, and whether it is the last.
@@ -298,7 +302,8 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 const PairItem I = pair_item<BK>(p, w);
                 UnionWalk<C::ROWS> it;
                 int len = 0;
-                if (it.init(p.row_ptr, I.rp, I.qb0, p.nb, p.nnz)) {
+                const bool ok = it.init(p.row_ptr, I.rp, I.qb0, p.nb, p.nnz);
+                if (it.any) {  // an item whose rows are all empty publishes an empty list
                     for (;;) {
                         int j, bits;
                         bool last, bad;
@@ -312,7 +317,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         if (last) break;
                     }
                     while (len % G) wlist[b * C::LIST_CAP + len++] = list_pack(0, 0);  // masked pad
-                } else {
+                } else if (!ok) {
                     atomicOr(p.gflags, kFlagIndex);
                 }
                 list_len[b] = len;
@@ -633,7 +638,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
                 if (row_valid && p.lse)
                     p.lse[I.row_base + qpos] = l > 0.f ? (m_used + lg2(l)) * 0.69314718055994531f : -INFINITY;
-            } else if (row_valid) {  // malformed layout: the row saw no key block
+            } else if (row_valid) {  // no row of this tile lists a key block: zero output
                 uint16_t* orow = p.o + (I.row_base + qpos) * HD;
                 for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
                 if (p.lse) p.lse[I.row_base + qpos] = -INFINITY;

@@ -220,8 +220,8 @@ int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float*
                     int32_t block_size, int32_t num_blocks, const int32_t* row_ptr,
                     const int32_t* col_idx, int64_t nnz, void* stream)
 {
-    if (!q || !k || !v || !o || !row_ptr || !col_idx) return S2_ERR_INVALID_ARG;
-    if (batch < 1 || heads < 1 || seq < 1 || nnz < 1 || !std::isfinite(scale) || !(scale > 0.f))
+    if (!q || !k || !v || !o || !row_ptr || (!col_idx && nnz > 0)) return S2_ERR_INVALID_ARG;
+    if (batch < 1 || heads < 1 || seq < 1 || nnz < 0 || !std::isfinite(scale) || !(scale > 0.f))
         return S2_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
     if (block_size != 64 && block_size != 128) return S2_ERR_UNSUPPORTED;
@@ -284,9 +284,10 @@ int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                    void* out, float* lse, void* workspace, size_t workspace_bytes,
                    int32_t num_splits, void* stream)
 {
-    if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !row_ptr || !col_idx || !out)
+    if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !row_ptr ||
+        (!col_idx && nnz > 0) || !out)
         return S2_ERR_INVALID_ARG;
-    if (batch < 1 || heads < 1 || max_pages < 1 || num_pages < 1 || num_blocks < 1 || nnz < 1 ||
+    if (batch < 1 || heads < 1 || max_pages < 1 || num_pages < 1 || num_blocks < 1 || nnz < 0 ||
         !std::isfinite(scale) || num_splits > kMaxSplits)
         return S2_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;

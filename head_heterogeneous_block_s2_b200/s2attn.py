@@ -6,7 +6,8 @@ stream, and turns status codes into exceptions. There is no fallback: if the
 library is missing or a call fails, it raises.
 
 Entry points mirror the C ABI in ``include/s2attn.h``:
-``build_layout`` (host), ``prefill``, ``decode``, ``decode_workspace_size``,
+``build_layout``, ``build_layout_ranges`` and ``build_layout_mask`` (host),
+``prefill``, ``decode``, ``decode_noalloc``, ``decode_workspace_size``,
 ``device_status`` and ``set_wait_timeout_ns``.
 """
 from __future__ import annotations
@@ -26,7 +27,8 @@ S2_OK = 0
 STATUS_NAMES = {0: "S2_OK", 1: "S2_ERR_INVALID_ARG", 2: "S2_ERR_UNSUPPORTED", 3: "S2_ERR_CAPACITY",
                 4: "S2_ERR_CUDA", 5: "S2_ERR_TIMEOUT", 6: "S2_ERR_DEVICE_INDEX"}
 
-EXPORTED = ("s2_status_string", "s2_build_layout", "s2_attn_prefill",
+EXPORTED = ("s2_status_string", "s2_build_layout", "s2_build_layout_ranges",
+            "s2_build_layout_mask", "s2_attn_prefill",
             "s2_attn_decode_workspace_size", "s2_attn_decode_auto_splits", "s2_attn_decode",
             "s2_device_status", "s2_set_wait_timeout_ns", "s2_version", "s2_attn_decode_noalloc")
 
@@ -41,6 +43,11 @@ class _LayoutDesc(ctypes.Structure):
     _fields_ = [("num_heads", ctypes.c_int32), ("block_size", ctypes.c_int32),
                 ("vertical_stride", ctypes.c_int32), ("local_blocks", ctypes.c_int32),
                 ("num_blocks", ctypes.c_int32), ("dense_head_mask", ctypes.c_void_p)]
+
+
+class _ContextRange(ctypes.Structure):
+    _fields_ = [("end_block", ctypes.c_int32), ("vertical_stride", ctypes.c_int32),
+                ("local_blocks", ctypes.c_int32), ("dense", ctypes.c_int32)]
 
 
 _lib = None
@@ -62,6 +69,10 @@ def load(path: str = LIB_PATH):
     lib.s2_version.argtypes = []
     lib.s2_build_layout.restype = ctypes.c_int
     lib.s2_build_layout.argtypes = [ctypes.POINTER(_LayoutDesc), vp, vp, i64, ctypes.POINTER(i64)]
+    lib.s2_build_layout_ranges.restype = ctypes.c_int
+    lib.s2_build_layout_ranges.argtypes = [i32, i32, vp, vp, vp, vp, i64, ctypes.POINTER(i64)]
+    lib.s2_build_layout_mask.restype = ctypes.c_int
+    lib.s2_build_layout_mask.argtypes = [i32, i32, vp, vp, vp, i64, ctypes.POINTER(i64)]
     lib.s2_attn_prefill.restype = ctypes.c_int
     lib.s2_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp, vp,
                                     i64, vp]
@@ -92,7 +103,11 @@ def _check(rc: int, what: str):
 
 @dataclasses.dataclass
 class Layout:
-    """Per-head compacted key-block lists (CSR) of one HHST layout."""
+    """Per-head compacted key-block lists (CSR) of one layout.
+
+    ``pattern`` says which builder made it: "hhst" (stride, local and
+    dense_heads are its parameters), "ranges" (``ranges`` holds the per-head
+    context ranges) or "mask"."""
     heads: int
     block_size: int
     stride: int
@@ -103,6 +118,8 @@ class Layout:
     col_idx: np.ndarray  # int32 [nnz]
     d_row_ptr: Optional[torch.Tensor] = None
     d_col_idx: Optional[torch.Tensor] = None
+    pattern: str = "hhst"
+    ranges: Optional[Tuple[Tuple[Tuple[int, int, int, bool], ...], ...]] = None
 
     @property
     def nnz(self) -> int:
@@ -114,7 +131,9 @@ class Layout:
 
     def to(self, device) -> "Layout":
         self.d_row_ptr = torch.from_numpy(self.row_ptr).to(device)
-        self.d_col_idx = torch.from_numpy(self.col_idx).to(device)
+        # an empty layout still gets a (never read) one-element buffer
+        col = self.col_idx if self.col_idx.size else np.zeros(1, dtype=np.int32)
+        self.d_col_idx = torch.from_numpy(col).to(device)
         return self
 
 
@@ -156,6 +175,65 @@ def build_layout(heads: int, block_size: int, stride: int, local: int, num_block
     return lay
 
 
+def _two_call(fn, heads: int, num_blocks: int, what: str):
+    """Run a builder twice (count, then fill) and return (row_ptr, col_idx)."""
+    nnz = ctypes.c_int64(0)
+    _check(fn(None, None, 0, ctypes.byref(nnz)), what)
+    row_ptr = np.zeros(heads * (num_blocks + 1), dtype=np.int32)
+    col_idx = np.zeros(max(1, nnz.value), dtype=np.int32)
+    _check(fn(row_ptr.ctypes.data, col_idx.ctypes.data, col_idx.size, ctypes.byref(nnz)), what)
+    return row_ptr, col_idx[:nnz.value].copy()
+
+
+def build_layout_ranges(ranges: Sequence[Sequence[Tuple[int, int, int, bool]]], block_size: int,
+                        num_blocks: int, device=None) -> Layout:
+    """Run s2_build_layout_ranges (host).
+
+    ``ranges[h]`` lists head h's context ranges as (end_block, stride, local,
+    dense) tuples, ends ascending, the last equal to ``num_blocks``; key block
+    j follows the range that holds it."""
+    lib = load()
+    heads = len(ranges)
+    ptr = np.zeros(heads + 1, dtype=np.int32)
+    flat = []
+    for h, head in enumerate(ranges):
+        for (e, st, lo, dn) in head:
+            flat.append((int(e), int(st), int(lo), int(bool(dn))))
+        ptr[h + 1] = len(flat)
+    arr = (_ContextRange * max(1, len(flat)))(*[_ContextRange(*t) for t in flat])
+
+    def fn(rp, ci, cap, nnz):
+        return lib.s2_build_layout_ranges(heads, num_blocks, ptr.ctypes.data,
+                                          ctypes.cast(arr, ctypes.c_void_p), rp, ci, cap, nnz)
+
+    row_ptr, col_idx = _two_call(fn, heads, num_blocks, "s2_build_layout_ranges")
+    frozen = tuple(tuple((int(e), int(st), int(lo), bool(dn)) for (e, st, lo, dn) in head)
+                   for head in ranges)
+    lay = Layout(heads, block_size, 0, 0, num_blocks, (), row_ptr, col_idx, pattern="ranges",
+                 ranges=frozen)
+    if device is not None:
+        lay.to(device)
+    return lay
+
+
+def build_layout_mask(block_mask: np.ndarray, block_size: int, device=None) -> Layout:
+    """Run s2_build_layout_mask (host) on a [heads, nb, nb] mask (nonzero = active)."""
+    lib = load()
+    m = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+    if m.ndim != 3 or m.shape[1] != m.shape[2]:
+        raise ValueError("block_mask must be [heads, num_blocks, num_blocks]")
+    heads, num_blocks = int(m.shape[0]), int(m.shape[1])
+
+    def fn(rp, ci, cap, nnz):
+        return lib.s2_build_layout_mask(heads, num_blocks, m.ctypes.data, rp, ci, cap, nnz)
+
+    row_ptr, col_idx = _two_call(fn, heads, num_blocks, "s2_build_layout_mask")
+    lay = Layout(heads, block_size, 0, 0, num_blocks, (), row_ptr, col_idx, pattern="mask")
+    if device is not None:
+        lay.to(device)
+    return lay
+
+
 # ------------------------------------------------------------------ kernels
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -186,6 +264,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: Layout,
     batch, heads, seq, hd = q.shape
     if k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v shapes differ")
+    if layout.heads != heads:
+        raise ValueError(f"layout has {layout.heads} heads, q has {heads}")
     if layout.d_row_ptr is None:
         layout.to(q.device)
     if out is None:
@@ -227,6 +307,8 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     num_pages, h2, page_size, hd2 = k_cache.shape
     if h2 != heads or hd2 != hd or v_cache.shape != k_cache.shape:
         raise ValueError("cache shape does not match q")
+    if layout.heads != heads:
+        raise ValueError(f"layout has {layout.heads} heads, q has {heads}")
     if layout.d_row_ptr is None:
         layout.to(q.device)
     if out is None:
@@ -274,6 +356,8 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     num_pages, h2, page_size, hd2 = k_cache.shape
     if h2 != heads or hd2 != hd or v_cache.shape != k_cache.shape:
         raise ValueError("cache shape does not match q")
+    if layout.heads != heads:
+        raise ValueError(f"layout has {layout.heads} heads, q has {heads}")
     if layout.d_row_ptr is None:
         layout.to(q.device)
     if out is None:

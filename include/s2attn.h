@@ -84,12 +84,67 @@ typedef struct s2_layout_desc {
  *     row_ptr[h*(nb+1) + nb] == row_ptr[(h+1)*(nb+1)] and row_ptr[0] == 0.
  *   col_idx [col_idx_cap] (host, written): active key blocks j, ascending within
  *     each list, so the diagonal block i is always last.
- *   *nnz_out = total entries. S2_ERR_CAPACITY when col_idx_cap < nnz.
- * Cost O(H * nb^2) rule evaluations; call once per layout and copy the arrays
- * to the device for the kernels.
+ *   *nnz_out = total entries. S2_ERR_CAPACITY when col_idx_cap < nnz, or when
+ *   nnz exceeds INT32_MAX (offsets are int32).
+ * S2_ERR_INVALID_ARG for a NULL desc or nnz_out, a parameter out of range, or
+ * col_idx given without row_ptr. The lists are enumerated directly (cost
+ * O(nnz)); call once per layout and copy the arrays to the device.
  */
 int s2_build_layout(const s2_layout_desc* desc, int32_t* row_ptr, int32_t* col_idx,
                     int64_t col_idx_cap, int64_t* nnz_out);
+
+/* One context range of a head's pattern (s2_build_layout_ranges). */
+typedef struct s2_context_range {
+    int32_t end_block;       /* exclusive end on the key-block axis; strictly ascending within
+                                a head, the head's last range ends at num_blocks */
+    int32_t vertical_stride; /* S >= 0; 0 = the range has no strided blocks */
+    int32_t local_blocks;    /* L >= 0 */
+    int32_t dense;           /* nonzero = every causal block of the range is active */
+} s2_context_range;
+
+/*
+ * Layouts customised per head and per context range. The arXiv abstract of
+ * "S2-Attention: Hardware-aware context sharding among attention heads" says
+ * the patterns can be set at both levels and gives no formula; the reading
+ * here: head h's ranges, ranges[range_ptr[h]] .. ranges[range_ptr[h+1] - 1],
+ * cut its key-block axis [0, num_blocks) into consecutive pieces, and key
+ * block j <= i is active for query block i of head h iff, with the (S, L,
+ * dense) of the range that holds j,
+ *
+ *     dense  or  i - j < L  or  (S > 0 and (j + h) mod S == 0).
+ *
+ * One range [0, nb) with S >= 1, L >= 1 is the HHST rule of s2_build_layout.
+ * A dense first range gives every head the opening blocks of the context; a
+ * range with S = 0 keeps only its local window.
+ *
+ *   range_ptr  host int32 [num_heads + 1] (read): range_ptr[0] == 0, at least
+ *              one range per head (range_ptr[h] < range_ptr[h+1]).
+ *   ranges     host [range_ptr[num_heads]] (read).
+ * Output arrays, the two-call protocol and S2_ERR_CAPACITY as s2_build_layout.
+ * A list may be empty (a range pattern may leave a query block with no key):
+ * the kernels then write a zero output row and LSE = -inf for its queries.
+ * S2_ERR_INVALID_ARG for NULL pointers, num_heads or num_blocks < 1, and
+ * ranges that are empty, not ascending, do not end at num_blocks, or have a
+ * negative S or L. Cost O(nnz + number of ranges * num_blocks).
+ */
+int s2_build_layout_ranges(int32_t num_heads, int32_t num_blocks, const int32_t* range_ptr,
+                           const s2_context_range* ranges, int32_t* row_ptr,
+                           int32_t* col_idx, int64_t col_idx_cap, int64_t* nnz_out);
+
+/*
+ * Layout from any per-head block mask (the generic form of a per-head
+ * pattern): block_mask is host uint8 [num_heads][num_blocks][num_blocks],
+ * nonzero at [h][i][j] when key block j is active for query block i of head
+ * h. Causality inside the diagonal block is still applied by the kernels.
+ * Entries above the diagonal (j > i) must be zero: the kernels treat every
+ * listed block other than the diagonal as fully visible, so such an entry is
+ * rejected with S2_ERR_INVALID_ARG rather than silently dropped. Output
+ * arrays, the two-call protocol and S2_ERR_CAPACITY as s2_build_layout; lists
+ * may be empty as in s2_build_layout_ranges. Cost O(num_heads * num_blocks^2).
+ */
+int s2_build_layout_mask(int32_t num_heads, int32_t num_blocks, const uint8_t* block_mask,
+                         int32_t* row_ptr, int32_t* col_idx, int64_t col_idx_cap,
+                         int64_t* nnz_out);
 
 /* ------------------------------------------------------------------------ */
 /* Prefill: block-sparse causal attention over whole sequences               */
@@ -104,11 +159,15 @@ int s2_build_layout(const s2_layout_desc* desc, int32_t* row_ptr, int32_t* col_i
  *             log-sum-exp of the scaled visible logits of each row (written).
  *   head_dim  64 or 128.  block_size 64 or 128.  seq % block_size == 0.
  *   num_blocks == seq / block_size.
- *   row_ptr, col_idx, nnz: the layout of s2_build_layout for (heads,
- *             block_size, num_blocks), copied to device memory (read).
+ *   row_ptr, col_idx, nnz: a layout from one of the s2_build_layout*
+ *             builders for (heads, num_blocks), copied to device memory
+ *             (read). Lists must be strictly ascending with j <= i; nnz may be
+ *             0 (then col_idx may be NULL). A query row whose list is empty
+ *             gets a zero output row and LSE = -inf.
  *   scale     multiplier of the logits (1/sqrt(head_dim) in the usual case).
  * Runs tcgen05 tensor-core tiles of 128 query rows; only the listed key blocks
  * are visited and causality is applied inside the diagonal block only.
+ * num_blocks is at most 2046 (union lists are staged in shared memory).
  */
 int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
                     int32_t batch, int32_t heads, int32_t seq, int32_t head_dim,
@@ -142,7 +201,9 @@ int32_t s2_attn_decode_auto_splits(int32_t batch, int32_t heads);
  *   ctx_lens     device int32 [batch] (read), 1 <= n <= min(max_pages *
  *                page_size, num_blocks * block_size).
  *   page_size 16.  head_dim 64 or 128.  block_size a multiple of page_size.
- *   row_ptr, col_idx, nnz: device layout for (heads, block_size, num_blocks).
+ *   row_ptr, col_idx, nnz: device layout for (heads, num_blocks) from one of
+ *                the s2_build_layout* builders; an empty list gives a zero
+ *                output and LSE = -inf.
  *   out          device bf16 [batch][heads][head_dim] (written).
  *   lse          device fp32 [batch][heads] or NULL (written).
  *   workspace    device, >= s2_attn_decode_workspace_size(...) bytes, 256-byte

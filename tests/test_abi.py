@@ -55,7 +55,7 @@ def _prefill(**over):
 @pytest.mark.parametrize("over,code", [
     (dict(q=None), 1), (dict(row_ptr=None), 1), (dict(batch=0), 1), (dict(seq=500), 1),
     (dict(nb=7), 1), (dict(hd=96), 2), (dict(bs=32), 2), (dict(q=(1 << 20) + 8), 1),
-    (dict(scale=float("nan")), 1), (dict(nnz=0), 1),
+    (dict(scale=float("nan")), 1), (dict(nnz=-1), 1), (dict(col_idx=None), 1),
 ])
 def test_prefill_rejects_bad_arguments_before_launch(over, code):
     assert _prefill(**over) == code
@@ -78,6 +78,7 @@ def _decode(**over):
     (dict(q=None), 1), (dict(bt=None), 1), (dict(page=32), 2), (dict(hd=80), 2),
     (dict(bs=24), 2), (dict(splits=2, ws=None), 1), (dict(splits=2, ws=1 << 20, ws_bytes=16), 3),
     (dict(splits=2, ws=(1 << 20) + 16, ws_bytes=1 << 20), 1), (dict(splits=1000), 1),
+    (dict(nnz=-1), 1), (dict(ci=None), 1),
 ])
 def test_decode_rejects_bad_arguments_before_launch(over, code):
     assert _decode(**over) == code
