@@ -28,14 +28,14 @@ namespace s2 {
 
 struct DecodeParams {
     const uint16_t* q;       // [batch][H][HD]
-    const uint16_t* k_cache; // [pages][H][16][HD]
+    const uint16_t* k_cache; // [pages][H_kv][16][HD]; query head h reads K/V head h / (H / H_kv)
     const uint16_t* v_cache;
     const int32_t* block_table;  // [batch][max_pages]
     const int32_t* ctx_lens;     // [batch]
     const int32_t* row_ptr;
     const int32_t* col_idx;
     int64_t nnz, num_pages;
-    int32_t batch, heads, max_pages, block_size, nb, num_splits;
+    int32_t batch, heads, heads_kv, max_pages, block_size, nb, num_splits;
     float scale_log2;
     uint16_t* out;   // [batch][H][HD] (num_splits == 1)
     float* lse;      // [batch][H] or null (num_splits == 1)
@@ -78,6 +78,7 @@ s2_decode_split_kernel(const DecodeParams p)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sp = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int H = p.heads;
+    const int hkv = h / (H / p.heads_kv);
 
     auto bar_full = [&](int st) { return sb + C::OFF_BAR + 8u * st; };
     auto bar_empty = [&](int st) { return sb + C::OFF_BAR + 8u * (C::NS + st); };
@@ -157,7 +158,7 @@ s2_decode_split_kernel(const DecodeParams p)
                 if (!mbar_wait(bar_empty(st), ((n / C::NS) & 1) ^ 1, ctl)) break;
                 meta[st] = make_int2(tok0, valid);
                 if (valid > 0) {
-                    const int64_t off = ((phys * H + h) * kPage) * HD;
+                    const int64_t off = ((phys * p.heads_kv + hkv) * kPage) * HD;
                     mbar_arrive_expect_tx(bar_full(st), C::STAGE_BYTES);
                     bulk_load(sb + st * C::STAGE_BYTES, p.k_cache + off, C::PAGE_BYTES, bar_full(st));
                     bulk_load(sb + st * C::STAGE_BYTES + C::PAGE_BYTES, p.v_cache + off, C::PAGE_BYTES,

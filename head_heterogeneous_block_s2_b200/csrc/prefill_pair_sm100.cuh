@@ -195,7 +195,8 @@ constexpr int kHeadMajorPairs = 64;
 struct PairItem {
     int qt0, qb0, rp;
     bool tile1;
-    int64_t row_base;
+    int bh, bkv;       // (batch, query head) and (batch, K/V head) plane indices
+    int64_t row_base;  // first output row of the plane: bh * seq
 };
 
 template <int BK>
@@ -215,6 +216,8 @@ __device__ __forceinline__ PairItem pair_item(const PrefillParams& p, int w)
     it.tile1 = it.qt0 + 1 < p.nqt;
     it.qb0 = (BK == 128) ? it.qt0 : 2 * it.qt0;
     it.rp = (bh % p.heads) * (p.nb + 1);
+    it.bh = bh;
+    it.bkv = (bh / p.heads) * p.heads_kv + (bh % p.heads) / (p.heads / p.heads_kv);
     it.row_base = (int64_t)bh * p.seq;
     return it;
 }
@@ -329,13 +332,13 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 for (int t = 0; t < (I.tile1 ? 2 : 1); ++t)
 #pragma unroll
                     for (int pn = 0; pn < HD / 64; ++pn)
-                        tma_load_2d(sb + C::OFF_Q + t * C::QBYTES + pn * (C::M * 128), &tmQ, pn * 64,
-                                    (int32_t)(I.row_base + (I.qt0 + t) * C::M), bar_q);
+                        tma_load_3d(sb + C::OFF_Q + t * C::QBYTES + pn * (C::M * 128), &tmQ, pn * 64,
+                                    (I.qt0 + t) * C::M, I.bh, bar_q);
                 if (w_next < num_items) {  // next item's Q into L2
                     const PairItem J = pair_item<BK>(p, w_next);
                     for (int t = 0; t < (J.tile1 ? 2 : 1); ++t)
                         for (int pn = 0; pn < HD / 64; ++pn)
-                            tma_prefetch_2d(&tmQ, pn * 64, (int32_t)(J.row_base + (J.qt0 + t) * C::M));
+                            tma_prefetch_3d(&tmQ, pn * 64, (J.qt0 + t) * C::M, J.bh);
                 }
                 w = w_next;
             }
@@ -361,17 +364,17 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         stop = true;
                         break;
                     }
-                    const int32_t krow = (int32_t)(I.row_base + (int64_t)list_j(L[e]) * BK);
+                    const int32_t krow = list_j(L[e]) * BK;
                     mbar_arrive_expect_tx(bar_kf(st), C::KVBYTES);
 #pragma unroll
                     for (int pn = 0; pn < HD / 64; ++pn)
-                        tma_load_2d(sb + C::OFF_K + pn * C::KPANEL + st * (BK * 128), &tmK, pn * 64, krow,
-                                    bar_kf(st));
+                        tma_load_3d(sb + C::OFF_K + pn * C::KPANEL + st * (BK * 128), &tmK, pn * 64, krow,
+                                    I.bkv, bar_kf(st));
                     mbar_arrive_expect_tx(bar_vf(st), C::KVBYTES);
 #pragma unroll
                     for (int pn = 0; pn < HD / 64; ++pn)
-                        tma_load_2d(sb + C::OFF_V + st * C::KVBYTES + pn * (BK * 128), &tmV, pn * 64,
-                                    krow, bar_vf(st));
+                        tma_load_3d(sb + C::OFF_V + st * C::KVBYTES + pn * (BK * 128), &tmV, pn * 64,
+                                    krow, I.bkv, bar_vf(st));
                 }
                 if (!stop) mbar_arrive(bar_le(b));
             }

@@ -91,13 +91,16 @@ int device_ready(int* dev_out)
 }
 
 // 2-D bf16 tensor map over [rows][cols], box [box_rows][64], SWIZZLE_128B.
-int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+// 3-D bf16 tensor map over [planes][seq][cols] (cols innermost), 64-column
+// SWIZZLE_128B boxes of box_rows rows; rows at or past seq read as zeros.
+int make_map(CUtensorMap* m, const void* base, uint64_t planes, uint64_t seq, uint64_t cols,
+             uint32_t box_rows)
 {
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+    const cuuint64_t dims[3] = {cols, seq, planes};
+    const cuuint64_t strides[2] = {cols * 2, seq * cols * 2};
+    const cuuint32_t box[3] = {64, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -111,10 +114,10 @@ int launch_prefill(const void* q, const void* k, const void* v, s2::PrefillParam
                    int attr_slot, cudaStream_t stream)
 {
     using C = s2::PairCfg<HD, BK>;
-    const uint64_t rows = (uint64_t)pp.batch * pp.heads * pp.seq;
+    const uint64_t qplanes = (uint64_t)pp.batch * pp.heads, kvplanes = (uint64_t)pp.batch * pp.heads_kv;
     CUtensorMap mq, mk, mv;
-    if (make_map(&mq, q, rows, HD, 128) || make_map(&mk, k, rows, HD, BK) ||
-        make_map(&mv, v, rows, HD, BK))
+    if (make_map(&mq, q, qplanes, pp.seq, HD, 128) || make_map(&mk, k, kvplanes, pp.seq, HD, BK) ||
+        make_map(&mv, v, kvplanes, pp.seq, HD, BK))
         return S2_ERR_CUDA;
     auto kern = s2::s2_prefill_pair_kernel<HD, BK>;
     {
@@ -215,19 +218,22 @@ int s2_device_status(int reset, uint32_t* flags_out)
     return S2_OK;
 }
 
-int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
-                    int32_t batch, int32_t heads, int32_t seq, int32_t head_dim, float scale,
-                    int32_t block_size, int32_t num_blocks, const int32_t* row_ptr,
-                    const int32_t* col_idx, int64_t nnz, void* stream)
+int s2_attn_prefill_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int32_t batch, int32_t heads, int32_t heads_kv, int32_t seq,
+                        int32_t head_dim, float scale, int32_t block_size, int32_t num_blocks,
+                        const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz, void* stream)
 {
     if (!q || !k || !v || !o || !row_ptr || (!col_idx && nnz > 0)) return S2_ERR_INVALID_ARG;
     if (batch < 1 || heads < 1 || seq < 1 || nnz < 0 || !std::isfinite(scale) || !(scale > 0.f))
         return S2_ERR_INVALID_ARG;
+    if (heads_kv < 1 || heads % heads_kv != 0) return S2_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
     if (block_size != 64 && block_size != 128) return S2_ERR_UNSUPPORTED;
     if (num_blocks > 2046) return S2_ERR_UNSUPPORTED;  // union lists are staged in shared memory
-    if (seq % block_size != 0 || num_blocks != seq / block_size) return S2_ERR_INVALID_ARG;
-    if ((int64_t)batch * heads * seq >= (int64_t)INT32_MAX) return S2_ERR_UNSUPPORTED;
+    if (num_blocks != (seq + block_size - 1) / block_size) return S2_ERR_INVALID_ARG;
+    // work items are counted in int on the device
+    if ((int64_t)batch * heads * (((seq + 127) / 128 + 1) / 2) >= (int64_t)(INT32_MAX / 2))
+        return S2_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return S2_ERR_INVALID_ARG;
@@ -243,6 +249,7 @@ int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float*
     pp.lse = lse;
     pp.batch = batch;
     pp.heads = heads;
+    pp.heads_kv = heads_kv;
     pp.seq = seq;
     pp.nb = num_blocks;
     pp.nqt = (seq + 127) / 128;
@@ -255,6 +262,15 @@ int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float*
     if (head_dim == 128 && block_size == 64) return launch_prefill<128, 64>(q, k, v, pp, dev, 1, st);
     if (head_dim == 64 && block_size == 128) return launch_prefill<64, 128>(q, k, v, pp, dev, 2, st);
     return launch_prefill<64, 64>(q, k, v, pp, dev, 3, st);
+}
+
+int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int32_t batch, int32_t heads, int32_t seq, int32_t head_dim, float scale,
+                    int32_t block_size, int32_t num_blocks, const int32_t* row_ptr,
+                    const int32_t* col_idx, int64_t nnz, void* stream)
+{
+    return s2_attn_prefill_gqa(q, k, v, o, lse, batch, heads, heads, seq, head_dim, scale,
+                               block_size, num_blocks, row_ptr, col_idx, nnz, stream);
 }
 
 int32_t s2_attn_decode_auto_splits(int32_t batch, int32_t heads)
@@ -276,13 +292,13 @@ size_t s2_attn_decode_workspace_size(int32_t batch, int32_t heads, int32_t head_
     return ws_bytes(batch, heads, head_dim, sp);
 }
 
-int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
-                   const int32_t* block_table, const int32_t* ctx_lens, int32_t batch,
-                   int32_t heads, int32_t head_dim, int32_t page_size, int32_t max_pages,
-                   int64_t num_pages, int32_t block_size, int32_t num_blocks,
-                   const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz, float scale,
-                   void* out, float* lse, void* workspace, size_t workspace_bytes,
-                   int32_t num_splits, void* stream)
+int s2_attn_decode_gqa(const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_table, const int32_t* ctx_lens, int32_t batch,
+                       int32_t heads, int32_t heads_kv, int32_t head_dim, int32_t page_size,
+                       int32_t max_pages, int64_t num_pages, int32_t block_size,
+                       int32_t num_blocks, const int32_t* row_ptr, const int32_t* col_idx,
+                       int64_t nnz, float scale, void* out, float* lse, void* workspace,
+                       size_t workspace_bytes, int32_t num_splits, void* stream)
 {
     if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !row_ptr ||
         (!col_idx && nnz > 0) || !out)
@@ -290,11 +306,12 @@ int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
     if (batch < 1 || heads < 1 || max_pages < 1 || num_pages < 1 || num_blocks < 1 || nnz < 0 ||
         !std::isfinite(scale) || num_splits > kMaxSplits)
         return S2_ERR_INVALID_ARG;
+    if (heads_kv < 1 || heads % heads_kv != 0) return S2_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
     if (page_size != s2::kPage) return S2_ERR_UNSUPPORTED;
     if (block_size < page_size || block_size % page_size != 0) return S2_ERR_UNSUPPORTED;
     if (batch > 65535 || heads > 65535) return S2_ERR_UNSUPPORTED;
-    if (num_pages * heads * page_size * head_dim >= (int64_t)1 << 62) return S2_ERR_INVALID_ARG;
+    if (num_pages * heads_kv * page_size * head_dim >= (int64_t)1 << 62) return S2_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return S2_ERR_INVALID_ARG;
@@ -321,6 +338,7 @@ int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
     dp.num_pages = num_pages;
     dp.batch = batch;
     dp.heads = heads;
+    dp.heads_kv = heads_kv;
     dp.max_pages = max_pages;
     dp.block_size = block_size;
     dp.nb = num_blocks;
@@ -335,6 +353,20 @@ int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
     dp.gflags = g_dev[dev].flags;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return head_dim == 128 ? launch_decode<128>(dp, dev, st) : launch_decode<64>(dp, dev, st);
+}
+
+int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* block_table, const int32_t* ctx_lens, int32_t batch,
+                   int32_t heads, int32_t head_dim, int32_t page_size, int32_t max_pages,
+                   int64_t num_pages, int32_t block_size, int32_t num_blocks,
+                   const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz, float scale,
+                   void* out, float* lse, void* workspace, size_t workspace_bytes,
+                   int32_t num_splits, void* stream)
+{
+    return s2_attn_decode_gqa(q, k_cache, v_cache, block_table, ctx_lens, batch, heads, heads,
+                              head_dim, page_size, max_pages, num_pages, block_size, num_blocks,
+                              row_ptr, col_idx, nnz, scale, out, lse, workspace, workspace_bytes,
+                              num_splits, stream);
 }
 
 }  // extern "C"

@@ -16,7 +16,7 @@ struct PrefillParams {
     int64_t nnz;
     uint16_t* o;  // bf16 bits
     float* lse;   // may be null
-    int32_t batch, heads, seq, nb, nqt;
+    int32_t batch, heads, heads_kv, seq, nb, nqt;  // query head h reads K/V head h / (heads / heads_kv)
     float scale_log2;  // scale * log2(e)
     uint64_t timeout_ns;
     uint32_t* gflags;

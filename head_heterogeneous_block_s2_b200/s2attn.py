@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "S2_OK", 1: "S2_ERR_INVALID_ARG", 2: "S2_ERR_UNSUPPORTED", 3:
                 4: "S2_ERR_CUDA", 5: "S2_ERR_TIMEOUT", 6: "S2_ERR_DEVICE_INDEX"}
 
 EXPORTED = ("s2_status_string", "s2_build_layout", "s2_build_layout_ranges",
-            "s2_build_layout_mask", "s2_attn_prefill",
+            "s2_build_layout_mask", "s2_attn_prefill", "s2_attn_prefill_gqa", "s2_attn_decode_gqa",
             "s2_attn_decode_workspace_size", "s2_attn_decode_auto_splits", "s2_attn_decode",
             "s2_device_status", "s2_set_wait_timeout_ns", "s2_version", "s2_attn_decode_noalloc")
 
@@ -76,6 +76,12 @@ def load(path: str = LIB_PATH):
     lib.s2_attn_prefill.restype = ctypes.c_int
     lib.s2_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp, vp,
                                     i64, vp]
+    lib.s2_attn_prefill_gqa.restype = ctypes.c_int
+    lib.s2_attn_prefill_gqa.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, i32,
+                                        vp, vp, i64, vp]
+    lib.s2_attn_decode_gqa.restype = ctypes.c_int
+    lib.s2_attn_decode_gqa.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i32,
+                                       i32, vp, vp, i64, f32, vp, vp, vp, sz, i32, vp]
     lib.s2_attn_decode_workspace_size.restype = sz
     lib.s2_attn_decode_workspace_size.argtypes = [i32, i32, i32, i32]
     lib.s2_attn_decode_auto_splits.restype = i32
@@ -258,12 +264,15 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: Layout,
             lse: Optional[torch.Tensor] = None, want_lse: bool = False):
     """s2_attn_prefill on [batch, heads, seq, head_dim] bf16 CUDA tensors.
 
+    k and v may have fewer heads (grouped K/V heads, s2_attn_prefill_gqa):
+    [batch, heads_kv, seq, head_dim] with heads_kv dividing heads.
     Returns out, or (out, lse) when ``want_lse`` or ``lse`` is given."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n)
     batch, heads, seq, hd = q.shape
-    if k.shape != q.shape or v.shape != q.shape:
-        raise ValueError("q, k, v shapes differ")
+    hkv = k.shape[1]
+    if k.shape != (batch, hkv, seq, hd) or v.shape != k.shape or heads % hkv:
+        raise ValueError("k, v must be [batch, heads_kv, seq, head_dim] with heads_kv | heads")
     if layout.heads != heads:
         raise ValueError(f"layout has {layout.heads} heads, q has {heads}")
     if layout.d_row_ptr is None:
@@ -276,11 +285,18 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: Layout,
     if lse is not None:
         _need(lse, "lse", torch.float32)
     sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
-    rc = load().s2_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), batch, heads, seq,
-                                hd, sc, layout.block_size, layout.num_blocks,
-                                _ptr(layout.d_row_ptr), _ptr(layout.d_col_idx), layout.nnz,
-                                _stream(q.device))
-    _check(rc, "s2_attn_prefill")
+    if hkv == heads:
+        rc = load().s2_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), batch, heads,
+                                    seq, hd, sc, layout.block_size, layout.num_blocks,
+                                    _ptr(layout.d_row_ptr), _ptr(layout.d_col_idx), layout.nnz,
+                                    _stream(q.device))
+        _check(rc, "s2_attn_prefill")
+    else:
+        rc = load().s2_attn_prefill_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), batch,
+                                        heads, hkv, seq, hd, sc, layout.block_size,
+                                        layout.num_blocks, _ptr(layout.d_row_ptr),
+                                        _ptr(layout.d_col_idx), layout.nnz, _stream(q.device))
+        _check(rc, "s2_attn_prefill_gqa")
     return (out, lse) if lse is not None else out
 
 
@@ -297,7 +313,8 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
            scale: Optional[float] = None, num_splits: int = 0,
            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
            want_lse: bool = False, workspace: Optional[torch.Tensor] = None):
-    """s2_attn_decode: q [batch, heads, D]; caches [pages, heads, 16, D];
+    """s2_attn_decode: q [batch, heads, D]; caches [pages, heads_kv, 16, D]
+    (heads_kv dividing heads; fewer heads = s2_attn_decode_gqa);
     block_table int32 [batch, max_pages]; ctx_lens int32 [batch] (all CUDA)."""
     for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
         _need(t, n)
@@ -305,7 +322,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     _need(ctx_lens, "ctx_lens", torch.int32)
     batch, heads, hd = q.shape
     num_pages, h2, page_size, hd2 = k_cache.shape
-    if h2 != heads or hd2 != hd or v_cache.shape != k_cache.shape:
+    if heads % h2 or hd2 != hd or v_cache.shape != k_cache.shape:
         raise ValueError("cache shape does not match q")
     if layout.heads != heads:
         raise ValueError(f"layout has {layout.heads} heads, q has {heads}")
@@ -323,13 +340,23 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
-    rc = load().s2_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
-                               _ptr(ctx_lens), batch, heads, hd, page_size, block_table.shape[1],
-                               num_pages, layout.block_size, layout.num_blocks,
-                               _ptr(layout.d_row_ptr), _ptr(layout.d_col_idx), layout.nnz, sc,
-                               _ptr(out), _ptr(lse), _ptr(workspace), ws_len, num_splits,
-                               _stream(q.device))
-    _check(rc, "s2_attn_decode")
+    if h2 == heads:
+        rc = load().s2_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                   _ptr(ctx_lens), batch, heads, hd, page_size, block_table.shape[1],
+                                   num_pages, layout.block_size, layout.num_blocks,
+                                   _ptr(layout.d_row_ptr), _ptr(layout.d_col_idx), layout.nnz, sc,
+                                   _ptr(out), _ptr(lse), _ptr(workspace), ws_len, num_splits,
+                                   _stream(q.device))
+        _check(rc, "s2_attn_decode")
+    else:
+        rc = load().s2_attn_decode_gqa(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                       _ptr(ctx_lens), batch, heads, h2, hd, page_size,
+                                       block_table.shape[1], num_pages, layout.block_size,
+                                       layout.num_blocks, _ptr(layout.d_row_ptr),
+                                       _ptr(layout.d_col_idx), layout.nnz, sc, _ptr(out),
+                                       _ptr(lse), _ptr(workspace), ws_len, num_splits,
+                                       _stream(q.device))
+        _check(rc, "s2_attn_decode_gqa")
     return (out, lse) if lse is not None else out
 
 

@@ -157,8 +157,9 @@ int s2_build_layout_mask(int32_t num_heads, int32_t num_blocks, const uint8_t* b
  *   o         device bf16 [batch][heads][seq][head_dim] (written).
  *   lse       device fp32 [batch][heads][seq] or NULL: natural-log
  *             log-sum-exp of the scaled visible logits of each row (written).
- *   head_dim  64 or 128.  block_size 64 or 128.  seq % block_size == 0.
- *   num_blocks == seq / block_size.
+ *   head_dim  64 or 128.  block_size 64 or 128.  Any seq >= 1: the last
+ *             block may be partial (its missing keys are never visible).
+ *   num_blocks == ceil(seq / block_size).
  *   row_ptr, col_idx, nnz: a layout from one of the s2_build_layout*
  *             builders for (heads, num_blocks), copied to device memory
  *             (read). Lists must be strictly ascending with j <= i; nnz may be
@@ -174,6 +175,20 @@ int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float*
                     float scale, int32_t block_size, int32_t num_blocks,
                     const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz,
                     void* stream);
+
+/*
+ * s2_attn_prefill with grouped key/value heads (GQA/MQA; the pages do not
+ * mention it): k and v are [batch][heads_kv][seq][head_dim], heads_kv divides
+ * heads, and query head h reads key/value head h / (heads / heads_kv). The
+ * layout (rows per query head) is applied per query head, so heads of one
+ * group may visit different key blocks. heads_kv == heads is s2_attn_prefill.
+ * S2_ERR_INVALID_ARG when heads_kv < 1 or does not divide heads.
+ */
+int s2_attn_prefill_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int32_t batch, int32_t heads, int32_t heads_kv, int32_t seq,
+                        int32_t head_dim, float scale, int32_t block_size, int32_t num_blocks,
+                        const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz,
+                        void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Decode: one query token per sequence over a paged KV cache               */
@@ -220,6 +235,22 @@ int s2_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                    int64_t nnz, float scale, void* out, float* lse,
                    void* workspace, size_t workspace_bytes, int32_t num_splits,
                    void* stream);
+
+/*
+ * s2_attn_decode with grouped key/value heads: the caches are
+ * [num_pages][heads_kv][page_size][head_dim] and query head h reads key/value
+ * head h / (heads / heads_kv) (heads_kv divides heads; S2_ERR_INVALID_ARG
+ * otherwise). Each query head walks its own layout row, so one group's heads
+ * may read different pages. heads_kv == heads is s2_attn_decode.
+ */
+int s2_attn_decode_gqa(const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_table, const int32_t* ctx_lens,
+                       int32_t batch, int32_t heads, int32_t heads_kv, int32_t head_dim,
+                       int32_t page_size, int32_t max_pages, int64_t num_pages,
+                       int32_t block_size, int32_t num_blocks, const int32_t* row_ptr,
+                       const int32_t* col_idx, int64_t nnz, float scale, void* out,
+                       float* lse, void* workspace, size_t workspace_bytes,
+                       int32_t num_splits, void* stream);
 
 /*
  * Decode that allocates nothing: s2_attn_decode with the split partials kept

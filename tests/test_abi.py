@@ -53,7 +53,7 @@ def _prefill(**over):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(q=None), 1), (dict(row_ptr=None), 1), (dict(batch=0), 1), (dict(seq=500), 1),
+    (dict(q=None), 1), (dict(row_ptr=None), 1), (dict(batch=0), 1), (dict(seq=600), 1),
     (dict(nb=7), 1), (dict(hd=96), 2), (dict(bs=32), 2), (dict(q=(1 << 20) + 8), 1),
     (dict(scale=float("nan")), 1), (dict(nnz=-1), 1), (dict(col_idx=None), 1),
 ])
@@ -91,3 +91,15 @@ def test_decode_workspace_size():
     auto = s2attn.decode_auto_splits(4, 8)
     assert 1 <= auto <= 16
     assert s2attn.decode_workspace_size(4, 8, 128, 0) == s2attn.decode_workspace_size(4, 8, 128, auto)
+
+
+def test_grouped_head_entry_points_reject_bad_head_counts():
+    lib = s2attn.load()
+    vp = ctypes.c_void_p
+    m = vp(1 << 20)
+    # 4 query heads over 3 K/V heads; 0 K/V heads
+    for hkv in (3, 0):
+        assert lib.s2_attn_prefill_gqa(m, m, m, m, None, 1, 4, hkv, 512, 64, 0.125, 64, 8, m, m,
+                                       60, None) == 1
+        assert lib.s2_attn_decode_gqa(m, m, m, m, m, 2, 4, hkv, 128, 16, 8, 16, 128, 1, m, m, 4,
+                                      0.1, m, None, None, 0, 1, None) == 1
