@@ -54,6 +54,9 @@ def _load():
     lib.s2o_decode_items.restype = i32
     lib.s2o_decode_items.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
                                      i64, vp, dbl, i64, vp, vp, vp, i32]
+    lib.s2o_backward.restype = i32
+    lib.s2o_backward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, vp, i64,
+                                 vp, dbl, vp, vp, vp, i32]
     lib.s2o_range_block_active.restype = i32
     lib.s2o_range_block_active.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp]
     lib.s2o_range_block_mask.restype = None
@@ -247,3 +250,31 @@ def decode_mask(q, k_cache, v_cache, block_table, ctx_lens, B, bmask, scale, ite
     if rc != 0:
         raise ValueError("oracle decode_mask rejected its arguments")
     return out, lse
+
+
+def backward(q, k, v, dout, B, scale, S=None, L=None, dense_heads=None, bmask=None, nthreads=0):
+    """Oracle gradients (dq, dk, dv) in fp64 of the masked softmax attention.
+
+    q, dout: [batch, H, seq, D]; k, v: [batch, Hkv, seq, D] (bf16). The block
+    rule is HHST (S, L, dense_heads) unless ``bmask`` [H, nbm, nbm] is given.
+    Returns dq [batch, H, seq, D], dk and dv [batch, Hkv, seq, D].
+    """
+    q, k, v, do = _bits(q), _bits(k), _bits(v), _bits(dout)
+    batch, H, seq, D = q.shape
+    Hkv = k.shape[1]
+    assert k.shape == (batch, Hkv, seq, D) and v.shape == k.shape and do.shape == q.shape
+    if bmask is not None:
+        bm = np.ascontiguousarray(np.asarray(bmask, dtype=np.uint8))
+        assert bm.ndim == 3 and bm.shape[0] == H and bm.shape[1] == bm.shape[2]
+        nbm, S_, L_, d = bm.shape[1], 0, 0, None
+    else:
+        bm, nbm, S_, L_, d = None, 0, int(S), int(L), _dense(H, dense_heads)
+    dq = np.empty((batch, H, seq, D), dtype=np.float64)
+    dk = np.empty((batch, Hkv, seq, D), dtype=np.float64)
+    dv = np.empty_like(dk)
+    rc = _load().s2o_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), batch, H, Hkv, seq, D, B, S_,
+                              L_, _ptr(d), nbm, _ptr(bm), float(scale), _ptr(dq), _ptr(dk),
+                              _ptr(dv), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle backward rejected its arguments")
+    return dq, dk, dv

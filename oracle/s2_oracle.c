@@ -44,6 +44,20 @@
  * zero output row and LSE = -inf: the softmax over an empty set is undefined,
  * and zero is the value whose weight in any later merge is nil.
  *
+ * Backward. The arXiv abstract reports training speedups, so the gradients of
+ * the same definition are part of the method. With an upstream gradient dO,
+ * P[q,k] = exp(s_qk - LSE_q) over the visible keys of row q, and
+ *
+ *     dV[k]  = sum_q P[q,k] dO[q]
+ *     dP[q,k] = dO[q] . V[k]
+ *     Dq     = sum_k P[q,k] dP[q,k]
+ *     dS[q,k] = P[q,k] (dP[q,k] - Dq)
+ *     dQ[q]  = scale * sum_k dS[q,k] K[k]
+ *     dK[k]  = scale * sum_q dS[q,k] Q[q]
+ *
+ * (the chain rule through the softmax and the scaled dot products; with
+ * grouped K/V heads, dK and dV of a K/V head sum over its query heads).
+ *
  * Every loop visits keys in ascending order; nothing is blocked, fused or
  * reordered beyond the definition.
  */
@@ -122,8 +136,9 @@ void s2o_range_block_mask(int64_t H, int64_t nb, const int64_t* range_ptr, const
 /* ------------------------------------------------------------------------- */
 
 typedef struct {
-    int kind; /* 0 = prefill rows, 1 = decode items */
-    const uint16_t *q, *k, *v;
+    int kind; /* 0 = prefill rows, 1 = decode items, 2 = backward planes */
+    const uint16_t *q, *k, *v, *dout;
+    double *dq, *dk, *dv; /* backward outputs */
     const int32_t *block_table, *ctx_lens;
     int64_t batch, H, seq, D, B, S, L, page_size, max_pages;
     const uint8_t* dense;
@@ -243,25 +258,97 @@ static int decode_item(const job_t* J, int64_t e, double* s, double* qd,
     return 0;
 }
 
+/* Backward item e = b * Hkv + g: every query head h of K/V head g (h / (H / Hkv)
+ * == g) and every row of batch entry b. dQ rows of those heads and the dK, dV
+ * rows of plane e are written by this item alone. */
+static void backward_plane(const job_t* J, int64_t e, double* s, double* p, double* qd,
+                           double* dod)
+{
+    const int64_t D = J->D, seq = J->seq, H = J->H, Hkv = J->Hkv, grp = H / Hkv;
+    const int64_t b = e / Hkv, g = e % Hkv;
+    const uint16_t* K = J->k + e * seq * D;
+    const uint16_t* V = J->v + e * seq * D;
+    double* dK = J->dk + e * seq * D;
+    double* dV = J->dv + e * seq * D;
+    for (int64_t t = 0; t < seq * D; ++t) dK[t] = dV[t] = 0.0;
+    for (int64_t h = g * grp; h < (g + 1) * grp; ++h) {
+        const int dense = J->dense ? J->dense[h] != 0 : 0;
+        const int64_t plane = b * H + h;
+        for (int64_t q = 0; q < seq; ++q) {
+            const int64_t i = q / J->B;
+            const uint16_t* Q = J->q + (plane * seq + q) * D;
+            const uint16_t* dO = J->dout + (plane * seq + q) * D;
+            double* dQ = J->dq + (plane * seq + q) * D;
+            for (int64_t d = 0; d < D; ++d) {
+                qd[d] = bf16_bits_to_double(Q[d]);
+                dod[d] = bf16_bits_to_double(dO[d]);
+                dQ[d] = 0.0;
+            }
+            /* forward softmax of row q */
+            double m = -INFINITY;
+            for (int64_t k = 0; k <= q; ++k) {
+                if (!visible(J, h, i, k / J->B, dense)) continue;
+                double dot = 0.0;
+                for (int64_t d = 0; d < D; ++d) dot += qd[d] * bf16_bits_to_double(K[k * D + d]);
+                s[k] = J->scale * dot;
+                if (s[k] > m) m = s[k];
+            }
+            if (m == -INFINITY) continue; /* no visible key: no gradient */
+            double den = 0.0;
+            for (int64_t k = 0; k <= q; ++k)
+                if (visible(J, h, i, k / J->B, dense)) den += exp(s[k] - m);
+            const double lse = m + log(den);
+            /* P, dP and Dq */
+            double Dq = 0.0;
+            for (int64_t k = 0; k <= q; ++k) {
+                if (!visible(J, h, i, k / J->B, dense)) continue;
+                const double pk = exp(s[k] - lse);
+                double dpk = 0.0;
+                for (int64_t d = 0; d < D; ++d) dpk += dod[d] * bf16_bits_to_double(V[k * D + d]);
+                p[k] = pk;
+                s[k] = dpk; /* s now holds dP */
+                Dq += pk * dpk;
+            }
+            /* dS, then the three products */
+            for (int64_t k = 0; k <= q; ++k) {
+                if (!visible(J, h, i, k / J->B, dense)) continue;
+                const double ds = p[k] * (s[k] - Dq);
+                for (int64_t d = 0; d < D; ++d) {
+                    dV[k * D + d] += p[k] * dod[d];
+                    dQ[d] += J->scale * ds * bf16_bits_to_double(K[k * D + d]);
+                    dK[k * D + d] += J->scale * ds * qd[d];
+                }
+            }
+        }
+    }
+}
+
 static void* worker(void* arg)
 {
     job_t* J = (job_t*)arg;
-    const int64_t span = J->kind == 0 ? J->seq
-                                      : J->max_pages * J->page_size;
+    const int64_t span = J->kind == 1 ? J->max_pages * J->page_size : J->seq;
     double* s = (double*)malloc(sizeof(double) * (size_t)(span > 0 ? span : 1));
+    double* p = (double*)malloc(sizeof(double) * (size_t)(span > 0 ? span : 1));
     double* qd = (double*)malloc(sizeof(double) * (size_t)J->D);
-    if (!s || !qd) {
+    double* dod = (double*)malloc(sizeof(double) * (size_t)J->D);
+    if (!s || !p || !qd || !dod) {
         pthread_mutex_lock(&J->lock);
         J->failed = 1;
         pthread_mutex_unlock(&J->lock);
         free(s);
+        free(p);
         free(qd);
+        free(dod);
         return NULL;
     }
     for (;;) {
         const int64_t t = take(J);
         if (t >= J->n_items) break;
         const int64_t id = J->items ? J->items[t] : t;
+        if (J->kind == 2) {
+            backward_plane(J, id, s, p, qd, dod);
+            continue;
+        }
         double* out = J->out + t * J->D;
         double* lse = J->lse + t;
         if (J->kind == 0) {
@@ -273,7 +360,9 @@ static void* worker(void* arg)
         }
     }
     free(s);
+    free(p);
     free(qd);
+    free(dod);
     return NULL;
 }
 
@@ -423,5 +512,31 @@ int s2o_decode_items_mask(const uint16_t* q, const uint16_t* k_cache, const uint
     J.batch = batch; J.H = H; J.Hkv = Hkv; J.D = D; J.page_size = page_size;
     J.max_pages = max_pages; J.B = B; J.bmask = bmask; J.nbm = nbm; J.scale = scale;
     J.n_items = n_items; J.items = items; J.out = out; J.lse = lse;
+    return run_job(&J, nthreads);
+}
+
+/* Backward oracle (the gradients in the header) under the HHST rule
+ * (bmask == NULL; S, L, dense as s2o_prefill_rows) or a block mask
+ * [H][nbm][nbm] (nbm >= ceil(seq / B)). q, dout: [batch][H][seq][D];
+ * k, v: [batch][Hkv][seq][D]. dq: [batch][H][seq][D]; dk, dv:
+ * [batch][Hkv][seq][D], fp64. The softmax is recomputed here in fp64 (no
+ * saved statistics are taken from the caller). Returns 0 or -1. */
+int s2o_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                 int64_t batch, int64_t H, int64_t Hkv, int64_t seq, int64_t D, int64_t B,
+                 int64_t S, int64_t L, const uint8_t* dense, int64_t nbm, const uint8_t* bmask,
+                 double scale, double* dq, double* dk, double* dv, int nthreads)
+{
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || batch < 1 || H < 1 || Hkv < 1 ||
+        H % Hkv != 0 || seq < 1 || D < 1 || B < 1)
+        return -1;
+    if (bmask ? nbm < (seq + B - 1) / B : (S < 1 || L < 1)) return -1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.kind = 2;
+    J.q = q; J.k = k; J.v = v; J.dout = dout;
+    J.dq = dq; J.dk = dk; J.dv = dv;
+    J.batch = batch; J.H = H; J.Hkv = Hkv; J.seq = seq; J.D = D; J.B = B;
+    J.S = S; J.L = L; J.dense = dense; J.bmask = bmask; J.nbm = nbm; J.scale = scale;
+    J.n_items = batch * Hkv; J.items = NULL;
     return run_job(&J, nthreads);
 }
