@@ -309,15 +309,56 @@ def run_ours(args, rank, world, dist):
         e2e_dec_ms = sum(e[1].elapsed_time(e[2]) for e in eevs) if wd else 0.0
         assert torch.equal(hout, out.cpu()), "e2e output differs from the device output"
 
+    # ---------------- backward (dQ, dK, dV) of a prefill workload, timed on its own
+    bwd_ms, bwd_steps, bwd_info = 0.0, 0, None
+    if args.backward != "none":
+        wb = wp if args.backward == "same" else synth.PREFILL_WORKLOADS[args.backward]
+        if wb is wp:
+            bq, bk_, bv, lay_b = q, k, v, lay_p
+        else:
+            bq, bk_, bv = synth.prefill_inputs(wb, device=dev)
+            lay_b = s2attn.build_layout(wb.heads, wb.block, wb.stride, wb.local, wb.num_blocks,
+                                        wb.dense_heads, device=dev)
+        lay_b.transposed(dev)
+        bo, blse = s2attn.prefill(bq, bk_, bv, lay_b, scale=wb.scale, want_lse=True)
+        gen = torch.Generator(device=dev).manual_seed(77)
+        bdo = torch.randn(bq.shape, generator=gen, device=dev).to(torch.bfloat16)
+        bdq, bdk, bdv = torch.empty_like(bq), torch.empty_like(bk_), torch.empty_like(bv)
+        bws = torch.empty(s2attn.backward_workspace_size(wb.batch, wb.heads, wb.seq),
+                          dtype=torch.uint8, device=dev)
+
+        def bwd():
+            s2attn.backward(bq, bk_, bv, bo, blse, bdo, lay_b, scale=wb.scale, dq=bdq, dk=bdk,
+                            dv=bdv, workspace=bws)
+
+        for _ in range(3):
+            bwd()
+        torch.cuda.synchronize()
+        bwd_steps = max(3, min(args.steps, args.bwd_steps))
+        bev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        if dist:
+            dist.barrier()
+        bev[0].record(stream)
+        for _ in range(bwd_steps):
+            bwd()
+        bev[1].record(stream)
+        torch.cuda.synchronize()
+        bwd_ms = bev[0].elapsed_time(bev[1])
+        rc, flags = s2attn.device_status(reset=True)
+        if rc != 0:
+            raise RuntimeError(f"device flags {flags:#x} after the backward")
+        bflops = prefill_flops(lay_b, wb)
+        bwd_info = (wb, bflops, prefill_issued_flops(lay_b, wb))
+
     # ---------------- max over ranks
-    vals = [total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms]
+    vals = [total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms]
     if dist:
         import torch.distributed as tdist
 
         t = torch.tensor(vals, dtype=torch.float64, device=dev)
         tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
         vals = t.tolist()
-    total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms = vals
+    total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms = vals
     clocks = sampler.summary()
     if rank != 0:
         return None
@@ -400,6 +441,27 @@ def run_ours(args, rank, world, dist):
                 "value": round(world * kv_bytes * e2e_steps / (e2e_dec_ms * 1e-3) / 1e9, 1),
                 "unit": "GB/s"},
         }
+    if bwd_info is not None:
+        wb, bflops, bissued = bwd_info
+        # dS needs S (recomputed), dP, and then dV, dK, dQ: 5 products of the
+        # forward's 2, so 2.5x its FLOPs; S and dP are computed by both backward
+        # kernels here, so 7 products are issued.
+        alg = 2.5 * bflops
+        per = alg / (bwd_ms / bwd_steps * 1e-3) / 1e12
+        line["backward"] = {
+            "value": round(world * alg * bwd_steps / (bwd_ms * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s",
+            "workload": wb.name,
+            "ms_per_call": round(bwd_ms / bwd_steps, 4),
+            "steps": bwd_steps,
+            "algorithmic_gflop_per_call": round(alg / 1e9, 3),
+            "issued_gflop_per_call": round(3.5 * bissued / 1e9, 3),
+            "kernels": "s2_bwd_stats_kernel + s2_bwd_dq_kernel + s2_bwd_dkv_kernel",
+            "roofline": {"bound": "tensor", "achieved": round(per, 2), "peak": tc_peak,
+                         "unit": "TFLOP/s", "frac": round(per / tc_peak, 4),
+                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
+        }
+        line["gpu_launches_backward"] = 3 * bwd_steps
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wp, args.cpu_seconds)
     return line
@@ -494,6 +556,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", default="same",
+                    help="prefill workload whose backward is timed separately ('same' = the "
+                         "prefill workload, 'none' = skip)")
+    ap.add_argument("--bwd-steps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

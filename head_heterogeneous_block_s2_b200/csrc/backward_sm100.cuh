@@ -1,0 +1,661 @@
+// backward_sm100.cuh -- block-sparse backward (dQ, dK, dV) of the HHST
+// attention on sm_100a.
+//
+// The arXiv abstract of "S2-Attention: Hardware-aware context sharding among
+// attention heads" reports training speedups over FlashAttention-2, so the
+// gradients run on the same compacted block lists as the forward. With the
+// forward's LSE and an upstream gradient dO, per visible (q, k):
+//
+//   P = exp(s - LSE_q),  dP = dO_q . V_k,  D_q = dO_q . O_q,  dS = P (dP - D_q)
+//   dQ_q = scale sum_k dS K_k,  dK_k = scale sum_q dS Q_q,  dV_k = sum_q P dO_q
+//
+// (D_q = sum_k P dP because O_q = sum_k P V_k.) Three kernels:
+//
+//   s2_bwd_stats_kernel  per query row: (LSE * log2 e, D_q) into a row-padded
+//                        fp32 workspace; rows past seq get (+inf, 0) so that
+//                        any P computed for them is exactly 0.
+//   s2_bwd_dq_kernel     one 128-row query tile per CTA, walking the union of
+//                        its query blocks' key-block lists (the forward's
+//                        lists): S = Q K^T and dP = dO V^T into TMEM, dS
+//                        (bf16) written back over S, dQ += dS K with dS read
+//                        from TMEM and K from shared memory as an MN-major B.
+//   s2_bwd_dkv_kernel    one 128-row key tile per CTA, walking the union of
+//                        its key blocks' transposed lists (query blocks that
+//                        list them): S^T = K Q^T and dP^T = V dO^T into TMEM,
+//                        P^T and dS^T (bf16) written back over them, then
+//                        dV += P^T dO and dK += dS^T Q with the A operands
+//                        read from TMEM.
+// dQ and dK/dV are computed by separate kernels (S and dP are recomputed by
+// both) so that no accumulator is shared between CTAs: no atomics, and the
+// results are deterministic.
+//
+// CTA = 8 warps: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer (one
+// thread), warp 2 builds the union list in shared memory before the main
+// loop, warps 4..7 the element-wise pass (thread = one tile row = one TMEM
+// lane) and the epilogue; warp 3 idles. With B = 64 a 128-row tile holds two
+// blocks and every row masks by its own block's tag. Every wait is bounded;
+// on a timeout the CTA drains its own copies and MMAs, frees TMEM and exits
+// with the device timeout flag set.
+#pragma once
+
+#include <climits>
+#include <cstdint>
+#include <cuda.h>
+
+#include "lists.cuh"
+#include "ptx.cuh"
+#include "umma.cuh"
+
+namespace s2 {
+
+struct BackwardParams {
+    const int32_t* row_ptr;  // key-block lists of query blocks (the forward's layout)
+    const int32_t* col_idx;
+    const int32_t* col_ptr;  // query-block lists of key blocks (its transpose)
+    const int32_t* row_idx;
+    int64_t nnz;
+    const uint16_t* o;     // [batch][heads][seq][HD] forward output (stats kernel)
+    const uint16_t* dout;  // [batch][heads][seq][HD] upstream gradient (stats kernel)
+    const float* lse;      // [batch][heads][seq] forward LSE, natural log (stats kernel)
+    float2* stats;         // [batch * heads][seq_pad]: (LSE * log2 e, D)
+    uint16_t* dq;          // [batch][heads][seq][HD]
+    uint16_t* dk;          // [batch][heads][seq][HD]
+    uint16_t* dv;
+    int32_t batch, heads, seq, seq_pad, nb, ntiles;
+    float scale;       // logit scale
+    float scale_log2;  // scale * log2 e
+    uint64_t timeout_ns;
+    uint32_t* gflags;
+};
+
+// Descriptor offset (16-byte units) of k-step kk (16 elements) of a K-major
+// SWIZZLE_128B operand of `rows` rows stored as 64-column panels.
+__device__ __forceinline__ uint64_t kstep(int kk, int rows)
+{
+    return (uint64_t)((((kk >> 2) * (rows * 128)) + (kk & 3) * 32) >> 4);
+}
+
+// ------------------------------------------------------------------ stats
+
+// One group of HD/8 threads per row (8 bf16 of dO and O per thread); the loop
+// runs warp by warp so that every lane of a warp takes part in each shuffle.
+template <int HD>
+__global__ void __launch_bounds__(256) s2_bwd_stats_kernel(const BackwardParams p)
+{
+    constexpr int TPR = HD / 8;
+    constexpr int RPW = 32 / TPR;  // rows per warp
+    const int64_t rows = (int64_t)p.batch * p.heads * p.seq_pad;
+    const int lane = threadIdx.x & 31, sub = lane % TPR;
+    const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t base = warp_id * RPW; base < rows; base += nwarps * RPW) {
+        const int64_t r = base + lane / TPR;
+        const int64_t bh = r / p.seq_pad;
+        const int q = (int)(r % p.seq_pad);
+        float d = 0.f;
+        if (r < rows && q < p.seq) {
+            const int64_t off = (bh * p.seq + q) * HD + sub * 8;
+            const uint4 a = *reinterpret_cast<const uint4*>(p.o + off);
+            const uint4 b = *reinterpret_cast<const uint4*>(p.dout + off);
+            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                d = fmaf(bf16lo(av[i]), bf16lo(bv[i]), fmaf(bf16hi(av[i]), bf16hi(bv[i]), d));
+        }
+#pragma unroll
+        for (int w = TPR / 2; w > 0; w >>= 1) d += __shfl_xor_sync(0xffffffffu, d, w);
+        if (sub == 0 && r < rows)
+            p.stats[r] = q < p.seq ? make_float2(p.lse[bh * p.seq + q] * 1.4426950408889634f, d)
+                                   : make_float2(INFINITY, 0.f);
+    }
+}
+
+// ------------------------------------------------------------------ dQ
+
+template <int HD, int BK>
+struct BwdQCfg {
+    static constexpr int M = 128;
+    static constexpr int ROWS = (BK == 128) ? 1 : 2;  // query blocks per tile
+    static constexpr uint32_t TBYTES = M * HD * 2;    // Q or dO tile
+    static constexpr uint32_t KVBYTES = BK * HD * 2;  // one K or V block
+    static constexpr int ST = 2;
+    static constexpr int LIST_CAP = 2048;
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_DO = TBYTES;
+    static constexpr uint32_t OFF_K = 2 * TBYTES;              // [stage][panel][BK rows x 128 B]
+    static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;
+    static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
+    static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_CAP * 4;
+    // barriers: qd_full, k_full[ST], v_full[ST], kv_empty[ST], s_full, ds_full, acc_done, drain
+    static constexpr int NBAR = 1 + 3 * ST + 4;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
+    static constexpr uint32_t SMEM = OFF_MISC + 32;
+    static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
+    static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_ACC = 2 * BK;
+    static constexpr uint32_t TMEM_COLS = (2 * BK + HD) <= 256 ? 256 : 512;
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
+
+template <int HD, int BK>
+__global__ void __launch_bounds__(256, 1)
+s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const BackwardParams p)
+{
+    using C = BwdQCfg<HD, BK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int BH = p.batch * p.heads;
+    const int qt = p.ntiles - 1 - (int)(blockIdx.x / BH);  // longest lists first
+    const int bh = (int)(blockIdx.x % BH);
+    const int h = bh % p.heads;
+
+    const uint32_t bar_qd = sb + C::OFF_BAR;
+    auto bar_kf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
+    auto bar_vf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + C::ST + s); };
+    auto bar_ke = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + 2 * C::ST + s); };
+    const uint32_t bar_s = sb + C::OFF_BAR + 8u * (1 + 3 * C::ST);
+    const uint32_t bar_ds = bar_s + 8u;
+    const uint32_t bar_acc = bar_s + 16u;
+    const uint32_t bar_dr = bar_s + 24u;
+    uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
+    int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2] list length
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
+    volatile int* abort_cta = misc + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_qd, 1);
+        for (int s = 0; s < C::ST; ++s) {
+            mbar_init(bar_kf(s), 1);
+            mbar_init(bar_vf(s), 1);
+            mbar_init(bar_ke(s), 1);
+        }
+        mbar_init(bar_s, 1);
+        mbar_init(bar_ds, 128);
+        mbar_init(bar_acc, 1);
+        mbar_init(bar_dr, 1);
+        *abort_cta = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 2 && lane == 0) {  // union of the tile's key-block lists
+        UnionWalk<C::ROWS> it;
+        int len = 0;
+        const bool ok = it.init(p.row_ptr, h * (p.nb + 1), qt * C::ROWS, p.nb, p.nnz);
+        if (!ok) atomicOr(p.gflags, kFlagIndex);
+        if (it.any) {
+            for (;;) {
+                int j, bits;
+                bool last, bad;
+                it.next(p.col_idx, j, bits, last, bad);
+                if (bad) atomicOr(p.gflags, kFlagIndex);
+                if (len >= C::LIST_CAP) {  // cannot happen when nb <= LIST_CAP
+                    atomicOr(p.gflags, kFlagIndex);
+                    break;
+                }
+                list[len++] = list_pack(j, bits);
+                if (last) break;
+            }
+        }
+        misc[2] = len;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int len = misc[2];
+    const WaitCtl ctl{p.timeout_ns, p.gflags, abort_cta};
+    constexpr uint64_t kDrainNs = 200000000ull;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && len > 0) {
+            mbar_arrive_expect_tx(bar_qd, 2 * C::TBYTES);
+#pragma unroll
+            for (int pn = 0; pn < HD / 64; ++pn) {
+                tma_load_3d(sb + C::OFF_Q + pn * (C::M * 128), &tmQ, pn * 64, qt * C::M, bh, bar_qd);
+                tma_load_3d(sb + C::OFF_DO + pn * (C::M * 128), &tmDO, pn * 64, qt * C::M, bh, bar_qd);
+            }
+            int n = 0;
+            for (; n < len; ++n) {
+                const int st = n % C::ST;
+                if (!mbar_wait(bar_ke(st), ((n / C::ST) & 1) ^ 1, ctl)) break;
+                const int32_t krow = list_j(list[n]) * BK;
+                mbar_arrive_expect_tx(bar_kf(st), C::KVBYTES);
+#pragma unroll
+                for (int pn = 0; pn < HD / 64; ++pn)
+                    tma_load_3d(sb + C::OFF_K + st * C::KVBYTES + pn * (BK * 128), &tmK, pn * 64, krow,
+                                bh, bar_kf(st));
+                mbar_arrive_expect_tx(bar_vf(st), C::KVBYTES);
+#pragma unroll
+                for (int pn = 0; pn < HD / 64; ++pn)
+                    tma_load_3d(sb + C::OFF_V + st * C::KVBYTES + pn * (BK * 128), &tmV, pn * 64, krow,
+                                bh, bar_vf(st));
+            }
+            if (*abort_cta) {  // let this CTA's own loads land before exit
+                mbar_drain(bar_qd, 0, kDrainNs);
+                for (int m = (n > C::ST ? n - C::ST : 0); m < n; ++m) {
+                    mbar_drain(bar_kf(m % C::ST), (m / C::ST) & 1, kDrainNs);
+                    mbar_drain(bar_vf(m % C::ST), (m / C::ST) & 1, kDrainNs);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && len > 0) {
+            constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S = Q K^T, dP = dO V^T
+            constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);  // dQ += dS K (K as MN-major B)
+            const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
+            const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
+            bool issued = false;
+            if (mbar_wait(bar_qd, 0, ctl)) {
+                for (int n = 0; n < len; ++n) {
+                    const int st = n % C::ST;
+                    const uint32_t par = (n / C::ST) & 1;
+                    if (!mbar_wait(bar_kf(st), par, ctl)) break;
+                    tc_fence_after();
+                    const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_bf16_ss(tmem + C::COL_S, dq_desc + kstep(kk, C::M), dk_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+                    issued = true;
+                    if (!mbar_wait(bar_vf(st), par, ctl)) break;
+                    tc_fence_after();
+                    const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_bf16_ss(tmem + C::COL_DP, ddo_desc + kstep(kk, C::M), dv_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+                    umma_commit(bar_s);
+                    if (!mbar_wait(bar_ds, n & 1, ctl)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t bk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_S + kk * 8, bk, idesc_q,
+                                     (n > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_ke(st));
+                }
+                if (!*abort_cta) umma_commit(bar_acc);
+            }
+            if (*abort_cta && issued) {
+                umma_commit(bar_dr);
+                mbar_drain(bar_dr, 0, kDrainNs);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ element-wise pass + epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const int qpos = qt * C::M + r;
+        const int rowbit = (BK == 128) ? 0 : (r >> 6);
+        const bool row_valid = qpos < p.seq;
+        const float sc = p.scale_log2;
+        float2 stat = make_float2(0.f, 0.f);
+        if (row_valid) stat = p.stats[(int64_t)bh * p.seq_pad + qpos];
+        bool fail = false;
+        for (int n = 0; n < len; ++n) {
+            const uint32_t ent = list[n];
+            if (!warp_wait(bar_s, n & 1, ctl)) {
+                fail = true;
+                break;
+            }
+            tc_fence_after();
+            const bool vis = row_valid && ((list_bits(ent) >> rowbit) & 1);
+            const int lim = qpos - list_j(ent) * BK;  // key column c visible iff c <= lim
+            // 64 columns at a time; dS of chunk ch (bf16 pairs) goes to columns
+            // 32 ch .. 32 ch + 31 of S, which are already read.
+#pragma unroll
+            for (int ch = 0; ch < BK / 64; ++ch) {
+                uint32_t sr[64], dp[64];
+                tmem_ld32(tl + C::COL_S + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(tl + C::COL_S + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_ld32(tl + C::COL_DP + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+                tmem_ld32(tl + C::COL_DP + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const int kc = 64 * ch + c;
+                    const float p0 = (vis && kc <= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -stat.x)) : 0.f;
+                    const float p1 = (vis && kc + 1 <= lim) ? ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -stat.x)) : 0.f;
+                    const float d0 = p0 * (__uint_as_float(dp[c]) - stat.y);
+                    const float d1 = p1 * (__uint_as_float(dp[c + 1]) - stat.y);
+                    sr[c / 2] = pack_bf16x2(d0, d1);  // slot c/2 <= c: already read
+                }
+                tmem_st32(tl + C::COL_S + 32 * ch, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_ds);
+        }
+        if (!fail) {
+            uint16_t* drow = p.dq + ((int64_t)bh * p.seq + qpos) * HD;
+            if (len > 0) {
+                if (warp_wait(bar_acc, 0, ctl)) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tl + C::COL_ACC + 32 * c, o);
+                        tmem_wait_ld();
+                        if (row_valid) {
+#pragma unroll
+                            for (int e2 = 0; e2 < 32; e2 += 8) {
+                                uint4 v;
+                                v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * p.scale, __uint_as_float(o[e2 + 1]) * p.scale);
+                                v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * p.scale, __uint_as_float(o[e2 + 3]) * p.scale);
+                                v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * p.scale, __uint_as_float(o[e2 + 5]) * p.scale);
+                                v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * p.scale, __uint_as_float(o[e2 + 7]) * p.scale);
+                                *reinterpret_cast<uint4*>(drow + 32 * c + e2) = v;
+                            }
+                        }
+                    }
+                }
+            } else if (row_valid) {  // no key block listed for this tile
+                for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(drow + d) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ dK, dV
+
+template <int HD, int BK>
+struct BwdKVCfg {
+    static constexpr int M = 128;
+    static constexpr int ROWS = (BK == 128) ? 1 : 2;   // key blocks per tile
+    static constexpr uint32_t TBYTES = M * HD * 2;     // K or V tile
+    static constexpr uint32_t QBYTES = BK * HD * 2;    // one query block of Q or dO
+    static constexpr uint32_t STATBYTES = BK * 8;      // (L2, D) per query
+    static constexpr int ST = 2;
+    static constexpr int LIST_CAP = 2048;
+    static constexpr uint32_t OFF_K = 0;
+    static constexpr uint32_t OFF_V = TBYTES;
+    static constexpr uint32_t OFF_Q = 2 * TBYTES;              // [stage][panel][BK rows x 128 B]
+    static constexpr uint32_t OFF_DO = OFF_Q + ST * QBYTES;
+    static constexpr uint32_t OFF_STAT = OFF_DO + ST * QBYTES;
+    static constexpr uint32_t OFF_LIST = OFF_STAT + ST * STATBYTES;
+    static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_CAP * 4;
+    // barriers: kv_full, q_full[ST], q_empty[ST], s_full, p_full, acc_done, drain
+    static constexpr int NBAR = 1 + 2 * ST + 4;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
+    static constexpr uint32_t SMEM = OFF_MISC + 32;
+    static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
+    static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_DV = 2 * BK, COL_DK = 2 * BK + HD;
+    static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD) <= 256 ? 256 : 512;
+    static_assert(2 * BK + 2 * HD <= 512, "TMEM budget");
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
+
+template <int HD, int BK>
+__global__ void __launch_bounds__(256, 1)
+s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const BackwardParams p)
+{
+    using C = BwdKVCfg<HD, BK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int BH = p.batch * p.heads;
+    const int kt = (int)(blockIdx.x / BH);
+    const int bh = (int)(blockIdx.x % BH);
+    const int h = bh % p.heads;
+
+    const uint32_t bar_kv = sb + C::OFF_BAR;
+    auto bar_qf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
+    auto bar_qe = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + C::ST + s); };
+    const uint32_t bar_s = sb + C::OFF_BAR + 8u * (1 + 2 * C::ST);
+    const uint32_t bar_p = bar_s + 8u;
+    const uint32_t bar_acc = bar_s + 16u;
+    const uint32_t bar_dr = bar_s + 24u;
+    uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
+    int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2] list length
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
+    volatile int* abort_cta = misc + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_kv, 1);
+        for (int s = 0; s < C::ST; ++s) {
+            mbar_init(bar_qf(s), 1);
+            mbar_init(bar_qe(s), 1);
+        }
+        mbar_init(bar_s, 1);
+        mbar_init(bar_p, 128);
+        mbar_init(bar_acc, 1);
+        mbar_init(bar_dr, 1);
+        *abort_cta = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 2 && lane == 0) {  // union of the tile's key blocks' query-block lists
+        UnionWalk<C::ROWS> it;
+        int len = 0;
+        const bool ok = it.init_transposed(p.col_ptr, h * (p.nb + 1), kt * C::ROWS, p.nb, p.nnz);
+        if (!ok) atomicOr(p.gflags, kFlagIndex);
+        if (it.any) {
+            for (;;) {
+                int i, bits;
+                bool last, bad;
+                it.next(p.row_idx, i, bits, last, bad);
+                if (bad) atomicOr(p.gflags, kFlagIndex);
+                if (len >= C::LIST_CAP) {
+                    atomicOr(p.gflags, kFlagIndex);
+                    break;
+                }
+                list[len++] = list_pack(i, bits);
+                if (last) break;
+            }
+        }
+        misc[2] = len;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int len = misc[2];
+    const WaitCtl ctl{p.timeout_ns, p.gflags, abort_cta};
+    constexpr uint64_t kDrainNs = 200000000ull;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && len > 0) {
+            mbar_arrive_expect_tx(bar_kv, 2 * C::TBYTES);
+#pragma unroll
+            for (int pn = 0; pn < HD / 64; ++pn) {
+                tma_load_3d(sb + C::OFF_K + pn * (C::M * 128), &tmK, pn * 64, kt * C::M, bh, bar_kv);
+                tma_load_3d(sb + C::OFF_V + pn * (C::M * 128), &tmV, pn * 64, kt * C::M, bh, bar_kv);
+            }
+            int n = 0;
+            for (; n < len; ++n) {
+                const int st = n % C::ST;
+                if (!mbar_wait(bar_qe(st), ((n / C::ST) & 1) ^ 1, ctl)) break;
+                const int i = list_j(list[n]);
+                mbar_arrive_expect_tx(bar_qf(st), 2 * C::QBYTES + C::STATBYTES);
+#pragma unroll
+                for (int pn = 0; pn < HD / 64; ++pn) {
+                    tma_load_3d(sb + C::OFF_Q + st * C::QBYTES + pn * (BK * 128), &tmQ, pn * 64, i * BK,
+                                bh, bar_qf(st));
+                    tma_load_3d(sb + C::OFF_DO + st * C::QBYTES + pn * (BK * 128), &tmDO, pn * 64, i * BK,
+                                bh, bar_qf(st));
+                }
+                bulk_load(sb + C::OFF_STAT + st * C::STATBYTES, p.stats + (int64_t)bh * p.seq_pad + i * BK,
+                          C::STATBYTES, bar_qf(st));
+            }
+            if (*abort_cta) {
+                mbar_drain(bar_kv, 0, kDrainNs);
+                for (int m = (n > C::ST ? n - C::ST : 0); m < n; ++m)
+                    mbar_drain(bar_qf(m % C::ST), (m / C::ST) & 1, kDrainNs);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && len > 0) {
+            constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
+            constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);   // dV += P^T dO, dK += dS^T Q
+            const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
+            const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
+            bool issued = false;
+            if (mbar_wait(bar_kv, 0, ctl)) {
+                for (int n = 0; n < len; ++n) {
+                    const int st = n % C::ST;
+                    if (!mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl)) break;
+                    tc_fence_after();
+                    const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
+                    const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+                    umma_commit(bar_s);
+                    issued = true;
+                    if (!mbar_wait(bar_p, n & 1, ctl)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, bdo, idesc_a,
+                                     (n > 0 || kk > 0) ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8, bq, idesc_a,
+                                     (n > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_qe(st));
+                }
+                if (!*abort_cta) umma_commit(bar_acc);
+            }
+            if (*abort_cta && issued) {
+                umma_commit(bar_dr);
+                mbar_drain(bar_dr, 0, kDrainNs);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ element-wise pass + epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const int kpos = kt * C::M + r;
+        const int kbit = (BK == 128) ? 0 : (r >> 6);
+        const bool row_valid = kpos < p.seq;
+        const float sc = p.scale_log2;
+        bool fail = false;
+        for (int n = 0; n < len; ++n) {
+            const int st = n % C::ST;
+            const uint32_t ent = list[n];
+            // the stage's query statistics came by bulk copy: observe its barrier
+            // too (already complete: the MMAs of this element waited for it)
+            if (!warp_wait(bar_qf(st), (n / C::ST) & 1, ctl) || !warp_wait(bar_s, n & 1, ctl)) {
+                fail = true;
+                break;
+            }
+            tc_fence_after();
+            const float2* stat = reinterpret_cast<const float2*>(smem + C::OFF_STAT + st * C::STATBYTES);
+            const bool vis = row_valid && ((list_bits(ent) >> kbit) & 1);
+            const int lim = kpos - list_j(ent) * BK;  // query column c visible iff c >= lim (k <= q)
+            // 64 columns at a time; P^T and dS^T of chunk ch (bf16 pairs) go to
+            // columns 32 ch .. 32 ch + 31 of S^T and dP^T, which are already read.
+#pragma unroll
+            for (int ch = 0; ch < BK / 64; ++ch) {
+                uint32_t sr[64], dp[64];
+                tmem_ld32(tl + C::COL_S + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(tl + C::COL_S + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_ld32(tl + C::COL_DP + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+                tmem_ld32(tl + C::COL_DP + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const int qc = 64 * ch + c;
+                    const float2 s0 = stat[qc], s1 = stat[qc + 1];
+                    const float p0 = (vis && qc >= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -s0.x)) : 0.f;
+                    const float p1 = (vis && qc + 1 >= lim) ? ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -s1.x)) : 0.f;
+                    const float d0 = p0 * (__uint_as_float(dp[c]) - s0.y);
+                    const float d1 = p1 * (__uint_as_float(dp[c + 1]) - s1.y);
+                    sr[c / 2] = pack_bf16x2(p0, p1);
+                    dp[c / 2] = pack_bf16x2(d0, d1);
+                }
+                tmem_st32(tl + C::COL_S + 32 * ch, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
+                tmem_st32(tl + C::COL_DP + 32 * ch, *reinterpret_cast<const uint32_t(*)[32]>(&dp[0]));
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_p);
+        }
+        if (!fail) {
+            const int64_t row = (int64_t)bh * p.seq + kpos;
+            if (len > 0) {
+                if (warp_wait(bar_acc, 0, ctl)) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        uint16_t* grow = (w == 0 ? p.dv : p.dk) + row * HD;
+                        const float f = w == 0 ? 1.0f : p.scale;
+                        const uint32_t col = w == 0 ? C::COL_DV : C::COL_DK;
+#pragma unroll
+                        for (int c = 0; c < HD / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(tl + col + 32 * c, o);
+                            tmem_wait_ld();
+                            if (row_valid) {
+#pragma unroll
+                                for (int e2 = 0; e2 < 32; e2 += 8) {
+                                    uint4 v;
+                                    v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * f, __uint_as_float(o[e2 + 1]) * f);
+                                    v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * f, __uint_as_float(o[e2 + 3]) * f);
+                                    v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * f, __uint_as_float(o[e2 + 5]) * f);
+                                    v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * f, __uint_as_float(o[e2 + 7]) * f);
+                                    *reinterpret_cast<uint4*>(grow + 32 * c + e2) = v;
+                                }
+                            }
+                        }
+                    }
+                }
+            } else if (row_valid) {  // no query block lists this tile's key blocks
+                for (int d = 0; d < HD; d += 8) {
+                    *reinterpret_cast<uint4*>(p.dk + row * HD + d) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(p.dv + row * HD + d) = make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace s2

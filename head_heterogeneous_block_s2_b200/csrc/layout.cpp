@@ -226,3 +226,47 @@ extern "C" int s2_build_layout_mask(int32_t num_heads, int32_t num_blocks,
     };
     return emit_csr(H, nb, count, fill, row_ptr, col_idx, col_idx_cap, nnz_out);
 }
+
+// ---------------------------------------------------------------------------
+// Transposed lists for the backward pass: for each head h and key block j, the
+// ascending query blocks i whose list holds j. A counting sort per head: count
+// the entries per j, turn the counts into offsets, then visit the rows in
+// ascending i so that every transposed list comes out ascending.
+// ---------------------------------------------------------------------------
+extern "C" int s2_build_layout_transpose(int32_t num_heads, int32_t num_blocks,
+                                         const int32_t* row_ptr, const int32_t* col_idx,
+                                         int64_t nnz, int32_t* col_ptr, int32_t* row_idx)
+{
+    if (!row_ptr || !col_ptr || num_heads < 1 || num_blocks < 1 || nnz < 0 || nnz > INT32_MAX ||
+        ((!col_idx || !row_idx) && nnz > 0))
+        return S2_ERR_INVALID_ARG;
+    const int64_t H = num_heads, nb = num_blocks;
+    // validate: global offsets, rows within [0, nnz], j ascending with j <= i
+    int64_t prev_end = 0;
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t i = 0; i < nb; ++i) {
+            const int64_t a = row_ptr[h * (nb + 1) + i], b = row_ptr[h * (nb + 1) + i + 1];
+            if (a != prev_end || b < a || b > nnz) return S2_ERR_INVALID_ARG;
+            prev_end = b;
+            for (int64_t e = a; e < b; ++e) {
+                const int32_t j = col_idx[e];
+                if (j < 0 || j > i || (e > a && j <= col_idx[e - 1])) return S2_ERR_INVALID_ARG;
+            }
+        }
+    if (prev_end != nnz) return S2_ERR_INVALID_ARG;
+    for (int64_t h = 0; h < H; ++h) {
+        int32_t* cp = col_ptr + h * (nb + 1);
+        for (int64_t j = 0; j <= nb; ++j) cp[j] = 0;
+        const int64_t base = row_ptr[h * (nb + 1)];
+        for (int64_t e = base; e < row_ptr[h * (nb + 1) + nb]; ++e) ++cp[col_idx[e] + 1];
+        cp[0] = (int32_t)base;
+        for (int64_t j = 1; j <= nb; ++j) cp[j] += cp[j - 1];
+        // fill: a running cursor per j (reuse the start offsets, then restore)
+        for (int64_t i = 0; i < nb; ++i)
+            for (int64_t e = row_ptr[h * (nb + 1) + i]; e < row_ptr[h * (nb + 1) + i + 1]; ++e)
+                row_idx[cp[col_idx[e]]++] = (int32_t)i;
+        for (int64_t j = nb; j > 0; --j) cp[j] = cp[j - 1];
+        cp[0] = (int32_t)base;
+    }
+    return S2_OK;
+}

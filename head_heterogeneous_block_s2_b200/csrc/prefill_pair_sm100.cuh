@@ -61,17 +61,11 @@
 #include <cuda.h>
 
 #include "ptx.cuh"
-#include "umma.cuh"  // PrefillParams, umma_sdesc, umma_idesc
+#include "lists.cuh"  // union lists of compacted key-block rows
+#include "umma.cuh"   // PrefillParams, umma_sdesc, umma_idesc
 
 namespace s2 {
 
-// Warp-wide bounded wait (every lane polls: measured faster than one lane
-// polling and broadcasting).
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl)
-{
-    const bool ok = mbar_wait(bar, parity, ctl);
-    return __all_sync(0xffffffffu, ok);
-}
 
 template <int HD, int BK>
 struct PairCfg {
@@ -107,77 +101,6 @@ struct PairCfg {
 };
 
 constexpr float kRescaleLog2 = 8.0f;
-
-// Union-list entry: key block j (bits 0..23), row tags (bits 24..27).
-__device__ __forceinline__ uint32_t list_pack(int j, int bits) { return (uint32_t)j | ((uint32_t)bits << 24); }
-__device__ __forceinline__ int list_j(uint32_t e) { return (int)(e & 0xFFFFFFu); }
-__device__ __forceinline__ int list_bits(uint32_t e) { return (int)((e >> 24) & 0xFu); }
-
-// Walks the ascending union of up to ROWS compacted lists (query blocks
-// qb0 .. qb0+ROWS-1 of one head) and tags each key block with the rows that
-// list it.
-template <int ROWS>
-struct UnionWalk {
-    int a[ROWS], e[ROWS];
-    int imax;
-
-    // Returns false for offsets outside [0, nnz]; `any` tells whether a list is non-empty.
-    bool any;
-
-    __device__ __forceinline__ bool init(const int32_t* row_ptr, int rp, int qb0, int nb, int64_t nnz)
-    {
-        bool ok = true;
-        any = false;
-        imax = -1;
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-            a[r] = e[r] = 0;
-            const int qb = qb0 + r;
-            if (qb < nb) {
-                a[r] = __ldg(row_ptr + rp + qb);
-                e[r] = __ldg(row_ptr + rp + qb + 1);
-                ok = ok && a[r] >= 0 && a[r] <= e[r] && e[r] <= nnz;
-                any = any || e[r] > a[r];
-                imax = qb;
-            }
-        }
-        if (!ok) {
-#pragma unroll
-            for (int r = 0; r < ROWS; ++r) a[r] = e[r] = 0;
-            any = false;
-        }
-        return ok;
-    }
-
-    // Next union element: key block j, row tag bits, and whether it is the last.
-    // A malformed entry (j outside [0, imax]) comes out as j = 0 with no tags.
-    __device__ __forceinline__ void next(const int32_t* col, int& j, int& bits, bool& last, bool& bad)
-    {
-        int jm = INT_MAX;
-        int cur[ROWS];
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-            cur[r] = a[r] < e[r] ? __ldg(col + a[r]) : INT_MAX;
-            jm = cur[r] < jm ? cur[r] : jm;
-        }
-        bits = 0;
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r)
-            if (cur[r] == jm) {
-                bits |= 1 << r;
-                ++a[r];
-            }
-        last = true;
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) last = last && a[r] >= e[r];
-        bad = jm < 0 || jm > imax;
-        if (bad) {
-            jm = 0;
-            bits = 0;
-        }
-        j = jm;
-    }
-};
 
 // Tile t's share of a union element's row tags.
 template <int BK>

@@ -1,6 +1,6 @@
 // s2attn.cu -- C ABI of the HHST sparse-attention library (see include/s2attn.h).
 //
-// Host side of the prefill and decode paths: argument validation, TMA tensor
+// Host side of the prefill, decode and backward paths: argument validation, TMA tensor
 // maps (encoded through the driver entry point, so the library does not link
 // libcuda and loads on machines without a GPU), launches, and the device
 // error flags shared by all kernels of this translation unit.
@@ -15,6 +15,7 @@
 
 #include "s2attn.h"
 #include "ptx.cuh"
+#include "backward_sm100.cuh"
 #include "decode.cuh"
 #include "prefill_pair_sm100.cuh"
 
@@ -39,6 +40,7 @@ struct DevInfo {
     int* sched = nullptr;
     bool prefill_attr_done[4] = {false, false, false, false};
     bool decode_attr_done[2] = {false, false};
+    bool backward_attr_done[4] = {false, false, false, false};
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -135,6 +137,47 @@ int launch_prefill(const void* q, const void* k, const void* v, s2::PrefillParam
     const uint64_t items = (uint64_t)pp.batch * pp.heads * ((pp.nqt + 1) / 2);
     const uint64_t grid = items < (uint64_t)g_dev[dev].num_sms ? items : (uint64_t)g_dev[dev].num_sms;
     kern<<<(unsigned)grid, 384, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
+    return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
+}
+
+// Backward: row statistics, then the dQ kernel and the dK/dV kernel (one CTA
+// per 128-row tile each; neither writes what the other reads).
+template <int HD, int BK>
+int launch_backward(const void* q, const void* k, const void* v, s2::BackwardParams& bp, int dev,
+                    int attr_slot, cudaStream_t stream)
+{
+    using CQ = s2::BwdQCfg<HD, BK>;
+    using CK = s2::BwdKVCfg<HD, BK>;
+    const uint64_t planes = (uint64_t)bp.batch * bp.heads;
+    CUtensorMap q128, do128, kbk, vbk, qbk, dobk, k128, v128;
+    if (make_map(&q128, q, planes, bp.seq, HD, 128) || make_map(&do128, bp.dout, planes, bp.seq, HD, 128) ||
+        make_map(&kbk, k, planes, bp.seq, HD, BK) || make_map(&vbk, v, planes, bp.seq, HD, BK) ||
+        make_map(&qbk, q, planes, bp.seq, HD, BK) || make_map(&dobk, bp.dout, planes, bp.seq, HD, BK) ||
+        make_map(&k128, k, planes, bp.seq, HD, 128) || make_map(&v128, v, planes, bp.seq, HD, 128))
+        return S2_ERR_CUDA;
+    auto kq = s2::s2_bwd_dq_kernel<HD, BK>;
+    auto kkv = s2::s2_bwd_dkv_kernel<HD, BK>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_dev[dev].backward_attr_done[attr_slot]) {
+            if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::SMEM_ALLOC) !=
+                    cudaSuccess ||
+                cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, CK::SMEM_ALLOC) !=
+                    cudaSuccess)
+                return S2_ERR_CUDA;
+            g_dev[dev].backward_attr_done[attr_slot] = true;
+        }
+    }
+    const int64_t rows = (int64_t)planes * bp.seq_pad;
+    const int64_t rows_per_cta = 256 / (HD / 8);
+    int64_t grid0 = (rows + rows_per_cta - 1) / rows_per_cta;
+    if (grid0 > (int64_t)g_dev[dev].num_sms * 16) grid0 = (int64_t)g_dev[dev].num_sms * 16;
+    s2::s2_bwd_stats_kernel<HD><<<(unsigned)grid0, 256, 0, stream>>>(bp);
+    if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
+    const uint64_t tiles = planes * (uint64_t)bp.ntiles;
+    kq<<<(unsigned)tiles, 256, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
+    if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
+    kkv<<<(unsigned)tiles, 256, CK::SMEM_ALLOC, stream>>>(qbk, dobk, k128, v128, bp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
@@ -262,6 +305,72 @@ int s2_attn_prefill_gqa(const void* q, const void* k, const void* v, void* o, fl
     if (head_dim == 128 && block_size == 64) return launch_prefill<128, 64>(q, k, v, pp, dev, 1, st);
     if (head_dim == 64 && block_size == 128) return launch_prefill<64, 128>(q, k, v, pp, dev, 2, st);
     return launch_prefill<64, 64>(q, k, v, pp, dev, 3, st);
+}
+
+size_t s2_attn_backward_workspace_size(int32_t batch, int32_t heads, int32_t seq)
+{
+    if (batch < 1 || heads < 1 || seq < 1) return 0;
+    const int64_t seq_pad = ((int64_t)seq + 127) / 128 * 128;
+    return (size_t)((int64_t)batch * heads * seq_pad * 8);
+}
+
+int s2_attn_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int32_t batch, int32_t heads,
+                     int32_t heads_kv, int32_t seq, int32_t head_dim, float scale,
+                     int32_t block_size, int32_t num_blocks, const int32_t* row_ptr,
+                     const int32_t* col_idx, const int32_t* col_ptr, const int32_t* row_idx,
+                     int64_t nnz, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !row_ptr || !col_ptr ||
+        ((!col_idx || !row_idx) && nnz > 0) || !workspace)
+        return S2_ERR_INVALID_ARG;
+    if (batch < 1 || heads < 1 || seq < 1 || nnz < 0 || !std::isfinite(scale) || !(scale > 0.f))
+        return S2_ERR_INVALID_ARG;
+    if (heads_kv < 1 || heads % heads_kv != 0) return S2_ERR_INVALID_ARG;
+    if (heads_kv != heads) return S2_ERR_UNSUPPORTED;  // grouped K/V heads: forward only
+    if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
+    if (block_size != 64 && block_size != 128) return S2_ERR_UNSUPPORTED;
+    if (num_blocks > 2046) return S2_ERR_UNSUPPORTED;  // union lists are staged in shared memory
+    if (num_blocks != (seq + block_size - 1) / block_size) return S2_ERR_INVALID_ARG;
+    const int64_t ntiles = ((int64_t)seq + 127) / 128;
+    if ((int64_t)batch * heads * ntiles >= (int64_t)INT32_MAX) return S2_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return S2_ERR_INVALID_ARG;
+    if (workspace_bytes < s2_attn_backward_workspace_size(batch, heads, seq)) return S2_ERR_CAPACITY;
+    int dev = 0;
+    int rc = device_ready(&dev);
+    if (rc) return rc;
+
+    s2::BackwardParams bp;
+    bp.row_ptr = row_ptr;
+    bp.col_idx = col_idx;
+    bp.col_ptr = col_ptr;
+    bp.row_idx = row_idx;
+    bp.nnz = nnz;
+    bp.o = static_cast<const uint16_t*>(o);
+    bp.dout = static_cast<const uint16_t*>(dout);
+    bp.lse = lse;
+    bp.stats = static_cast<float2*>(workspace);
+    bp.dq = static_cast<uint16_t*>(dq);
+    bp.dk = static_cast<uint16_t*>(dk);
+    bp.dv = static_cast<uint16_t*>(dv);
+    bp.batch = batch;
+    bp.heads = heads;
+    bp.seq = seq;
+    bp.seq_pad = (int32_t)(ntiles * 128);
+    bp.nb = num_blocks;
+    bp.ntiles = (int32_t)ntiles;
+    bp.scale = scale;
+    bp.scale_log2 = scale * 1.4426950408889634f;
+    bp.timeout_ns = g_timeout_ns.load();
+    bp.gflags = g_dev[dev].flags;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (head_dim == 128 && block_size == 128) return launch_backward<128, 128>(q, k, v, bp, dev, 0, st);
+    if (head_dim == 128 && block_size == 64) return launch_backward<128, 64>(q, k, v, bp, dev, 1, st);
+    if (head_dim == 64 && block_size == 128) return launch_backward<64, 128>(q, k, v, bp, dev, 2, st);
+    return launch_backward<64, 64>(q, k, v, bp, dev, 3, st);
 }
 
 int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,

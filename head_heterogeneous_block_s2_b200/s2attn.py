@@ -28,7 +28,9 @@ STATUS_NAMES = {0: "S2_OK", 1: "S2_ERR_INVALID_ARG", 2: "S2_ERR_UNSUPPORTED", 3:
                 4: "S2_ERR_CUDA", 5: "S2_ERR_TIMEOUT", 6: "S2_ERR_DEVICE_INDEX"}
 
 EXPORTED = ("s2_status_string", "s2_build_layout", "s2_build_layout_ranges",
-            "s2_build_layout_mask", "s2_attn_prefill", "s2_attn_prefill_gqa", "s2_attn_decode_gqa",
+            "s2_build_layout_mask", "s2_build_layout_transpose", "s2_attn_prefill",
+            "s2_attn_prefill_gqa", "s2_attn_decode_gqa", "s2_attn_backward",
+            "s2_attn_backward_workspace_size",
             "s2_attn_decode_workspace_size", "s2_attn_decode_auto_splits", "s2_attn_decode",
             "s2_device_status", "s2_set_wait_timeout_ns", "s2_version", "s2_attn_decode_noalloc")
 
@@ -76,6 +78,13 @@ def load(path: str = LIB_PATH):
     lib.s2_attn_prefill.restype = ctypes.c_int
     lib.s2_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, i32, vp, vp,
                                     i64, vp]
+    lib.s2_build_layout_transpose.restype = ctypes.c_int
+    lib.s2_build_layout_transpose.argtypes = [i32, i32, vp, vp, i64, vp, vp]
+    lib.s2_attn_backward_workspace_size.restype = sz
+    lib.s2_attn_backward_workspace_size.argtypes = [i32, i32, i32]
+    lib.s2_attn_backward.restype = ctypes.c_int
+    lib.s2_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                     f32, i32, i32, vp, vp, vp, vp, i64, vp, sz, vp]
     lib.s2_attn_prefill_gqa.restype = ctypes.c_int
     lib.s2_attn_prefill_gqa.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, i32,
                                         vp, vp, i64, vp]
@@ -126,6 +135,26 @@ class Layout:
     d_col_idx: Optional[torch.Tensor] = None
     pattern: str = "hhst"
     ranges: Optional[Tuple[Tuple[Tuple[int, int, int, bool], ...], ...]] = None
+    # transposed lists (query blocks listing each key block), for the backward
+    t_col_ptr: Optional[np.ndarray] = None
+    t_row_idx: Optional[np.ndarray] = None
+    d_t_col_ptr: Optional[torch.Tensor] = None
+    d_t_row_idx: Optional[torch.Tensor] = None
+
+    def transposed(self, device=None) -> "Layout":
+        """Build (once) the transposed lists with s2_build_layout_transpose and
+        copy them to ``device``."""
+        if self.t_col_ptr is None:
+            self.t_col_ptr = np.zeros(self.heads * (self.num_blocks + 1), dtype=np.int32)
+            self.t_row_idx = np.zeros(max(1, self.nnz), dtype=np.int32)
+            _check(load().s2_build_layout_transpose(
+                self.heads, self.num_blocks, self.row_ptr.ctypes.data,
+                self.col_idx.ctypes.data if self.nnz else None, self.nnz,
+                self.t_col_ptr.ctypes.data, self.t_row_idx.ctypes.data), "s2_build_layout_transpose")
+        if device is not None and (self.d_t_col_ptr is None or self.d_t_col_ptr.device != torch.device(device)):
+            self.d_t_col_ptr = torch.from_numpy(self.t_col_ptr).to(device)
+            self.d_t_row_idx = torch.from_numpy(self.t_row_idx).to(device)
+        return self
 
     @property
     def nnz(self) -> int:
@@ -298,6 +327,51 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: Layout,
                                         _ptr(layout.d_col_idx), layout.nnz, _stream(q.device))
         _check(rc, "s2_attn_prefill_gqa")
     return (out, lse) if lse is not None else out
+
+
+def backward_workspace_size(batch: int, heads: int, seq: int) -> int:
+    return int(load().s2_attn_backward_workspace_size(batch, heads, seq))
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+             lse: torch.Tensor, dout: torch.Tensor, layout: Layout,
+             scale: Optional[float] = None, dq: Optional[torch.Tensor] = None,
+             dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None):
+    """s2_attn_backward: gradients (dq, dk, dv) of ``prefill`` for the upstream
+    gradient ``dout``, given the forward's output ``o`` and ``lse``."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, n)
+    _need(lse, "lse", torch.float32)
+    batch, heads, seq, hd = q.shape
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        if t.shape != q.shape:
+            raise ValueError(f"{n} shape differs from q")
+    if lse.shape != (batch, heads, seq):
+        raise ValueError("lse must be [batch, heads, seq]")
+    if layout.heads != heads:
+        raise ValueError(f"layout has {layout.heads} heads, q has {heads}")
+    if layout.d_row_ptr is None:
+        layout.to(q.device)
+    layout.transposed(q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, n)
+    ws_bytes = backward_workspace_size(batch, heads, seq)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    ws_len = workspace.numel() * workspace.element_size()
+    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    rc = load().s2_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), batch, heads, heads, seq, hd, sc,
+                                 layout.block_size, layout.num_blocks, _ptr(layout.d_row_ptr),
+                                 _ptr(layout.d_col_idx), _ptr(layout.d_t_col_ptr),
+                                 _ptr(layout.d_t_row_idx), layout.nnz, _ptr(workspace), ws_len,
+                                 _stream(q.device))
+    _check(rc, "s2_attn_backward")
+    return dq, dk, dv
 
 
 def decode_auto_splits(batch: int, heads: int) -> int:

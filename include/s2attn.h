@@ -146,6 +146,21 @@ int s2_build_layout_mask(int32_t num_heads, int32_t num_blocks, const uint8_t* b
                          int32_t* row_ptr, int32_t* col_idx, int64_t col_idx_cap,
                          int64_t* nnz_out);
 
+/*
+ * Transposed lists for the backward pass: for each head h and key block j,
+ * the ascending query blocks i whose list (in row_ptr/col_idx, from any of
+ * the builders above) holds j.
+ *   row_ptr, col_idx, nnz  host layout (read); lists must be strictly
+ *                          ascending with 0 <= j <= i and global offsets.
+ *   col_ptr  host int32 [num_heads * (num_blocks + 1)] (written): global
+ *            offsets into row_idx, col_ptr[h*(nb+1) + j] .. col_ptr[h*(nb+1) + j + 1].
+ *   row_idx  host int32 [nnz] (written).
+ * S2_ERR_INVALID_ARG for NULL pointers or a malformed layout. Cost O(nnz + H nb).
+ */
+int s2_build_layout_transpose(int32_t num_heads, int32_t num_blocks, const int32_t* row_ptr,
+                              const int32_t* col_idx, int64_t nnz, int32_t* col_ptr,
+                              int32_t* row_idx);
+
 /* ------------------------------------------------------------------------ */
 /* Prefill: block-sparse causal attention over whole sequences               */
 /* ------------------------------------------------------------------------ */
@@ -189,6 +204,49 @@ int s2_attn_prefill_gqa(const void* q, const void* k, const void* v, void* o, fl
                         int32_t head_dim, float scale, int32_t block_size, int32_t num_blocks,
                         const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz,
                         void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Backward: gradients of the prefill                                        */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of device workspace s2_attn_backward needs: 8 bytes per query row,
+ * rows padded to a multiple of 128 per (batch, head). */
+size_t s2_attn_backward_workspace_size(int32_t batch, int32_t heads, int32_t seq);
+
+/*
+ * dQ, dK, dV of s2_attn_prefill. The arXiv abstract of "S2-Attention:
+ * Hardware-aware context sharding among attention heads" reports training
+ * speedups; the gradients are those of the same masked softmax attention:
+ * with P = exp(scale Q K^T - LSE) over the visible keys and D = rowsum(dO * O),
+ *     dV = P^T dO,   dS = P * (dO V^T - D),   dQ = scale dS K,   dK = scale dS^T Q.
+ *
+ *   q, k, v, o  device bf16 [batch][heads][seq][head_dim] (read): the forward's
+ *               inputs and output.
+ *   dout        device bf16 [batch][heads][seq][head_dim] (read): dL/dO.
+ *   lse         device fp32 [batch][heads][seq] (read): the forward's LSE.
+ *   dq, dk, dv  device bf16 [batch][heads][seq][head_dim] (written).
+ *   heads_kv    must equal heads (grouped K/V heads: S2_ERR_UNSUPPORTED).
+ *   seq, head_dim, scale, block_size, num_blocks: as s2_attn_prefill.
+ *   row_ptr, col_idx, nnz  device layout the forward used (read).
+ *   col_ptr, row_idx       device transposed layout from
+ *                          s2_build_layout_transpose (read).
+ *   workspace   device, >= s2_attn_backward_workspace_size(batch, heads, seq)
+ *               bytes, 256-byte aligned (scratch, clobbered).
+ * Runs three kernels: row statistics (D, LSE in the log2 domain), dQ over the
+ * query tiles' key-block lists, and dK/dV over the key tiles' transposed
+ * lists; S and dP are recomputed by both, so no accumulator is shared between
+ * CTAs (no atomics; results are deterministic). Rows with an empty list get
+ * zero gradients. Errors: S2_ERR_INVALID_ARG (null pointers, sizes, alignment,
+ * a bad scale), S2_ERR_CAPACITY (workspace too small), S2_ERR_UNSUPPORTED
+ * (head_dim, block_size, grouped heads), S2_ERR_CUDA (launch failure).
+ */
+int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                     int32_t batch, int32_t heads, int32_t heads_kv, int32_t seq,
+                     int32_t head_dim, float scale, int32_t block_size, int32_t num_blocks,
+                     const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_ptr,
+                     const int32_t* row_idx, int64_t nnz, void* workspace,
+                     size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Decode: one query token per sequence over a paged KV cache               */

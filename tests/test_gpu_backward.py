@@ -1,0 +1,109 @@
+"""Backward parity: dQ, dK, dV from the sm_100a kernels (through the C ABI)
+against the fp64 oracle's gradients of the same masked attention.
+
+Tolerance. The kernels round P and dS to bf16 as MMA operands (relative
+error up to 2^-9 each), accumulate in fp32 and round the gradients to bf16
+once; gradient entries reach a few units on these unit-normal inputs, so the
+bar is relative to the reference's scale: max-abs <= 2e-2 * max(1, max|ref|)
+and mean-abs <= 2e-3 * max(1, mean|ref|).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from head_heterogeneous_block_s2_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def grad_parity(name, got, ref):
+    got = got.detach().double().cpu().numpy().reshape(ref.shape)
+    assert np.isfinite(got).all(), f"{name}: non-finite"
+    err = np.abs(got - ref)
+    mx_ref, mean_ref = float(np.abs(ref).max()), float(np.abs(ref).mean())
+    mx, mean = float(err.max()), float(err.mean())
+    print(f"{name}: max-abs {mx:.3e} (ref max {mx_ref:.3f}) mean-abs {mean:.3e} (ref mean {mean_ref:.3f})")
+    assert mx <= 2e-2 * max(1.0, mx_ref), f"{name}: max-abs {mx:.3e}"
+    assert mean <= 2e-3 * max(1.0, mean_ref), f"{name}: mean-abs {mean:.3e}"
+
+
+def run_backward(s2, w, lay, q, k, v, do, bmask=None):
+    qc, kc, vc, doc = (t.cuda() for t in (q, k, v, do))
+    o, lse = s2.prefill(qc, kc, vc, lay, scale=w.scale, want_lse=True)
+    dq, dk, dv = s2.backward(qc, kc, vc, o, lse, doc, lay, scale=w.scale)
+    torch.cuda.synchronize()
+    if bmask is None:
+        ref = oracle.backward(q, k, v, do, w.block, w.scale, S=w.stride, L=w.local,
+                              dense_heads=w.dense_heads)
+    else:
+        ref = oracle.backward(q, k, v, do, w.block, w.scale, bmask=bmask)
+    for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        grad_parity(name, g, r)
+    return dq, dk, dv
+
+
+def upstream(w, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn((w.batch, w.heads, w.seq, w.head_dim), generator=g).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("hd", [64, 128])
+@pytest.mark.parametrize("bk", [64, 128])
+@pytest.mark.parametrize("S,L,dense", [(4, 1, ()), (3, 2, (1,))])
+def test_small_shapes_all_gradients(s2gpu, hd, bk, S, L, dense):
+    seq = 9 * 64 if bk == 64 else 5 * 128
+    w = synth.PrefillWorkload("t", 2, 3, hd, seq, bk, S, L, dense_heads=dense, seed=90)
+    q, k, v = synth.prefill_inputs(w)
+    lay = s2gpu.build_layout(3, bk, S, L, w.seq // bk, dense, device="cuda")
+    run_backward(s2gpu, w, lay, q, k, v, upstream(w, 1))
+
+
+@pytest.mark.parametrize("bk", [64, 128])
+@pytest.mark.parametrize("seq", [1, 100, 333])
+def test_ragged_lengths(s2gpu, bk, seq):
+    w = synth.PrefillWorkload("t", 1, 2, 128, seq, bk, 2, 1, seed=91)
+    q, k, v = synth.prefill_inputs(w)
+    lay = s2gpu.build_layout(2, bk, 2, 1, -(-seq // bk), device="cuda")
+    run_backward(s2gpu, w, lay, q, k, v, upstream(w, 2))
+
+
+@pytest.mark.parametrize("bk", [64, 128])
+def test_mask_layout_with_empty_rows(s2gpu, bk):
+    nb, H = 8, 3
+    rng = np.random.default_rng(7)
+    m = np.tril(rng.random((H, nb, nb)) < 0.4).astype(np.uint8)
+    m[0, 2] = 0      # an empty query block
+    m[1, :, 3] = 0   # a key block nobody lists
+    m[2, :4] = 0     # whole tiles with no key
+    w = synth.PrefillWorkload("t", 1, H, 128, nb * bk, bk, 1, 1, seed=92)
+    q, k, v = synth.prefill_inputs(w)
+    lay = s2gpu.build_layout_mask(m, bk, device="cuda")
+    dq, dk, dv = run_backward(s2gpu, w, lay, q, k, v, upstream(w, 3), bmask=m)
+    assert (dk[0, 1, 3 * bk:4 * bk] == 0).all() and (dv[0, 1, 3 * bk:4 * bk] == 0).all()
+
+
+def test_stride_one_matches_autograd_of_causal_sdpa(s2gpu):
+    w = synth.PrefillWorkload("t", 1, 2, 128, 512, 128, 1, 1, seed=93)
+    q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
+    do = upstream(w, 4).cuda()
+    lay = s2gpu.build_layout(2, 128, 1, 1, 4, device="cuda")
+    o, lse = s2gpu.prefill(q, k, v, lay, scale=w.scale, want_lse=True)
+    dq, dk, dv = s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale)
+    qf, kf, vf = (t.float().requires_grad_() for t in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(qf, kf, vf, is_causal=True, scale=w.scale)
+    (ref * do.float()).sum().backward()
+    for g, r in ((dq, qf.grad), (dk, kf.grad), (dv, vf.grad)):
+        assert (g.float() - r).abs().max().item() <= 2e-2 * max(1.0, r.abs().max().item())
+
+
+def test_backward_is_deterministic(s2gpu):
+    w = synth.PrefillWorkload("t", 1, 4, 128, 1024, 64, 4, 2, seed=94)
+    q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
+    do = upstream(w, 5).cuda()
+    lay = s2gpu.build_layout(4, 64, 4, 2, 16, device="cuda")
+    o, lse = s2gpu.prefill(q, k, v, lay, scale=w.scale, want_lse=True)
+    a = s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale)
+    b = s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
