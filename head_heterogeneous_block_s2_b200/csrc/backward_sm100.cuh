@@ -53,6 +53,7 @@ struct BackwardParams {
     const int32_t* col_idx;
     const int32_t* col_ptr;  // query-block lists of key blocks (its transpose)
     const int32_t* row_idx;
+    const int32_t* key_tiles;  // B = 64: [heads][ntiles][2] key blocks of each key tile (-1: none)
     int64_t nnz;
     const uint16_t* o;     // [batch][heads][seq][HD] forward output (stats kernel)
     const uint16_t* dout;  // [batch][heads][seq][HD] upstream gradient (stats kernel)
@@ -421,6 +422,18 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const int kt = (int)(blockIdx.x / BH);
     const int bh = (int)(blockIdx.x % BH);
     const int h = bh % p.heads;
+    // Key blocks of this tile: one 128-row block, or two 64-row blocks chosen on
+    // the host so that their transposed lists overlap (see s2_build_key_tiles).
+    int kb[C::ROWS];
+    if (C::ROWS == 1) {
+        kb[0] = kt;
+    } else {
+#pragma unroll
+        for (int r = 0; r < C::ROWS; ++r) {
+            kb[r] = __ldg(p.key_tiles + ((int64_t)h * p.ntiles + kt) * C::ROWS + r);
+            if (kb[r] >= p.nb) kb[r] = -1;
+        }
+    }
 
     const uint32_t bar_kv = sb + C::OFF_BAR;
     auto bar_qf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
@@ -454,7 +467,7 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     if (warp == 2 && lane == 0) {  // union of the tile's key blocks' query-block lists
         UnionWalk<C::ROWS> it;
         int len = 0;
-        const bool ok = it.init_transposed(p.col_ptr, h * (p.nb + 1), kt * C::ROWS, p.nb, p.nnz);
+        const bool ok = it.init_transposed(p.col_ptr, h * (p.nb + 1), kb, p.nb, p.nnz);
         if (!ok) atomicOr(p.gflags, kFlagIndex);
         if (it.any) {
             for (;;) {
@@ -484,10 +497,20 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         // ------------------------------------------------------------ producer
         if (lane == 0 && len > 0) {
             mbar_arrive_expect_tx(bar_kv, 2 * C::TBYTES);
+            int kany = 0;  // a missing block loads a present one's rows (finite data, masked)
 #pragma unroll
-            for (int pn = 0; pn < HD / 64; ++pn) {
-                tma_load_3d(sb + C::OFF_K + pn * (C::M * 128), &tmK, pn * 64, kt * C::M, bh, bar_kv);
-                tma_load_3d(sb + C::OFF_V + pn * (C::M * 128), &tmV, pn * 64, kt * C::M, bh, bar_kv);
+            for (int r = 0; r < C::ROWS; ++r)
+                if (kb[r] >= 0) kany = kb[r];
+#pragma unroll
+            for (int r = 0; r < C::ROWS; ++r) {
+                const int32_t krow = (kb[r] >= 0 ? kb[r] : kany) * BK;
+#pragma unroll
+                for (int pn = 0; pn < HD / 64; ++pn) {
+                    tma_load_3d(sb + C::OFF_K + pn * (C::M * 128) + r * (BK * 128), &tmK, pn * 64, krow, bh,
+                                bar_kv);
+                    tma_load_3d(sb + C::OFF_V + pn * (C::M * 128) + r * (BK * 128), &tmV, pn * 64, krow, bh,
+                                bar_kv);
+                }
             }
             int n = 0;
             for (; n < len; ++n) {
@@ -566,9 +589,9 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        const int kpos = kt * C::M + r;
         const int kbit = (BK == 128) ? 0 : (r >> 6);
-        const bool row_valid = kpos < p.seq;
+        const int kpos = kb[kbit] * BK + (r % BK);
+        const bool row_valid = kb[kbit] >= 0 && kpos < p.seq;
         const float sc = p.scale_log2;
         bool fail = false;
         for (int n = 0; n < len; ++n) {

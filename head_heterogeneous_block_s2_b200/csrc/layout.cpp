@@ -8,8 +8,10 @@
 // or every block 0..i for a dense head. This file enumerates them directly in
 // ascending order (strided ones first, then the local run), which is O(nnz)
 // rather than a test of every (i, j) pair, and emits CSR offsets.
+#include <algorithm>
 #include <climits>
 #include <cstdint>
+#include <vector>
 
 #include "s2attn.h"
 
@@ -267,6 +269,38 @@ extern "C" int s2_build_layout_transpose(int32_t num_heads, int32_t num_blocks,
                 row_idx[cp[col_idx[e]]++] = (int32_t)i;
         for (int64_t j = nb; j > 0; --j) cp[j] = cp[j - 1];
         cp[0] = (int32_t)base;
+    }
+    return S2_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Key tiles of the backward's dK/dV kernel for 64-row blocks: each 128-row key
+// tile holds two key blocks and walks the union of their transposed lists, so
+// blocks whose lists overlap should share a tile. Per head, the blocks are
+// ordered by transposed-list length (longest first, then by j) and paired
+// consecutively: under HHST the strided blocks j and j + S pair up (both are
+// listed by nearly every later query block) and the other blocks pair with
+// their neighbours (overlapping local windows).
+// ---------------------------------------------------------------------------
+extern "C" int s2_build_key_tiles(int32_t num_heads, int32_t num_blocks, const int32_t* col_ptr,
+                                  int32_t* key_tiles)
+{
+    if (!col_ptr || !key_tiles || num_heads < 1 || num_blocks < 1) return S2_ERR_INVALID_ARG;
+    const int64_t H = num_heads, nb = num_blocks, ntk = (nb + 1) / 2;
+    std::vector<int32_t> order((size_t)nb);
+    for (int64_t h = 0; h < H; ++h) {
+        const int32_t* cp = col_ptr + h * (nb + 1);
+        for (int64_t j = 0; j < nb; ++j) {
+            if (cp[j + 1] < cp[j]) return S2_ERR_INVALID_ARG;
+            order[(size_t)j] = (int32_t)j;
+        }
+        std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) {
+            return cp[a + 1] - cp[a] > cp[b + 1] - cp[b];
+        });
+        for (int64_t t = 0; t < ntk; ++t) {
+            key_tiles[(h * ntk + t) * 2] = order[(size_t)(2 * t)];
+            key_tiles[(h * ntk + t) * 2 + 1] = 2 * t + 1 < nb ? order[(size_t)(2 * t + 1)] : -1;
+        }
     }
     return S2_OK;
 }

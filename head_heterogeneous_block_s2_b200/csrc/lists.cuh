@@ -49,17 +49,31 @@ struct UnionWalk {
         return ok;
     }
 
-    // Transposed lists of key blocks kb0..: the same walk, valid range [kb0, nb - 1].
-    __device__ __forceinline__ bool init_transposed(const int32_t* col_ptr, int rp, int kb0, int nb,
+    // Transposed lists of the key blocks kb[0..ROWS-1] (kb[r] < 0: no block):
+    // the same walk, valid range [smallest key block, nb - 1].
+    __device__ __forceinline__ bool init_transposed(const int32_t* col_ptr, int rp, const int* kb, int nb,
                                                     int64_t nnz)
     {
-        const bool ok = init_rows(col_ptr, rp, kb0, nb, nnz);
-        imin = kb0;
+        const bool ok = init_rows(col_ptr, rp, kb, nb, nnz);
+        imin = INT_MAX;
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r)
+            if (kb[r] >= 0 && kb[r] < imin) imin = kb[r];
         imax = nb - 1;
         return ok;
     }
 
     __device__ __forceinline__ bool init_rows(const int32_t* row_ptr, int rp, int qb0, int nb, int64_t nnz)
+    {
+        int rows[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) rows[r] = qb0 + r;
+        return init_rows(row_ptr, rp, rows, nb, nnz);
+    }
+
+    // CSR rows rows[0..ROWS-1] (a row outside [0, nb) is absent).
+    __device__ __forceinline__ bool init_rows(const int32_t* row_ptr, int rp, const int* rows, int nb,
+                                              int64_t nnz)
     {
         bool ok = true;
         any = false;
@@ -67,8 +81,8 @@ struct UnionWalk {
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
             a[r] = e[r] = 0;
-            const int qb = qb0 + r;
-            if (qb < nb) {
+            const int qb = rows[r];
+            if (qb >= 0 && qb < nb) {
                 a[r] = __ldg(row_ptr + rp + qb);
                 e[r] = __ldg(row_ptr + rp + qb + 1);
                 ok = ok && a[r] >= 0 && a[r] <= e[r] && e[r] <= nnz;

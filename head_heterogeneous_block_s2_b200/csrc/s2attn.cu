@@ -149,11 +149,10 @@ int launch_backward(const void* q, const void* k, const void* v, s2::BackwardPar
     using CQ = s2::BwdQCfg<HD, BK>;
     using CK = s2::BwdKVCfg<HD, BK>;
     const uint64_t planes = (uint64_t)bp.batch * bp.heads;
-    CUtensorMap q128, do128, kbk, vbk, qbk, dobk, k128, v128;
+    CUtensorMap q128, do128, kbk, vbk, qbk, dobk;
     if (make_map(&q128, q, planes, bp.seq, HD, 128) || make_map(&do128, bp.dout, planes, bp.seq, HD, 128) ||
         make_map(&kbk, k, planes, bp.seq, HD, BK) || make_map(&vbk, v, planes, bp.seq, HD, BK) ||
-        make_map(&qbk, q, planes, bp.seq, HD, BK) || make_map(&dobk, bp.dout, planes, bp.seq, HD, BK) ||
-        make_map(&k128, k, planes, bp.seq, HD, 128) || make_map(&v128, v, planes, bp.seq, HD, 128))
+        make_map(&qbk, q, planes, bp.seq, HD, BK) || make_map(&dobk, bp.dout, planes, bp.seq, HD, BK))
         return S2_ERR_CUDA;
     auto kq = s2::s2_bwd_dq_kernel<HD, BK>;
     auto kkv = s2::s2_bwd_dkv_kernel<HD, BK>;
@@ -177,7 +176,7 @@ int launch_backward(const void* q, const void* k, const void* v, s2::BackwardPar
     const uint64_t tiles = planes * (uint64_t)bp.ntiles;
     kq<<<(unsigned)tiles, 256, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
     if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
-    kkv<<<(unsigned)tiles, 256, CK::SMEM_ALLOC, stream>>>(qbk, dobk, k128, v128, bp);
+    kkv<<<(unsigned)tiles, 256, CK::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
@@ -319,10 +318,11 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
                      int32_t heads_kv, int32_t seq, int32_t head_dim, float scale,
                      int32_t block_size, int32_t num_blocks, const int32_t* row_ptr,
                      const int32_t* col_idx, const int32_t* col_ptr, const int32_t* row_idx,
-                     int64_t nnz, void* workspace, size_t workspace_bytes, void* stream)
+                     const int32_t* key_tiles, int64_t nnz, void* workspace,
+                     size_t workspace_bytes, void* stream)
 {
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !row_ptr || !col_ptr ||
-        ((!col_idx || !row_idx) && nnz > 0) || !workspace)
+        ((!col_idx || !row_idx) && nnz > 0) || !workspace || (block_size == 64 && !key_tiles))
         return S2_ERR_INVALID_ARG;
     if (batch < 1 || heads < 1 || seq < 1 || nnz < 0 || !std::isfinite(scale) || !(scale > 0.f))
         return S2_ERR_INVALID_ARG;
@@ -348,6 +348,7 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
     bp.col_idx = col_idx;
     bp.col_ptr = col_ptr;
     bp.row_idx = row_idx;
+    bp.key_tiles = key_tiles;
     bp.nnz = nnz;
     bp.o = static_cast<const uint16_t*>(o);
     bp.dout = static_cast<const uint16_t*>(dout);

@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "S2_OK", 1: "S2_ERR_INVALID_ARG", 2: "S2_ERR_UNSUPPORTED", 3:
 EXPORTED = ("s2_status_string", "s2_build_layout", "s2_build_layout_ranges",
             "s2_build_layout_mask", "s2_build_layout_transpose", "s2_attn_prefill",
             "s2_attn_prefill_gqa", "s2_attn_decode_gqa", "s2_attn_backward",
-            "s2_attn_backward_workspace_size",
+            "s2_attn_backward_workspace_size", "s2_build_key_tiles",
             "s2_attn_decode_workspace_size", "s2_attn_decode_auto_splits", "s2_attn_decode",
             "s2_device_status", "s2_set_wait_timeout_ns", "s2_version", "s2_attn_decode_noalloc")
 
@@ -80,11 +80,13 @@ def load(path: str = LIB_PATH):
                                     i64, vp]
     lib.s2_build_layout_transpose.restype = ctypes.c_int
     lib.s2_build_layout_transpose.argtypes = [i32, i32, vp, vp, i64, vp, vp]
+    lib.s2_build_key_tiles.restype = ctypes.c_int
+    lib.s2_build_key_tiles.argtypes = [i32, i32, vp, vp]
     lib.s2_attn_backward_workspace_size.restype = sz
     lib.s2_attn_backward_workspace_size.argtypes = [i32, i32, i32]
     lib.s2_attn_backward.restype = ctypes.c_int
     lib.s2_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
-                                     f32, i32, i32, vp, vp, vp, vp, i64, vp, sz, vp]
+                                     f32, i32, i32, vp, vp, vp, vp, vp, i64, vp, sz, vp]
     lib.s2_attn_prefill_gqa.restype = ctypes.c_int
     lib.s2_attn_prefill_gqa.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, i32,
                                         vp, vp, i64, vp]
@@ -138,22 +140,29 @@ class Layout:
     # transposed lists (query blocks listing each key block), for the backward
     t_col_ptr: Optional[np.ndarray] = None
     t_row_idx: Optional[np.ndarray] = None
+    t_key_tiles: Optional[np.ndarray] = None  # [heads, ceil(nb / 2), 2] (s2_build_key_tiles)
     d_t_col_ptr: Optional[torch.Tensor] = None
     d_t_row_idx: Optional[torch.Tensor] = None
+    d_t_key_tiles: Optional[torch.Tensor] = None
 
     def transposed(self, device=None) -> "Layout":
-        """Build (once) the transposed lists with s2_build_layout_transpose and
-        copy them to ``device``."""
+        """Build (once) the transposed lists (s2_build_layout_transpose) and the
+        backward's key tiles (s2_build_key_tiles), and copy them to ``device``."""
         if self.t_col_ptr is None:
+            lib = load()
             self.t_col_ptr = np.zeros(self.heads * (self.num_blocks + 1), dtype=np.int32)
             self.t_row_idx = np.zeros(max(1, self.nnz), dtype=np.int32)
-            _check(load().s2_build_layout_transpose(
+            _check(lib.s2_build_layout_transpose(
                 self.heads, self.num_blocks, self.row_ptr.ctypes.data,
                 self.col_idx.ctypes.data if self.nnz else None, self.nnz,
                 self.t_col_ptr.ctypes.data, self.t_row_idx.ctypes.data), "s2_build_layout_transpose")
+            self.t_key_tiles = np.zeros((self.heads, (self.num_blocks + 1) // 2, 2), dtype=np.int32)
+            _check(lib.s2_build_key_tiles(self.heads, self.num_blocks, self.t_col_ptr.ctypes.data,
+                                          self.t_key_tiles.ctypes.data), "s2_build_key_tiles")
         if device is not None and (self.d_t_col_ptr is None or self.d_t_col_ptr.device != torch.device(device)):
             self.d_t_col_ptr = torch.from_numpy(self.t_col_ptr).to(device)
             self.d_t_row_idx = torch.from_numpy(self.t_row_idx).to(device)
+            self.d_t_key_tiles = torch.from_numpy(self.t_key_tiles).to(device)
         return self
 
     @property
@@ -368,7 +377,8 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                                  _ptr(dq), _ptr(dk), _ptr(dv), batch, heads, heads, seq, hd, sc,
                                  layout.block_size, layout.num_blocks, _ptr(layout.d_row_ptr),
                                  _ptr(layout.d_col_idx), _ptr(layout.d_t_col_ptr),
-                                 _ptr(layout.d_t_row_idx), layout.nnz, _ptr(workspace), ws_len,
+                                 _ptr(layout.d_t_row_idx), _ptr(layout.d_t_key_tiles), layout.nnz,
+                                 _ptr(workspace), ws_len,
                                  _stream(q.device))
     _check(rc, "s2_attn_backward")
     return dq, dk, dv

@@ -161,6 +161,22 @@ int s2_build_layout_transpose(int32_t num_heads, int32_t num_blocks, const int32
                               const int32_t* col_idx, int64_t nnz, int32_t* col_ptr,
                               int32_t* row_idx);
 
+/*
+ * Key tiles of the backward for block_size 64: the dK/dV kernel works on
+ * 128-row key tiles of two 64-row key blocks and walks the union of their
+ * transposed lists, so blocks whose lists overlap should share a tile. Per
+ * head, blocks are ordered by transposed-list length (longest first, ties by
+ * j) and paired consecutively (under HHST: strided blocks j and j + S, and
+ * neighbouring local-only blocks).
+ *   col_ptr    host transposed offsets from s2_build_layout_transpose (read).
+ *   key_tiles  host int32 [num_heads][ceil(num_blocks / 2)][2] (written): the
+ *              two key blocks of each tile; -1 for the missing second block
+ *              when num_blocks is odd. Every block appears exactly once.
+ * S2_ERR_INVALID_ARG for NULL pointers, sizes < 1 or decreasing offsets.
+ */
+int s2_build_key_tiles(int32_t num_heads, int32_t num_blocks, const int32_t* col_ptr,
+                       int32_t* key_tiles);
+
 /* ------------------------------------------------------------------------ */
 /* Prefill: block-sparse causal attention over whole sequences               */
 /* ------------------------------------------------------------------------ */
@@ -230,6 +246,8 @@ size_t s2_attn_backward_workspace_size(int32_t batch, int32_t heads, int32_t seq
  *   row_ptr, col_idx, nnz  device layout the forward used (read).
  *   col_ptr, row_idx       device transposed layout from
  *                          s2_build_layout_transpose (read).
+ *   key_tiles              device key tiles from s2_build_key_tiles (read;
+ *                          required when block_size is 64, ignored otherwise).
  *   workspace   device, >= s2_attn_backward_workspace_size(batch, heads, seq)
  *               bytes, 256-byte aligned (scratch, clobbered).
  * Runs three kernels: row statistics (D, LSE in the log2 domain), dQ over the
@@ -245,8 +263,8 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
                      int32_t batch, int32_t heads, int32_t heads_kv, int32_t seq,
                      int32_t head_dim, float scale, int32_t block_size, int32_t num_blocks,
                      const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_ptr,
-                     const int32_t* row_idx, int64_t nnz, void* workspace,
-                     size_t workspace_bytes, void* stream);
+                     const int32_t* row_idx, const int32_t* key_tiles, int64_t nnz,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Decode: one query token per sequence over a paged KV cache               */

@@ -63,3 +63,26 @@ def test_transpose_rejects_malformed_layouts():
     assert _raw([0, 2, 3], [0, 1, 1], 1, 2) == 1   # j > i in row 0
     assert _raw([0, 1, 4], [0, 0, 1, 1], 1, 2) == 1  # duplicate
     assert _raw([1, 1, 2], [0, 0], 1, 2) == 1      # offsets not starting at 0
+
+
+@pytest.mark.parametrize("args", [(16, 64, 8, 2, 128, ()), (5, 64, 3, 2, 37, (4,)), (3, 64, 4, 1, 1, ())])
+def test_key_tiles_cover_every_block_once(args):
+    lay = s2attn.build_layout(*args).transposed()
+    kt = lay.t_key_tiles
+    H, nb = lay.heads, lay.num_blocks
+    assert kt.shape == (H, (nb + 1) // 2, 2)
+    for h in range(H):
+        got = sorted(int(x) for x in kt[h].reshape(-1) if x >= 0)
+        assert got == list(range(nb))
+        assert (kt[h].reshape(-1) < 0).sum() == (nb % 2)
+
+
+def test_key_tiles_pair_strided_blocks_under_hhst():
+    # B 64, S 8, L 2: strided blocks of head h are j = -h mod 8; they pair with j + 8
+    lay = s2attn.build_layout(16, 64, 8, 2, 128).transposed()
+    for h in (0, 3, 9):
+        j0 = (-h) % 8
+        strided = list(range(j0, 126, 8))
+        tiles = [tuple(t) for t in lay.t_key_tiles[h]]
+        for a, b in zip(strided[0:-1:2], strided[1::2]):
+            assert (a, b) in tiles
