@@ -29,10 +29,13 @@
 // both) so that no accumulator is shared between CTAs: no atomics, and the
 // results are deterministic.
 //
-// CTA = 8 warps: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer (one
+// CTA = 12 warps: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer (one
 // thread), warp 2 builds the union list in shared memory before the main
-// loop, warps 4..7 the element-wise pass (thread = one tile row = one TMEM
-// lane) and the epilogue; warp 3 idles. With B = 64 a 128-row tile holds two
+// loop, warps 4..11 the element-wise passes and the epilogue: thread = one
+// tile row = one TMEM lane, warps 4..7 on the first half of the columns and
+// warps 8..11 on the second (two warps per SM sub-partition hide the
+// exponential and TMEM latencies; a single warpgroup was measured to leave
+// the tensor core idle most of the time); warp 3 idles. With B = 64 a 128-row tile holds two
 // blocks and every row masks by its own block's tag. Every wait is bounded;
 // on a timeout the CTA drains its own copies and MMAs, frees TMEM and exits
 // with the device timeout flag set.
@@ -58,7 +61,7 @@ struct BackwardParams {
     const uint16_t* o;     // [batch][heads][seq][HD] forward output (stats kernel)
     const uint16_t* dout;  // [batch][heads][seq][HD] upstream gradient (stats kernel)
     const float* lse;      // [batch][heads][seq] forward LSE, natural log (stats kernel)
-    float2* stats;         // [batch * heads][seq_pad]: (LSE * log2 e, D)
+    float* stats;          // [batch * heads][seq_pad / 128][2][128]: LSE * log2 e, then D
     uint16_t* dq;          // [batch][heads][seq][HD]
     uint16_t* dk;          // [batch][heads][seq][HD]
     uint16_t* dv;
@@ -74,6 +77,40 @@ struct BackwardParams {
 __device__ __forceinline__ uint64_t kstep(int kk, int rows)
 {
     return (uint64_t)((((kk >> 2) * (rows * 128)) + (kk & 3) * 32) >> 4);
+}
+
+// N consecutive 32-bit TMEM columns of this thread's lane (N = 16, 32 or 64).
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N])
+{
+    if constexpr (N == 16) {
+        tmem_ld16(taddr, r);
+    } else {
+#pragma unroll
+        for (int c = 0; c < N / 32; ++c)
+            tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[N])
+{
+    if constexpr (N == 16) {
+        tmem_st16(taddr, r);
+    } else {
+#pragma unroll
+        for (int c = 0; c < N / 32; ++c)
+            tmem_st32(taddr + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&r[32 * c]));
+    }
+}
+
+// TMEM column of k-step kk (16 rows of K) of a bf16 A operand written by the
+// two element-wise warpgroups: half g = kk / (BK / 32) of the BK columns was
+// packed into the first BK / 4 columns of that half's own range.
+template <int BK>
+__host__ __device__ constexpr uint32_t packed_col(int kk)
+{
+    return (uint32_t)((kk / (BK / 32)) * (BK / 2) + (kk % (BK / 32)) * 8);
 }
 
 // ------------------------------------------------------------------ stats
@@ -105,9 +142,11 @@ __global__ void __launch_bounds__(256) s2_bwd_stats_kernel(const BackwardParams 
         }
 #pragma unroll
         for (int w = TPR / 2; w > 0; w >>= 1) d += __shfl_xor_sync(0xffffffffu, d, w);
-        if (sub == 0 && r < rows)
-            p.stats[r] = q < p.seq ? make_float2(p.lse[bh * p.seq + q] * 1.4426950408889634f, d)
-                                   : make_float2(INFINITY, 0.f);
+        if (sub == 0 && r < rows) {  // planar per 128-row tile: 128 values of L2, then 128 of D
+            float* t = p.stats + (r / 128) * 256 + (r % 128);
+            t[0] = q < p.seq ? p.lse[bh * p.seq + q] * 1.4426950408889634f : INFINITY;
+            t[128] = q < p.seq ? d : 0.f;
+        }
     }
 }
 
@@ -126,9 +165,11 @@ struct BwdQCfg {
     static constexpr uint32_t OFF_K = 2 * TBYTES;              // [stage][panel][BK rows x 128 B]
     static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
-    static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_CAP * 4;
-    // barriers: qd_full, k_full[ST], v_full[ST], kv_empty[ST], s_full, ds_full, acc_done, drain
-    static constexpr int NBAR = 1 + 3 * ST + 4;
+    static constexpr uint32_t OFF_SCR = OFF_LIST + LIST_CAP * 4;  // list-merge scratch (ROWS > 1)
+    static constexpr uint32_t OFF_BAR = OFF_SCR + (ROWS > 1 ? ROWS * LIST_CAP * 4 : 0);
+    // barriers: qd_full, k_full[ST], v_full[ST], kv_empty[ST], s_full, ds_full, acc_done, drain,
+    // dp_full
+    static constexpr int NBAR = 1 + 3 * ST + 5;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
@@ -138,7 +179,7 @@ struct BwdQCfg {
 };
 
 template <int HD, int BK>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const BackwardParams p)
@@ -162,12 +203,14 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t bar_ds = bar_s + 8u;
     const uint32_t bar_acc = bar_s + 16u;
     const uint32_t bar_dr = bar_s + 24u;
+    const uint32_t bar_dp = bar_s + 32u;
     uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2] list length
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
     volatile int* abort_cta = misc + 1;
 
     if (threadIdx.x == 0) {
+        mbar_init(bar_dp, 1);
         mbar_init(bar_qd, 1);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_kf(s), 1);
@@ -175,7 +218,7 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mbar_init(bar_ke(s), 1);
         }
         mbar_init(bar_s, 1);
-        mbar_init(bar_ds, 128);
+        mbar_init(bar_ds, 256);
         mbar_init(bar_acc, 1);
         mbar_init(bar_dr, 1);
         *abort_cta = 0;
@@ -185,26 +228,22 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 2 && lane == 0) {  // union of the tile's key-block lists
-        UnionWalk<C::ROWS> it;
-        int len = 0;
-        const bool ok = it.init(p.row_ptr, h * (p.nb + 1), qt * C::ROWS, p.nb, p.nnz);
-        if (!ok) atomicOr(p.gflags, kFlagIndex);
-        if (it.any) {
-            for (;;) {
-                int j, bits;
-                bool last, bad;
-                it.next(p.col_idx, j, bits, last, bad);
-                if (bad) atomicOr(p.gflags, kFlagIndex);
-                if (len >= C::LIST_CAP) {  // cannot happen when nb <= LIST_CAP
-                    atomicOr(p.gflags, kFlagIndex);
-                    break;
-                }
-                list[len++] = list_pack(j, bits);
-                if (last) break;
-            }
+    if (threadIdx.x == 0) {  // Q and dO of the tile do not depend on the list: load them now
+        mbar_arrive_expect_tx(bar_qd, 2 * C::TBYTES);
+#pragma unroll
+        for (int pn = 0; pn < HD / 64; ++pn) {
+            tma_load_3d(sb + C::OFF_Q + pn * (C::M * 128), &tmQ, pn * 64, qt * C::M, bh, bar_qd);
+            tma_load_3d(sb + C::OFF_DO + pn * (C::M * 128), &tmDO, pn * 64, qt * C::M, bh, bar_qd);
         }
-        misc[2] = len;
+    }
+    if (warp == 2) {  // union of the tile's key-block lists
+        int rows[C::ROWS];
+#pragma unroll
+        for (int r = 0; r < C::ROWS; ++r) rows[r] = qt * C::ROWS + r;
+        const int n = warp_union_list<C::ROWS>(p.row_ptr, p.col_idx, h * (p.nb + 1), rows, p.nb, p.nnz,
+                                               0, min(qt * C::ROWS + C::ROWS, p.nb) - 1, list, C::LIST_CAP,
+                                               reinterpret_cast<int32_t*>(smem + C::OFF_SCR), p.gflags);
+        if (lane == 0) misc[2] = n;
     }
     tc_fence_before();
     __syncthreads();
@@ -216,13 +255,8 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        if (lane == 0 && len == 0) mbar_drain(bar_qd, 0, kDrainNs);  // nothing to do: let Q, dO land
         if (lane == 0 && len > 0) {
-            mbar_arrive_expect_tx(bar_qd, 2 * C::TBYTES);
-#pragma unroll
-            for (int pn = 0; pn < HD / 64; ++pn) {
-                tma_load_3d(sb + C::OFF_Q + pn * (C::M * 128), &tmQ, pn * 64, qt * C::M, bh, bar_qd);
-                tma_load_3d(sb + C::OFF_DO + pn * (C::M * 128), &tmDO, pn * 64, qt * C::M, bh, bar_qd);
-            }
             int n = 0;
             for (; n < len; ++n) {
                 const int st = n % C::ST;
@@ -256,35 +290,51 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
             const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
             bool issued = false;
-            if (mbar_wait(bar_qd, 0, ctl)) {
+            // S(n) and dP(n) are committed separately so that the element-wise
+            // warps start on P while dP is still running. Order per element n:
+            // [dS(n) ready] S(n+1), dQ(n), dP(n+1): S(n+1) only overwrites S(n),
+            // which the warps have finished with; dS(n) sits in dP's columns
+            // and dP(n+1) is issued after dQ(n) has read it.
+            auto issue_s = [&](int n) {
+                const int st = n % C::ST;
+                if (!mbar_wait(bar_kf(st), (n / C::ST) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_bf16_ss(tmem + C::COL_S, dq_desc + kstep(kk, C::M), dk_desc + kstep(kk, BK), idesc_s,
+                                 kk > 0 ? 1u : 0u);
+                umma_commit(bar_s);
+                issued = true;
+                return true;
+            };
+            auto issue_dp = [&](int n) {
+                const int st = n % C::ST;
+                if (!mbar_wait(bar_vf(st), (n / C::ST) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_bf16_ss(tmem + C::COL_DP, ddo_desc + kstep(kk, C::M), dv_desc + kstep(kk, BK),
+                                 idesc_s, kk > 0 ? 1u : 0u);
+                umma_commit(bar_dp);
+                return true;
+            };
+            if (mbar_wait(bar_qd, 0, ctl) && issue_s(0) && issue_dp(0)) {
                 for (int n = 0; n < len; ++n) {
                     const int st = n % C::ST;
-                    const uint32_t par = (n / C::ST) & 1;
-                    if (!mbar_wait(bar_kf(st), par, ctl)) break;
-                    tc_fence_after();
-                    const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ss(tmem + C::COL_S, dq_desc + kstep(kk, C::M), dk_desc + kstep(kk, BK),
-                                     idesc_s, kk > 0 ? 1u : 0u);
-                    issued = true;
-                    if (!mbar_wait(bar_vf(st), par, ctl)) break;
-                    tc_fence_after();
-                    const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ss(tmem + C::COL_DP, ddo_desc + kstep(kk, C::M), dv_desc + kstep(kk, BK),
-                                     idesc_s, kk > 0 ? 1u : 0u);
-                    umma_commit(bar_s);
+                    const bool more = n + 1 < len;
                     if (!mbar_wait(bar_ds, n & 1, ctl)) break;
                     tc_fence_after();
+                    if (more && !issue_s(n + 1)) break;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t bk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_S + kk * 8, bk, idesc_q,
+                        umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
                                      (n > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(bar_ke(st));
+                    if (more && !issue_dp(n + 1)) break;
                 }
                 if (!*abort_cta) umma_commit(bar_acc);
             }
@@ -295,16 +345,21 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         __syncwarp();
     } else if (warp >= 4) {
-        // ------------------------------------------------------------ element-wise pass + epilogue
-        const int quad = warp & 3;
+        // ------------------------------------------------------------ element-wise passes + epilogue
+        constexpr int HALF = BK / 2;  // key columns per warpgroup
+        const int quad = warp & 3, g = (warp - 4) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const int qpos = qt * C::M + r;
         const int rowbit = (BK == 128) ? 0 : (r >> 6);
         const bool row_valid = qpos < p.seq;
         const float sc = p.scale_log2;
-        float2 stat = make_float2(0.f, 0.f);
-        if (row_valid) stat = p.stats[(int64_t)bh * p.seq_pad + qpos];
+        float lx = 0.f, dy = 0.f;  // this row's LSE * log2 e and D
+        if (row_valid) {
+            const float* sp = p.stats + ((int64_t)bh * p.ntiles + qt) * 256 + r;
+            lx = sp[0];
+            dy = sp[128];
+        }
         bool fail = false;
         for (int n = 0; n < len; ++n) {
             const uint32_t ent = list[n];
@@ -314,41 +369,47 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
             tc_fence_after();
             const bool vis = row_valid && ((list_bits(ent) >> rowbit) & 1);
-            const int lim = qpos - list_j(ent) * BK;  // key column c visible iff c <= lim
-            // 64 columns at a time; dS of chunk ch (bf16 pairs) goes to columns
-            // 32 ch .. 32 ch + 31 of S, which are already read.
+            const int lim = qpos - list_j(ent) * BK - g * HALF;  // column c of this half visible iff c <= lim
+            // P pass (needs S only; dP may still be running): P as bf16 pairs in registers
+            uint32_t sr[HALF], pk[HALF / 2];
+            tmem_ld_cols<HALF>(tl + C::COL_S + g * HALF, sr);
+            tmem_wait_ld();
 #pragma unroll
-            for (int ch = 0; ch < BK / 64; ++ch) {
-                uint32_t sr[64], dp[64];
-                tmem_ld32(tl + C::COL_S + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(tl + C::COL_S + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_ld32(tl + C::COL_DP + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-                tmem_ld32(tl + C::COL_DP + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const int kc = 64 * ch + c;
-                    const float p0 = (vis && kc <= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -stat.x)) : 0.f;
-                    const float p1 = (vis && kc + 1 <= lim) ? ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -stat.x)) : 0.f;
-                    const float d0 = p0 * (__uint_as_float(dp[c]) - stat.y);
-                    const float d1 = p1 * (__uint_as_float(dp[c + 1]) - stat.y);
-                    sr[c / 2] = pack_bf16x2(d0, d1);  // slot c/2 <= c: already read
-                }
-                tmem_st32(tl + C::COL_S + 32 * ch, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
+            for (int c = 0; c < HALF; c += 2) {
+                const float p0 = (vis && c <= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -lx)) : 0.f;
+                const float p1 = (vis && c + 1 <= lim) ? ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -lx)) : 0.f;
+                pk[c / 2] = pack_bf16x2(p0, p1);
             }
+            if (!warp_wait(bar_dp, n & 1, ctl)) {
+                fail = true;
+                break;
+            }
+            tc_fence_after();
+            // dS pass: dS = P (dP - D), bf16 pairs over the first HALF/2 columns
+            // of this half of dP (already read)
+            tmem_ld_cols<HALF>(tl + C::COL_DP + g * HALF, sr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < HALF; c += 2) {
+                const float d0 = bf16lo(pk[c / 2]) * (__uint_as_float(sr[c]) - dy);
+                const float d1 = bf16hi(pk[c / 2]) * (__uint_as_float(sr[c + 1]) - dy);
+                pk[c / 2] = pack_bf16x2(d0, d1);
+            }
+            tmem_st_cols<HALF / 2>(tl + C::COL_DP + g * HALF, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_ds);
         }
         if (!fail) {
-            uint16_t* drow = p.dq + ((int64_t)bh * p.seq + qpos) * HD;
+            // warpgroup g stores output columns g * HD/2 .. (g + 1) * HD/2 - 1
+            uint16_t* drow = p.dq + ((int64_t)bh * p.seq + qpos) * HD + g * (HD / 2);
             if (len > 0) {
                 if (warp_wait(bar_acc, 0, ctl)) {
                     tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
+                    for (int c = 0; c < HD / 64; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(tl + C::COL_ACC + 32 * c, o);
+                        tmem_ld32(tl + C::COL_ACC + g * (HD / 2) + 32 * c, o);
                         tmem_wait_ld();
                         if (row_valid) {
 #pragma unroll
@@ -364,7 +425,7 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     }
                 }
             } else if (row_valid) {  // no key block listed for this tile
-                for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(drow + d) = make_uint4(0, 0, 0, 0);
+                for (int d = 0; d < HD / 2; d += 8) *reinterpret_cast<uint4*>(drow + d) = make_uint4(0, 0, 0, 0);
             }
         }
         tc_fence_before();
@@ -385,7 +446,7 @@ struct BwdKVCfg {
     static constexpr int ROWS = (BK == 128) ? 1 : 2;   // key blocks per tile
     static constexpr uint32_t TBYTES = M * HD * 2;     // K or V tile
     static constexpr uint32_t QBYTES = BK * HD * 2;    // one query block of Q or dO
-    static constexpr uint32_t STATBYTES = BK * 8;      // (L2, D) per query
+    static constexpr uint32_t STATBYTES = BK * 8;      // L2 of the BK queries, then their D
     static constexpr int ST = 2;
     static constexpr int LIST_CAP = 2048;
     static constexpr uint32_t OFF_K = 0;
@@ -394,9 +455,10 @@ struct BwdKVCfg {
     static constexpr uint32_t OFF_DO = OFF_Q + ST * QBYTES;
     static constexpr uint32_t OFF_STAT = OFF_DO + ST * QBYTES;
     static constexpr uint32_t OFF_LIST = OFF_STAT + ST * STATBYTES;
-    static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_CAP * 4;
-    // barriers: kv_full, q_full[ST], q_empty[ST], s_full, p_full, acc_done, drain
-    static constexpr int NBAR = 1 + 2 * ST + 4;
+    static constexpr uint32_t OFF_SCR = OFF_LIST + LIST_CAP * 4;  // list-merge scratch (ROWS > 1)
+    static constexpr uint32_t OFF_BAR = OFF_SCR + (ROWS > 1 ? ROWS * LIST_CAP * 4 : 0);
+    // barriers: kv_full, q_full[ST], q_empty[ST], s_full, p_full, acc_done, drain, dp_full, ds_full
+    static constexpr int NBAR = 1 + 2 * ST + 6;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
@@ -407,7 +469,7 @@ struct BwdKVCfg {
 };
 
 template <int HD, int BK>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const BackwardParams p)
@@ -442,19 +504,23 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const uint32_t bar_p = bar_s + 8u;
     const uint32_t bar_acc = bar_s + 16u;
     const uint32_t bar_dr = bar_s + 24u;
+    const uint32_t bar_dp = bar_s + 32u;
+    const uint32_t bar_ds = bar_s + 40u;
     uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2] list length
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
     volatile int* abort_cta = misc + 1;
 
     if (threadIdx.x == 0) {
+        mbar_init(bar_dp, 1);
+        mbar_init(bar_ds, 256);
         mbar_init(bar_kv, 1);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_qf(s), 1);
             mbar_init(bar_qe(s), 1);
         }
         mbar_init(bar_s, 1);
-        mbar_init(bar_p, 128);
+        mbar_init(bar_p, 256);
         mbar_init(bar_acc, 1);
         mbar_init(bar_dr, 1);
         *abort_cta = 0;
@@ -464,26 +530,31 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 2 && lane == 0) {  // union of the tile's key blocks' query-block lists
-        UnionWalk<C::ROWS> it;
-        int len = 0;
-        const bool ok = it.init_transposed(p.col_ptr, h * (p.nb + 1), kb, p.nb, p.nnz);
-        if (!ok) atomicOr(p.gflags, kFlagIndex);
-        if (it.any) {
-            for (;;) {
-                int i, bits;
-                bool last, bad;
-                it.next(p.row_idx, i, bits, last, bad);
-                if (bad) atomicOr(p.gflags, kFlagIndex);
-                if (len >= C::LIST_CAP) {
-                    atomicOr(p.gflags, kFlagIndex);
-                    break;
-                }
-                list[len++] = list_pack(i, bits);
-                if (last) break;
+    if (threadIdx.x == 0) {  // K and V of the tile do not depend on the list: load them now
+        mbar_arrive_expect_tx(bar_kv, 2 * C::TBYTES);
+        int kany = 0;  // a missing block loads a present one's rows (finite data, masked)
+#pragma unroll
+        for (int r = 0; r < C::ROWS; ++r)
+            if (kb[r] >= 0) kany = kb[r];
+#pragma unroll
+        for (int r = 0; r < C::ROWS; ++r) {
+            const int32_t krow = (kb[r] >= 0 ? kb[r] : kany) * BK;
+#pragma unroll
+            for (int pn = 0; pn < HD / 64; ++pn) {
+                tma_load_3d(sb + C::OFF_K + pn * (C::M * 128) + r * (BK * 128), &tmK, pn * 64, krow, bh, bar_kv);
+                tma_load_3d(sb + C::OFF_V + pn * (C::M * 128) + r * (BK * 128), &tmV, pn * 64, krow, bh, bar_kv);
             }
         }
-        misc[2] = len;
+    }
+    if (warp == 2) {  // union of the tile's key blocks' query-block lists
+        int lo = INT_MAX;
+#pragma unroll
+        for (int r = 0; r < C::ROWS; ++r)
+            if (kb[r] >= 0 && kb[r] < lo) lo = kb[r];
+        const int n = warp_union_list<C::ROWS>(p.col_ptr, p.row_idx, h * (p.nb + 1), kb, p.nb, p.nnz,
+                                               lo, p.nb - 1, list, C::LIST_CAP,
+                                               reinterpret_cast<int32_t*>(smem + C::OFF_SCR), p.gflags);
+        if (lane == 0) misc[2] = n;
     }
     tc_fence_before();
     __syncthreads();
@@ -495,23 +566,8 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        if (lane == 0 && len == 0) mbar_drain(bar_kv, 0, kDrainNs);  // nothing to do: let K, V land
         if (lane == 0 && len > 0) {
-            mbar_arrive_expect_tx(bar_kv, 2 * C::TBYTES);
-            int kany = 0;  // a missing block loads a present one's rows (finite data, masked)
-#pragma unroll
-            for (int r = 0; r < C::ROWS; ++r)
-                if (kb[r] >= 0) kany = kb[r];
-#pragma unroll
-            for (int r = 0; r < C::ROWS; ++r) {
-                const int32_t krow = (kb[r] >= 0 ? kb[r] : kany) * BK;
-#pragma unroll
-                for (int pn = 0; pn < HD / 64; ++pn) {
-                    tma_load_3d(sb + C::OFF_K + pn * (C::M * 128) + r * (BK * 128), &tmK, pn * 64, krow, bh,
-                                bar_kv);
-                    tma_load_3d(sb + C::OFF_V + pn * (C::M * 128) + r * (BK * 128), &tmV, pn * 64, krow, bh,
-                                bar_kv);
-                }
-            }
             int n = 0;
             for (; n < len; ++n) {
                 const int st = n % C::ST;
@@ -525,8 +581,9 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     tma_load_3d(sb + C::OFF_DO + st * C::QBYTES + pn * (BK * 128), &tmDO, pn * 64, i * BK,
                                 bh, bar_qf(st));
                 }
-                bulk_load(sb + C::OFF_STAT + st * C::STATBYTES, p.stats + (int64_t)bh * p.seq_pad + i * BK,
-                          C::STATBYTES, bar_qf(st));
+                const float* sx = p.stats + ((int64_t)bh * p.ntiles + (i * BK) / 128) * 256 + (i * BK) % 128;
+                bulk_load(sb + C::OFF_STAT + st * C::STATBYTES, sx, BK * 4, bar_qf(st));
+                bulk_load(sb + C::OFF_STAT + st * C::STATBYTES + BK * 4, sx + 128, BK * 4, bar_qf(st));
             }
             if (*abort_cta) {
                 mbar_drain(bar_kv, 0, kDrainNs);
@@ -543,38 +600,58 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
             const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
             bool issued = false;
-            if (mbar_wait(bar_kv, 0, ctl)) {
+            // S^T(n) and dP^T(n) are committed separately so that the element-wise
+            // warps compute P^T while dP^T is still running. Order per element n:
+            // [P^T(n) ready] dV(n); [dS^T(n) ready] S^T(n+1), dK(n), dP^T(n+1).
+            // S^T(n+1) overwrites P^T(n) only after dV(n) and the dS pass have
+            // read it; dP^T(n+1) overwrites dS^T(n) after dK(n) (MMAs of one
+            // thread run in issue order).
+            auto issue_st = [&](int n) {
+                const int st = n % C::ST;
+                if (!mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK), idesc_s,
+                                 kk > 0 ? 1u : 0u);
+                umma_commit(bar_s);
+                issued = true;
+                return true;
+            };
+            auto issue_dpt = [&](int n) {  // stage already waited for by issue_st(n)
+                const int st = n % C::ST;
+                const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
+                                 idesc_s, kk > 0 ? 1u : 0u);
+                umma_commit(bar_dp);
+            };
+            if (mbar_wait(bar_kv, 0, ctl) && issue_st(0)) {
+                issue_dpt(0);
                 for (int n = 0; n < len; ++n) {
                     const int st = n % C::ST;
-                    if (!mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl)) break;
-                    tc_fence_after();
-                    const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
-                    const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK),
-                                     idesc_s, kk > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
-                                     idesc_s, kk > 0 ? 1u : 0u);
-                    umma_commit(bar_s);
-                    issued = true;
+                    const bool more = n + 1 < len;
                     if (!mbar_wait(bar_p, n & 1, ctl)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, bdo, idesc_a,
+                        umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
                                      (n > 0 || kk > 0) ? 1u : 0u);
                     }
+                    if (!mbar_wait(bar_ds, n & 1, ctl)) break;
+                    tc_fence_after();
+                    if (more && !issue_st(n + 1)) break;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8, bq, idesc_a,
+                        umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + packed_col<BK>(kk), bq, idesc_a,
                                      (n > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(bar_qe(st));
+                    if (more) issue_dpt(n + 1);
                 }
                 if (!*abort_cta) umma_commit(bar_acc);
             }
@@ -585,8 +662,9 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
         __syncwarp();
     } else if (warp >= 4) {
-        // ------------------------------------------------------------ element-wise pass + epilogue
-        const int quad = warp & 3;
+        // ------------------------------------------------------------ element-wise passes + epilogue
+        constexpr int HALF = BK / 2;  // query columns per warpgroup
+        const int quad = warp & 3, g = (warp - 4) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const int kbit = (BK == 128) ? 0 : (r >> 6);
@@ -604,71 +682,81 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 break;
             }
             tc_fence_after();
-            const float2* stat = reinterpret_cast<const float2*>(smem + C::OFF_STAT + st * C::STATBYTES);
+            const float* sx = reinterpret_cast<const float*>(smem + C::OFF_STAT + st * C::STATBYTES) + g * HALF;
+            const float* sy = sx + BK;
             const bool vis = row_valid && ((list_bits(ent) >> kbit) & 1);
-            const int lim = kpos - list_j(ent) * BK;  // query column c visible iff c >= lim (k <= q)
-            // 64 columns at a time; P^T and dS^T of chunk ch (bf16 pairs) go to
-            // columns 32 ch .. 32 ch + 31 of S^T and dP^T, which are already read.
+            const int lim = kpos - list_j(ent) * BK - g * HALF;  // column c of this half visible iff c >= lim
+            // P pass (needs S^T only): P^T as bf16 pairs over the first HALF/2
+            // columns of this half of S^T (already read), kept in registers too
+            uint32_t sr[HALF], pk[HALF / 2];
+            tmem_ld_cols<HALF>(tl + C::COL_S + g * HALF, sr);
+            tmem_wait_ld();
 #pragma unroll
-            for (int ch = 0; ch < BK / 64; ++ch) {
-                uint32_t sr[64], dp[64];
-                tmem_ld32(tl + C::COL_S + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(tl + C::COL_S + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_ld32(tl + C::COL_DP + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-                tmem_ld32(tl + C::COL_DP + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const int qc = 64 * ch + c;
-                    const float2 s0 = stat[qc], s1 = stat[qc + 1];
-                    const float p0 = (vis && qc >= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -s0.x)) : 0.f;
-                    const float p1 = (vis && qc + 1 >= lim) ? ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -s1.x)) : 0.f;
-                    const float d0 = p0 * (__uint_as_float(dp[c]) - s0.y);
-                    const float d1 = p1 * (__uint_as_float(dp[c + 1]) - s1.y);
-                    sr[c / 2] = pack_bf16x2(p0, p1);
-                    dp[c / 2] = pack_bf16x2(d0, d1);
-                }
-                tmem_st32(tl + C::COL_S + 32 * ch, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
-                tmem_st32(tl + C::COL_DP + 32 * ch, *reinterpret_cast<const uint32_t(*)[32]>(&dp[0]));
+            for (int c = 0; c < HALF; c += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(sx + c);
+                const float p0 = (vis && c >= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -x.x)) : 0.f;
+                const float p1 = (vis && c + 1 >= lim) ? ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -x.y)) : 0.f;
+                const float p2 = (vis && c + 2 >= lim) ? ex2(fmaf(__uint_as_float(sr[c + 2]), sc, -x.z)) : 0.f;
+                const float p3 = (vis && c + 3 >= lim) ? ex2(fmaf(__uint_as_float(sr[c + 3]), sc, -x.w)) : 0.f;
+                pk[c / 2] = pack_bf16x2(p0, p1);
+                pk[c / 2 + 1] = pack_bf16x2(p2, p3);
             }
+            tmem_st_cols<HALF / 2>(tl + C::COL_S + g * HALF, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p);
+            if (!warp_wait(bar_dp, n & 1, ctl)) {
+                fail = true;
+                break;
+            }
+            tc_fence_after();
+            // dS pass: dS^T = P^T (dP^T - D) over the first HALF/2 columns of this half of dP^T
+            tmem_ld_cols<HALF>(tl + C::COL_DP + g * HALF, sr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < HALF; c += 4) {
+                const float4 y = *reinterpret_cast<const float4*>(sy + c);
+                const float d0 = bf16lo(pk[c / 2]) * (__uint_as_float(sr[c]) - y.x);
+                const float d1 = bf16hi(pk[c / 2]) * (__uint_as_float(sr[c + 1]) - y.y);
+                const float d2 = bf16lo(pk[c / 2 + 1]) * (__uint_as_float(sr[c + 2]) - y.z);
+                const float d3 = bf16hi(pk[c / 2 + 1]) * (__uint_as_float(sr[c + 3]) - y.w);
+                pk[c / 2] = pack_bf16x2(d0, d1);
+                pk[c / 2 + 1] = pack_bf16x2(d2, d3);
+            }
+            tmem_st_cols<HALF / 2>(tl + C::COL_DP + g * HALF, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_ds);
         }
         if (!fail) {
+            // warpgroup 0 stores dV, warpgroup 1 stores dK (times the scale)
             const int64_t row = (int64_t)bh * p.seq + kpos;
+            uint16_t* grow = (g == 0 ? p.dv : p.dk) + row * HD;
             if (len > 0) {
                 if (warp_wait(bar_acc, 0, ctl)) {
                     tc_fence_after();
+                    const float f = g == 0 ? 1.0f : p.scale;
+                    const uint32_t col = g == 0 ? C::COL_DV : C::COL_DK;
 #pragma unroll
-                    for (int w = 0; w < 2; ++w) {
-                        uint16_t* grow = (w == 0 ? p.dv : p.dk) + row * HD;
-                        const float f = w == 0 ? 1.0f : p.scale;
-                        const uint32_t col = w == 0 ? C::COL_DV : C::COL_DK;
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tl + col + 32 * c, o);
+                        tmem_wait_ld();
+                        if (row_valid) {
 #pragma unroll
-                        for (int c = 0; c < HD / 32; ++c) {
-                            uint32_t o[32];
-                            tmem_ld32(tl + col + 32 * c, o);
-                            tmem_wait_ld();
-                            if (row_valid) {
-#pragma unroll
-                                for (int e2 = 0; e2 < 32; e2 += 8) {
-                                    uint4 v;
-                                    v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * f, __uint_as_float(o[e2 + 1]) * f);
-                                    v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * f, __uint_as_float(o[e2 + 3]) * f);
-                                    v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * f, __uint_as_float(o[e2 + 5]) * f);
-                                    v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * f, __uint_as_float(o[e2 + 7]) * f);
-                                    *reinterpret_cast<uint4*>(grow + 32 * c + e2) = v;
-                                }
+                            for (int e2 = 0; e2 < 32; e2 += 8) {
+                                uint4 v;
+                                v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * f, __uint_as_float(o[e2 + 1]) * f);
+                                v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * f, __uint_as_float(o[e2 + 3]) * f);
+                                v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * f, __uint_as_float(o[e2 + 5]) * f);
+                                v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * f, __uint_as_float(o[e2 + 7]) * f);
+                                *reinterpret_cast<uint4*>(grow + 32 * c + e2) = v;
                             }
                         }
                     }
                 }
             } else if (row_valid) {  // no query block lists this tile's key blocks
-                for (int d = 0; d < HD; d += 8) {
-                    *reinterpret_cast<uint4*>(p.dk + row * HD + d) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(p.dv + row * HD + d) = make_uint4(0, 0, 0, 0);
-                }
+                for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(grow + d) = make_uint4(0, 0, 0, 0);
             }
         }
         tc_fence_before();

@@ -128,4 +128,79 @@ struct UnionWalk {
     }
 };
 
+// Warp-cooperative version of the walk, for a list built once per CTA before
+// the main loop: all 32 lanes copy the CSR rows rows[0..ROWS-1] (coalesced)
+// into `scratch` (ROWS * cap ints) and lane 0 merges them from shared memory,
+// which avoids a dependent global load per element. Writes the tagged union
+// into `list` and returns its length on every lane. Rows outside [0, nb) are
+// absent; offsets outside [0, nnz], lists longer than cap and elements
+// outside [lo, hi] set kFlagIndex (a bad element becomes lo with no tags).
+template <int ROWS>
+__device__ __forceinline__ int warp_union_list(const int32_t* row_ptr, const int32_t* col, int rp,
+                                               const int* rows, int nb, int64_t nnz, int lo, int hi,
+                                               uint32_t* list, int cap, int32_t* scratch,
+                                               uint32_t* gflags)
+{
+    const int lane = threadIdx.x & 31;
+    int a[ROWS], n[ROWS];
+    bool ok = true;
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+        a[r] = n[r] = 0;
+        if (rows[r] >= 0 && rows[r] < nb) {
+            const int b0 = __ldg(row_ptr + rp + rows[r]), b1 = __ldg(row_ptr + rp + rows[r] + 1);
+            ok = ok && b0 >= 0 && b0 <= b1 && b1 <= nnz && b1 - b0 <= cap;
+            a[r] = b0;
+            n[r] = b1 - b0;
+        }
+    }
+    if (!ok) {
+        if (lane == 0) atomicOr(gflags, kFlagIndex);
+        return 0;
+    }
+    auto checked = [&](int j, int bits) {
+        if (j < lo || j > hi) {
+            atomicOr(gflags, kFlagIndex);
+            return list_pack(lo, 0);
+        }
+        return list_pack(j, bits);
+    };
+    if (ROWS == 1) {
+        for (int t = lane; t < n[0]; t += 32) list[t] = checked(__ldg(col + a[0] + t), 1);
+        __syncwarp();
+        return n[0];
+    }
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+        for (int t = lane; t < n[r]; t += 32) scratch[r * cap + t] = __ldg(col + a[r] + t);
+    __syncwarp();
+    int len = 0;
+    if (lane == 0) {
+        int i[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) i[r] = 0;
+        for (;;) {
+            int jm = INT_MAX;
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r)
+                if (i[r] < n[r]) jm = min(jm, scratch[r * cap + i[r]]);
+            if (jm == INT_MAX) break;
+            int bits = 0;
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r)
+                if (i[r] < n[r] && scratch[r * cap + i[r]] == jm) {
+                    bits |= 1 << r;
+                    ++i[r];
+                }
+            if (len >= cap) {  // cannot happen for ascending lists with nb <= cap
+                atomicOr(gflags, kFlagIndex);
+                break;
+            }
+            list[len++] = checked(jm, bits);
+        }
+    }
+    __syncwarp();
+    return __shfl_sync(0xffffffffu, len, 0);
+}
+
 }  // namespace s2

@@ -174,9 +174,9 @@ int launch_backward(const void* q, const void* k, const void* v, s2::BackwardPar
     s2::s2_bwd_stats_kernel<HD><<<(unsigned)grid0, 256, 0, stream>>>(bp);
     if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
     const uint64_t tiles = planes * (uint64_t)bp.ntiles;
-    kq<<<(unsigned)tiles, 256, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
+    kq<<<(unsigned)tiles, 384, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
     if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
-    kkv<<<(unsigned)tiles, 256, CK::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
+    kkv<<<(unsigned)tiles, 384, CK::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
@@ -353,7 +353,7 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
     bp.o = static_cast<const uint16_t*>(o);
     bp.dout = static_cast<const uint16_t*>(dout);
     bp.lse = lse;
-    bp.stats = static_cast<float2*>(workspace);
+    bp.stats = static_cast<float*>(workspace);
     bp.dq = static_cast<uint16_t*>(dq);
     bp.dk = static_cast<uint16_t*>(dk);
     bp.dv = static_cast<uint16_t*>(dv);
