@@ -168,8 +168,8 @@ struct BwdQCfg {
     static constexpr uint32_t OFF_SCR = OFF_LIST + LIST_CAP * 4;  // list-merge scratch (ROWS > 1)
     static constexpr uint32_t OFF_BAR = OFF_SCR + (ROWS > 1 ? ROWS * LIST_CAP * 4 : 0);
     // barriers: qd_full, k_full[ST], v_full[ST], kv_empty[ST], s_full, ds_full, acc_done, drain,
-    // dp_full
-    static constexpr int NBAR = 1 + 3 * ST + 5;
+    // dp_full, s_free
+    static constexpr int NBAR = 1 + 3 * ST + 6;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
@@ -204,6 +204,7 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t bar_acc = bar_s + 16u;
     const uint32_t bar_dr = bar_s + 24u;
     const uint32_t bar_dp = bar_s + 32u;
+    const uint32_t bar_sfree = bar_s + 40u;
     uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2] list length
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
@@ -211,6 +212,7 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
     if (threadIdx.x == 0) {
         mbar_init(bar_dp, 1);
+        mbar_init(bar_sfree, 256);
         mbar_init(bar_qd, 1);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_kf(s), 1);
@@ -292,9 +294,10 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             bool issued = false;
             // S(n) and dP(n) are committed separately so that the element-wise
             // warps start on P while dP is still running. Order per element n:
-            // [dS(n) ready] S(n+1), dQ(n), dP(n+1): S(n+1) only overwrites S(n),
-            // which the warps have finished with; dS(n) sits in dP's columns
-            // and dP(n+1) is issued after dQ(n) has read it.
+            // [S(n) read out] S(n+1); [dS(n) ready] dQ(n), dP(n+1). The warps
+            // keep P in registers, so S(n+1) may overwrite S(n) as soon as they
+            // have loaded it; dS(n) sits in dP's columns and dP(n+1) is issued
+            // after dQ(n) has read it.
             auto issue_s = [&](int n) {
                 const int st = n % C::ST;
                 if (!mbar_wait(bar_kf(st), (n / C::ST) & 1, ctl)) return false;
@@ -324,9 +327,13 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 for (int n = 0; n < len; ++n) {
                     const int st = n % C::ST;
                     const bool more = n + 1 < len;
+                    if (more) {
+                        if (!mbar_wait(bar_sfree, n & 1, ctl)) break;
+                        tc_fence_after();
+                        if (!issue_s(n + 1)) break;
+                    }
                     if (!mbar_wait(bar_ds, n & 1, ctl)) break;
                     tc_fence_after();
-                    if (more && !issue_s(n + 1)) break;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t bk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
@@ -374,6 +381,8 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             uint32_t sr[HALF], pk[HALF / 2];
             tmem_ld_cols<HALF>(tl + C::COL_S + g * HALF, sr);
             tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar_sfree);  // S(n) is in registers: S(n+1) may be written
 #pragma unroll
             for (int c = 0; c < HALF; c += 2) {
                 const float p0 = (vis && c <= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -lx)) : 0.f;
@@ -602,10 +611,10 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             bool issued = false;
             // S^T(n) and dP^T(n) are committed separately so that the element-wise
             // warps compute P^T while dP^T is still running. Order per element n:
-            // [P^T(n) ready] dV(n); [dS^T(n) ready] S^T(n+1), dK(n), dP^T(n+1).
-            // S^T(n+1) overwrites P^T(n) only after dV(n) and the dS pass have
-            // read it; dP^T(n+1) overwrites dS^T(n) after dK(n) (MMAs of one
-            // thread run in issue order).
+            // [P^T(n) ready] dV(n), S^T(n+1); [dS^T(n) ready] dK(n), dP^T(n+1).
+            // S^T(n+1) overwrites P^T(n) after dV(n) has read it (MMAs of one
+            // thread run in issue order; the warps keep P in registers for the
+            // dS pass); dP^T(n+1) overwrites dS^T(n) after dK(n).
             auto issue_st = [&](int n) {
                 const int st = n % C::ST;
                 if (!mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl)) return false;
@@ -641,9 +650,9 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
                                      (n > 0 || kk > 0) ? 1u : 0u);
                     }
+                    if (more && !issue_st(n + 1)) break;
                     if (!mbar_wait(bar_ds, n & 1, ctl)) break;
                     tc_fence_after();
-                    if (more && !issue_st(n + 1)) break;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
