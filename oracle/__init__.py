@@ -54,6 +54,9 @@ def _load():
     lib.s2o_decode_items.restype = i32
     lib.s2o_decode_items.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
                                      i64, vp, dbl, i64, vp, vp, vp, i32]
+    lib.s2o_chunk_rows.restype = i32
+    lib.s2o_chunk_rows.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64,
+                                   i64, vp, i64, vp, dbl, vp, vp, i32]
     lib.s2o_backward.restype = i32
     lib.s2o_backward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, vp, i64,
                                  vp, dbl, vp, vp, vp, i32]
@@ -278,3 +281,35 @@ def backward(q, k, v, dout, B, scale, S=None, L=None, dense_heads=None, bmask=No
     if rc != 0:
         raise ValueError("oracle backward rejected its arguments")
     return dq, dk, dv
+
+
+def chunk(q, k_cache, v_cache, block_table, ctx_lens, q_start, B, scale, S=None, L=None,
+          dense_heads=None, bmask=None, nthreads=0):
+    """Oracle chunked prefill over a paged cache.
+
+    q: [total_q, H, D] packed chunk rows (sequence s owns rows
+    q_start[s]..q_start[s+1]-1, the last tokens of its ctx_lens[s]-token
+    context); caches [pages, Hkv, page_size, D]. Returns (out [total_q, H, D],
+    lse [total_q, H]).
+    """
+    q, kc, vc = _bits(q), _bits(k_cache), _bits(v_cache)
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    cl = np.ascontiguousarray(np.asarray(ctx_lens, dtype=np.int32))
+    qs = np.ascontiguousarray(np.asarray(q_start, dtype=np.int32))
+    total_q, H, D = q.shape
+    _, Hkv, page_size, D2 = kc.shape
+    assert D2 == D and vc.shape == kc.shape and qs[-1] == total_q
+    batch = cl.size
+    if bmask is not None:
+        bm = np.ascontiguousarray(np.asarray(bmask, dtype=np.uint8))
+        nbm, S_, L_, d = bm.shape[1], 0, 0, None
+    else:
+        bm, nbm, S_, L_, d = None, 0, int(S), int(L), _dense(H, dense_heads)
+    out = np.zeros((total_q, H, D), dtype=np.float64)
+    lse = np.empty((total_q, H), dtype=np.float64)
+    rc = _load().s2o_chunk_rows(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), _ptr(cl), _ptr(qs), batch, H,
+                                Hkv, D, page_size, bt.shape[1], B, S_, L_, _ptr(d), nbm, _ptr(bm),
+                                float(scale), _ptr(out), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle chunk rejected its arguments")
+    return out, lse

@@ -136,10 +136,10 @@ void s2o_range_block_mask(int64_t H, int64_t nb, const int64_t* range_ptr, const
 /* ------------------------------------------------------------------------- */
 
 typedef struct {
-    int kind; /* 0 = prefill rows, 1 = decode items, 2 = backward planes */
+    int kind; /* 0 = prefill rows, 1 = decode items, 2 = backward planes, 3 = chunk rows */
     const uint16_t *q, *k, *v, *dout;
     double *dq, *dk, *dv; /* backward outputs */
-    const int32_t *block_table, *ctx_lens;
+    const int32_t *block_table, *ctx_lens, *q_start;
     int64_t batch, H, seq, D, B, S, L, page_size, max_pages;
     const uint8_t* dense;
     const uint8_t* bmask; /* NULL: the block rule above; else [H][nbm][nbm] */
@@ -210,26 +210,22 @@ static void prefill_row(const job_t* J, int64_t r, double* s, double* qd,
     *lse = m + log(den);
 }
 
-/* Decode item e = seq_index * H + h: the query of sequence s sits at position
- * n-1 (n = ctx_lens[s]) and sees keys 0..n-1, token t being row t % page_size
- * of page block_table[s][t / page_size] in a [pages][Hkv][page_size][D] cache,
- * key/value head h / (H / Hkv). */
-static int decode_item(const job_t* J, int64_t e, double* s, double* qd,
-                       double* out, double* lse)
+/* One query of sequence sq and head h at position pos of a paged context:
+ * keys 0..pos, token t being row t % page_size of page block_table[sq][t /
+ * page_size] in a [pages][Hkv][page_size][D] cache, key/value head
+ * h / (H / Hkv). Q points at the query's D bf16 values. */
+static int paged_row(const job_t* J, int64_t sq, int64_t h, int64_t pos, const uint16_t* Q,
+                     double* s, double* qd, double* out, double* lse)
 {
     const int64_t D = J->D, H = J->H, P = J->page_size;
-    const int64_t sq = e / H, h = e % H;
-    const int64_t n = J->ctx_lens[sq];
-    if (n < 1) return -1;
-    const int64_t i = (n - 1) / J->B;
+    const int64_t i = pos / J->B;
     const int dense = J->dense ? J->dense[h] != 0 : 0;
     const int64_t Hkv = J->Hkv, kvh = h / (H / Hkv);
-    const uint16_t* Q = J->q + e * D;
 
     for (int64_t d = 0; d < D; ++d) qd[d] = bf16_bits_to_double(Q[d]);
 
     double m = -INFINITY;
-    for (int64_t k = 0; k < n; ++k) {
+    for (int64_t k = 0; k <= pos; ++k) {
         if (!visible(J, h, i, k / J->B, dense)) continue;
         const int64_t page = J->block_table[sq * J->max_pages + k / P];
         if (page < 0) return -1;
@@ -241,7 +237,7 @@ static int decode_item(const job_t* J, int64_t e, double* s, double* qd,
     }
     double den = 0.0;
     for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
-    for (int64_t k = 0; k < n; ++k) {
+    for (int64_t k = 0; k <= pos; ++k) {
         if (!visible(J, h, i, k / J->B, dense)) continue;
         const int64_t page = J->block_table[sq * J->max_pages + k / P];
         const uint16_t* Vrow = J->v + ((page * Hkv + kvh) * P + k % P) * D;
@@ -256,6 +252,32 @@ static int decode_item(const job_t* J, int64_t e, double* s, double* qd,
     for (int64_t d = 0; d < D; ++d) out[d] /= den;
     *lse = m + log(den);
     return 0;
+}
+
+/* Decode item e = seq_index * H + h: the query of sequence s sits at position
+ * n-1 (n = ctx_lens[s]) and sees keys 0..n-1 of its paged context. */
+static int decode_item(const job_t* J, int64_t e, double* s, double* qd,
+                       double* out, double* lse)
+{
+    const int64_t sq = e / J->H, h = e % J->H;
+    const int64_t n = J->ctx_lens[sq];
+    if (n < 1) return -1;
+    return paged_row(J, sq, h, n - 1, J->q + e * J->D, s, qd, out, lse);
+}
+
+/* Chunk item e = t * H + h, t a row of the packed chunk queries: sequence sq
+ * holds rows q_start[sq] .. q_start[sq+1]-1, its last chunk of a context of
+ * n = ctx_lens[sq] tokens, so row t sits at position n - (q_start[sq+1] - t). */
+static int chunk_item(const job_t* J, int64_t e, double* s, double* qd, double* out,
+                      double* lse)
+{
+    const int64_t t = e / J->H, h = e % J->H;
+    int64_t sq = 0;
+    while (sq + 1 < J->batch && J->q_start[sq + 1] <= t) ++sq;
+    const int64_t n = J->ctx_lens[sq];
+    const int64_t pos = n - (J->q_start[sq + 1] - t);
+    if (pos < 0 || pos >= n) return -1;
+    return paged_row(J, sq, h, pos, J->q + e * J->D, s, qd, out, lse);
 }
 
 /* Backward item e = b * Hkv + g: every query head h of K/V head g (h / (H / Hkv)
@@ -326,7 +348,7 @@ static void backward_plane(const job_t* J, int64_t e, double* s, double* p, doub
 static void* worker(void* arg)
 {
     job_t* J = (job_t*)arg;
-    const int64_t span = J->kind == 1 ? J->max_pages * J->page_size : J->seq;
+    const int64_t span = (J->kind == 1 || J->kind == 3) ? J->max_pages * J->page_size : J->seq;
     double* s = (double*)malloc(sizeof(double) * (size_t)(span > 0 ? span : 1));
     double* p = (double*)malloc(sizeof(double) * (size_t)(span > 0 ? span : 1));
     double* qd = (double*)malloc(sizeof(double) * (size_t)J->D);
@@ -353,7 +375,8 @@ static void* worker(void* arg)
         double* lse = J->lse + t;
         if (J->kind == 0) {
             prefill_row(J, id, s, qd, out, lse);
-        } else if (decode_item(J, id, s, qd, out, lse) != 0) {
+        } else if ((J->kind == 1 ? decode_item(J, id, s, qd, out, lse)
+                                 : chunk_item(J, id, s, qd, out, lse)) != 0) {
             pthread_mutex_lock(&J->lock);
             J->failed = 1;
             pthread_mutex_unlock(&J->lock);
@@ -538,5 +561,42 @@ int s2o_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const 
     J.batch = batch; J.H = H; J.Hkv = Hkv; J.seq = seq; J.D = D; J.B = B;
     J.S = S; J.L = L; J.dense = dense; J.bmask = bmask; J.nbm = nbm; J.scale = scale;
     J.n_items = batch * Hkv; J.items = NULL;
+    return run_job(&J, nthreads);
+}
+
+/* Chunked-prefill oracle: each sequence s appends a chunk of
+ * q_start[s+1] - q_start[s] query tokens at the end of a paged context of
+ * ctx_lens[s] tokens (the chunk's own keys and values already in the cache);
+ * every chunk row attends to keys 0..its position under the HHST rule
+ * (bmask == NULL; S, L, dense) or a block mask [H][nbm][nbm].
+ * q: [total_q][H][D] packed rows (total_q = q_start[batch]); caches
+ * [num_pages][Hkv][page_size][D]; out [total_q][H][D], lse [total_q][H].
+ * Returns 0 or -1 (a chunk longer than its context, a bad page id, ...). */
+int s2o_chunk_rows(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                   const int32_t* block_table, const int32_t* ctx_lens, const int32_t* q_start,
+                   int64_t batch, int64_t H, int64_t Hkv, int64_t D, int64_t page_size,
+                   int64_t max_pages, int64_t B, int64_t S, int64_t L, const uint8_t* dense,
+                   int64_t nbm, const uint8_t* bmask, double scale, double* out, double* lse,
+                   int nthreads)
+{
+    if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !q_start || !out || !lse ||
+        batch < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || D < 1 || page_size < 1 ||
+        max_pages < 1 || B < 1 || q_start[0] != 0)
+        return -1;
+    if (bmask ? nbm < 1 : (S < 1 || L < 1)) return -1;
+    for (int64_t s = 0; s < batch; ++s) {
+        const int64_t ql = q_start[s + 1] - q_start[s];
+        if (ql < 0 || ctx_lens[s] < ql || ctx_lens[s] > max_pages * page_size) return -1;
+        if (bmask && ctx_lens[s] > 0 && (ctx_lens[s] - 1) / B >= nbm) return -1;
+    }
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.kind = 3;
+    J.q = q; J.k = k_cache; J.v = v_cache;
+    J.block_table = block_table; J.ctx_lens = ctx_lens; J.q_start = q_start;
+    J.batch = batch; J.H = H; J.Hkv = Hkv; J.D = D; J.page_size = page_size;
+    J.max_pages = max_pages; J.B = B; J.S = S; J.L = L; J.dense = dense;
+    J.bmask = bmask; J.nbm = nbm; J.scale = scale;
+    J.n_items = q_start[batch] * H; J.items = NULL; J.out = out; J.lse = lse;
     return run_job(&J, nthreads);
 }
