@@ -76,6 +76,29 @@ def decode_counts(lay, w, ctx_lens):
     return tokens, pages
 
 
+def chunk_flops(lay, w, ctx_lens, qlens) -> int:
+    """Algorithmic FLOPs of a chunked prefill: 4*D per visible (chunk row, key)
+    pair, a row at position pos seeing B keys of each listed block below its own
+    block and pos - i*B + 1 keys of its own block i when listed."""
+    H, nb, B = lay.heads, lay.num_blocks, w.block
+    nfull = np.zeros((H, nb), dtype=np.int64)
+    diag = np.zeros((H, nb), dtype=np.int64)
+    for h in range(H):
+        for i in range(nb):
+            r = lay.row(h, i)
+            nfull[h, i] = int((r < i).sum())
+            diag[h, i] = int((r == i).any())
+    pairs = 0
+    for n, ql in zip(ctx_lens, qlens):
+        c0 = n - ql
+        for i in range(c0 // B, (n - 1) // B + 1 if ql else 0):
+            a, b = max(c0, i * B), min(n, (i + 1) * B)
+            rows = b - a
+            tri = (a - i * B + 1 + b - i * B) * rows // 2  # sum of pos - iB + 1 over the rows
+            pairs += int((rows * nfull[:, i] * B + diag[:, i] * tri).sum())
+    return 4 * w.head_dim * pairs
+
+
 def source_sha() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "head_heterogeneous_block_s2_b200", "csrc")
@@ -350,15 +373,51 @@ def run_ours(args, rank, world, dist):
         bflops = prefill_flops(lay_b, wb)
         bwd_info = (wb, bflops, prefill_issued_flops(lay_b, wb))
 
+    # ---------------- chunked prefill over the paged cache, timed on its own
+    chunk_ms, chunk_steps, chunk_info = 0.0, 0, None
+    if args.chunk != "none":
+        wc = synth.CHUNK_WORKLOADS[args.chunk]
+        ci = synth.chunk_inputs(wc, synth.CHUNK_LEN[wc.name], device=dev)
+        nb_c = -(-wc.ctx_max // wc.block)
+        lay_c = s2attn.build_layout(wc.heads, wc.block, wc.stride, wc.local, nb_c, wc.dense_heads,
+                                    device=dev)
+        cout = torch.empty_like(ci.q)
+
+        def chunk_call():
+            s2attn.chunk_prefill(ci.q, ci.k_cache, ci.v_cache, ci.block_table, ci.ctx_lens,
+                                 ci.q_start, lay_c, ci.max_q_len, scale=wc.scale, out=cout)
+
+        for _ in range(3):
+            chunk_call()
+        torch.cuda.synchronize()
+        chunk_steps = max(3, min(args.steps, args.bwd_steps))
+        cev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        if dist:
+            dist.barrier()
+        cev[0].record(stream)
+        for _ in range(chunk_steps):
+            chunk_call()
+        cev[1].record(stream)
+        torch.cuda.synchronize()
+        chunk_ms = cev[0].elapsed_time(cev[1])
+        rc, flags = s2attn.device_status(reset=True)
+        if rc != 0:
+            raise RuntimeError(f"device flags {flags:#x} after the chunked prefill")
+        ctx_h = ci.ctx_lens.cpu().tolist()
+        qs = ci.q_start.cpu().tolist()
+        qlens = [qs[i + 1] - qs[i] for i in range(len(ctx_h))]
+        chunk_info = (wc, chunk_flops(lay_c, wc, ctx_h, qlens), sum(qlens))
+        del ci, cout
+
     # ---------------- max over ranks
-    vals = [total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms]
+    vals = [total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms, chunk_ms]
     if dist:
         import torch.distributed as tdist
 
         t = torch.tensor(vals, dtype=torch.float64, device=dev)
         tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
         vals = t.tolist()
-    total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms = vals
+    total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms, chunk_ms = vals
     clocks = sampler.summary()
     if rank != 0:
         return None
@@ -462,6 +521,27 @@ def run_ours(args, rank, world, dist):
                          "peak_source": f"{peak_src} bf16_tflops_sustained"},
         }
         line["gpu_launches_backward"] = 3 * bwd_steps
+    if chunk_info is not None:
+        wc, cflops, total_q = chunk_info
+        per = cflops / (chunk_ms / chunk_steps * 1e-3) / 1e12
+        line["chunk"] = {
+            "value": round(world * cflops * chunk_steps / (chunk_ms * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s",
+            "workload": wc.name,
+            "ms_per_call": round(chunk_ms / chunk_steps, 4),
+            "steps": chunk_steps,
+            "chunk_rows": total_q,
+            "algorithmic_gflop_per_call": round(cflops / 1e9, 3),
+            "config": {"batch": wc.batch, "heads": wc.heads, "head_dim": wc.head_dim,
+                       "ctx": [wc.ctx_min, wc.ctx_max], "chunk": synth.CHUNK_LEN[wc.name],
+                       "page": wc.page_size, "block": wc.block, "stride": wc.stride,
+                       "local": wc.local},
+            "kernels": "s2_chunk_prefill_kernel",
+            "roofline": {"bound": "tensor", "achieved": round(per, 2), "peak": tc_peak,
+                         "unit": "TFLOP/s", "frac": round(per / tc_peak, 4),
+                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
+        }
+        line["gpu_launches_chunk"] = chunk_steps
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wp, args.cpu_seconds)
     return line
@@ -560,6 +640,8 @@ def main():
                     help="prefill workload whose backward is timed separately ('same' = the "
                          "prefill workload, 'none' = skip)")
     ap.add_argument("--bwd-steps", type=int, default=20)
+    ap.add_argument("--chunk", default="chunk_paged", choices=["chunk_paged", "none"],
+                    help="chunked prefill over the paged cache, timed separately")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -16,6 +16,7 @@
 #include "s2attn.h"
 #include "ptx.cuh"
 #include "backward_sm100.cuh"
+#include "chunk_sm100.cuh"
 #include "decode.cuh"
 #include "prefill_pair_sm100.cuh"
 
@@ -41,6 +42,7 @@ struct DevInfo {
     bool prefill_attr_done[4] = {false, false, false, false};
     bool decode_attr_done[2] = {false, false};
     bool backward_attr_done[4] = {false, false, false, false};
+    bool chunk_attr_done[4] = {false, false, false, false};
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -101,6 +103,20 @@ int make_map(CUtensorMap* m, const void* base, uint64_t planes, uint64_t seq, ui
     const cuuint64_t dims[3] = {cols, seq, planes};
     const cuuint64_t strides[2] = {cols * 2, seq * cols * 2};
     const cuuint32_t box[3] = {64, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? S2_OK : S2_ERR_CUDA;
+}
+
+// Packed chunk rows [rows][heads][cols]: one head's 128 consecutive rows per box.
+int make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads, uint64_t cols)
+{
+    const cuuint64_t dims[3] = {cols, heads, rows};
+    const cuuint64_t strides[2] = {cols * 2, heads * cols * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -177,6 +193,34 @@ int launch_backward(const void* q, const void* k, const void* v, s2::BackwardPar
     kq<<<(unsigned)tiles, 384, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
     if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
     kkv<<<(unsigned)tiles, 384, CK::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
+    return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
+}
+
+// Chunked prefill: one CTA per (tile slot, head, sequence); slots past a
+// sequence's chunk exit at once.
+template <int HD, int BK>
+int launch_chunk(const void* q, const void* kc, const void* vc, s2::ChunkParams& cp, int dev, int attr_slot,
+                 cudaStream_t stream)
+{
+    using C = s2::ChunkCfg<HD, BK>;
+    CUtensorMap mq, mk, mv;
+    const uint64_t planes = (uint64_t)cp.num_pages * cp.heads_kv;
+    if (make_rows_map(&mq, q, (uint64_t)cp.total_q, cp.heads, HD) ||
+        make_map(&mk, kc, planes, s2::kChunkPage, HD, s2::kChunkPage) ||
+        make_map(&mv, vc, planes, s2::kChunkPage, HD, s2::kChunkPage))
+        return S2_ERR_CUDA;
+    auto kern = s2::s2_chunk_prefill_kernel<HD, BK>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_dev[dev].chunk_attr_done[attr_slot]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
+                cudaSuccess)
+                return S2_ERR_CUDA;
+            g_dev[dev].chunk_attr_done[attr_slot] = true;
+        }
+    }
+    const dim3 grid((unsigned)((cp.max_q_len + 127) / 128 + 1), (unsigned)cp.heads, (unsigned)cp.batch);
+    kern<<<grid, 256, C::SMEM_ALLOC, stream>>>(mq, mk, mv, cp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
@@ -381,6 +425,61 @@ int s2_attn_prefill(const void* q, const void* k, const void* v, void* o, float*
 {
     return s2_attn_prefill_gqa(q, k, v, o, lse, batch, heads, heads, seq, head_dim, scale,
                                block_size, num_blocks, row_ptr, col_idx, nnz, stream);
+}
+
+int s2_attn_chunk_prefill(const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_table, const int32_t* ctx_lens, const int32_t* q_start,
+                          int32_t batch, int32_t heads, int32_t heads_kv, int32_t head_dim,
+                          int32_t page_size, int32_t max_pages, int64_t num_pages, int32_t max_q_len,
+                          int64_t total_q, int32_t block_size, int32_t num_blocks,
+                          const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz, float scale,
+                          void* out, float* lse, void* stream)
+{
+    if (!q || !k_cache || !v_cache || !block_table || !ctx_lens || !q_start || !row_ptr ||
+        (!col_idx && nnz > 0) || !out)
+        return S2_ERR_INVALID_ARG;
+    if (batch < 1 || heads < 1 || max_pages < 1 || num_pages < 1 || num_blocks < 1 || nnz < 0 ||
+        max_q_len < 1 || total_q < 1 || !std::isfinite(scale) || !(scale > 0.f))
+        return S2_ERR_INVALID_ARG;
+    if (heads_kv < 1 || heads % heads_kv != 0) return S2_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
+    if (page_size != s2::kChunkPage) return S2_ERR_UNSUPPORTED;
+    if (block_size != 64 && block_size != 128) return S2_ERR_UNSUPPORTED;
+    if (num_blocks > 2046) return S2_ERR_UNSUPPORTED;  // union lists are staged in shared memory
+    if (batch > 65535 || heads > 65535 || total_q >= INT32_MAX / 2 || max_q_len > (1 << 24))
+        return S2_ERR_UNSUPPORTED;
+    if (num_pages * heads_kv >= (int64_t)INT32_MAX) return S2_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return S2_ERR_INVALID_ARG;
+    int dev = 0;
+    int rc = device_ready(&dev);
+    if (rc) return rc;
+    s2::ChunkParams cp;
+    cp.row_ptr = row_ptr;
+    cp.col_idx = col_idx;
+    cp.nnz = nnz;
+    cp.block_table = block_table;
+    cp.ctx_lens = ctx_lens;
+    cp.q_start = q_start;
+    cp.out = static_cast<uint16_t*>(out);
+    cp.lse = lse;
+    cp.num_pages = num_pages;
+    cp.total_q = total_q;
+    cp.batch = batch;
+    cp.heads = heads;
+    cp.heads_kv = heads_kv;
+    cp.max_pages = max_pages;
+    cp.nb = num_blocks;
+    cp.max_q_len = max_q_len;
+    cp.scale_log2 = scale * 1.4426950408889634f;
+    cp.timeout_ns = g_timeout_ns.load();
+    cp.gflags = g_dev[dev].flags;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (head_dim == 128 && block_size == 128) return launch_chunk<128, 128>(q, k_cache, v_cache, cp, dev, 0, st);
+    if (head_dim == 128 && block_size == 64) return launch_chunk<128, 64>(q, k_cache, v_cache, cp, dev, 1, st);
+    if (head_dim == 64 && block_size == 128) return launch_chunk<64, 128>(q, k_cache, v_cache, cp, dev, 2, st);
+    return launch_chunk<64, 64>(q, k_cache, v_cache, cp, dev, 3, st);
 }
 
 int32_t s2_attn_decode_auto_splits(int32_t batch, int32_t heads)

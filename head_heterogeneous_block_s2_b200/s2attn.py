@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "S2_OK", 1: "S2_ERR_INVALID_ARG", 2: "S2_ERR_UNSUPPORTED", 3:
 EXPORTED = ("s2_status_string", "s2_build_layout", "s2_build_layout_ranges",
             "s2_build_layout_mask", "s2_build_layout_transpose", "s2_attn_prefill",
             "s2_attn_prefill_gqa", "s2_attn_decode_gqa", "s2_attn_backward",
-            "s2_attn_backward_workspace_size", "s2_build_key_tiles",
+            "s2_attn_backward_workspace_size", "s2_build_key_tiles", "s2_attn_chunk_prefill",
             "s2_attn_decode_workspace_size", "s2_attn_decode_auto_splits", "s2_attn_decode",
             "s2_device_status", "s2_set_wait_timeout_ns", "s2_version", "s2_attn_decode_noalloc")
 
@@ -93,6 +93,9 @@ def load(path: str = LIB_PATH):
     lib.s2_attn_decode_gqa.restype = ctypes.c_int
     lib.s2_attn_decode_gqa.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i32,
                                        i32, vp, vp, i64, f32, vp, vp, vp, sz, i32, vp]
+    lib.s2_attn_chunk_prefill.restype = ctypes.c_int
+    lib.s2_attn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64,
+                                          i32, i64, i32, i32, vp, vp, i64, f32, vp, vp, vp]
     lib.s2_attn_decode_workspace_size.restype = sz
     lib.s2_attn_decode_workspace_size.argtypes = [i32, i32, i32, i32]
     lib.s2_attn_decode_auto_splits.restype = i32
@@ -382,6 +385,48 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                                  _stream(q.device))
     _check(rc, "s2_attn_backward")
     return dq, dk, dv
+
+
+def chunk_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                  block_table: torch.Tensor, ctx_lens: torch.Tensor, q_start: torch.Tensor,
+                  layout: Layout, max_q_len: int, scale: Optional[float] = None,
+                  out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                  want_lse: bool = False):
+    """s2_attn_chunk_prefill: q [total_q, heads, D] packed chunk rows; caches
+    [pages, heads_kv, 16, D]; block_table int32 [batch, max_pages]; ctx_lens
+    int32 [batch] (contexts including the chunks); q_start int32 [batch + 1]
+    (all CUDA). ``max_q_len`` bounds the chunk lengths."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n)
+    for t, n in ((block_table, "block_table"), (ctx_lens, "ctx_lens"), (q_start, "q_start")):
+        _need(t, n, torch.int32)
+    total_q, heads, hd = q.shape
+    num_pages, hkv, page_size, hd2 = k_cache.shape
+    if heads % hkv or hd2 != hd or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape does not match q")
+    batch = ctx_lens.numel()
+    if q_start.numel() != batch + 1:
+        raise ValueError("q_start must have batch + 1 entries")
+    if layout.heads != heads:
+        raise ValueError(f"layout has {layout.heads} heads, q has {heads}")
+    if layout.d_row_ptr is None:
+        layout.to(q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out")
+    if lse is None and want_lse:
+        lse = torch.empty((total_q, heads), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    rc = load().s2_attn_chunk_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                      _ptr(ctx_lens), _ptr(q_start), batch, heads, hkv, hd, page_size,
+                                      block_table.shape[1], num_pages, int(max_q_len), total_q,
+                                      layout.block_size, layout.num_blocks, _ptr(layout.d_row_ptr),
+                                      _ptr(layout.d_col_idx), layout.nnz, sc, _ptr(out), _ptr(lse),
+                                      _stream(q.device))
+    _check(rc, "s2_attn_chunk_prefill")
+    return (out, lse) if lse is not None else out
 
 
 def decode_auto_splits(batch: int, heads: int) -> int:

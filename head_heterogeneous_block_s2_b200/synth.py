@@ -30,6 +30,7 @@ with round-to-nearest-even (torch's fp32 -> bf16 conversion).
 from __future__ import annotations
 
 import dataclasses
+import itertools
 import math
 from typing import Dict, Optional, Sequence, Tuple
 
@@ -103,8 +104,15 @@ PREFILL_LONG_131K = PrefillWorkload("prefill_long_131k", 1, 32, 128, 131072, 128
                                     seed=3, planted=True)
 DECODE_PAGED = DecodeWorkload("decode_paged", 64, 32, 128, 4096, 32768, 16, 128, 16, 4, seed=4)
 
+# Chunked prefill over the paged cache (serving): 16 sequences with contexts
+# U[4096, 32768], each ending in a chunk of the last 2048 tokens; same pattern
+# and page layout as decode_paged.
+CHUNK_PAGED = DecodeWorkload("chunk_paged", 16, 32, 128, 4096, 32768, 16, 128, 16, 4, seed=5)
+CHUNK_LEN = {"chunk_paged": 2048}
+
 PREFILL_WORKLOADS = {w.name: w for w in (TINY, PREFILL_1P3B, PREFILL_7B_HYBRID, PREFILL_LONG_131K)}
 DECODE_WORKLOADS = {DECODE_PAGED.name: DECODE_PAGED}
+CHUNK_WORKLOADS = {CHUNK_PAGED.name: CHUNK_PAGED}
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -197,3 +205,27 @@ def decode_inputs(w: DecodeWorkload, device="cpu", ctx_lens: Optional[Sequence[i
             cache[p0:p1] = torch.randn((p1 - p0,) + shape[1:], generator=g, device=device,
                                        dtype=torch.float32)
     return DecodeInputs(q, k_cache, v_cache, bt.to(device), cl.to(torch.int32).to(device))
+
+
+@dataclasses.dataclass
+class ChunkInputs:
+    q: torch.Tensor            # [total_q, heads, head_dim] packed chunk rows
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block_table: torch.Tensor
+    ctx_lens: torch.Tensor     # contexts including the chunks
+    q_start: torch.Tensor      # [batch + 1]
+    max_q_len: int
+
+
+def chunk_inputs(w: DecodeWorkload, chunk: int, device="cpu") -> ChunkInputs:
+    """Chunked-prefill inputs: the paged contexts of ``w`` (as decode_inputs)
+    and, per sequence, a chunk of its last min(chunk, context) tokens as
+    packed N(0,1) query rows."""
+    d = decode_inputs(w, device=device)
+    cl = d.ctx_lens.cpu().tolist()
+    qlen = [min(chunk, n) for n in cl]
+    q_start = torch.tensor([0] + list(itertools.accumulate(qlen)), dtype=torch.int32)
+    g = _gen(w.seed + 1000, device)
+    q = _normal_bf16((int(q_start[-1]), w.heads, w.head_dim), g, device)
+    return ChunkInputs(q, d.k_cache, d.v_cache, d.block_table, d.ctx_lens, q_start.to(device), max(qlen))

@@ -222,6 +222,52 @@ int s2_attn_prefill_gqa(const void* q, const void* k, const void* v, void* o, fl
                         void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Chunked prefill: a chunk of queries per sequence over a paged KV cache    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Each sequence s appends a chunk of q_start[s+1] - q_start[s] query tokens at
+ * the end of its context of ctx_lens[s] tokens, whose keys and values (the
+ * chunk's own included) are already in the paged cache. Chunk row t of
+ * sequence s sits at position ctx_lens[s] - (q_start[s+1] - t) and attends to
+ * keys 0..position under the layout (query block = position / block_size),
+ * with token causality inside the diagonal block: the prefill definition
+ * restricted to the chunk rows. One-token chunks are decode. Serving prefills
+ * long prompts this way; the arXiv abstract of "S2-Attention: Hardware-aware
+ * context sharding among attention heads" reports 7B inference in vLLM, and
+ * PagedAttention is in its reference list.
+ *
+ *   q            device bf16 [total_q][heads][head_dim] (read): packed rows.
+ *   k_cache,     device bf16 [num_pages][heads_kv][page_size][head_dim] (read),
+ *   v_cache      as s2_attn_decode_gqa (heads_kv divides heads).
+ *   block_table  device int32 [batch][max_pages] (read).
+ *   ctx_lens     device int32 [batch] (read): context length including the chunk.
+ *   q_start      device int32 [batch + 1] (read): q_start[0] = 0, ascending,
+ *                q_start[batch] = total_q, and each chunk no longer than
+ *                max_q_len or its context.
+ *   max_q_len    host bound on the chunk lengths (sizes the grid).
+ *   page_size 16. head_dim 64 or 128. block_size 64 or 128.
+ *   row_ptr, col_idx, nnz, num_blocks: device layout covering the longest
+ *                context ((ctx_len - 1) / block_size < num_blocks).
+ *   out          device bf16 [total_q][heads][head_dim] (written).
+ *   lse          device fp32 [total_q][heads] or NULL (written).
+ * Cache rows past a context inside its last page may hold anything: the
+ * kernel never lets them reach the output. A sequence whose q_start, length
+ * or page ids are out of range is skipped and reported by s2_device_status as
+ * S2_ERR_DEVICE_INDEX. Errors before launch: S2_ERR_INVALID_ARG (null
+ * pointers, sizes, alignment, scale), S2_ERR_UNSUPPORTED (head_dim,
+ * block_size, page_size, num_blocks > 2046, sizes past the int32 ranges).
+ */
+int s2_attn_chunk_prefill(const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_table, const int32_t* ctx_lens,
+                          const int32_t* q_start, int32_t batch, int32_t heads, int32_t heads_kv,
+                          int32_t head_dim, int32_t page_size, int32_t max_pages,
+                          int64_t num_pages, int32_t max_q_len, int64_t total_q,
+                          int32_t block_size, int32_t num_blocks, const int32_t* row_ptr,
+                          const int32_t* col_idx, int64_t nnz, float scale, void* out,
+                          float* lse, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Backward: gradients of the prefill                                        */
 /* ------------------------------------------------------------------------ */
 
