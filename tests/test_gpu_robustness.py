@@ -100,3 +100,55 @@ def test_bad_context_length_is_flagged(s2gpu):
     rc, flags = s2gpu.device_status(reset=True)
     assert rc == S2_ERR_DEVICE_INDEX and flags == 2
     assert torch.isfinite(out.float()).all()
+
+
+def test_backward_wait_timeout_is_reported_and_recoverable(s2gpu):
+    w = synth.PrefillWorkload("t", 1, 4, 128, 2048, 128, 1, 1, seed=31)  # dense: long lists
+    q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
+    lay = s2gpu.build_layout(4, 128, 1, 1, 16, device="cuda")
+    o, lse = s2gpu.prefill(q, k, v, lay, scale=w.scale, want_lse=True)
+    do = torch.randn_like(q, dtype=torch.float32).to(torch.bfloat16)
+    s2gpu.set_wait_timeout_ns(0)
+    try:
+        s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale)
+        rc, flags = s2gpu.device_status(reset=True)
+    finally:
+        s2gpu.set_wait_timeout_ns(500_000_000)
+    assert rc == S2_ERR_TIMEOUT and flags & 1
+    a = s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale)
+    b = s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y) and torch.isfinite(x.float()).all()
+
+
+def test_chunk_wait_timeout_is_reported_and_recoverable(s2gpu):
+    wd = synth.DecodeWorkload("t", 2, 4, 128, 1, 4096, 16, 128, 1, 1, dense_heads=(0, 1, 2, 3), seed=32)
+    ctx = [4000, 4096]
+    d = synth.decode_inputs(wd, ctx_lens=ctx)
+    lay = s2gpu.build_layout(4, 128, 1, 1, wd.num_blocks, (0, 1, 2, 3), device="cuda")
+    q = torch.randn(600, 4, 128).to(torch.bfloat16)
+    q_start = torch.tensor([0, 300, 600], dtype=torch.int32)
+    args = (q.cuda(), d.k_cache.cuda(), d.v_cache.cuda(), d.block_table.cuda(), d.ctx_lens.cuda(),
+            q_start.cuda(), lay, 300)
+    s2gpu.set_wait_timeout_ns(0)
+    try:
+        s2gpu.chunk_prefill(*args, scale=wd.scale)
+        rc, flags = s2gpu.device_status(reset=True)
+    finally:
+        s2gpu.set_wait_timeout_ns(500_000_000)
+    assert rc == S2_ERR_TIMEOUT and flags & 1
+    out = s2gpu.chunk_prefill(*args, scale=wd.scale)
+    ref, _ = oracle.chunk(q, d.k_cache, d.v_cache, d.block_table.cpu().numpy(), ctx, q_start.numpy(),
+                          128, wd.scale, S=1, L=1, dense_heads=(0, 1, 2, 3))
+    parity(out.reshape(-1, 128), ref.reshape(-1, 128))
+
+
+def test_malformed_transposed_layout_is_flagged_not_faulted(s2gpu):
+    w = synth.PrefillWorkload("t", 1, 2, 128, 512, 128, 2, 1, seed=33)
+    q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
+    lay = s2gpu.build_layout(2, 128, 2, 1, 4, device="cuda").transposed("cuda")
+    o, lse = s2gpu.prefill(q, k, v, lay, scale=w.scale, want_lse=True)
+    lay.d_t_row_idx[1] = 1 << 20  # a query block far outside the layout
+    s2gpu.backward(q, k, v, o, lse, torch.ones_like(q), lay, scale=w.scale)
+    rc, flags = s2gpu.device_status(reset=True)
+    assert rc == S2_ERR_DEVICE_INDEX and flags == 2
