@@ -165,11 +165,12 @@ __device__ __forceinline__ int warp_union_list(const int32_t* row_ptr, const int
         }
         return list_pack(j, bits);
     };
-    if (ROWS == 1) {
+    if constexpr (ROWS == 1) {
         for (int t = lane; t < n[0]; t += 32) list[t] = checked(__ldg(col + a[0] + t), 1);
         __syncwarp();
         return n[0];
     }
+    else {
 #pragma unroll
     for (int r = 0; r < ROWS; ++r)
         for (int t = lane; t < n[r]; t += 32) scratch[r * cap + t] = __ldg(col + a[r] + t);
@@ -201,6 +202,7 @@ __device__ __forceinline__ int warp_union_list(const int32_t* row_ptr, const int
     }
     __syncwarp();
     return __shfl_sync(0xffffffffu, len, 0);
+    }
 }
 
 }  // namespace s2

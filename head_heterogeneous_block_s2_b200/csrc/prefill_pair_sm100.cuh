@@ -90,12 +90,18 @@ struct PairCfg {
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
-    static constexpr uint32_t TMEM_COLS = (2 * NK + 2 * HD) <= 256 ? 256 : 512;
+    // (2 NK of S, 2 HD of O, and HD of Q when it fits; see Q_IN_TMEM)
+    static constexpr uint32_t TMEM_COLS = (2 * NK + 3 * HD) <= 256 ? 256 : 512;
     // list_empty arrivals per item: K/V producer, MMA issuer, 8 softmax warps
     static constexpr uint32_t LIST_CONSUMERS = 10;
     __host__ __device__ static constexpr uint32_t colS(int t) { return (uint32_t)(t * NK); }
     __host__ __device__ static constexpr uint32_t colO(int t) { return (uint32_t)(2 * NK + t * HD); }
+    // With 64-key blocks TMEM has room for both tiles' Q (HD/2 columns each):
+    // S = Q K^T then reads Q from TMEM and only K from shared memory.
+    static constexpr bool Q_IN_TMEM = 2 * NK + 2 * HD + HD <= 512;
+    __host__ __device__ static constexpr uint32_t colQ(int t) { return (uint32_t)(2 * NK + 2 * HD + t * (HD / 2)); }
     static_assert(2 * NK + 2 * HD <= 512, "TMEM budget");
+    static_assert(!Q_IN_TMEM || 2 * NK + 3 * HD <= (int)TMEM_COLS, "Q columns inside the allocation");
     static_assert(ST % G == 0, "groups must not wrap the stage ring");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
@@ -323,10 +329,14 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
                 const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * (BK * 128), 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    umma_bf16_ss(tmem + C::colS(t), dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
-                                 dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4), idesc_s,
-                                 kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint64_t bk = dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4);
+                    if constexpr (C::Q_IN_TMEM)
+                        umma_bf16_ts(tmem + C::colS(t), tmem + C::colQ(t) + kk * 8, bk, idesc_s, kk > 0 ? 1u : 0u);
+                    else
+                        umma_bf16_ss(tmem + C::colS(t), dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
+                                     bk, idesc_s, kk > 0 ? 1u : 0u);
+                }
                 umma_commit(bar_sf(t));
                 issued = true;
             };
@@ -358,6 +368,20 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     mbar_arrive(bar_le(b));
                     continue;
                 }
+                if constexpr (C::Q_IN_TMEM) {
+                    // Q of both tiles into TMEM (after the previous item's S MMAs, in
+                    // issue order), then the shared-memory Q buffer is free at once.
+                    tc_fence_after();
+                    const bool two = pair_item<BK>(p, list_item[b]).tile1;
+                    for (int t = 0; t < (two ? 2 : 1); ++t) {
+                        const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < HD / 16; ++kk)
+                            tmem_cp_128x256b(tmem + C::colQ(t) + kk * 8,
+                                             dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4));
+                    }
+                    umma_commit(bar_qe);
+                }
                 const int ngroups = len / G;
                 first_pv[0] = first_pv[1] = true;
                 auto gbits = [&](int g) {
@@ -386,7 +410,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     const int nbits = last ? 0 : gbits(g + 1);
                     const int st = n % C::ST;
                     const int st1 = (n + G) % C::ST;
-                    if (last) umma_commit(bar_qe);  // no more S MMAs of this item read Q
+                    if (last && !C::Q_IN_TMEM) umma_commit(bar_qe);  // no more S MMAs of this item read Q
                     bool v_ready = false, k_next_ready = false;
                     if (bits == 0) {  // malformed group no tile sees: let its loads land first
                         if (!wait_k(n) || !wait_v(n)) {

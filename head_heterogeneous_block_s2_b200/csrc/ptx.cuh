@@ -214,6 +214,14 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
+// Copy a 128-row x 32-byte slab (one 16-element k-step of a bf16 operand)
+// from shared memory, described by a matrix descriptor, into 8 TMEM columns
+// of lanes 0..127: the layout of an A operand read from TMEM.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 op this thread issued so far has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar)
 {
