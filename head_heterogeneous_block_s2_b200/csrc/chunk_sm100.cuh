@@ -21,12 +21,18 @@
 // shared memory before the P V product uses them (their P is 0 anyway, but
 // 0 times a NaN would not be).
 //
-// CTA = 8 warps: warp 0 lane 0 loads Q and streams K (3 stages), warp 3
+// CTA = 12 warps: warp 0 lane 0 loads Q and streams K (3 stages), warp 3
 // lane 0 streams V (2 stages), warp 1 owns TMEM and issues tcgen05.mma
 // (S = Q K^T into one of two TMEM buffers, O += P V with P from TMEM), warp 2
-// builds the union list, warps 4..7 run the online softmax (thread = row =
-// TMEM lane) and the epilogue. S is double-buffered, so the softmax of one
-// key block overlaps the MMAs of the next.
+// builds the union list, warps 4..11 run the online softmax and the epilogue:
+// thread = row = TMEM lane, warps 4..7 on the first half of each block's
+// columns and warps 8..11 on the second; the two halves of a row exchange
+// their maxima through shared memory once per block (an mbarrier of the 256
+// softmax threads, waited with the same bound as every other wait, so a CTA
+// that gives up cannot strand the others) and keep partial sums that meet in
+// the epilogue. S is
+// double-buffered, so the softmax of one key block overlaps the MMAs of the
+// next.
 #pragma once
 
 #include <climits>
@@ -70,10 +76,12 @@ struct ChunkCfg {
     static constexpr uint32_t OFF_V = OFF_K + KST * KVBYTES;
     static constexpr uint32_t OFF_LIST = OFF_V + VST * KVBYTES;
     static constexpr uint32_t OFF_SCR = OFF_LIST + LIST_CAP * 4;
-    static constexpr uint32_t OFF_BAR = OFF_SCR + (ROWS > 1 ? ROWS * LIST_CAP * 4 : 0);
+    // exchange slots [3][2][128] floats: row maxima by block parity, then partial sums
+    static constexpr uint32_t OFF_XCH = OFF_SCR + (ROWS > 1 ? ROWS * LIST_CAP * 4 : 0);
+    static constexpr uint32_t OFF_BAR = OFF_XCH + 3 * 2 * 128 * 4;
     // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full,
-    // pv_done, drain
-    static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 5;
+    // pv_done, drain, xch[2], xch_sum
+    static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 8;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
@@ -85,7 +93,7 @@ struct ChunkCfg {
 };
 
 template <int HD, int BK>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const ChunkParams p)
 {
@@ -121,6 +129,8 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     const uint32_t bar_p = sb + C::OFF_BAR + 8u * (3 + 2 * C::KST + 2 * C::VST);
     const uint32_t bar_pv = bar_p + 8u;
     const uint32_t bar_dr = bar_p + 16u;
+    auto bar_x = [&](int b) { return bar_p + 24u + 8u * b; };  // max exchange, by block parity
+    const uint32_t bar_xl = bar_p + 40u;                        // partial-sum exchange
     uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2] list length
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
@@ -138,9 +148,12 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         }
         mbar_init(bar_sf(0), 1);
         mbar_init(bar_sf(1), 1);
-        mbar_init(bar_p, 128);
+        mbar_init(bar_p, 256);
         mbar_init(bar_pv, 1);
         mbar_init(bar_dr, 1);
+        mbar_init(bar_x(0), 256);
+        mbar_init(bar_x(1), 256);
+        mbar_init(bar_xl, 256);
         *abort_cta = 0;
         fence_mbar_init();
         // Q of the tile: chunk row of position t*128 is q0 + t*128 - c0 (may be
@@ -247,7 +260,9 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t dv = umma_sdesc(sb + C::OFF_V + vs * C::KVBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_O, tmem + C::colS(e & 1) + kk * 8, dv, idesc_o,
+                        // the two softmax halves packed P into the first quarter of each half
+                        const uint32_t pcol = (kk / (BK / 32)) * (BK / 2) + (kk % (BK / 32)) * 8;
+                        umma_bf16_ts(tmem + C::COL_O, tmem + C::colS(e & 1) + pcol, dv, idesc_o,
                                      (e > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(bar_ve(vs));
@@ -263,15 +278,17 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         __syncwarp();
     } else if (warp >= 4) {
         // ------------------------------------------------------------ online softmax + epilogue
-        const int quad = warp & 3;
+        constexpr int HALF = BK / 2;  // key columns per warpgroup
+        const int quad = warp & 3, g = (warp - 4) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);  // [slot][half][row]
         const int pos = t * C::M + r;
         const int rowbit = (BK == 128) ? 0 : (r >> 6);
         const bool row_valid = pos >= c0 && pos < n;
         const float sc = p.scale_log2;  // > 0
         const int n16 = ((n + kChunkPage - 1) / kChunkPage) * kChunkPage;  // end of the last loaded page
-        float m_used = -1e30f, l = 0.f;
+        float m_used = -1e30f, l = 0.f;  // l: this half's partial row sum
         bool fail = false;
         for (int e = 0; e < len; ++e) {
             const uint32_t ent = list[e];
@@ -282,39 +299,50 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 break;
             }
             tc_fence_after();
-            uint32_t sr[BK];
+            uint32_t sr[HALF];
 #pragma unroll
-            for (int c = 0; c < BK / 32; ++c)
-                tmem_ld32(tl + C::colS(b) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+            for (int c = 0; c < HALF / 32; ++c)
+                tmem_ld32(tl + C::colS(b) + g * HALF + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
             tmem_wait_ld();
             const bool vis = row_valid && ((list_bits(ent) >> rowbit) & 1);
-            const int lim = pos - j * BK;  // key column c visible iff c <= lim
+            const int lim = pos - j * BK - g * HALF;  // column c of this half visible iff c <= lim
 #pragma unroll
-            for (int c = 0; c < BK; ++c)
+            for (int c = 0; c < HALF; ++c)
                 if (!(vis && c <= lim)) sr[c] = 0xff800000u;  // -inf
             float mx = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < BK; c += 2) mx = fmax3(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+            for (int c = 0; c < HALF; c += 2) mx = fmax3(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+            // the row's maximum over both halves (slots alternate by block parity, so
+            // a slot is rewritten only after its reader has passed the next barrier)
+            xch[(b * 2 + g) * 128 + r] = mx;
+            mbar_arrive(bar_x(b));
+            if (!warp_wait(bar_x(b), (e >> 1) & 1, ctl)) {
+                fail = true;
+                break;
+            }
+            mx = fmaxf(mx, xch[(b * 2 + (g ^ 1)) * 128 + r]);
             const float m_cand = fmaxf(m_used, mx * sc);
             const bool move = m_cand - m_used > 8.0f;  // rescale O only when the max grew by > 2^8
             const float alpha = move ? ex2(m_used - m_cand) : 1.0f;
             if (move) m_used = m_cand;
             float rs = 0.f;
 #pragma unroll
-            for (int c = 0; c < BK / 2; ++c) {
+            for (int c = 0; c < HALF / 2; ++c) {
                 const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sc, -m_used));
                 const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sc, -m_used));
                 rs += p0 + p1;
                 sr[c] = pack_bf16x2(p0, p1);  // slot c <= 2c: already read
             }
             l = l * alpha + rs;
-#pragma unroll
-            for (int c = 0; c < BK / 64; ++c)
-                tmem_st32(tl + C::colS(b) + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&sr[32 * c]));
+            if constexpr (HALF / 2 == 32) {
+                tmem_st32(tl + C::colS(b) + g * HALF, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
+            } else {
+                tmem_st16(tl + C::colS(b) + g * HALF, *reinterpret_cast<const uint32_t(*)[16]>(&sr[0]));
+            }
             // Rows of this block past the context inside its last loaded page hold
             // stale cache data: zero them in V before the P V product reads them.
             const int z0 = n - j * BK, z1 = min(BK, n16 - j * BK);
-            if (z0 < z1) {
+            if (z0 < z1 && g == 0) {
                 const int vs = e % C::VST;
                 if (!warp_wait(bar_vf(vs), (e / C::VST) & 1, ctl)) {
                     fail = true;
@@ -330,7 +358,7 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 }
                 fence_proxy_async_smem();
             }
-            // O is stable once PV(e-1) is done: rescale it if the max moved
+            // O is stable once PV(e-1) is done: each half rescales its HD/2 columns
             if (e > 0 && !warp_wait(bar_pv, (e - 1) & 1, ctl)) {
                 fail = true;
                 break;
@@ -338,31 +366,37 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             tc_fence_after();
             if (e > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
+                for (int c = 0; c < HD / 64; ++c) {
                     uint32_t o[32];
-                    tmem_ld32(tl + C::COL_O + 32 * c, o);
+                    tmem_ld32(tl + C::COL_O + g * (HD / 2) + 32 * c, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e2 = 0; e2 < 32; ++e2) o[e2] = __float_as_uint(__uint_as_float(o[e2]) * alpha);
-                    tmem_st32(tl + C::COL_O + 32 * c, o);
+                    tmem_st32(tl + C::COL_O + g * (HD / 2) + 32 * c, o);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p);
         }
+        if (!fail) {  // the two halves' partial sums meet
+            xch[(4 + g) * 128 + r] = l;  // slot 2: never used by the max exchange
+            mbar_arrive(bar_xl);
+            fail = !warp_wait(bar_xl, 0, ctl);
+            l += xch[(4 + (g ^ 1)) * 128 + r];
+        }
         if (!fail) {
             // every lane takes part in the waits and TMEM loads; only chunk rows store
             const bool acc_ok = len > 0 && warp_wait(bar_pv, (len - 1) & 1, ctl);
             const int64_t orow = (int64_t)(q0 + pos - c0) * p.heads + h;
-            uint16_t* og = p.out + orow * HD;
+            uint16_t* og = p.out + orow * HD + g * (HD / 2);
             if (acc_ok) {
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.0f / l : 0.f;
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
+                for (int c = 0; c < HD / 64; ++c) {
                     uint32_t o[32];
-                    tmem_ld32(tl + C::COL_O + 32 * c, o);
+                    tmem_ld32(tl + C::COL_O + g * (HD / 2) + 32 * c, o);
                     tmem_wait_ld();
                     if (row_valid) {
 #pragma unroll
@@ -376,11 +410,11 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                         }
                     }
                 }
-                if (row_valid && p.lse)
+                if (row_valid && g == 0 && p.lse)
                     p.lse[orow] = l > 0.f ? (m_used + lg2(l)) * 0.69314718055994531f : -INFINITY;
             } else if (len == 0 && row_valid) {  // no key block listed for this tile
-                for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(og + d) = make_uint4(0, 0, 0, 0);
-                if (p.lse) p.lse[orow] = -INFINITY;
+                for (int d = 0; d < HD / 2; d += 8) *reinterpret_cast<uint4*>(og + d) = make_uint4(0, 0, 0, 0);
+                if (g == 0 && p.lse) p.lse[orow] = -INFINITY;
             }
         }
         tc_fence_before();

@@ -220,7 +220,7 @@ int launch_chunk(const void* q, const void* kc, const void* vc, s2::ChunkParams&
         }
     }
     const dim3 grid((unsigned)((cp.max_q_len + 127) / 128 + 1), (unsigned)cp.heads, (unsigned)cp.batch);
-    kern<<<grid, 256, C::SMEM_ALLOC, stream>>>(mq, mk, mv, cp);
+    kern<<<grid, 384, C::SMEM_ALLOC, stream>>>(mq, mk, mv, cp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
