@@ -99,13 +99,22 @@ def chunk_flops(lay, w, ctx_lens, qlens) -> int:
     return 4 * w.head_dim * pairs
 
 
-def source_sha() -> str:
+# Sources each kernel is compiled from (its ncu traffic figure stays valid while
+# these files are unchanged).
+KERNEL_SOURCES = {
+    "s2_prefill_pair_kernel": ("prefill_pair_sm100.cuh", "lists.cuh", "ptx.cuh", "umma.cuh"),
+    "s2_decode_split_kernel": ("decode.cuh", "ptx.cuh"),
+    "s2_bwd": ("backward_sm100.cuh", "lists.cuh", "ptx.cuh", "umma.cuh"),
+    "s2_chunk_prefill_kernel": ("chunk_sm100.cuh", "lists.cuh", "ptx.cuh", "umma.cuh"),
+}
+
+
+def source_sha(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "head_heterogeneous_block_s2_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".cpp")):
-            h.update(fn.encode())
-            h.update(open(os.path.join(csrc, fn), "rb").read())
+    for fn in sorted(KERNEL_SOURCES[kernel]):
+        h.update(fn.encode())
+        h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -125,7 +134,7 @@ def load_traffic(kernel: str, workload: str):
         return None
     d = json.load(open(p))
     e = d.get(f"{kernel}@{workload}")
-    if not e or e.get("source_sha") != source_sha():
+    if not e or e.get("source_sha") != source_sha(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -518,6 +527,7 @@ def run_ours(args, rank, world, dist):
             "kernels": "s2_bwd_stats_kernel + s2_bwd_dq_kernel + s2_bwd_dkv_kernel",
             "roofline": {"bound": "tensor", "achieved": round(per, 2), "peak": tc_peak,
                          "unit": "TFLOP/s", "frac": round(per / tc_peak, 4),
+                         "traffic": load_traffic("s2_bwd", wb.name),
                          "peak_source": f"{peak_src} bf16_tflops_sustained"},
         }
         line["gpu_launches_backward"] = 3 * bwd_steps
@@ -539,6 +549,7 @@ def run_ours(args, rank, world, dist):
             "kernels": "s2_chunk_prefill_kernel",
             "roofline": {"bound": "tensor", "achieved": round(per, 2), "peak": tc_peak,
                          "unit": "TFLOP/s", "frac": round(per / tc_peak, 4),
+                         "traffic": load_traffic("s2_chunk_prefill_kernel", wc.name),
                          "peak_source": f"{peak_src} bf16_tflops_sustained"},
         }
         line["gpu_launches_chunk"] = chunk_steps
