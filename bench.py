@@ -118,6 +118,18 @@ def source_sha(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
+def max_over_ranks(vals, dist, device):
+    """Element-wise maximum of per-rank timings (one all-reduce; identity on
+    one process). Every rank must call it, with the same number of values."""
+    if dist is None:
+        return list(vals)
+    import torch
+
+    t = torch.tensor(list(vals), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -420,12 +432,7 @@ def run_ours(args, rank, world, dist):
 
     # ---------------- max over ranks
     vals = [total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms, chunk_ms]
-    if dist:
-        import torch.distributed as tdist
-
-        t = torch.tensor(vals, dtype=torch.float64, device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        vals = t.tolist()
+    vals = max_over_ranks(vals, dist, dev)
     total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms, chunk_ms = vals
     clocks = sampler.summary()
     if rank != 0:
