@@ -63,9 +63,9 @@ struct BackwardParams {
     const float* lse;      // [batch][heads][seq] forward LSE, natural log (stats kernel)
     float* stats;          // [batch * heads][seq_pad / 128][2][128]: LSE * log2 e, then D
     uint16_t* dq;          // [batch][heads][seq][HD]
-    uint16_t* dk;          // [batch][heads][seq][HD]
+    uint16_t* dk;          // [batch][heads_kv][seq][HD]: summed over each K/V head's query heads
     uint16_t* dv;
-    int32_t batch, heads, seq, seq_pad, nb, ntiles;
+    int32_t batch, heads, heads_kv, seq, seq_pad, nb, ntiles;  // query head h reads K/V head h / (heads / heads_kv)
     float scale;       // logit scale
     float scale_log2;  // scale * log2 e
     uint64_t timeout_ns;
@@ -194,6 +194,7 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int qt = p.ntiles - 1 - (int)(blockIdx.x / BH);  // longest lists first
     const int bh = (int)(blockIdx.x % BH);
     const int h = bh % p.heads;
+    const int bkv = (bh / p.heads) * p.heads_kv + h / (p.heads / p.heads_kv);  // K/V plane
 
     const uint32_t bar_qd = sb + C::OFF_BAR;
     auto bar_kf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
@@ -268,12 +269,12 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
                 for (int pn = 0; pn < HD / 64; ++pn)
                     tma_load_3d(sb + C::OFF_K + st * C::KVBYTES + pn * (BK * 128), &tmK, pn * 64, krow,
-                                bh, bar_kf(st));
+                                bkv, bar_kf(st));
                 mbar_arrive_expect_tx(bar_vf(st), C::KVBYTES);
 #pragma unroll
                 for (int pn = 0; pn < HD / 64; ++pn)
                     tma_load_3d(sb + C::OFF_V + st * C::KVBYTES + pn * (BK * 128), &tmV, pn * 64, krow,
-                                bh, bar_vf(st));
+                                bkv, bar_vf(st));
             }
             if (*abort_cta) {  // let this CTA's own loads land before exit
                 mbar_drain(bar_qd, 0, kDrainNs);
@@ -457,7 +458,7 @@ struct BwdKVCfg {
     static constexpr uint32_t QBYTES = BK * HD * 2;    // one query block of Q or dO
     static constexpr uint32_t STATBYTES = BK * 8;      // L2 of the BK queries, then their D
     static constexpr int ST = 2;
-    static constexpr int LIST_CAP = 2048;
+    static constexpr int LIST_CAP = 4096;  // grouped heads: the lists of every query head of the group
     static constexpr uint32_t OFF_K = 0;
     static constexpr uint32_t OFF_V = TBYTES;
     static constexpr uint32_t OFF_Q = 2 * TBYTES;              // [stage][panel][BK rows x 128 B]
@@ -489,10 +490,14 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                                                ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int BH = p.batch * p.heads;
-    const int kt = (int)(blockIdx.x / BH);
-    const int bh = (int)(blockIdx.x % BH);
-    const int h = bh % p.heads;
+    // One key tile of one K/V plane; with grouped heads the tile collects the
+    // gradients of every query head of its group (list entries carry the head).
+    const int BHk = p.batch * p.heads_kv;
+    const int kt = (int)(blockIdx.x / BHk);
+    const int bkv = (int)(blockIdx.x % BHk);
+    const int grp = p.heads / p.heads_kv;
+    const int h = (bkv % p.heads_kv) * grp;         // first query head of the group
+    const int bq0 = (bkv / p.heads_kv) * p.heads + h;  // its (batch, head) plane
     // Key blocks of this tile: one 128-row block, or two 64-row blocks chosen on
     // the host so that their transposed lists overlap (see s2_build_key_tiles).
     int kb[C::ROWS];
@@ -550,8 +555,8 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             const int32_t krow = (kb[r] >= 0 ? kb[r] : kany) * BK;
 #pragma unroll
             for (int pn = 0; pn < HD / 64; ++pn) {
-                tma_load_3d(sb + C::OFF_K + pn * (C::M * 128) + r * (BK * 128), &tmK, pn * 64, krow, bh, bar_kv);
-                tma_load_3d(sb + C::OFF_V + pn * (C::M * 128) + r * (BK * 128), &tmV, pn * 64, krow, bh, bar_kv);
+                tma_load_3d(sb + C::OFF_K + pn * (C::M * 128) + r * (BK * 128), &tmK, pn * 64, krow, bkv, bar_kv);
+                tma_load_3d(sb + C::OFF_V + pn * (C::M * 128) + r * (BK * 128), &tmV, pn * 64, krow, bkv, bar_kv);
             }
         }
     }
@@ -560,10 +565,16 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 #pragma unroll
         for (int r = 0; r < C::ROWS; ++r)
             if (kb[r] >= 0 && kb[r] < lo) lo = kb[r];
-        const int n = warp_union_list<C::ROWS>(p.col_ptr, p.row_idx, h * (p.nb + 1), kb, p.nb, p.nnz,
-                                               lo, p.nb - 1, list, C::LIST_CAP,
-                                               reinterpret_cast<int32_t*>(smem + C::OFF_SCR), p.gflags);
-        if (lane == 0) misc[2] = n;
+        int total = 0;
+        for (int hh = 0; hh < grp; ++hh) {  // the group's query heads, one list after another
+            const int n = warp_union_list<C::ROWS>(p.col_ptr, p.row_idx, (h + hh) * (p.nb + 1), kb, p.nb, p.nnz,
+                                                   lo, p.nb - 1, list + total, C::LIST_CAP - total,
+                                                   reinterpret_cast<int32_t*>(smem + C::OFF_SCR), p.gflags);
+            for (int t = lane; t < n; t += 32) list[total + t] |= (uint32_t)hh << 28;
+            __syncwarp();
+            total += n;
+        }
+        if (lane == 0) misc[2] = total;
     }
     tc_fence_before();
     __syncthreads();
@@ -582,15 +593,16 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 const int st = n % C::ST;
                 if (!mbar_wait(bar_qe(st), ((n / C::ST) & 1) ^ 1, ctl)) break;
                 const int i = list_j(list[n]);
+                const int bq = bq0 + (int)(list[n] >> 28);  // query plane of this entry
                 mbar_arrive_expect_tx(bar_qf(st), 2 * C::QBYTES + C::STATBYTES);
 #pragma unroll
                 for (int pn = 0; pn < HD / 64; ++pn) {
                     tma_load_3d(sb + C::OFF_Q + st * C::QBYTES + pn * (BK * 128), &tmQ, pn * 64, i * BK,
-                                bh, bar_qf(st));
+                                bq, bar_qf(st));
                     tma_load_3d(sb + C::OFF_DO + st * C::QBYTES + pn * (BK * 128), &tmDO, pn * 64, i * BK,
-                                bh, bar_qf(st));
+                                bq, bar_qf(st));
                 }
-                const float* sx = p.stats + ((int64_t)bh * p.ntiles + (i * BK) / 128) * 256 + (i * BK) % 128;
+                const float* sx = p.stats + ((int64_t)bq * p.ntiles + (i * BK) / 128) * 256 + (i * BK) % 128;
                 bulk_load(sb + C::OFF_STAT + st * C::STATBYTES, sx, BK * 4, bar_qf(st));
                 bulk_load(sb + C::OFF_STAT + st * C::STATBYTES + BK * 4, sx + 128, BK * 4, bar_qf(st));
             }
@@ -739,7 +751,7 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
         if (!fail) {
             // warpgroup 0 stores dV, warpgroup 1 stores dK (times the scale)
-            const int64_t row = (int64_t)bh * p.seq + kpos;
+            const int64_t row = (int64_t)bkv * p.seq + kpos;
             uint16_t* grow = (g == 0 ? p.dv : p.dk) + row * HD;
             if (len > 0) {
                 if (warp_wait(bar_acc, 0, ctl)) {

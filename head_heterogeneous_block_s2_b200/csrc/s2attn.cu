@@ -164,10 +164,10 @@ int launch_backward(const void* q, const void* k, const void* v, s2::BackwardPar
 {
     using CQ = s2::BwdQCfg<HD, BK>;
     using CK = s2::BwdKVCfg<HD, BK>;
-    const uint64_t planes = (uint64_t)bp.batch * bp.heads;
+    const uint64_t planes = (uint64_t)bp.batch * bp.heads, kvplanes = (uint64_t)bp.batch * bp.heads_kv;
     CUtensorMap q128, do128, kbk, vbk, qbk, dobk;
     if (make_map(&q128, q, planes, bp.seq, HD, 128) || make_map(&do128, bp.dout, planes, bp.seq, HD, 128) ||
-        make_map(&kbk, k, planes, bp.seq, HD, BK) || make_map(&vbk, v, planes, bp.seq, HD, BK) ||
+        make_map(&kbk, k, kvplanes, bp.seq, HD, BK) || make_map(&vbk, v, kvplanes, bp.seq, HD, BK) ||
         make_map(&qbk, q, planes, bp.seq, HD, BK) || make_map(&dobk, bp.dout, planes, bp.seq, HD, BK))
         return S2_ERR_CUDA;
     auto kq = s2::s2_bwd_dq_kernel<HD, BK>;
@@ -189,10 +189,9 @@ int launch_backward(const void* q, const void* k, const void* v, s2::BackwardPar
     if (grid0 > (int64_t)g_dev[dev].num_sms * 16) grid0 = (int64_t)g_dev[dev].num_sms * 16;
     s2::s2_bwd_stats_kernel<HD><<<(unsigned)grid0, 256, 0, stream>>>(bp);
     if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
-    const uint64_t tiles = planes * (uint64_t)bp.ntiles;
-    kq<<<(unsigned)tiles, 384, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
+    kq<<<(unsigned)(planes * bp.ntiles), 384, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
     if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
-    kkv<<<(unsigned)tiles, 384, CK::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
+    kkv<<<(unsigned)(kvplanes * bp.ntiles), 384, CK::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
@@ -371,7 +370,9 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
     if (batch < 1 || heads < 1 || seq < 1 || nnz < 0 || !std::isfinite(scale) || !(scale > 0.f))
         return S2_ERR_INVALID_ARG;
     if (heads_kv < 1 || heads % heads_kv != 0) return S2_ERR_INVALID_ARG;
-    if (heads_kv != heads) return S2_ERR_UNSUPPORTED;  // grouped K/V heads: forward only
+    // grouped heads: a key tile walks every query head's list of its group (tags of 4 bits)
+    if (heads / heads_kv > 16 || (heads != heads_kv && (int64_t)(heads / heads_kv) * num_blocks > 4096))
+        return S2_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
     if (block_size != 64 && block_size != 128) return S2_ERR_UNSUPPORTED;
     if (num_blocks > 2046) return S2_ERR_UNSUPPORTED;  // union lists are staged in shared memory
@@ -403,6 +404,7 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
     bp.dv = static_cast<uint16_t*>(dv);
     bp.batch = batch;
     bp.heads = heads;
+    bp.heads_kv = heads_kv;
     bp.seq = seq;
     bp.seq_pad = (int32_t)(ntiles * 128);
     bp.nb = num_blocks;

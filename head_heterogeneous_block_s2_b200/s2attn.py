@@ -351,12 +351,17 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
              dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
              workspace: Optional[torch.Tensor] = None):
     """s2_attn_backward: gradients (dq, dk, dv) of ``prefill`` for the upstream
-    gradient ``dout``, given the forward's output ``o`` and ``lse``."""
+    gradient ``dout``, given the forward's output ``o`` and ``lse``. k and v
+    may have fewer heads (grouped K/V heads): dk and dv then sum over each K/V
+    head's query heads."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
         _need(t, n)
     _need(lse, "lse", torch.float32)
     batch, heads, seq, hd = q.shape
-    for t, n in ((k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+    hkv = k.shape[1]
+    if k.shape != (batch, hkv, seq, hd) or v.shape != k.shape or heads % hkv:
+        raise ValueError("k, v must be [batch, heads_kv, seq, head_dim] with heads_kv | heads")
+    for t, n in ((o, "o"), (dout, "dout")):
         if t.shape != q.shape:
             raise ValueError(f"{n} shape differs from q")
     if lse.shape != (batch, heads, seq):
@@ -377,7 +382,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     ws_len = workspace.numel() * workspace.element_size()
     sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
     rc = load().s2_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
-                                 _ptr(dq), _ptr(dk), _ptr(dv), batch, heads, heads, seq, hd, sc,
+                                 _ptr(dq), _ptr(dk), _ptr(dv), batch, heads, hkv, seq, hd, sc,
                                  layout.block_size, layout.num_blocks, _ptr(layout.d_row_ptr),
                                  _ptr(layout.d_col_idx), _ptr(layout.d_t_col_ptr),
                                  _ptr(layout.d_t_row_idx), _ptr(layout.d_t_key_tiles), layout.nnz,

@@ -282,12 +282,18 @@ size_t s2_attn_backward_workspace_size(int32_t batch, int32_t heads, int32_t seq
  * with P = exp(scale Q K^T - LSE) over the visible keys and D = rowsum(dO * O),
  *     dV = P^T dO,   dS = P * (dO V^T - D),   dQ = scale dS K,   dK = scale dS^T Q.
  *
- *   q, k, v, o  device bf16 [batch][heads][seq][head_dim] (read): the forward's
- *               inputs and output.
+ *   q, o        device bf16 [batch][heads][seq][head_dim] (read): the forward's
+ *               queries and output.
+ *   k, v        device bf16 [batch][heads_kv][seq][head_dim] (read).
  *   dout        device bf16 [batch][heads][seq][head_dim] (read): dL/dO.
  *   lse         device fp32 [batch][heads][seq] (read): the forward's LSE.
- *   dq, dk, dv  device bf16 [batch][heads][seq][head_dim] (written).
- *   heads_kv    must equal heads (grouped K/V heads: S2_ERR_UNSUPPORTED).
+ *   dq          device bf16 [batch][heads][seq][head_dim] (written).
+ *   dk, dv      device bf16 [batch][heads_kv][seq][head_dim] (written): with
+ *               grouped heads (heads_kv < heads, query head h reading K/V head
+ *               h / (heads / heads_kv)) they sum over the group's query heads.
+ *   heads_kv    divides heads; a group is at most 16 query heads and, when
+ *               heads_kv < heads, (heads / heads_kv) * num_blocks <= 4096
+ *               (S2_ERR_UNSUPPORTED otherwise).
  *   seq, head_dim, scale, block_size, num_blocks: as s2_attn_prefill.
  *   row_ptr, col_idx, nnz  device layout the forward used (read).
  *   col_ptr, row_idx       device transposed layout from
@@ -302,7 +308,7 @@ size_t s2_attn_backward_workspace_size(int32_t batch, int32_t heads, int32_t seq
  * CTAs (no atomics; results are deterministic). Rows with an empty list get
  * zero gradients. Errors: S2_ERR_INVALID_ARG (null pointers, sizes, alignment,
  * a bad scale), S2_ERR_CAPACITY (workspace too small), S2_ERR_UNSUPPORTED
- * (head_dim, block_size, grouped heads), S2_ERR_CUDA (launch failure).
+ * (head_dim, block_size, group limits above), S2_ERR_CUDA (launch failure).
  */
 int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,

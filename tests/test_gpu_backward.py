@@ -107,3 +107,22 @@ def test_backward_is_deterministic(s2gpu):
     b = s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("hkv", [1, 2])
+@pytest.mark.parametrize("bk", [64, 128])
+def test_grouped_kv_heads(s2gpu, hkv, bk):
+    H, seq = 4, 9 * 64 if bk == 64 else 5 * 128
+    w = synth.PrefillWorkload("t", 2, H, 128, seq, bk, 3, 1, dense_heads=(1,), seed=95)
+    q, k, v = synth.prefill_inputs(w)
+    k, v = k[:, :hkv].contiguous(), v[:, :hkv].contiguous()
+    do = upstream(w, 6)
+    lay = s2gpu.build_layout(H, bk, 3, 1, seq // bk, (1,), device="cuda")
+    qc, kc, vc, doc = (t.cuda() for t in (q, k, v, do))
+    o, lse = s2gpu.prefill(qc, kc, vc, lay, scale=w.scale, want_lse=True)
+    dq, dk, dv = s2gpu.backward(qc, kc, vc, o, lse, doc, lay, scale=w.scale)
+    torch.cuda.synchronize()
+    assert dk.shape == k.shape and dv.shape == v.shape
+    ref = oracle.backward(q, k, v, do, bk, w.scale, S=3, L=1, dense_heads=(1,))
+    for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        grad_parity(name, g, r)
