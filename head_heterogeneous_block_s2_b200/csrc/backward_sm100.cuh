@@ -174,7 +174,11 @@ struct BwdQCfg {
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
     static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_ACC = 2 * BK;
-    static constexpr uint32_t TMEM_COLS = (2 * BK + HD) <= 256 ? 256 : 512;
+    // Q and dO, the A operands of every S and dP MMA of the CTA, sit in TMEM
+    // (HD/2 columns each): those MMAs read only K or V from shared memory.
+    static constexpr uint32_t COL_QA = 2 * BK + HD, COL_DOA = 2 * BK + HD + HD / 2;
+    static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD) <= 256 ? 256 : 512;
+    static_assert(2 * BK + 2 * HD <= 512, "TMEM budget");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
@@ -306,7 +310,7 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk)
-                    umma_bf16_ss(tmem + C::COL_S, dq_desc + kstep(kk, C::M), dk_desc + kstep(kk, BK), idesc_s,
+                    umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_QA + kk * 8, dk_desc + kstep(kk, BK), idesc_s,
                                  kk > 0 ? 1u : 0u);
                 umma_commit(bar_s);
                 issued = true;
@@ -319,12 +323,22 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk)
-                    umma_bf16_ss(tmem + C::COL_DP, ddo_desc + kstep(kk, C::M), dv_desc + kstep(kk, BK),
+                    umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_DOA + kk * 8, dv_desc + kstep(kk, BK),
                                  idesc_s, kk > 0 ? 1u : 0u);
                 umma_commit(bar_dp);
                 return true;
             };
-            if (mbar_wait(bar_qd, 0, ctl) && issue_s(0) && issue_dp(0)) {
+            const bool qd_ok = mbar_wait(bar_qd, 0, ctl);
+            if (qd_ok) {  // Q and dO into TMEM (in issue order before every MMA that reads them)
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    tmem_cp_128x256b(tmem + C::COL_QA + kk * 8, dq_desc + kstep(kk, C::M));
+                    tmem_cp_128x256b(tmem + C::COL_DOA + kk * 8, ddo_desc + kstep(kk, C::M));
+                }
+                issued = true;
+            }
+            if (qd_ok && issue_s(0) && issue_dp(0)) {
                 for (int n = 0; n < len; ++n) {
                     const int st = n % C::ST;
                     const bool more = n + 1 < len;
@@ -473,7 +487,11 @@ struct BwdKVCfg {
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
     static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_DV = 2 * BK, COL_DK = 2 * BK + HD;
-    static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD) <= 256 ? 256 : 512;
+    // When TMEM has room (B = 64, or head_dim 64), K and V, the A operands of
+    // every S^T and dP^T MMA of the CTA, sit in TMEM (HD/2 columns each).
+    static constexpr bool A_IN_TMEM = 2 * BK + 3 * HD <= 512;
+    static constexpr uint32_t COL_KA = 2 * BK + 2 * HD, COL_VA = 2 * BK + 2 * HD + HD / 2;
+    static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD + (A_IN_TMEM ? HD : 0)) <= 256 ? 256 : 512;
     static_assert(2 * BK + 2 * HD <= 512, "TMEM budget");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
@@ -633,9 +651,14 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 tc_fence_after();
                 const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK), idesc_s,
-                                 kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    if constexpr (C::A_IN_TMEM)
+                        umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_KA + kk * 8, dq_desc + kstep(kk, BK), idesc_s,
+                                     kk > 0 ? 1u : 0u);
+                    else
+                        umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK), idesc_s,
+                                     kk > 0 ? 1u : 0u);
+                }
                 umma_commit(bar_s);
                 issued = true;
                 return true;
@@ -644,12 +667,27 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 const int st = n % C::ST;
                 const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
-                                 idesc_s, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    if constexpr (C::A_IN_TMEM)
+                        umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_VA + kk * 8, ddo_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+                    else
+                        umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+                }
                 umma_commit(bar_dp);
             };
-            if (mbar_wait(bar_kv, 0, ctl) && issue_st(0)) {
+            const bool kv_ok = mbar_wait(bar_kv, 0, ctl);
+            if (kv_ok && C::A_IN_TMEM) {  // K and V into TMEM, before every MMA that reads them
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    tmem_cp_128x256b(tmem + C::COL_KA + kk * 8, dk_desc + kstep(kk, C::M));
+                    tmem_cp_128x256b(tmem + C::COL_VA + kk * 8, dv_desc + kstep(kk, C::M));
+                }
+                issued = true;
+            }
+            if (kv_ok && issue_st(0)) {
                 issue_dpt(0);
                 for (int n = 0; n < len; ++n) {
                     const int st = n % C::ST;

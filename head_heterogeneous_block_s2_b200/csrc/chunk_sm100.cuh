@@ -87,8 +87,9 @@ struct ChunkCfg {
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
     __host__ __device__ static constexpr uint32_t colS(int b) { return (uint32_t)(b * BK); }
     static constexpr uint32_t COL_O = 2 * BK;
-    static constexpr uint32_t TMEM_COLS = (2 * BK + HD) <= 256 ? 256 : 512;
-    static_assert(2 * BK + HD <= 512, "TMEM budget");
+    static constexpr uint32_t COL_QA = 2 * BK + HD;  // Q, the A operand of every S MMA (HD/2 columns)
+    static constexpr uint32_t TMEM_COLS = (2 * BK + HD + HD / 2) <= 256 ? 256 : 512;
+    static_assert(2 * BK + HD + HD / 2 <= 512, "TMEM budget");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
@@ -244,14 +245,25 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint64_t off_q = (uint64_t)((((kk >> 2) * (C::M * 128)) + (kk & 3) * 32) >> 4);
                     const uint64_t off_k = (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4);
-                    umma_bf16_ss(tmem + C::colS(e & 1), dq + off_q, dk + off_k, idesc_s, kk > 0 ? 1u : 0u);
+                    (void)off_q;
+                    umma_bf16_ts(tmem + C::colS(e & 1), tmem + C::COL_QA + kk * 8, dk + off_k, idesc_s,
+                                 kk > 0 ? 1u : 0u);
                 }
                 umma_commit(bar_ke(st));
                 umma_commit(bar_sf(e & 1));
                 issued = true;
                 return true;
             };
-            if (mbar_wait(bar_q, 0, ctl) && issue_s(0) && (len < 2 || issue_s(1))) {
+            const bool q_ok = mbar_wait(bar_q, 0, ctl);
+            if (q_ok) {  // Q into TMEM, in issue order before every S MMA
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    tmem_cp_128x256b(tmem + C::COL_QA + kk * 8,
+                                     dq + (uint64_t)((((kk >> 2) * (C::M * 128)) + (kk & 3) * 32) >> 4));
+                issued = true;
+            }
+            if (q_ok && issue_s(0) && (len < 2 || issue_s(1))) {
                 for (int e = 0; e < len; ++e) {
                     const int vs = e % C::VST;
                     if (!mbar_wait(bar_p, e & 1, ctl)) break;
