@@ -24,14 +24,17 @@
 //   warp 2      scheduler, list builder and Q producer: takes the next item
 //               from the work counter, writes the item's union list and index
 //               into a double-buffered shared-memory list, loads the item's Q
-//               tiles once the previous item's S MMAs release the buffer, and
-//               prefetches the next item's Q into L2.
+//               tiles once the previous item releases the shared-memory Q
+//               buffer, and prefetches the next item's Q into L2.
 //   warp 0      K/V producer: K and V of each union block, item after item,
 //               into an ST-stage ring (TMA, SWIZZLE_128B, 64-column panels).
 //   warp 1      owns TMEM; one thread issues tcgen05.mma:
-//               S_t = Q_t K^T (A and B from shared memory) into TMEM, and
-//               O_t += P_t V with P_t read from TMEM (A operand) and V from
-//               shared memory (MN-major B operand).
+//               S_t = Q_t K^T into TMEM (with 64-key blocks Q_t is first
+//               copied into TMEM by tcgen05.cp and the MMA reads only K from
+//               shared memory, which frees the Q buffer at the start of the
+//               item; with 128-key blocks both operands come from shared
+//               memory), and O_t += P_t V with P_t read from TMEM (A operand)
+//               and V from shared memory (MN-major B operand).
 //   warps 4..7  softmax of tile 0, warps 8..11 softmax of tile 1: thread = one
 //               query row = one TMEM lane. Loads its S row of a group, masks
 //               (union tag bit of its query block; token causality where the
@@ -43,8 +46,9 @@
 // its tile, the tensor core runs the other tile's MMAs.
 //
 // Ordering facts the pipeline relies on:
-//  * tcgen05.mma ops of one thread execute in issue order and a commit tracks
-//    all earlier ones. S_t(next) is issued after PV_t(current), so when the
+//  * tcgen05.mma and tcgen05.cp ops of one thread execute in issue order and a
+//    commit tracks all earlier ones (so the next item's Q copy lands after
+//    the current item's last S MMA has read Q from TMEM). S_t(next) is issued after PV_t(current), so when the
 //    softmax sees S_t(next) complete, PV_t(current) has finished: P_t's TMEM
 //    columns (aliased on S_t) are free and O_t is stable for a rescale.
 //  * A tile's first P of the next item is published only after its warpgroup

@@ -6,9 +6,11 @@ stream, and turns status codes into exceptions. There is no fallback: if the
 library is missing or a call fails, it raises.
 
 Entry points mirror the C ABI in ``include/s2attn.h``:
-``build_layout``, ``build_layout_ranges`` and ``build_layout_mask`` (host),
-``prefill``, ``decode``, ``decode_noalloc``, ``decode_workspace_size``,
-``device_status`` and ``set_wait_timeout_ns``.
+``build_layout``, ``build_layout_ranges``, ``build_layout_mask`` and
+``Layout.transposed`` (host; the last also builds the backward's key tiles),
+``prefill`` (grouped K/V heads when k, v have fewer heads), ``backward``,
+``chunk_prefill``, ``decode``, ``decode_noalloc``, ``decode_workspace_size``,
+``backward_workspace_size``, ``device_status`` and ``set_wait_timeout_ns``.
 """
 from __future__ import annotations
 
