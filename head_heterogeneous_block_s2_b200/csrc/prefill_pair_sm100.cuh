@@ -88,9 +88,9 @@ struct PairCfg {
     static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;  // [stage][panel][BK rows x 128 B]
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
     static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
-    // barriers: q_full, q_empty, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2],
-    // pv_done[2], drain, list_full[2], list_empty[2]
-    static constexpr int NBAR = 2 + 3 * ST + 6 + 1 + 4;
+    // barriers: q_full, q_empty, kv_full[ST] (K and V of a stage), kv_empty[ST], s_full[2],
+    // p_full[2], pv_done[2], drain, list_full[2], list_empty[2]
+    static constexpr int NBAR = 2 + 2 * ST + 6 + 1 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
@@ -171,15 +171,17 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
     const uint32_t bar_q = sb + C::OFF_BAR;
     const uint32_t bar_qe = sb + C::OFF_BAR + 8u;
+    // K and V of a stage land on one barrier: the MMA thread waits once per
+    // block (the loads run well ahead of it; a separate V barrier only added a
+    // wait to its critical path).
     auto bar_kf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + s); };
-    auto bar_vf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + C::ST + s); };
-    auto bar_ke = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + 2 * C::ST + s); };
-    auto bar_sf = [&](int t) { return sb + C::OFF_BAR + 8u * (2 + 3 * C::ST + t); };
-    auto bar_pf = [&](int t) { return sb + C::OFF_BAR + 8u * (4 + 3 * C::ST + t); };
-    auto bar_pv = [&](int t) { return sb + C::OFF_BAR + 8u * (6 + 3 * C::ST + t); };
-    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (8 + 3 * C::ST);
-    auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (9 + 3 * C::ST + b); };
-    auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (11 + 3 * C::ST + b); };
+    auto bar_ke = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + C::ST + s); };
+    auto bar_sf = [&](int t) { return sb + C::OFF_BAR + 8u * (2 + 2 * C::ST + t); };
+    auto bar_pf = [&](int t) { return sb + C::OFF_BAR + 8u * (4 + 2 * C::ST + t); };
+    auto bar_pv = [&](int t) { return sb + C::OFF_BAR + 8u * (6 + 2 * C::ST + t); };
+    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (8 + 2 * C::ST);
+    auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (9 + 2 * C::ST + b); };
+    auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (11 + 2 * C::ST + b); };
     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
     // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
@@ -193,7 +195,6 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         mbar_init(bar_qe, 1);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_kf(s), 1);
-            mbar_init(bar_vf(s), 1);
             mbar_init(bar_ke(s), 1);
         }
         for (int t = 0; t < 2; ++t) {
@@ -298,24 +299,21 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         break;
                     }
                     const int32_t krow = list_j(L[e]) * BK;
-                    mbar_arrive_expect_tx(bar_kf(st), C::KVBYTES);
+                    mbar_arrive_expect_tx(bar_kf(st), 2 * C::KVBYTES);
 #pragma unroll
                     for (int pn = 0; pn < HD / 64; ++pn)
                         tma_load_3d(sb + C::OFF_K + pn * C::KPANEL + st * (BK * 128), &tmK, pn * 64, krow,
                                     I.bkv, bar_kf(st));
-                    mbar_arrive_expect_tx(bar_vf(st), C::KVBYTES);
 #pragma unroll
                     for (int pn = 0; pn < HD / 64; ++pn)
                         tma_load_3d(sb + C::OFF_V + st * C::KVBYTES + pn * (BK * 128), &tmV, pn * 64,
-                                    krow, I.bkv, bar_vf(st));
+                                    krow, I.bkv, bar_kf(st));
                 }
                 if (!stop) mbar_arrive(bar_le(b));
             }
             if (*abort_cta)  // let this CTA's own loads land before exit
-                for (int m = (n > C::ST ? n - C::ST : 0); m < n; ++m) {
+                for (int m = (n > C::ST ? n - C::ST : 0); m < n; ++m)
                     mbar_drain(bar_kf(m % C::ST), (m / C::ST) & 1, kDrainNs);
-                    mbar_drain(bar_vf(m % C::ST), (m / C::ST) & 1, kDrainNs);
-                }
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -399,11 +397,6 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         if (!mbar_wait(bar_kf((n0 + i) % C::ST), ((n0 + i) / C::ST) & 1, ctl)) return false;
                     return true;
                 };
-                auto wait_v = [&](int n0) {
-                    for (int i = 0; i < G; ++i)
-                        if (!mbar_wait(bar_vf((n0 + i) % C::ST), ((n0 + i) / C::ST) & 1, ctl)) return false;
-                    return true;
-                };
                 int bits = gbits(0);
                 if (!wait_k(n)) break;
                 tc_fence_after();
@@ -415,9 +408,11 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     const int st = n % C::ST;
                     const int st1 = (n + G) % C::ST;
                     if (last && !C::Q_IN_TMEM) umma_commit(bar_qe);  // no more S MMAs of this item read Q
-                    bool v_ready = false, k_next_ready = false;
+                    // K and V of this group landed together: S of the group was issued
+                    // after waiting for them (or the malformed case below waits)
+                    bool k_next_ready = false;
                     if (bits == 0) {  // malformed group no tile sees: let its loads land first
-                        if (!wait_k(n) || !wait_v(n)) {
+                        if (!wait_k(n)) {
                             fail = true;
                             break;
                         }
@@ -426,10 +421,6 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     for (int t = 0; t < 2 && !fail; ++t) {
                         if (tile_sees<BK>(bits, t)) {
                             if (!mbar_wait(bar_pf(t), pvc[t] & 1, ctl)) { fail = true; break; }
-                            if (!v_ready) {
-                                if (!wait_v(n)) { fail = true; break; }
-                                v_ready = true;
-                            }
                             tc_fence_after();
                             issue_pv(t, st);
                         }
