@@ -353,7 +353,6 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     umma_bf16_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, dv, idesc_o,
                                  kk > 0 ? 1u : acc0);
                 }
-                umma_commit(bar_pv(t));
                 ++pvc[t];
                 first_pv[t] = false;
             };
@@ -442,7 +441,13 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     }
                     bits = nbits;
                 }
-                if (!fail) mbar_arrive(bar_le(b));
+                if (!fail) {
+                    // O_t of this item is complete once its last PV is: one commit per
+                    // tile and item (the softmax reads O only in the epilogue)
+                    for (int t = 0; t < 2; ++t)
+                        if (!first_pv[t]) umma_commit(bar_pv(t));
+                    mbar_arrive(bar_le(b));
+                }
             }
             if (*abort_cta && issued) {
                 umma_commit(bar_dr);
@@ -458,6 +463,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const float sc = p.scale_log2;              // > 0
         int cnt = 0;                                // S_t groups processed (all items)
+        int n_ep = 0;                               // items with a PV of this tile (pv_done phases)
         bool fail = false;
         int k = 0;
         for (; !fail; ++k) {
@@ -560,7 +566,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_le(b));
             if (cnt_item > 0) {
-                if (!warp_wait(bar_pv(t), (cnt - 1) & 1, ctl)) break;
+                if (!warp_wait(bar_pv(t), (n_ep++) & 1, ctl)) break;
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.0f / l : 0.f;
                 uint16_t* orow = p.o + (I.row_base + qpos) * HD;
