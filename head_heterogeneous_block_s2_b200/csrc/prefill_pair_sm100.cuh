@@ -28,7 +28,11 @@
 //               buffer, and prefetches the next item's Q into L2.
 //   warp 0      K/V producer: K and V of each union block, item after item,
 //               into an ST-stage ring (TMA, SWIZZLE_128B, 64-column panels).
-//   warp 1      owns TMEM; one thread issues tcgen05.mma:
+//   warp 1      owns TMEM; one thread issues tcgen05.mma (with 64-key blocks
+//               it issues tile 0's and one thread of warp 3 tile 1's, each
+//               walking the same union list, so neither tile's chain of waits
+//               and issues stalls behind the other's; a K/V stage and the Q
+//               buffer are then released when both issuers have committed):
 //               S_t = Q_t K^T into TMEM (with 64-key blocks Q_t is first
 //               copied into TMEM by tcgen05.cp and the MMA reads only K from
 //               shared memory, which frees the Q buffer at the start of the
@@ -41,13 +45,12 @@
 //               key block reaches its own block), keeps a running max and sum
 //               in the log2 domain, writes P (bf16 pairs) over the S columns
 //               in TMEM, and at the end normalises O and stores it with the LSE.
-//   warp 3      idle (it only takes part in block-wide barriers).
-// The two softmax warpgroups ping-pong: while one computes exponentials for
-// its tile, the tensor core runs the other tile's MMAs.
+// Warp 3 is otherwise idle. The two softmax warpgroups ping-pong: while one
+// computes exponentials for its tile, the tensor core runs the other tile's MMAs.
 //
 // Ordering facts the pipeline relies on:
 //  * tcgen05.mma and tcgen05.cp ops of one thread execute in issue order and a
-//    commit tracks all earlier ones (so the next item's Q copy lands after
+//    commit tracks all earlier ones of that thread (so the next item's Q copy lands after
 //    the current item's last S MMA has read Q from TMEM). S_t(next) is issued after PV_t(current), so when the
 //    softmax sees S_t(next) complete, PV_t(current) has finished: P_t's TMEM
 //    columns (aliased on S_t) are free and O_t is stable for a rescale.
@@ -89,20 +92,27 @@ struct PairCfg {
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
     static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
     // barriers: q_full, q_empty, kv_full[ST] (K and V of a stage), kv_empty[ST], s_full[2],
-    // p_full[2], pv_done[2], drain, list_full[2], list_empty[2]
-    static constexpr int NBAR = 2 + 2 * ST + 6 + 1 + 4;
+    // p_full[2], pv_done[2], drain[2], list_full[2], list_empty[2]
+    static constexpr int NBAR = 2 + 2 * ST + 6 + 2 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
     // (2 NK of S, 2 HD of O, and HD of Q when it fits; see Q_IN_TMEM)
     static constexpr uint32_t TMEM_COLS = (2 * NK + 3 * HD) <= 256 ? 256 : 512;
-    // list_empty arrivals per item: K/V producer, MMA issuer, 8 softmax warps
-    static constexpr uint32_t LIST_CONSUMERS = 10;
+    // MMA issuer threads. With 64-key blocks the single issuer's chain of waits
+    // and issues bounded the kernel (measured: one issuer per tile ran 13%
+    // faster); with 128-key blocks each group's MMAs are twice as long and one
+    // issuer keeps the tiles' MMAs apart, so one softmax warpgroup computes while
+    // the other tile's MMAs run (measured: two issuers 10% slower there).
+    static constexpr int ISSUERS = BK == 64 ? 2 : 1;
+    // list_empty arrivals per item: K/V producer, MMA issuer(s), 8 softmax warps
+    static constexpr uint32_t LIST_CONSUMERS = 9 + ISSUERS;
     __host__ __device__ static constexpr uint32_t colS(int t) { return (uint32_t)(t * NK); }
     __host__ __device__ static constexpr uint32_t colO(int t) { return (uint32_t)(2 * NK + t * HD); }
     // With 64-key blocks TMEM has room for both tiles' Q (HD/2 columns each):
     // S = Q K^T then reads Q from TMEM and only K from shared memory.
     static constexpr bool Q_IN_TMEM = 2 * NK + 2 * HD + HD <= 512;
+    static_assert(ISSUERS == 1 || Q_IN_TMEM, "the two-issuer path reads Q from TMEM");
     __host__ __device__ static constexpr uint32_t colQ(int t) { return (uint32_t)(2 * NK + 2 * HD + t * (HD / 2)); }
     static_assert(2 * NK + 2 * HD <= 512, "TMEM budget");
     static_assert(!Q_IN_TMEM || 2 * NK + 3 * HD <= (int)TMEM_COLS, "Q columns inside the allocation");
@@ -179,9 +189,9 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     auto bar_sf = [&](int t) { return sb + C::OFF_BAR + 8u * (2 + 2 * C::ST + t); };
     auto bar_pf = [&](int t) { return sb + C::OFF_BAR + 8u * (4 + 2 * C::ST + t); };
     auto bar_pv = [&](int t) { return sb + C::OFF_BAR + 8u * (6 + 2 * C::ST + t); };
-    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (8 + 2 * C::ST);
-    auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (9 + 2 * C::ST + b); };
-    auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (11 + 2 * C::ST + b); };
+    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (8 + 2 * C::ST);  // [2]: one per MMA issuer
+    auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (10 + 2 * C::ST + b); };
+    auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (12 + 2 * C::ST + b); };
     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
     // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
@@ -192,10 +202,10 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        mbar_init(bar_qe, 1);
+        mbar_init(bar_qe, C::ISSUERS);  // one commit per MMA issuer
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_kf(s), 1);
-            mbar_init(bar_ke(s), 1);
+            mbar_init(bar_ke(s), C::ISSUERS);  // one commit per MMA issuer
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar_sf(t), 1);
@@ -205,6 +215,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             mbar_init(bar_le(t), C::LIST_CONSUMERS);
         }
         mbar_init(bar_dr, 1);
+        mbar_init(bar_dr + 8u, 1);
         *abort_cta = 0;
         fence_mbar_init();
     }
@@ -316,142 +327,267 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     mbar_drain(bar_kf(m % C::ST), (m / C::ST) & 1, kDrainNs);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc(128, C::NK, 0, 0);
-            constexpr uint32_t idesc_o = umma_idesc(128, HD, 0, 1);
-            constexpr int KSTEPS_BLK = BK / 16;  // PV k-steps per key block
-            bool issued = false, fail = false;
-            int pvc[2] = {0, 0};  // PV groups issued per tile (all items)
-            bool first_pv[2] = {true, true};
-            int n = 0;            // union elements consumed (all items); a multiple of G
-            // S_t = Q_t K^T over the G blocks of the group starting at stage st (N = 128).
-            auto issue_s = [&](int t, int st) {
-                const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
-                const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * (BK * 128), 16, 1024);
+    } else if (warp == 1 || (C::ISSUERS == 2 && warp == 3)) {
+        // ------------------------------------------------------------ MMA issuer(s)
+        // Two code paths, each the faster one measured for its block size: a
+        // generic loop over a tile range ran slower than either.
+        if constexpr (C::ISSUERS == 2) {
+            // One thread per tile (warp 1: tile 0, warp 3: tile 1), each walking
+            // the same union list; Q is in TMEM (Q_IN_TMEM holds for 64-key
+            // blocks), so S reads only K from shared memory.
+            if (lane == 0) {
+                const int T = warp == 1 ? 0 : 1;
+                constexpr uint32_t idesc_s = umma_idesc(128, C::NK, 0, 0);
+                constexpr uint32_t idesc_o = umma_idesc(128, HD, 0, 1);
+                constexpr int KSTEPS_BLK = BK / 16;  // PV k-steps per key block
+                bool issued = false, fail = false;
+                int pvc = 0;          // PV groups issued for tile T (all items)
+                bool first_pv = true;
+                int n = 0;            // union elements consumed (all items); a multiple of G
+                // S_T = Q_T K^T over the G blocks of the group starting at stage st.
+                auto issue_s = [&](int st) {
+                    const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * (BK * 128), 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint64_t bk = dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4);
-                    if constexpr (C::Q_IN_TMEM)
-                        umma_bf16_ts(tmem + C::colS(t), tmem + C::colQ(t) + kk * 8, bk, idesc_s, kk > 0 ? 1u : 0u);
-                    else
-                        umma_bf16_ss(tmem + C::colS(t), dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
-                                     bk, idesc_s, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(bar_sf(t));
-                issued = true;
-            };
-            // O_t += P_t V over the group's G blocks (stages st .. st+G-1).
-            auto issue_pv = [&](int t, int st) {
-                const uint32_t acc0 = first_pv[t] ? 0u : 1u;
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        const uint64_t bk = dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4);
+                        umma_bf16_ts(tmem + C::colS(T), tmem + C::colQ(T) + kk * 8, bk, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar_sf(T));
+                    issued = true;
+                };
+                // O_T += P_T V over the group's G blocks (stages st .. st+G-1).
+                auto issue_pv = [&](int st) {
+                    const uint32_t acc0 = first_pv ? 0u : 1u;
 #pragma unroll
-                for (int kk = 0; kk < C::NK / 16; ++kk) {
-                    const int s = st + kk / KSTEPS_BLK;
-                    const uint64_t dv = umma_sdesc(sb + C::OFF_V + s * C::KVBYTES + (kk % KSTEPS_BLK) * 2048,
-                                                   BK * 128, 1024);
-                    umma_bf16_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, dv, idesc_o,
-                                 kk > 0 ? 1u : acc0);
-                }
-                ++pvc[t];
-                first_pv[t] = false;
-            };
-            int k = 0;
-            for (; !fail; ++k) {
-                const int b = k & 1;
-                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
-                if (list_item[b] < 0) break;
-                const uint32_t* L = list + b * C::LIST_CAP;
-                const int len = list_len[b];
-                if (!mbar_wait(bar_q, k & 1, ctl)) break;
-                if (len == 0) {
-                    umma_commit(bar_qe);
-                    mbar_arrive(bar_le(b));
-                    continue;
-                }
-                if constexpr (C::Q_IN_TMEM) {
-                    // Q of both tiles into TMEM (after the previous item's S MMAs, in
-                    // issue order), then the shared-memory Q buffer is free at once.
+                    for (int kk = 0; kk < C::NK / 16; ++kk) {
+                        const int s = st + kk / KSTEPS_BLK;
+                        const uint64_t dv = umma_sdesc(sb + C::OFF_V + s * C::KVBYTES + (kk % KSTEPS_BLK) * 2048,
+                                                       BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::colO(T), tmem + C::colS(T) + kk * 8, dv, idesc_o,
+                                     kk > 0 ? 1u : acc0);
+                    }
+                    ++pvc;
+                    first_pv = false;
+                };
+                int k = 0;
+                for (; !fail; ++k) {
+                    const int b = k & 1;
+                    if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                    if (list_item[b] < 0) break;
+                    const uint32_t* L = list + b * C::LIST_CAP;
+                    const int len = list_len[b];
+                    if (!mbar_wait(bar_q, k & 1, ctl)) break;
+                    if (len == 0) {
+                        umma_commit(bar_qe);
+                        mbar_arrive(bar_le(b));
+                        continue;
+                    }
+                    const bool mine = T == 0 || pair_item<BK>(p, list_item[b]).tile1;  // tile T exists
+                    // Q_T into TMEM (after this tile's previous S MMAs, in issue order),
+                    // then this issuer's share of the shared-memory Q buffer is free.
                     tc_fence_after();
-                    const bool two = pair_item<BK>(p, list_item[b]).tile1;
-                    for (int t = 0; t < (two ? 2 : 1); ++t) {
-                        const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
+                    if (mine) {
+                        const uint64_t dq = umma_sdesc(sb + C::OFF_Q + T * C::QBYTES, 16, 1024);
 #pragma unroll
                         for (int kk = 0; kk < HD / 16; ++kk)
-                            tmem_cp_128x256b(tmem + C::colQ(t) + kk * 8,
+                            tmem_cp_128x256b(tmem + C::colQ(T) + kk * 8,
                                              dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4));
                     }
                     umma_commit(bar_qe);
-                }
-                const int ngroups = len / G;
-                first_pv[0] = first_pv[1] = true;
-                auto gbits = [&](int g) {
-                    int bits = 0;
+                    const int ngroups = len / G;
+                    first_pv = true;
+                    auto gbits = [&](int g) {
+                        int bits = 0;
 #pragma unroll
-                    for (int i = 0; i < G; ++i) bits |= list_bits(L[g * G + i]);
-                    return bits;
-                };
-                auto wait_k = [&](int n0) {
-                    for (int i = 0; i < G; ++i)
-                        if (!mbar_wait(bar_kf((n0 + i) % C::ST), ((n0 + i) / C::ST) & 1, ctl)) return false;
-                    return true;
-                };
-                int bits = gbits(0);
-                if (!wait_k(n)) break;
-                tc_fence_after();
-                for (int t = 0; t < 2; ++t)
-                    if (tile_sees<BK>(bits, t)) issue_s(t, n % C::ST);
-                for (int g = 0;; ++g, n += G) {
-                    const bool last = g + 1 == ngroups;
-                    const int nbits = last ? 0 : gbits(g + 1);
-                    const int st = n % C::ST;
-                    const int st1 = (n + G) % C::ST;
-                    if (last && !C::Q_IN_TMEM) umma_commit(bar_qe);  // no more S MMAs of this item read Q
-                    // K and V of this group landed together: S of the group was issued
-                    // after waiting for them (or the malformed case below waits)
-                    bool k_next_ready = false;
-                    if (bits == 0) {  // malformed group no tile sees: let its loads land first
-                        if (!wait_k(n)) {
-                            fail = true;
+                        for (int i = 0; i < G; ++i) bits |= list_bits(L[g * G + i]);
+                        return bits;
+                    };
+                    auto wait_k = [&](int n0) {
+                        for (int i = 0; i < G; ++i)
+                            if (!mbar_wait(bar_kf((n0 + i) % C::ST), ((n0 + i) / C::ST) & 1, ctl)) return false;
+                        return true;
+                    };
+                    int bits = gbits(0);
+                    if (mine && tile_sees<BK>(bits, T)) {
+                        if (!wait_k(n)) break;
+                        tc_fence_after();
+                        issue_s(n % C::ST);
+                    }
+                    for (int g = 0;; ++g, n += G) {
+                        const bool last = g + 1 == ngroups;
+                        const int nbits = last ? 0 : gbits(g + 1);
+                        const int st = n % C::ST;
+                        const int st1 = (n + G) % C::ST;
+                        if (!(mine && tile_sees<BK>(bits, T))) {
+                            // a group this tile skips: let its loads land before releasing the stage
+                            if (!wait_k(n)) {
+                                fail = true;
+                                break;
+                            }
+                        } else {
+                            if (!mbar_wait(bar_pf(T), pvc & 1, ctl)) { fail = true; break; }
+                            tc_fence_after();
+                            issue_pv(st);
+                        }
+                        for (int i = 0; i < G; ++i) umma_commit(bar_ke(st + i));
+                        if (!last && mine && tile_sees<BK>(nbits, T)) {
+                            if (!wait_k(n + G)) { fail = true; break; }
+                            tc_fence_after();
+                            issue_s(st1);
+                        }
+                        if (last) {
+                            n += G;
                             break;
                         }
+                        bits = nbits;
                     }
-                    const int last_t = tile_sees<BK>(bits, 1) ? 1 : (tile_sees<BK>(bits, 0) ? 0 : 1);
-                    for (int t = 0; t < 2 && !fail; ++t) {
-                        if (tile_sees<BK>(bits, t)) {
-                            if (!mbar_wait(bar_pf(t), pvc[t] & 1, ctl)) { fail = true; break; }
-                            tc_fence_after();
-                            issue_pv(t, st);
-                        }
-                        if (t == last_t)
-                            for (int i = 0; i < G; ++i) umma_commit(bar_ke(st + i));
-                        if (!last && tile_sees<BK>(nbits, t)) {
-                            if (!k_next_ready) {
-                                if (!wait_k(n + G)) { fail = true; break; }
-                                k_next_ready = true;
-                                tc_fence_after();
-                            }
-                            issue_s(t, st1);
-                        }
+                    if (!fail) {
+                        // O_T of this item is complete once its last PV is
+                        if (!first_pv) umma_commit(bar_pv(T));
+                        mbar_arrive(bar_le(b));
                     }
-                    if (fail) break;
-                    if (last) {
-                        n += G;
-                        break;
-                    }
-                    bits = nbits;
                 }
-                if (!fail) {
-                    // O_t of this item is complete once its last PV is: one commit per
-                    // tile and item (the softmax reads O only in the epilogue)
-                    for (int t = 0; t < 2; ++t)
-                        if (!first_pv[t]) umma_commit(bar_pv(t));
-                    mbar_arrive(bar_le(b));
+                if (*abort_cta && issued) {
+                    umma_commit(bar_dr + 8u * T);
+                    mbar_drain(bar_dr + 8u * T, 0, kDrainNs);
                 }
             }
-            if (*abort_cta && issued) {
-                umma_commit(bar_dr);
-                mbar_drain(bar_dr, 0, kDrainNs);
+        } else {
+            if (lane == 0) {
+                constexpr uint32_t idesc_s = umma_idesc(128, C::NK, 0, 0);
+                constexpr uint32_t idesc_o = umma_idesc(128, HD, 0, 1);
+                constexpr int KSTEPS_BLK = BK / 16;  // PV k-steps per key block
+                bool issued = false, fail = false;
+                int pvc[2] = {0, 0};  // PV groups issued per tile (all items)
+                bool first_pv[2] = {true, true};
+                int n = 0;            // union elements consumed (all items); a multiple of G
+                // S_t = Q_t K^T over the G blocks of the group starting at stage st (N = 128).
+                auto issue_s = [&](int t, int st) {
+                    const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
+                    const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * (BK * 128), 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        const uint64_t bk = dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4);
+                        if constexpr (C::Q_IN_TMEM)
+                            umma_bf16_ts(tmem + C::colS(t), tmem + C::colQ(t) + kk * 8, bk, idesc_s, kk > 0 ? 1u : 0u);
+                        else
+                            umma_bf16_ss(tmem + C::colS(t), dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
+                                         bk, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar_sf(t));
+                    issued = true;
+                };
+                // O_t += P_t V over the group's G blocks (stages st .. st+G-1).
+                auto issue_pv = [&](int t, int st) {
+                    const uint32_t acc0 = first_pv[t] ? 0u : 1u;
+#pragma unroll
+                    for (int kk = 0; kk < C::NK / 16; ++kk) {
+                        const int s = st + kk / KSTEPS_BLK;
+                        const uint64_t dv = umma_sdesc(sb + C::OFF_V + s * C::KVBYTES + (kk % KSTEPS_BLK) * 2048,
+                                                       BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, dv, idesc_o,
+                                     kk > 0 ? 1u : acc0);
+                    }
+                    ++pvc[t];
+                    first_pv[t] = false;
+                };
+                int k = 0;
+                for (; !fail; ++k) {
+                    const int b = k & 1;
+                    if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                    if (list_item[b] < 0) break;
+                    const uint32_t* L = list + b * C::LIST_CAP;
+                    const int len = list_len[b];
+                    if (!mbar_wait(bar_q, k & 1, ctl)) break;
+                    if (len == 0) {
+                        umma_commit(bar_qe);
+                        mbar_arrive(bar_le(b));
+                        continue;
+                    }
+                    if constexpr (C::Q_IN_TMEM) {
+                        // Q of both tiles into TMEM (after the previous item's S MMAs, in
+                        // issue order), then the shared-memory Q buffer is free at once.
+                        tc_fence_after();
+                        const bool two = pair_item<BK>(p, list_item[b]).tile1;
+                        for (int t = 0; t < (two ? 2 : 1); ++t) {
+                            const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < HD / 16; ++kk)
+                                tmem_cp_128x256b(tmem + C::colQ(t) + kk * 8,
+                                                 dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4));
+                        }
+                        umma_commit(bar_qe);
+                    }
+                    const int ngroups = len / G;
+                    first_pv[0] = first_pv[1] = true;
+                    auto gbits = [&](int g) {
+                        int bits = 0;
+#pragma unroll
+                        for (int i = 0; i < G; ++i) bits |= list_bits(L[g * G + i]);
+                        return bits;
+                    };
+                    auto wait_k = [&](int n0) {
+                        for (int i = 0; i < G; ++i)
+                            if (!mbar_wait(bar_kf((n0 + i) % C::ST), ((n0 + i) / C::ST) & 1, ctl)) return false;
+                        return true;
+                    };
+                    int bits = gbits(0);
+                    if (!wait_k(n)) break;
+                    tc_fence_after();
+                    for (int t = 0; t < 2; ++t)
+                        if (tile_sees<BK>(bits, t)) issue_s(t, n % C::ST);
+                    for (int g = 0;; ++g, n += G) {
+                        const bool last = g + 1 == ngroups;
+                        const int nbits = last ? 0 : gbits(g + 1);
+                        const int st = n % C::ST;
+                        const int st1 = (n + G) % C::ST;
+                        if (last && !C::Q_IN_TMEM) umma_commit(bar_qe);  // no more S MMAs of this item read Q
+                        // K and V of this group landed together: S of the group was issued
+                        // after waiting for them (or the malformed case below waits)
+                        bool k_next_ready = false;
+                        if (bits == 0) {  // malformed group no tile sees: let its loads land first
+                            if (!wait_k(n)) {
+                                fail = true;
+                                break;
+                            }
+                        }
+                        const int last_t = tile_sees<BK>(bits, 1) ? 1 : (tile_sees<BK>(bits, 0) ? 0 : 1);
+                        for (int t = 0; t < 2 && !fail; ++t) {
+                            if (tile_sees<BK>(bits, t)) {
+                                if (!mbar_wait(bar_pf(t), pvc[t] & 1, ctl)) { fail = true; break; }
+                                tc_fence_after();
+                                issue_pv(t, st);
+                            }
+                            if (t == last_t)
+                                for (int i = 0; i < G; ++i) umma_commit(bar_ke(st + i));
+                            if (!last && tile_sees<BK>(nbits, t)) {
+                                if (!k_next_ready) {
+                                    if (!wait_k(n + G)) { fail = true; break; }
+                                    k_next_ready = true;
+                                    tc_fence_after();
+                                }
+                                issue_s(t, st1);
+                            }
+                        }
+                        if (fail) break;
+                        if (last) {
+                            n += G;
+                            break;
+                        }
+                        bits = nbits;
+                    }
+                    if (!fail) {
+                        // O_t of this item is complete once its last PV is: one commit per
+                        // tile and item (the softmax reads O only in the epilogue)
+                        for (int t = 0; t < 2; ++t)
+                            if (!first_pv[t]) umma_commit(bar_pv(t));
+                        mbar_arrive(bar_le(b));
+                    }
+                }
+                if (*abort_cta && issued) {
+                    umma_commit(bar_dr);
+                    mbar_drain(bar_dr, 0, kDrainNs);
+                }
             }
         }
         __syncwarp();
