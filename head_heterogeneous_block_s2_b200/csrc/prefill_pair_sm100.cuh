@@ -28,32 +28,41 @@
 //               buffer, and prefetches the next item's Q into L2.
 //   warp 0      K/V producer: K and V of each union block, item after item,
 //               into an ST-stage ring (TMA, SWIZZLE_128B, 64-column panels).
-//   warp 1      owns TMEM; one thread issues tcgen05.mma (with 64-key blocks
-//               it issues tile 0's and one thread of warp 3 tile 1's, each
-//               walking the same union list, so neither tile's chain of waits
-//               and issues stalls behind the other's; a K/V stage and the Q
-//               buffer are then released when both issuers have committed):
-//               S_t = Q_t K^T into TMEM (with 64-key blocks Q_t is first
-//               copied into TMEM by tcgen05.cp and the MMA reads only K from
-//               shared memory, which frees the Q buffer at the start of the
-//               item; with 128-key blocks both operands come from shared
-//               memory), and O_t += P_t V with P_t read from TMEM (A operand)
-//               and V from shared memory (MN-major B operand).
+//   warp 1      owns TMEM; one thread issues the tcgen05.mma ops
+//               S_t = Q_t K^T into TMEM and O_t += P_t V with P_t read from
+//               TMEM (A operand) and V from shared memory (MN-major B operand).
 //   warps 4..7  softmax of tile 0, warps 8..11 softmax of tile 1: thread = one
 //               query row = one TMEM lane. Loads its S row of a group, masks
 //               (union tag bit of its query block; token causality where the
 //               key block reaches its own block), keeps a running max and sum
 //               in the log2 domain, writes P (bf16 pairs) over the S columns
 //               in TMEM, and at the end normalises O and stores it with the LSE.
-// Warp 3 is otherwise idle. The two softmax warpgroups ping-pong: while one
-// computes exponentials for its tile, the tensor core runs the other tile's MMAs.
 //
-// Ordering facts the pipeline relies on:
+// Two pipelines, chosen by block size (PairCfg):
+//  * 64-key blocks (SDB): each tile has two S buffers in TMEM, and S of the
+//    tile's next two blocks is issued ahead of the softmax, so the tensor core
+//    computes S of block i+1 while the softmax works on block i. One thread of
+//    warp 1 issues tile 0's MMAs and one of warp 3 tile 1's, each walking the
+//    same union list; a K/V stage and the Q buffer are released when both
+//    have committed. Q stays in shared memory (TMEM is full).
+//  * 128-key blocks: one S buffer per tile and one issuer for both tiles; the
+//    two softmax warpgroups ping-pong (while one computes exponentials for its
+//    tile, the tensor core runs the other tile's MMAs). When TMEM has room
+//    (head dim 64), Q is copied into TMEM by tcgen05.cp at the start of the
+//    item and S reads only K from shared memory. Warp 3 is idle.
+//
+// Ordering facts the pipelines rely on:
 //  * tcgen05.mma and tcgen05.cp ops of one thread execute in issue order and a
-//    commit tracks all earlier ones of that thread (so the next item's Q copy lands after
-//    the current item's last S MMA has read Q from TMEM). S_t(next) is issued after PV_t(current), so when the
+//    commit tracks all earlier ones of that thread (so the next item's Q copy
+//    lands after the current item's last S MMA has read Q from TMEM).
+//  * One S buffer: S_t(next) is issued after PV_t(current), so when the
 //    softmax sees S_t(next) complete, PV_t(current) has finished: P_t's TMEM
 //    columns (aliased on S_t) are free and O_t is stable for a rescale.
+//  * Two S buffers: S_t(i+2) is issued after PV_t(i) (same buffer). The
+//    softmax waits for PV_t(i-1)'s own commit before it rescales O_t at block
+//    i and before the epilogue; S_t(i) complete implies PV_t(i-2) complete, so
+//    that barrier's phase cannot alias. Every S/P barrier is per buffer, for
+//    the same reason.
 //  * A tile's first P of the next item is published only after its warpgroup
 //    has read O out of TMEM (tcgen05.wait::ld) for the previous item, so the
 //    next item's first PV (which overwrites O) cannot race the epilogue.
@@ -91,31 +100,33 @@ struct PairCfg {
     static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;  // [stage][panel][BK rows x 128 B]
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
     static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
-    // barriers: q_full, q_empty, kv_full[ST] (K and V of a stage), kv_empty[ST], s_full[2],
-    // p_full[2], pv_done[2], drain[2], list_full[2], list_empty[2]
-    static constexpr int NBAR = 2 + 2 * ST + 6 + 2 + 4;
+    // barriers: q_full, q_empty, kv_full[ST] (K and V of a stage), kv_empty[ST],
+    // s_full[2][2], p_full[2][2], pv_done[2][2] ([tile][S buffer]), drain[2],
+    // list_full[2], list_empty[2]
+    static constexpr int NBAR = 2 + 2 * ST + 12 + 2 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
-    // (2 NK of S, 2 HD of O, and HD of Q when it fits; see Q_IN_TMEM)
-    static constexpr uint32_t TMEM_COLS = (2 * NK + 3 * HD) <= 256 ? 256 : 512;
-    // MMA issuer threads. With 64-key blocks the single issuer's chain of waits
-    // and issues bounded the kernel (measured: one issuer per tile ran 13%
-    // faster); with 128-key blocks each group's MMAs are twice as long and one
-    // issuer keeps the tiles' MMAs apart, so one softmax warpgroup computes while
-    // the other tile's MMAs run (measured: two issuers 10% slower there).
-    static constexpr int ISSUERS = BK == 64 ? 2 : 1;
+    // S double-buffered per tile (64-key blocks): the S MMA of a tile's next
+    // block runs while the softmax works on the current one, so a tile's chain
+    // is no longer S -> softmax -> PV -> S. Takes 4 NK + 2 HD TMEM columns, so
+    // Q stays in shared memory. This pipeline has one MMA issuer per tile
+    // (warp 1: tile 0, warp 3: tile 1).
+    static constexpr bool SDB = BK == 64 && 4 * NK + 2 * HD <= 512;
+    static constexpr int SBUF = SDB ? 2 : 1;
+    static constexpr int ISSUERS = SDB ? 2 : 1;
     // list_empty arrivals per item: K/V producer, MMA issuer(s), 8 softmax warps
     static constexpr uint32_t LIST_CONSUMERS = 9 + ISSUERS;
-    __host__ __device__ static constexpr uint32_t colS(int t) { return (uint32_t)(t * NK); }
-    __host__ __device__ static constexpr uint32_t colO(int t) { return (uint32_t)(2 * NK + t * HD); }
-    // With 64-key blocks TMEM has room for both tiles' Q (HD/2 columns each):
-    // S = Q K^T then reads Q from TMEM and only K from shared memory.
-    static constexpr bool Q_IN_TMEM = 2 * NK + 2 * HD + HD <= 512;
-    static_assert(ISSUERS == 1 || Q_IN_TMEM, "the two-issuer path reads Q from TMEM");
+    __host__ __device__ static constexpr uint32_t colS(int t, int u = 0) { return (uint32_t)((t * SBUF + u) * NK); }
+    __host__ __device__ static constexpr uint32_t colO(int t) { return (uint32_t)(2 * SBUF * NK + t * HD); }
+    // Without S double-buffering, when TMEM has room for both tiles' Q (HD/2
+    // columns each) S = Q K^T reads Q from TMEM and only K from shared memory.
+    static constexpr bool Q_IN_TMEM = !SDB && 2 * NK + 3 * HD <= 512;
     __host__ __device__ static constexpr uint32_t colQ(int t) { return (uint32_t)(2 * NK + 2 * HD + t * (HD / 2)); }
-    static_assert(2 * NK + 2 * HD <= 512, "TMEM budget");
-    static_assert(!Q_IN_TMEM || 2 * NK + 3 * HD <= (int)TMEM_COLS, "Q columns inside the allocation");
+    static constexpr int TMEM_NEED = 2 * SBUF * NK + 2 * HD + (Q_IN_TMEM ? HD : 0);
+    static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
+    static_assert(TMEM_NEED <= 512, "TMEM budget");
+    static_assert(!SDB || G == 1, "the double-buffered pipeline walks single blocks");
     static_assert(ST % G == 0, "groups must not wrap the stage ring");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
@@ -186,12 +197,13 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     // wait to its critical path).
     auto bar_kf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + s); };
     auto bar_ke = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + C::ST + s); };
-    auto bar_sf = [&](int t) { return sb + C::OFF_BAR + 8u * (2 + 2 * C::ST + t); };
-    auto bar_pf = [&](int t) { return sb + C::OFF_BAR + 8u * (4 + 2 * C::ST + t); };
-    auto bar_pv = [&](int t) { return sb + C::OFF_BAR + 8u * (6 + 2 * C::ST + t); };
-    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (8 + 2 * C::ST);  // [2]: one per MMA issuer
-    auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (10 + 2 * C::ST + b); };
-    auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (12 + 2 * C::ST + b); };
+    // [tile][S buffer]
+    auto bar_sf = [&](int t, int u = 0) { return sb + C::OFF_BAR + 8u * (2 + 2 * C::ST + 2 * t + u); };
+    auto bar_pf = [&](int t, int u = 0) { return sb + C::OFF_BAR + 8u * (6 + 2 * C::ST + 2 * t + u); };
+    auto bar_pv = [&](int t, int u = 0) { return sb + C::OFF_BAR + 8u * (10 + 2 * C::ST + 2 * t + u); };
+    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (14 + 2 * C::ST);  // [2]: one per MMA issuer
+    auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (16 + 2 * C::ST + b); };
+    auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (18 + 2 * C::ST + b); };
     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
     // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
@@ -208,9 +220,11 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             mbar_init(bar_ke(s), C::ISSUERS);  // one commit per MMA issuer
         }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(bar_sf(t), 1);
-            mbar_init(bar_pf(t), 128);
-            mbar_init(bar_pv(t), 1);
+            for (int u = 0; u < 2; ++u) {
+                mbar_init(bar_sf(t, u), 1);
+                mbar_init(bar_pf(t, u), 128);
+                mbar_init(bar_pv(t, u), 1);
+            }
             mbar_init(bar_lf(t), 1);
             mbar_init(bar_le(t), C::LIST_CONSUMERS);
         }
@@ -329,123 +343,94 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         __syncwarp();
     } else if (warp == 1 || (C::ISSUERS == 2 && warp == 3)) {
         // ------------------------------------------------------------ MMA issuer(s)
-        // Two code paths, each the faster one measured for its block size: a
-        // generic loop over a tile range ran slower than either.
-        if constexpr (C::ISSUERS == 2) {
+        if constexpr (C::SDB) {
             // One thread per tile (warp 1: tile 0, warp 3: tile 1), each walking
-            // the same union list; Q is in TMEM (Q_IN_TMEM holds for 64-key
-            // blocks), so S reads only K from shared memory.
+            // the same union list. S of the i-th block a tile sees goes to its S
+            // buffer i & 1 and is issued up to two blocks ahead of the PVs: S of
+            // block i + 2 reuses the buffer of block i, so it is issued after
+            // PV_i (in issue order it then runs after PV_i has read P_i).
             if (lane == 0) {
                 const int T = warp == 1 ? 0 : 1;
                 constexpr uint32_t idesc_s = umma_idesc(128, C::NK, 0, 0);
                 constexpr uint32_t idesc_o = umma_idesc(128, HD, 0, 1);
-                constexpr int KSTEPS_BLK = BK / 16;  // PV k-steps per key block
                 bool issued = false, fail = false;
-                int pvc = 0;          // PV groups issued for tile T (all items)
-                bool first_pv = true;
-                int n = 0;            // union elements consumed (all items); a multiple of G
-                // S_T = Q_T K^T over the G blocks of the group starting at stage st.
+                int sc = 0;  // S MMAs issued for tile T (all items)
+                int pc = 0;  // PV MMAs issued for tile T (all items)
+                int n0 = 0;  // union elements of the earlier items
+                const uint64_t dq = umma_sdesc(sb + C::OFF_Q + T * C::QBYTES, 16, 1024);
                 auto issue_s = [&](int st) {
                     const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * (BK * 128), 16, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
-                        const uint64_t bk = dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4);
-                        umma_bf16_ts(tmem + C::colS(T), tmem + C::colQ(T) + kk * 8, bk, idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(bar_sf(T));
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_bf16_ss(tmem + C::colS(T, sc & 1), dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
+                                     dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
+                    umma_commit(bar_sf(T, sc & 1));
+                    ++sc;
                     issued = true;
                 };
-                // O_T += P_T V over the group's G blocks (stages st .. st+G-1).
-                auto issue_pv = [&](int st) {
-                    const uint32_t acc0 = first_pv ? 0u : 1u;
+                // O_T (+)= P_T V; the per-PV commit lets the softmax wait for O before
+                // a rescale and before the epilogue.
+                auto issue_pv = [&](int st, bool first) {
 #pragma unroll
-                    for (int kk = 0; kk < C::NK / 16; ++kk) {
-                        const int s = st + kk / KSTEPS_BLK;
-                        const uint64_t dv = umma_sdesc(sb + C::OFF_V + s * C::KVBYTES + (kk % KSTEPS_BLK) * 2048,
-                                                       BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::colO(T), tmem + C::colS(T) + kk * 8, dv, idesc_o,
-                                     kk > 0 ? 1u : acc0);
-                    }
-                    ++pvc;
-                    first_pv = false;
+                    for (int kk = 0; kk < C::NK / 16; ++kk)
+                        umma_bf16_ts(tmem + C::colO(T), tmem + C::colS(T, pc & 1) + kk * 8,
+                                     umma_sdesc(sb + C::OFF_V + st * C::KVBYTES + kk * 2048, BK * 128, 1024),
+                                     idesc_o, (kk > 0 || !first) ? 1u : 0u);
+                    umma_commit(bar_pv(T, pc & 1));
+                    ++pc;
                 };
-                int k = 0;
-                for (; !fail; ++k) {
+                for (int k = 0; !fail; ++k) {
                     const int b = k & 1;
                     if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
                     if (list_item[b] < 0) break;
                     const uint32_t* L = list + b * C::LIST_CAP;
                     const int len = list_len[b];
                     if (!mbar_wait(bar_q, k & 1, ctl)) break;
-                    if (len == 0) {
-                        umma_commit(bar_qe);
-                        mbar_arrive(bar_le(b));
-                        continue;
-                    }
                     const bool mine = T == 0 || pair_item<BK>(p, list_item[b]).tile1;  // tile T exists
-                    // Q_T into TMEM (after this tile's previous S MMAs, in issue order),
-                    // then this issuer's share of the shared-memory Q buffer is free.
-                    tc_fence_after();
-                    if (mine) {
-                        const uint64_t dq = umma_sdesc(sb + C::OFF_Q + T * C::QBYTES, 16, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk)
-                            tmem_cp_128x256b(tmem + C::colQ(T) + kk * 8,
-                                             dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4));
-                    }
-                    umma_commit(bar_qe);
-                    const int ngroups = len / G;
-                    first_pv = true;
-                    auto gbits = [&](int g) {
-                        int bits = 0;
-#pragma unroll
-                        for (int i = 0; i < G; ++i) bits |= list_bits(L[g * G + i]);
-                        return bits;
-                    };
-                    auto wait_k = [&](int n0) {
-                        for (int i = 0; i < G; ++i)
-                            if (!mbar_wait(bar_kf((n0 + i) % C::ST), ((n0 + i) / C::ST) & 1, ctl)) return false;
+                    auto seen = [&](int e) { return mine && tile_sees<BK>(list_bits(L[e]), T); };
+                    int s_next = 0;      // next element to look at for an S MMA
+                    int ss = 0, ps = 0;  // S and PV MMAs of this item
+                    bool q_done = false;
+                    // S for the next blocks tile T sees: at most two ahead of the PVs,
+                    // and only blocks whose stage this thread has already released
+                    // (element s_next loads once element s_next - ST is released), so
+                    // the wait below never waits on this thread's own progress.
+                    auto ahead = [&](int e_done) {
+                        while (ss - ps < 2) {
+                            while (s_next < len && !seen(s_next)) ++s_next;
+                            if (s_next >= len || s_next > e_done + C::ST) break;
+                            const int n = n0 + s_next;
+                            if (!mbar_wait(bar_kf(n % C::ST), (n / C::ST) & 1, ctl)) return false;
+                            tc_fence_after();
+                            issue_s(n % C::ST);
+                            ++ss;
+                            ++s_next;
+                        }
+                        if (!q_done && s_next >= len) {  // no more S MMAs of this item read Q_T
+                            umma_commit(bar_qe);
+                            q_done = true;
+                        }
                         return true;
                     };
-                    int bits = gbits(0);
-                    if (mine && tile_sees<BK>(bits, T)) {
-                        if (!wait_k(n)) break;
-                        tc_fence_after();
-                        issue_s(n % C::ST);
-                    }
-                    for (int g = 0;; ++g, n += G) {
-                        const bool last = g + 1 == ngroups;
-                        const int nbits = last ? 0 : gbits(g + 1);
-                        const int st = n % C::ST;
-                        const int st1 = (n + G) % C::ST;
-                        if (!(mine && tile_sees<BK>(bits, T))) {
-                            // a group this tile skips: let its loads land before releasing the stage
-                            if (!wait_k(n)) {
-                                fail = true;
-                                break;
-                            }
-                        } else {
-                            if (!mbar_wait(bar_pf(T), pvc & 1, ctl)) { fail = true; break; }
+                    if (!ahead(-1)) break;
+                    for (int e = 0; e < len; ++e) {
+                        const int n = n0 + e, st = n % C::ST;
+                        if (seen(e)) {
+                            if (!mbar_wait(bar_pf(T, pc & 1), (pc >> 1) & 1, ctl)) { fail = true; break; }
                             tc_fence_after();
-                            issue_pv(st);
-                        }
-                        for (int i = 0; i < G; ++i) umma_commit(bar_ke(st + i));
-                        if (!last && mine && tile_sees<BK>(nbits, T)) {
-                            if (!wait_k(n + G)) { fail = true; break; }
-                            tc_fence_after();
-                            issue_s(st1);
-                        }
-                        if (last) {
-                            n += G;
+                            issue_pv(st, ps == 0);
+                            ++ps;
+                        } else if (!mbar_wait(bar_kf(st), (n / C::ST) & 1, ctl)) {
+                            // a block tile T skips: its loads land before the stage is released
+                            fail = true;
                             break;
                         }
-                        bits = nbits;
+                        umma_commit(bar_ke(st));
+                        if (!ahead(e)) { fail = true; break; }
                     }
-                    if (!fail) {
-                        // O_T of this item is complete once its last PV is
-                        if (!first_pv) umma_commit(bar_pv(T));
-                        mbar_arrive(bar_le(b));
-                    }
+                    if (fail) break;
+                    n0 += len;
+                    mbar_arrive(bar_le(b));
                 }
                 if (*abort_cta && issued) {
                     umma_commit(bar_dr + 8u * T);
@@ -626,7 +611,10 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         bits |= list_bits(ent[i]);
                     }
                     if (!tile_sees<BK>(bits, t)) continue;
-                    if (!warp_wait(bar_sf(t), cnt & 1, ctl)) {
+                    // S buffer of this block and the phase of its barriers
+                    const int u = C::SDB ? (cnt & 1) : 0;
+                    const uint32_t par = C::SDB ? ((cnt >> 1) & 1) : (cnt & 1);
+                    if (!warp_wait(bar_sf(t, u), par, ctl)) {
                         fail = true;
                         break;
                     }
@@ -634,7 +622,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     uint32_t sr[C::NK];  // S row; packed P overwrites its front as it is consumed
 #pragma unroll
                     for (int c = 0; c < C::NK / 32; ++c)
-                        tmem_ld32(tl + C::colS(t) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+                        tmem_ld32(tl + C::colS(t, u) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
                     tmem_wait_ld();
                     bool vis[G];
                     int lim[G];  // key column c of block i visible iff vis[i] && c <= lim[i]
@@ -677,10 +665,21 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     // P (bf16 pairs) over the first NK/2 columns of S_t.
 #pragma unroll
                     for (int c = 0; c < C::NK / 64; ++c)
-                        tmem_st32(tl + C::colS(t) + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&sr[32 * c]));
+                        tmem_st32(tl + C::colS(t, u) + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&sr[32 * c]));
                     static_assert(C::NK % 64 == 0, "P stored in 32-column chunks");
                     if (cnt_item > 0 && __any_sync(0xffffffffu, move)) {
-                        // O_t is stable: S_t of this group completed after PV_t of the last one.
+                        // O_t must hold PV_t of the previous block and no later one (the
+                        // next PV waits for this block's P). Single S buffer: S_t of this
+                        // block was issued after that PV, so it has completed. Double
+                        // buffer: wait for that PV's commit (the PV before it completed
+                        // before this block's S did, so the phase cannot alias).
+                        if constexpr (C::SDB) {
+                            if (!warp_wait(bar_pv(t, (cnt - 1) & 1), ((cnt - 1) >> 1) & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
 #pragma unroll
                         for (int c = 0; c < HD / 32; ++c) {
                             uint32_t o[32];
@@ -693,7 +692,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(bar_pf(t));
+                    mbar_arrive(bar_pf(t, u));
                     ++cnt;
                     ++cnt_item;
                 }
@@ -702,7 +701,11 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_le(b));
             if (cnt_item > 0) {
-                if (!warp_wait(bar_pv(t), (n_ep++) & 1, ctl)) break;
+                // O_t complete: the commit after this item's last PV (single S buffer:
+                // one commit per item; double buffer: one per PV, the last one's phase)
+                const bool ok = C::SDB ? warp_wait(bar_pv(t, (cnt - 1) & 1), ((cnt - 1) >> 1) & 1, ctl)
+                                       : warp_wait(bar_pv(t), (n_ep++) & 1, ctl);
+                if (!ok) break;
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.0f / l : 0.f;
                 uint16_t* orow = p.o + (I.row_base + qpos) * HD;
