@@ -20,7 +20,7 @@
 // S MMAs overlap the current item's last groups and epilogue and the load
 // balances itself (item order: see pair_item).
 //
-// CTA = 12 warps:
+// CTA = 12 warps (14 with 64-key blocks):
 //   warp 2      scheduler, list builder and Q producer: takes the next item
 //               from the work counter, writes the item's union list and index
 //               into a double-buffered shared-memory list, loads the item's Q
@@ -40,11 +40,14 @@
 //
 // Two pipelines, chosen by block size (PairCfg):
 //  * 64-key blocks (SDB): each tile has two S buffers in TMEM, and S of the
-//    tile's next two blocks is issued ahead of the softmax, so the tensor core
-//    computes S of block i+1 while the softmax works on block i. One thread of
-//    warp 1 issues tile 0's MMAs and one of warp 3 tile 1's, each walking the
-//    same union list; a K/V stage and the Q buffer are released when both
-//    have committed. Q stays in shared memory (TMEM is full).
+//    tile's next blocks is issued ahead of the softmax, so the tensor core
+//    computes S of block i+1 while the softmax works on block i. With 64-key
+//    blocks a single thread's chain of barrier waits, commits and MMA issues
+//    (about 0.1-0.2k cycles each) was the limit, so four threads issue: per
+//    tile one for S (warps 1 and 3) and one for PV (warps 12 and 13), each
+//    walking the same union list; a K/V stage is released when all four have
+//    committed, the Q buffer when both S issuers have. Q stays in shared
+//    memory (TMEM is full).
 //  * 128-key blocks: one S buffer per tile and one issuer for both tiles; the
 //    two softmax warpgroups ping-pong (while one computes exponentials for its
 //    tile, the tensor core runs the other tile's MMAs). When TMEM has room
@@ -58,11 +61,11 @@
 //  * One S buffer: S_t(next) is issued after PV_t(current), so when the
 //    softmax sees S_t(next) complete, PV_t(current) has finished: P_t's TMEM
 //    columns (aliased on S_t) are free and O_t is stable for a rescale.
-//  * Two S buffers: S_t(i+2) is issued after PV_t(i) (same buffer). The
-//    softmax waits for PV_t(i-1)'s own commit before it rescales O_t at block
-//    i and before the epilogue; S_t(i) complete implies PV_t(i-2) complete, so
-//    that barrier's phase cannot alias. Every S/P barrier is per buffer, for
-//    the same reason.
+//  * Two S buffers: S_t(i+2) is issued once PV_t(i) (same buffer) has
+//    completed. The softmax waits for PV_t(i-1)'s own commit before it
+//    rescales O_t at block i and before the epilogue; S_t(i) complete implies
+//    PV_t(i-2) complete, so that barrier's phase cannot alias. Every S/P/PV
+//    barrier is per buffer, for the same reason.
 //  * A tile's first P of the next item is published only after its warpgroup
 //    has read O out of TMEM (tcgen05.wait::ld) for the previous item, so the
 //    next item's first PV (which overwrites O) cannot race the epilogue.
@@ -101,22 +104,27 @@ struct PairCfg {
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
     static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
     // barriers: q_full, q_empty, kv_full[ST] (K and V of a stage), kv_empty[ST],
-    // s_full[2][2], p_full[2][2], pv_done[2][2] ([tile][S buffer]), drain[2],
-    // list_full[2], list_empty[2]
-    static constexpr int NBAR = 2 + 2 * ST + 12 + 2 + 4;
+    // s_full[2][2], p_full[2][2], pv_done[2][2] ([tile][S buffer]), drain[4]
+    // (one per MMA issuer), list_full[2], list_empty[2]
+    static constexpr int NBAR = 2 + 2 * ST + 12 + 4 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
     // S double-buffered per tile (64-key blocks): the S MMA of a tile's next
     // block runs while the softmax works on the current one, so a tile's chain
     // is no longer S -> softmax -> PV -> S. Takes 4 NK + 2 HD TMEM columns, so
-    // Q stays in shared memory. This pipeline has one MMA issuer per tile
-    // (warp 1: tile 0, warp 3: tile 1).
+    // Q stays in shared memory. This pipeline has four MMA issuer threads, an
+    // S issuer and a PV issuer per tile (warps 1 and 3: S of tiles 0 and 1;
+    // warps 12 and 13: PV of tiles 0 and 1), in a 14-warp CTA.
     static constexpr bool SDB = BK == 64 && 4 * NK + 2 * HD <= 512;
     static constexpr int SBUF = SDB ? 2 : 1;
-    static constexpr int ISSUERS = SDB ? 2 : 1;
+    static constexpr int THREADS = SDB ? 448 : 384;
+    // threads that commit once per union element to kv_empty (and S issuers:
+    // once per item to q_empty)
+    static constexpr uint32_t KV_RELEASERS = SDB ? 4 : 1;
+    static constexpr uint32_t Q_RELEASERS = SDB ? 2 : 1;
     // list_empty arrivals per item: K/V producer, MMA issuer(s), 8 softmax warps
-    static constexpr uint32_t LIST_CONSUMERS = 9 + ISSUERS;
+    static constexpr uint32_t LIST_CONSUMERS = 9 + KV_RELEASERS;
     __host__ __device__ static constexpr uint32_t colS(int t, int u = 0) { return (uint32_t)((t * SBUF + u) * NK); }
     __host__ __device__ static constexpr uint32_t colO(int t) { return (uint32_t)(2 * SBUF * NK + t * HD); }
     // Without S double-buffering, when TMEM has room for both tiles' Q (HD/2
@@ -177,7 +185,7 @@ __device__ __forceinline__ PairItem pair_item(const PrefillParams& p, int w)
 }
 
 template <int HD, int BK>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(PairCfg<HD, BK>::THREADS, 1)
 s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const PrefillParams p)
 {
@@ -201,9 +209,9 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     auto bar_sf = [&](int t, int u = 0) { return sb + C::OFF_BAR + 8u * (2 + 2 * C::ST + 2 * t + u); };
     auto bar_pf = [&](int t, int u = 0) { return sb + C::OFF_BAR + 8u * (6 + 2 * C::ST + 2 * t + u); };
     auto bar_pv = [&](int t, int u = 0) { return sb + C::OFF_BAR + 8u * (10 + 2 * C::ST + 2 * t + u); };
-    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (14 + 2 * C::ST);  // [2]: one per MMA issuer
-    auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (16 + 2 * C::ST + b); };
-    auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (18 + 2 * C::ST + b); };
+    const uint32_t bar_dr = sb + C::OFF_BAR + 8u * (14 + 2 * C::ST);  // [4]: one per MMA issuer
+    auto bar_lf = [&](int b) { return sb + C::OFF_BAR + 8u * (18 + 2 * C::ST + b); };
+    auto bar_le = [&](int b) { return sb + C::OFF_BAR + 8u * (20 + 2 * C::ST + b); };
     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
     // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
@@ -214,10 +222,10 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        mbar_init(bar_qe, C::ISSUERS);  // one commit per MMA issuer
+        mbar_init(bar_qe, C::Q_RELEASERS);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_kf(s), 1);
-            mbar_init(bar_ke(s), C::ISSUERS);  // one commit per MMA issuer
+            mbar_init(bar_ke(s), C::KV_RELEASERS);
         }
         for (int t = 0; t < 2; ++t) {
             for (int u = 0; u < 2; ++u) {
@@ -228,8 +236,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             mbar_init(bar_lf(t), 1);
             mbar_init(bar_le(t), C::LIST_CONSUMERS);
         }
-        mbar_init(bar_dr, 1);
-        mbar_init(bar_dr + 8u, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(bar_dr + 8u * i, 1);
         *abort_cta = 0;
         fence_mbar_init();
     }
@@ -341,100 +348,105 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     mbar_drain(bar_kf(m % C::ST), (m / C::ST) & 1, kDrainNs);
         }
         __syncwarp();
-    } else if (warp == 1 || (C::ISSUERS == 2 && warp == 3)) {
+    } else if (warp == 1 || (C::SDB && (warp == 3 || warp >= 12))) {
         // ------------------------------------------------------------ MMA issuer(s)
         if constexpr (C::SDB) {
-            // One thread per tile (warp 1: tile 0, warp 3: tile 1), each walking
-            // the same union list. S of the i-th block a tile sees goes to its S
-            // buffer i & 1 and is issued up to two blocks ahead of the PVs: S of
-            // block i + 2 reuses the buffer of block i, so it is issued after
-            // PV_i (in issue order it then runs after PV_i has read P_i).
+            // Per tile an S issuer (warp 1: tile 0, warp 3: tile 1) and a PV issuer
+            // (warp 12: tile 0, warp 13: tile 1), each walking the same union list.
+            // The i-th S of a tile goes to its S buffer i & 1; S_{i+2} reuses the
+            // buffer of block i, so the S issuer waits for PV_i's commit first
+            // (the two threads' MMAs have no issue-order relation). Both commit
+            // kv_empty once per union element: a stage is free when K (read by
+            // S) and V (read by PV) of both tiles are done.
+            const bool s_role = warp == 1 || warp == 3;
+            const int T = s_role ? (warp == 1 ? 0 : 1) : warp - 12;
+            const uint32_t my_dr = bar_dr + 8u * (s_role ? T : 2 + T);
             if (lane == 0) {
-                const int T = warp == 1 ? 0 : 1;
                 constexpr uint32_t idesc_s = umma_idesc(128, C::NK, 0, 0);
                 constexpr uint32_t idesc_o = umma_idesc(128, HD, 0, 1);
                 bool issued = false, fail = false;
-                int sc = 0;  // S MMAs issued for tile T (all items)
-                int pc = 0;  // PV MMAs issued for tile T (all items)
-                int n0 = 0;  // union elements of the earlier items
+                int cnt = 0;  // S (or PV) MMAs of tile T issued so far (all items)
+                int n0 = 0;   // union elements of the earlier items
                 const uint64_t dq = umma_sdesc(sb + C::OFF_Q + T * C::QBYTES, 16, 1024);
-                auto issue_s = [&](int st) {
-                    const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * (BK * 128), 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ss(tmem + C::colS(T, sc & 1), dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
-                                     dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
-                    umma_commit(bar_sf(T, sc & 1));
-                    ++sc;
-                    issued = true;
-                };
-                // O_T (+)= P_T V; the per-PV commit lets the softmax wait for O before
-                // a rescale and before the epilogue.
-                auto issue_pv = [&](int st, bool first) {
-#pragma unroll
-                    for (int kk = 0; kk < C::NK / 16; ++kk)
-                        umma_bf16_ts(tmem + C::colO(T), tmem + C::colS(T, pc & 1) + kk * 8,
-                                     umma_sdesc(sb + C::OFF_V + st * C::KVBYTES + kk * 2048, BK * 128, 1024),
-                                     idesc_o, (kk > 0 || !first) ? 1u : 0u);
-                    umma_commit(bar_pv(T, pc & 1));
-                    ++pc;
-                };
                 for (int k = 0; !fail; ++k) {
                     const int b = k & 1;
                     if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
                     if (list_item[b] < 0) break;
                     const uint32_t* L = list + b * C::LIST_CAP;
                     const int len = list_len[b];
-                    if (!mbar_wait(bar_q, k & 1, ctl)) break;
                     const bool mine = T == 0 || pair_item<BK>(p, list_item[b]).tile1;  // tile T exists
-                    auto seen = [&](int e) { return mine && tile_sees<BK>(list_bits(L[e]), T); };
-                    int s_next = 0;      // next element to look at for an S MMA
-                    int ss = 0, ps = 0;  // S and PV MMAs of this item
-                    bool q_done = false;
-                    // S for the next blocks tile T sees: at most two ahead of the PVs,
-                    // and only blocks whose stage this thread has already released
-                    // (element s_next loads once element s_next - ST is released), so
-                    // the wait below never waits on this thread's own progress.
-                    auto ahead = [&](int e_done) {
-                        while (ss - ps < 2) {
-                            while (s_next < len && !seen(s_next)) ++s_next;
-                            if (s_next >= len || s_next > e_done + C::ST) break;
-                            const int n = n0 + s_next;
-                            if (!mbar_wait(bar_kf(n % C::ST), (n / C::ST) & 1, ctl)) return false;
-                            tc_fence_after();
-                            issue_s(n % C::ST);
-                            ++ss;
-                            ++s_next;
-                        }
-                        if (!q_done && s_next >= len) {  // no more S MMAs of this item read Q_T
-                            umma_commit(bar_qe);
-                            q_done = true;
-                        }
-                        return true;
-                    };
-                    if (!ahead(-1)) break;
+                    int last_seen = -1;  // last element tile T sees in this item
+                    if (s_role) {
+                        if (!mbar_wait(bar_q, k & 1, ctl)) break;
+                        for (int e = len - 1; mine && e >= 0; --e)
+                            if (tile_sees<BK>(list_bits(L[e]), T)) {
+                                last_seen = e;
+                                break;
+                            }
+                        if (last_seen < 0) umma_commit(bar_qe);  // Q_T unused in this item
+                    }
+                    bool first = true;
                     for (int e = 0; e < len; ++e) {
                         const int n = n0 + e, st = n % C::ST;
-                        if (seen(e)) {
-                            if (!mbar_wait(bar_pf(T, pc & 1), (pc >> 1) & 1, ctl)) { fail = true; break; }
+                        const bool sees = mine && tile_sees<BK>(list_bits(L[e]), T);
+                        if (s_role) {
+                            // S buffer cnt & 1 is free once PV_{cnt-2} completed (PV_{cnt-4}
+                            // completed before S_{cnt-2} was issued: no phase aliasing)
+                            if (sees && cnt >= 2 &&
+                                !mbar_wait(bar_pv(T, cnt & 1), ((cnt - 2) >> 1) & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
+                            if (!mbar_wait(bar_kf(st), (n / C::ST) & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
+                            if (sees) {
+                                tc_fence_after();
+                                const uint64_t dk = umma_sdesc(sb + C::OFF_K + st * (BK * 128), 16, 1024);
+#pragma unroll
+                                for (int kk = 0; kk < HD / 16; ++kk)
+                                    umma_bf16_ss(tmem + C::colS(T, cnt & 1),
+                                                 dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4),
+                                                 dk + (((kk >> 2) * C::KPANEL + (kk & 3) * 32) >> 4), idesc_s,
+                                                 kk > 0 ? 1u : 0u);
+                                umma_commit(bar_sf(T, cnt & 1));
+                                ++cnt;
+                                issued = true;
+                                if (e == last_seen) umma_commit(bar_qe);  // no more S of this item reads Q_T
+                            }
+                        } else if (sees) {
+                            if (!mbar_wait(bar_pf(T, cnt & 1), (cnt >> 1) & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
                             tc_fence_after();
-                            issue_pv(st, ps == 0);
-                            ++ps;
+#pragma unroll
+                            for (int kk = 0; kk < C::NK / 16; ++kk)
+                                umma_bf16_ts(tmem + C::colO(T), tmem + C::colS(T, cnt & 1) + kk * 8,
+                                             umma_sdesc(sb + C::OFF_V + st * C::KVBYTES + kk * 2048, BK * 128, 1024),
+                                             idesc_o, (kk > 0 || !first) ? 1u : 0u);
+                            // the softmax waits on this before an O rescale and the epilogue,
+                            // the S issuer before reusing the buffer
+                            umma_commit(bar_pv(T, cnt & 1));
+                            ++cnt;
+                            first = false;
+                            issued = true;
                         } else if (!mbar_wait(bar_kf(st), (n / C::ST) & 1, ctl)) {
                             // a block tile T skips: its loads land before the stage is released
+                            // (so this arrival cannot count toward an earlier use of the stage)
                             fail = true;
                             break;
                         }
                         umma_commit(bar_ke(st));
-                        if (!ahead(e)) { fail = true; break; }
                     }
                     if (fail) break;
                     n0 += len;
                     mbar_arrive(bar_le(b));
                 }
                 if (*abort_cta && issued) {
-                    umma_commit(bar_dr + 8u * T);
-                    mbar_drain(bar_dr + 8u * T, 0, kDrainNs);
+                    umma_commit(my_dr);
+                    mbar_drain(my_dr, 0, kDrainNs);
                 }
             }
         } else {

@@ -152,7 +152,7 @@ int launch_prefill(const void* q, const void* k, const void* v, s2::PrefillParam
     // static share of the tile pairs.
     const uint64_t items = (uint64_t)pp.batch * pp.heads * ((pp.nqt + 1) / 2);
     const uint64_t grid = items < (uint64_t)g_dev[dev].num_sms ? items : (uint64_t)g_dev[dev].num_sms;
-    kern<<<(unsigned)grid, 384, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
+    kern<<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, pp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
