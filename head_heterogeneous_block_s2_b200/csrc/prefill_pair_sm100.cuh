@@ -721,20 +721,53 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.0f / l : 0.f;
                 uint16_t* orow = p.o + (I.row_base + qpos) * HD;
+                if constexpr (C::SDB) {
+                    // Each thread writes its own row: 32-byte stores (whole L2 sectors,
+                    // half the store instructions of 16-byte ones) when O is 32-byte
+                    // aligned, and 64 columns loaded per tcgen05 wait. (The 128-key
+                    // kernel is at its register cap and keeps 32-column loads and
+                    // 16-byte stores: the wider form spilled and ran 7% slower there.)
+                    const bool st32 = (reinterpret_cast<uintptr_t>(p.o) & 31u) == 0;
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tl + C::colO(t) + 32 * c, o);
-                    tmem_wait_ld();
-                    if (row_valid) {
+                    for (int c = 0; c < HD / 64; ++c) {
+                        uint32_t o[64];
+                        tmem_ld32(tl + C::colO(t) + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                        tmem_ld32(tl + C::colO(t) + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+                        tmem_wait_ld();
+                        if (row_valid) {
 #pragma unroll
-                        for (int e2 = 0; e2 < 32; e2 += 8) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * inv, __uint_as_float(o[e2 + 1]) * inv);
-                            v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * inv, __uint_as_float(o[e2 + 3]) * inv);
-                            v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * inv, __uint_as_float(o[e2 + 5]) * inv);
-                            v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * inv, __uint_as_float(o[e2 + 7]) * inv);
-                            *reinterpret_cast<uint4*>(orow + 32 * c + e2) = v;
+                            for (int e2 = 0; e2 < 64; e2 += 16) {
+                                uint32_t w[8];
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    w[i] = pack_bf16x2(__uint_as_float(o[e2 + 2 * i]) * inv,
+                                                       __uint_as_float(o[e2 + 2 * i + 1]) * inv);
+                                if (st32) {
+                                    st_global_v8(orow + 64 * c + e2, w);
+                                } else {
+                                    *reinterpret_cast<uint4*>(orow + 64 * c + e2) = make_uint4(w[0], w[1], w[2], w[3]);
+                                    *reinterpret_cast<uint4*>(orow + 64 * c + e2 + 8) =
+                                        make_uint4(w[4], w[5], w[6], w[7]);
+                                }
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tl + C::colO(t) + 32 * c, o);
+                        tmem_wait_ld();
+                        if (row_valid) {
+#pragma unroll
+                            for (int e2 = 0; e2 < 32; e2 += 8) {
+                                uint4 v;
+                                v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * inv, __uint_as_float(o[e2 + 1]) * inv);
+                                v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * inv, __uint_as_float(o[e2 + 3]) * inv);
+                                v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * inv, __uint_as_float(o[e2 + 5]) * inv);
+                                v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * inv, __uint_as_float(o[e2 + 7]) * inv);
+                                *reinterpret_cast<uint4*>(orow + 32 * c + e2) = v;
+                            }
                         }
                     }
                 }

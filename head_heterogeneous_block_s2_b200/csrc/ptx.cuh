@@ -309,6 +309,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     return r;
 }
 
+// 32-byte global store (sm_100 256-bit store); addr must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* addr, const uint32_t (&w)[8])
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(addr), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
 // Two floats -> packed bf16x2 (round to nearest even), low half = a.
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
 {

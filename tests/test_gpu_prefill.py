@@ -73,6 +73,23 @@ def test_repeated_calls_are_deterministic(s2gpu):
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("bk", [64, 128])
+def test_output_only_16_byte_aligned(s2gpu, bk):
+    # The epilogue stores whole 32-byte sectors when O is 32-byte aligned and
+    # falls back to 16-byte stores otherwise; both must write the same bytes.
+    w = synth.PrefillWorkload("t", 1, 3, 128, 640, bk, 3, 1, seed=11)
+    q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
+    lay = s2gpu.build_layout(w.heads, w.block, w.stride, w.local, w.num_blocks, w.dense_heads, device="cuda")
+    ref = s2gpu.prefill(q, k, v, lay, scale=w.scale)
+    buf = torch.full((q.numel() + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = buf[8:].view(q.shape)  # 16 bytes past a 512-byte-aligned allocation
+    assert out.data_ptr() % 32 == 16
+    s2gpu.prefill(q, k, v, lay, scale=w.scale, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    assert torch.isnan(buf[:8].float()).all()  # nothing written before O
+
+
 def sample_rows(w, seed, blocks_random=6, per_block=16):
     rng = np.random.default_rng(seed)
     rows = []
