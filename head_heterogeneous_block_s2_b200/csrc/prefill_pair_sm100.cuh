@@ -667,10 +667,22 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int q = 0; q < C::NK / 2; ++q) {  // column pair (2q, 2q+1)
-                        const float p0 = ex2(fmaf(__uint_as_float(sr[2 * q]), sc, neg_m));
-                        const float p1 = ex2(fmaf(__uint_as_float(sr[2 * q + 1]), sc, neg_m));
-                        rs[(2 * q) & 3] += p0;
-                        rs[(2 * q + 1) & 3] += p1;
+                        float p0, p1;
+                        if constexpr (C::SDB) {
+                            // packed pair FMA and ADD: 5 instructions per pair instead of 7
+                            // (this loop's instruction count, not the exponential unit,
+                            // is what the softmax spends its time on)
+                            float x0, x1;
+                            ffma2(x0, x1, __uint_as_float(sr[2 * q]), __uint_as_float(sr[2 * q + 1]), sc, neg_m);
+                            p0 = ex2(x0);
+                            p1 = ex2(x1);
+                            fadd2(rs[(q & 1) * 2], rs[(q & 1) * 2 + 1], p0, p1);
+                        } else {
+                            p0 = ex2(fmaf(__uint_as_float(sr[2 * q]), sc, neg_m));
+                            p1 = ex2(fmaf(__uint_as_float(sr[2 * q + 1]), sc, neg_m));
+                            rs[(2 * q) & 3] += p0;
+                            rs[(2 * q + 1) & 3] += p1;
+                        }
                         sr[q] = pack_bf16x2(p0, p1);  // slot q <= 2q: already read
                     }
                     l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));

@@ -309,6 +309,31 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     return r;
 }
 
+// Packed fp32 pair arithmetic (sm_100 f32x2): (d0, d1) = (a0, a1) * b + c.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b, float c)
+{
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %4};\n\t"
+        "mov.b64 rc, {%5, %5};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// (d0, d1) += (a0, a1), packed.
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1)
+{
+    asm("{\n\t.reg .b64 ra, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rd, {%0, %1};\n\t"
+        "add.rn.f32x2 rd, rd, ra;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1));
+}
+
 // 32-byte global store (sm_100 256-bit store); addr must be 32-byte aligned.
 __device__ __forceinline__ void st_global_v8(void* addr, const uint32_t (&w)[8])
 {
