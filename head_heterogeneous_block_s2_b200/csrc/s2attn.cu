@@ -218,8 +218,13 @@ int launch_chunk(const void* q, const void* kc, const void* vc, s2::ChunkParams&
             g_dev[dev].chunk_attr_done[attr_slot] = true;
         }
     }
-    const dim3 grid((unsigned)((cp.max_q_len + 127) / 128 + 1), (unsigned)cp.heads, (unsigned)cp.batch);
-    kern<<<grid, 384, C::SMEM_ALLOC, stream>>>(mq, mk, mv, cp);
+    // Persistent: at most one CTA per SM; the kernel counts the items (tile
+    // pairs x heads) from the device-side chunk metadata, bounded here by the
+    // largest chunk (a chunk of L rows spans at most L / 128 + 2 tiles).
+    const uint64_t pairs_max = ((uint64_t)(cp.max_q_len + 127) / 128 + 2) / 2;
+    const uint64_t items = (uint64_t)cp.batch * cp.heads * pairs_max;
+    const uint64_t grid = items < (uint64_t)g_dev[dev].num_sms ? items : (uint64_t)g_dev[dev].num_sms;
+    kern<<<(unsigned)grid, 384, C::SMEM_ALLOC, stream>>>(mq, mk, mv, cp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
@@ -477,6 +482,7 @@ int s2_attn_chunk_prefill(const void* q, const void* k_cache, const void* v_cach
     cp.scale_log2 = scale * 1.4426950408889634f;
     cp.timeout_ns = g_timeout_ns.load();
     cp.gflags = g_dev[dev].flags;
+    cp.sched = g_dev[dev].sched + 2 * (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 128 && block_size == 128) return launch_chunk<128, 128>(q, k_cache, v_cache, cp, dev, 0, st);
     if (head_dim == 128 && block_size == 64) return launch_chunk<128, 64>(q, k_cache, v_cache, cp, dev, 1, st);

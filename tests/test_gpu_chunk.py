@@ -69,6 +69,17 @@ def test_chunks_of_every_shape(s2gpu, D, B):
     case(s2gpu, ctx, qlen, D=D, B=B, S=3, L=1, dense=(1,), seed=B + D)
 
 
+def test_many_sequences_with_empty_chunks(s2gpu):
+    # more than 32 sequences (items are mapped by a warp-wide prefix over the
+    # sequences, 32 at a time) and some chunks of zero rows
+    rng = np.random.default_rng(21)
+    ctx = [int(c) for c in rng.integers(1, 400, size=37)]
+    qlen = [int(rng.integers(0, c + 1)) for c in ctx]
+    qlen[3] = qlen[20] = qlen[36] = 0
+    qlen[0] = ctx[0]
+    case(s2gpu, ctx, qlen, H=2, D=64, B=64, S=3, L=1, seed=21)
+
+
 def test_grouped_kv_heads(s2gpu):
     case(s2gpu, [700, 260], [300, 260], H=8, hkv=2, seed=5)
 
