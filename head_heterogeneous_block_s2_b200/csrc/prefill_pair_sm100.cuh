@@ -66,6 +66,12 @@
 //    rescales O_t at block i and before the epilogue; S_t(i) complete implies
 //    PV_t(i-2) complete, so that barrier's phase cannot alias. Every S/P/PV
 //    barrier is per buffer, for the same reason.
+//  * Every issuing thread waits for each union element's loads, in order, and
+//    commits kv_empty for it, including elements its tile skips: a stage can
+//    then never be refilled before every thread has passed it, which keeps
+//    each kv_full parity wait within one phase of the element it wants. (An S
+//    thread that skipped unseen elements could see a stage one phase behind
+//    as complete, or, waiting on them, one phase ahead that needs its own S.)
 //  * A tile's first P of the next item is published only after its warpgroup
 //    has read O out of TMEM (tcgen05.wait::ld) for the previous item, so the
 //    next item's first PV (which overwrites O) cannot race the epilogue.
