@@ -14,11 +14,12 @@
 //   s2_bwd_stats_kernel  per query row: (LSE * log2 e, D_q) into a row-padded
 //                        fp32 workspace; rows past seq get (+inf, 0) so that
 //                        any P computed for them is exactly 0.
-//   s2_bwd_dq_kernel     one 128-row query tile per CTA, walking the union of
-//                        its query blocks' key-block lists (the forward's
-//                        lists): S = Q K^T and dP = dO V^T into TMEM, dS
-//                        (bf16) written back over S, dQ += dS K with dS read
-//                        from TMEM and K from shared memory as an MN-major B.
+//   s2_bwd_dq_kernel     persistent; one 128-row query tile per work item,
+//                        walking the union of its query blocks' key-block
+//                        lists (the forward's lists): S = Q K^T and dP = dO V^T
+//                        into TMEM, dS (bf16) written back over dP, dQ += dS K
+//                        with dS read from TMEM and K from shared memory as an
+//                        MN-major B.
 //   s2_bwd_dkv_kernel    one 128-row key tile per CTA, walking the union of
 //                        its key blocks' transposed lists (query blocks that
 //                        list them): S^T = K Q^T and dP^T = V dO^T into TMEM,
@@ -30,8 +31,8 @@
 // results are deterministic.
 //
 // CTA = 12 warps: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer (one
-// thread), warp 2 builds the union list in shared memory before the main
-// loop, warps 4..11 the element-wise passes and the epilogue: thread = one
+// thread), warp 2 builds the union list in shared memory (in the dQ kernel:
+// item after item, double-buffered, and loads the item's Q and dO), warps 4..11 the element-wise passes and the epilogue: thread = one
 // tile row = one TMEM lane, warps 4..7 on the first half of the columns and
 // warps 8..11 on the second (two warps per SM sub-partition hide the
 // exponential and TMEM latencies; a single warpgroup was measured to leave
@@ -70,6 +71,7 @@ struct BackwardParams {
     float scale_log2;  // scale * log2 e
     uint64_t timeout_ns;
     uint32_t* gflags;
+    int* sched;  // dQ kernel work counter {next item, CTAs done}, zero at launch
 };
 
 // Descriptor offset (16-byte units) of k-step kk (16 elements) of a K-major
@@ -160,21 +162,22 @@ struct BwdQCfg {
     static constexpr uint32_t KVBYTES = BK * HD * 2;  // one K or V block
     static constexpr int ST = 2;
     static constexpr int LIST_CAP = 2048;
+    static constexpr uint32_t LIST_BYTES = 2 * LIST_CAP * 4;  // double-buffered
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_DO = TBYTES;
     static constexpr uint32_t OFF_K = 2 * TBYTES;              // [stage][panel][BK rows x 128 B]
     static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
-    static constexpr uint32_t OFF_SCR = OFF_LIST + LIST_CAP * 4;  // list-merge scratch (ROWS > 1)
-    static constexpr uint32_t OFF_BAR = OFF_SCR + (ROWS > 1 ? ROWS * LIST_CAP * 4 : 0);
-    // barriers: qd_full, k_full[ST], v_full[ST], kv_empty[ST], s_full, ds_full, acc_done, drain,
-    // dp_full, s_free
-    static constexpr int NBAR = 1 + 3 * ST + 6;
+    static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
+    // barriers: qd_full, qd_empty, k_full[ST], v_full[ST], kv_empty[ST], s_full, ds_full, acc_done,
+    // drain, dp_full, s_free, list_full[2], list_empty[2]
+    static constexpr int NBAR = 2 + 3 * ST + 6 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
+    static constexpr uint32_t LIST_CONSUMERS = 10;  // producer, MMA issuer, 8 element-wise warps
     static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_ACC = 2 * BK;
-    // Q and dO, the A operands of every S and dP MMA of the CTA, sit in TMEM
+    // Q and dO, the A operands of every S and dP MMA of an item, sit in TMEM
     // (HD/2 columns each): those MMAs read only K or V from shared memory.
     static constexpr uint32_t COL_QA = 2 * BK + HD, COL_DOA = 2 * BK + HD + HD / 2;
     static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD) <= 256 ? 256 : 512;
@@ -182,6 +185,10 @@ struct BwdQCfg {
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
+// Persistent: each CTA takes work items (one 128-row query tile of one plane,
+// the tiles with the longest lists first) from a device counter; a warp
+// builds the next item's union list and loads its Q and dO while the current
+// item runs, so items follow one another without a prologue.
 template <int HD, int BK>
 __global__ void __launch_bounds__(384, 1)
 s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
@@ -195,30 +202,34 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t sb = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int BH = p.batch * p.heads;
-    const int qt = p.ntiles - 1 - (int)(blockIdx.x / BH);  // longest lists first
-    const int bh = (int)(blockIdx.x % BH);
-    const int h = bh % p.heads;
-    const int bkv = (bh / p.heads) * p.heads_kv + h / (p.heads / p.heads_kv);  // K/V plane
+    const int num_items = p.ntiles * BH;
+    auto item_qt = [&](int w) { return p.ntiles - 1 - w / BH; };  // longest lists first
+    auto item_bh = [&](int w) { return w % BH; };
 
     const uint32_t bar_qd = sb + C::OFF_BAR;
-    auto bar_kf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
-    auto bar_vf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + C::ST + s); };
-    auto bar_ke = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + 2 * C::ST + s); };
-    const uint32_t bar_s = sb + C::OFF_BAR + 8u * (1 + 3 * C::ST);
+    const uint32_t bar_qe = sb + C::OFF_BAR + 8u;
+    auto bar_kf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + s); };
+    auto bar_vf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + C::ST + s); };
+    auto bar_ke = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + 2 * C::ST + s); };
+    const uint32_t bar_s = sb + C::OFF_BAR + 8u * (2 + 3 * C::ST);
     const uint32_t bar_ds = bar_s + 8u;
     const uint32_t bar_acc = bar_s + 16u;
     const uint32_t bar_dr = bar_s + 24u;
     const uint32_t bar_dp = bar_s + 32u;
     const uint32_t bar_sfree = bar_s + 40u;
-    uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
-    int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2] list length
+    auto bar_lf = [&](int b) { return bar_s + 48u + 8u * b; };
+    auto bar_le = [&](int b) { return bar_s + 64u + 8u * b; };
+    const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
+    // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
+    int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
     volatile int* abort_cta = misc + 1;
+    volatile int* list_len = misc + 2;
+    volatile int* list_item = misc + 4;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar_dp, 1);
-        mbar_init(bar_sfree, 256);
         mbar_init(bar_qd, 1);
+        mbar_init(bar_qe, 1);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_kf(s), 1);
             mbar_init(bar_vf(s), 1);
@@ -228,6 +239,12 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mbar_init(bar_ds, 256);
         mbar_init(bar_acc, 1);
         mbar_init(bar_dr, 1);
+        mbar_init(bar_dp, 1);
+        mbar_init(bar_sfree, 256);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_lf(b), 1);
+            mbar_init(bar_le(b), C::LIST_CONSUMERS);
+        }
         *abort_cta = 0;
         fence_mbar_init();
     }
@@ -235,77 +252,125 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (threadIdx.x == 0) {  // Q and dO of the tile do not depend on the list: load them now
-        mbar_arrive_expect_tx(bar_qd, 2 * C::TBYTES);
-#pragma unroll
-        for (int pn = 0; pn < HD / 64; ++pn) {
-            tma_load_3d(sb + C::OFF_Q + pn * (C::M * 128), &tmQ, pn * 64, qt * C::M, bh, bar_qd);
-            tma_load_3d(sb + C::OFF_DO + pn * (C::M * 128), &tmDO, pn * 64, qt * C::M, bh, bar_qd);
-        }
-    }
-    if (warp == 2) {  // union of the tile's key-block lists
-        int rows[C::ROWS];
-#pragma unroll
-        for (int r = 0; r < C::ROWS; ++r) rows[r] = qt * C::ROWS + r;
-        const int n = warp_union_list<C::ROWS>(p.row_ptr, p.col_idx, h * (p.nb + 1), rows, p.nb, p.nnz,
-                                               0, min(qt * C::ROWS + C::ROWS, p.nb) - 1, list, C::LIST_CAP,
-                                               reinterpret_cast<int32_t*>(smem + C::OFF_SCR), p.gflags);
-        if (lane == 0) misc[2] = n;
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int len = misc[2];
     const WaitCtl ctl{p.timeout_ns, p.gflags, abort_cta};
     constexpr uint64_t kDrainNs = 200000000ull;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0 && len == 0) mbar_drain(bar_qd, 0, kDrainNs);  // nothing to do: let Q, dO land
-        if (lane == 0 && len > 0) {
-            int n = 0;
-            for (; n < len; ++n) {
-                const int st = n % C::ST;
-                if (!mbar_wait(bar_ke(st), ((n / C::ST) & 1) ^ 1, ctl)) break;
-                const int32_t krow = list_j(list[n]) * BK;
-                mbar_arrive_expect_tx(bar_kf(st), C::KVBYTES);
+    if (warp == 2) {
+        // ------------------------------------------------------------ items, union lists, Q and dO
+        if (lane == 0) {
+            int k = 0;
+            uint32_t* wlist = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
+            int w = blockIdx.x;  // first item static, the rest from the work counter
+            for (;; ++k) {
+                const int b = k & 1;
+                // list buffer b is free once item k-2 is consumed
+                if (!mbar_wait(bar_le(b), ((k >> 1) & 1) ^ 1, ctl)) break;
+                if (w >= num_items) {  // tell every role there is no more work
+                    list_item[b] = -1;
+                    list_len[b] = 0;
+                    mbar_arrive(bar_lf(b));
+                    break;
+                }
+                const int w_next = (int)gridDim.x + atomicAdd(p.sched, 1);
+                const int qt = item_qt(w), bh = item_bh(w), h = bh % p.heads;
+                UnionWalk<C::ROWS> it;
+                int len = 0;
+                const bool ok = it.init(p.row_ptr, h * (p.nb + 1), qt * C::ROWS, p.nb, p.nnz);
+                if (it.any) {
+                    for (;;) {
+                        int j, bits;
+                        bool last, bad;
+                        it.next(p.col_idx, j, bits, last, bad);
+                        if (bad) atomicOr(p.gflags, kFlagIndex);
+                        if (len >= C::LIST_CAP - 1) {  // cannot happen when nb <= LIST_CAP - 1
+                            atomicOr(p.gflags, kFlagIndex);
+                            last = true;
+                        }
+                        wlist[b * C::LIST_CAP + len++] = list_pack(j, bits);
+                        if (last) break;
+                    }
+                } else if (!ok) {
+                    atomicOr(p.gflags, kFlagIndex);
+                }
+                list_len[b] = len;
+                list_item[b] = w;
+                mbar_arrive(bar_lf(b));
+                // Q and dO of the tile, once the previous item's copies into TMEM are done
+                if (!mbar_wait(bar_qe, (k & 1) ^ 1, ctl)) break;
+                mbar_arrive_expect_tx(bar_qd, 2 * C::TBYTES);
 #pragma unroll
-                for (int pn = 0; pn < HD / 64; ++pn)
-                    tma_load_3d(sb + C::OFF_K + st * C::KVBYTES + pn * (BK * 128), &tmK, pn * 64, krow,
-                                bkv, bar_kf(st));
-                mbar_arrive_expect_tx(bar_vf(st), C::KVBYTES);
-#pragma unroll
-                for (int pn = 0; pn < HD / 64; ++pn)
-                    tma_load_3d(sb + C::OFF_V + st * C::KVBYTES + pn * (BK * 128), &tmV, pn * 64, krow,
-                                bkv, bar_vf(st));
+                for (int pn = 0; pn < HD / 64; ++pn) {
+                    tma_load_3d(sb + C::OFF_Q + pn * (C::M * 128), &tmQ, pn * 64, qt * C::M, bh, bar_qd);
+                    tma_load_3d(sb + C::OFF_DO + pn * (C::M * 128), &tmDO, pn * 64, qt * C::M, bh, bar_qd);
+                }
+                w = w_next;
             }
-            if (*abort_cta) {  // let this CTA's own loads land before exit
-                mbar_drain(bar_qd, 0, kDrainNs);
+            if (*abort_cta && k > 0) mbar_drain(bar_qd, (k - 1) & 1, kDrainNs);
+        }
+        __syncwarp();
+    } else if (warp == 0) {
+        // ------------------------------------------------------------ K and V producer
+        if (lane == 0) {
+            int n = 0, k = 0;
+            bool stop = false;
+            for (; !stop; ++k) {
+                const int b = k & 1;
+                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                const int w = list_item[b];
+                if (w < 0) break;
+                const int bh = item_bh(w);
+                const int bkv = (bh / p.heads) * p.heads_kv + (bh % p.heads) / (p.heads / p.heads_kv);
+                const uint32_t* L = list + b * C::LIST_CAP;
+                const int len = list_len[b];
+                for (int e = 0; e < len; ++e, ++n) {
+                    const int st = n % C::ST;
+                    if (!mbar_wait(bar_ke(st), ((n / C::ST) & 1) ^ 1, ctl)) {
+                        stop = true;
+                        break;
+                    }
+                    const int32_t krow = list_j(L[e]) * BK;
+                    mbar_arrive_expect_tx(bar_kf(st), C::KVBYTES);
+#pragma unroll
+                    for (int pn = 0; pn < HD / 64; ++pn)
+                        tma_load_3d(sb + C::OFF_K + st * C::KVBYTES + pn * (BK * 128), &tmK, pn * 64, krow,
+                                    bkv, bar_kf(st));
+                    mbar_arrive_expect_tx(bar_vf(st), C::KVBYTES);
+#pragma unroll
+                    for (int pn = 0; pn < HD / 64; ++pn)
+                        tma_load_3d(sb + C::OFF_V + st * C::KVBYTES + pn * (BK * 128), &tmV, pn * 64, krow,
+                                    bkv, bar_vf(st));
+                }
+                if (!stop) mbar_arrive(bar_le(b));
+            }
+            if (*abort_cta)  // let this CTA's own loads land before exit
                 for (int m = (n > C::ST ? n - C::ST : 0); m < n; ++m) {
                     mbar_drain(bar_kf(m % C::ST), (m / C::ST) & 1, kDrainNs);
                     mbar_drain(bar_vf(m % C::ST), (m / C::ST) & 1, kDrainNs);
                 }
-            }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && len > 0) {
+        if (lane == 0) {
             constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S = Q K^T, dP = dO V^T
             constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);  // dQ += dS K (K as MN-major B)
             const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
             const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
-            bool issued = false;
-            // S(n) and dP(n) are committed separately so that the element-wise
-            // warps start on P while dP is still running. Order per element n:
-            // [S(n) read out] S(n+1); [dS(n) ready] dQ(n), dP(n+1). The warps
-            // keep P in registers, so S(n+1) may overwrite S(n) as soon as they
-            // have loaded it; dS(n) sits in dP's columns and dP(n+1) is issued
-            // after dQ(n) has read it.
-            auto issue_s = [&](int n) {
-                const int st = n % C::ST;
-                if (!mbar_wait(bar_kf(st), (n / C::ST) & 1, ctl)) return false;
+            bool issued = false, fail = false;
+            // Element G (counted over all items) uses stage G % ST; S(G) and dP(G)
+            // are committed separately so that the element-wise warps start on P
+            // while dP is still running. Order per element: [S(G) read out]
+            // S(G+1); [dS(G) ready] dQ(G), dP(G+1). The warps keep P in
+            // registers, so S(G+1) may overwrite S(G) as soon as they have
+            // loaded it; dS(G) sits in dP's columns and dP(G+1) is issued after
+            // dQ(G) has read it.
+            auto issue_s = [&](int G) {
+                const int st = G % C::ST;
+                if (!mbar_wait(bar_kf(st), (G / C::ST) & 1, ctl)) return false;
                 tc_fence_after();
                 const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
 #pragma unroll
@@ -316,9 +381,9 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 issued = true;
                 return true;
             };
-            auto issue_dp = [&](int n) {
-                const int st = n % C::ST;
-                if (!mbar_wait(bar_vf(st), (n / C::ST) & 1, ctl)) return false;
+            auto issue_dp = [&](int G) {
+                const int st = G % C::ST;
+                if (!mbar_wait(bar_vf(st), (G / C::ST) & 1, ctl)) return false;
                 tc_fence_after();
                 const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
 #pragma unroll
@@ -328,37 +393,65 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 umma_commit(bar_dp);
                 return true;
             };
-            const bool qd_ok = mbar_wait(bar_qd, 0, ctl);
-            if (qd_ok) {  // Q and dO into TMEM (in issue order before every MMA that reads them)
+            int G = 0;
+            for (int k = 0; !fail; ++k) {
+                const int b = k & 1;
+                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                if (list_item[b] < 0) break;
+                const int len = list_len[b];
+                if (!mbar_wait(bar_qd, k & 1, ctl)) break;
+                // Q and dO into TMEM (after the previous item's MMAs that read them,
+                // in issue order); the shared-memory buffers are then free.
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     tmem_cp_128x256b(tmem + C::COL_QA + kk * 8, dq_desc + kstep(kk, C::M));
                     tmem_cp_128x256b(tmem + C::COL_DOA + kk * 8, ddo_desc + kstep(kk, C::M));
                 }
+                umma_commit(bar_qe);
                 issued = true;
-            }
-            if (qd_ok && issue_s(0) && issue_dp(0)) {
-                for (int n = 0; n < len; ++n) {
-                    const int st = n % C::ST;
-                    const bool more = n + 1 < len;
-                    if (more) {
-                        if (!mbar_wait(bar_sfree, n & 1, ctl)) break;
-                        tc_fence_after();
-                        if (!issue_s(n + 1)) break;
-                    }
-                    if (!mbar_wait(bar_ds, n & 1, ctl)) break;
+                if (len > 0) {
+                    // S's columns are free once the warps have loaded S of the previous
+                    // element; dP's (its dS) were read by its dQ, issued before.
+                    if (G > 0 && !mbar_wait(bar_sfree, (G - 1) & 1, ctl)) break;
                     tc_fence_after();
+                    if (!issue_s(G) || !issue_dp(G)) break;
+                    for (int n = 0; n < len; ++n, ++G) {
+                        const int st = G % C::ST;
+                        const bool more = n + 1 < len;
+                        if (more) {
+                            if (!mbar_wait(bar_sfree, G & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
+                            tc_fence_after();
+                            if (!issue_s(G + 1)) {
+                                fail = true;
+                                break;
+                            }
+                        }
+                        if (!mbar_wait(bar_ds, G & 1, ctl)) {
+                            fail = true;
+                            break;
+                        }
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t bk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
-                                     (n > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t bk =
+                                umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
+                            umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
+                                         (n > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(bar_ke(st));
+                        if (more && !issue_dp(G + 1)) {
+                            fail = true;
+                            break;
+                        }
                     }
-                    umma_commit(bar_ke(st));
-                    if (more && !issue_dp(n + 1)) break;
+                    if (fail) break;
+                    umma_commit(bar_acc);  // dQ of this item is complete once its last MMA is
                 }
-                if (!*abort_cta) umma_commit(bar_acc);
+                mbar_arrive(bar_le(b));
             }
             if (*abort_cta && issued) {
                 umma_commit(bar_dr);
@@ -372,79 +465,91 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int quad = warp & 3, g = (warp - 4) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        const int qpos = qt * C::M + r;
-        const int rowbit = (BK == 128) ? 0 : (r >> 6);
-        const bool row_valid = qpos < p.seq;
         const float sc = p.scale_log2;
-        float lx = 0.f, dy = 0.f;  // this row's LSE * log2 e and D
-        if (row_valid) {
-            const float* sp = p.stats + ((int64_t)bh * p.ntiles + qt) * 256 + r;
-            lx = sp[0];
-            dy = sp[128];
-        }
+        const int rowbit = (BK == 128) ? 0 : (r >> 6);
         bool fail = false;
-        for (int n = 0; n < len; ++n) {
-            const uint32_t ent = list[n];
-            if (!warp_wait(bar_s, n & 1, ctl)) {
-                fail = true;
-                break;
+        int G = 0, n_acc = 0;  // elements, and items with a dQ accumulation, so far
+        for (int k = 0; !fail; ++k) {
+            const int b = k & 1;
+            if (!warp_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+            const int w = list_item[b];
+            if (w < 0) break;
+            const int qt = item_qt(w), bh = item_bh(w);
+            const int qpos = qt * C::M + r;
+            const bool row_valid = qpos < p.seq;
+            float lx = 0.f, dy = 0.f;  // this row's LSE * log2 e and D
+            if (row_valid) {
+                const float* sp = p.stats + ((int64_t)bh * p.ntiles + qt) * 256 + r;
+                lx = sp[0];
+                dy = sp[128];
             }
-            tc_fence_after();
-            const bool vis = row_valid && ((list_bits(ent) >> rowbit) & 1);
-            const int lim = qpos - list_j(ent) * BK - g * HALF;  // column c of this half visible iff c <= lim
-            // P pass (needs S only; dP may still be running): P as bf16 pairs in registers
-            uint32_t sr[HALF], pk[HALF / 2];
-            tmem_ld_cols<HALF>(tl + C::COL_S + g * HALF, sr);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar_sfree);  // S(n) is in registers: S(n+1) may be written
+            const uint32_t* L = list + b * C::LIST_CAP;
+            const int len = list_len[b];
+            for (int n = 0; n < len; ++n, ++G) {
+                const uint32_t ent = L[n];
+                if (!warp_wait(bar_s, G & 1, ctl)) {
+                    fail = true;
+                    break;
+                }
+                tc_fence_after();
+                const bool vis = row_valid && ((list_bits(ent) >> rowbit) & 1);
+                const int lim = qpos - list_j(ent) * BK - g * HALF;  // column c of this half visible iff c <= lim
+                // P pass (needs S only; dP may still be running): P as bf16 pairs in registers
+                uint32_t sr[HALF], pk[HALF / 2];
+                tmem_ld_cols<HALF>(tl + C::COL_S + g * HALF, sr);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar_sfree);  // S(G) is in registers: S(G+1) may be written
 #pragma unroll
-            for (int c = 0; c < HALF; c += 2) {
-                const float p0 = (vis && c <= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -lx)) : 0.f;
-                const float p1 = (vis && c + 1 <= lim) ? ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -lx)) : 0.f;
-                pk[c / 2] = pack_bf16x2(p0, p1);
-            }
-            if (!warp_wait(bar_dp, n & 1, ctl)) {
-                fail = true;
-                break;
-            }
-            tc_fence_after();
-            // dS pass: dS = P (dP - D), bf16 pairs over the first HALF/2 columns
-            // of this half of dP (already read)
-            tmem_ld_cols<HALF>(tl + C::COL_DP + g * HALF, sr);
-            tmem_wait_ld();
+                for (int c = 0; c < HALF; c += 2) {
+                    const float p0 = (vis && c <= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -lx)) : 0.f;
+                    const float p1 = (vis && c + 1 <= lim) ? ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -lx)) : 0.f;
+                    pk[c / 2] = pack_bf16x2(p0, p1);
+                }
+                if (!warp_wait(bar_dp, G & 1, ctl)) {
+                    fail = true;
+                    break;
+                }
+                tc_fence_after();
+                // dS pass: dS = P (dP - D), bf16 pairs over the first HALF/2 columns
+                // of this half of dP (already read)
+                tmem_ld_cols<HALF>(tl + C::COL_DP + g * HALF, sr);
+                tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < HALF; c += 2) {
-                const float d0 = bf16lo(pk[c / 2]) * (__uint_as_float(sr[c]) - dy);
-                const float d1 = bf16hi(pk[c / 2]) * (__uint_as_float(sr[c + 1]) - dy);
-                pk[c / 2] = pack_bf16x2(d0, d1);
+                for (int c = 0; c < HALF; c += 2) {
+                    const float d0 = bf16lo(pk[c / 2]) * (__uint_as_float(sr[c]) - dy);
+                    const float d1 = bf16hi(pk[c / 2]) * (__uint_as_float(sr[c + 1]) - dy);
+                    pk[c / 2] = pack_bf16x2(d0, d1);
+                }
+                tmem_st_cols<HALF / 2>(tl + C::COL_DP + g * HALF, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_ds);
             }
-            tmem_st_cols<HALF / 2>(tl + C::COL_DP + g * HALF, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar_ds);
-        }
-        if (!fail) {
-            // warpgroup g stores output columns g * HD/2 .. (g + 1) * HD/2 - 1
+            if (fail) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_le(b));
+            // warpgroup g stores output columns g * HD/2 .. (g + 1) * HD/2 - 1; the
+            // next item's first dQ MMA (which overwrites the accumulator) waits
+            // for this warpgroup's first dS of that item, so it follows these loads
             uint16_t* drow = p.dq + ((int64_t)bh * p.seq + qpos) * HD + g * (HD / 2);
             if (len > 0) {
-                if (warp_wait(bar_acc, 0, ctl)) {
-                    tc_fence_after();
+                if (!warp_wait(bar_acc, (n_acc++) & 1, ctl)) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < HD / 64; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tl + C::COL_ACC + g * (HD / 2) + 32 * c, o);
-                        tmem_wait_ld();
-                        if (row_valid) {
+                for (int c = 0; c < HD / 64; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tl + C::COL_ACC + g * (HD / 2) + 32 * c, o);
+                    tmem_wait_ld();
+                    if (row_valid) {
 #pragma unroll
-                            for (int e2 = 0; e2 < 32; e2 += 8) {
-                                uint4 v;
-                                v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * p.scale, __uint_as_float(o[e2 + 1]) * p.scale);
-                                v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * p.scale, __uint_as_float(o[e2 + 3]) * p.scale);
-                                v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * p.scale, __uint_as_float(o[e2 + 5]) * p.scale);
-                                v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * p.scale, __uint_as_float(o[e2 + 7]) * p.scale);
-                                *reinterpret_cast<uint4*>(drow + 32 * c + e2) = v;
-                            }
+                        for (int e2 = 0; e2 < 32; e2 += 8) {
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * p.scale, __uint_as_float(o[e2 + 1]) * p.scale);
+                            v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * p.scale, __uint_as_float(o[e2 + 3]) * p.scale);
+                            v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * p.scale, __uint_as_float(o[e2 + 5]) * p.scale);
+                            v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * p.scale, __uint_as_float(o[e2 + 7]) * p.scale);
+                            *reinterpret_cast<uint4*>(drow + 32 * c + e2) = v;
                         }
                     }
                 }
@@ -459,6 +564,16 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    if (threadIdx.x == 0) {
+        // The last CTA to finish resets the counter for the next launch on this slot
+        // (every CTA has stopped taking items by now).
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+            atomicExch(p.sched, 0);
+            atomicExch(p.sched + 1, 0);
+            __threadfence();
+        }
     }
 }
 

@@ -189,14 +189,16 @@ int launch_backward(const void* q, const void* k, const void* v, s2::BackwardPar
     if (grid0 > (int64_t)g_dev[dev].num_sms * 16) grid0 = (int64_t)g_dev[dev].num_sms * 16;
     s2::s2_bwd_stats_kernel<HD><<<(unsigned)grid0, 256, 0, stream>>>(bp);
     if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
-    kq<<<(unsigned)(planes * bp.ntiles), 384, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
+    // dQ: persistent, at most one CTA per SM (work counter slot in bp.sched)
+    const uint64_t qitems = planes * (uint64_t)bp.ntiles;
+    const uint64_t qgrid = qitems < (uint64_t)g_dev[dev].num_sms ? qitems : (uint64_t)g_dev[dev].num_sms;
+    kq<<<(unsigned)qgrid, 384, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
     if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
     kkv<<<(unsigned)(kvplanes * bp.ntiles), 384, CK::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
-// Chunked prefill: one CTA per (tile slot, head, sequence); slots past a
-// sequence's chunk exit at once.
+// Chunked prefill: persistent CTAs over (sequence, head, tile pair) items.
 template <int HD, int BK>
 int launch_chunk(const void* q, const void* kc, const void* vc, s2::ChunkParams& cp, int dev, int attr_slot,
                  cudaStream_t stream)
@@ -418,6 +420,7 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
     bp.scale_log2 = scale * 1.4426950408889634f;
     bp.timeout_ns = g_timeout_ns.load();
     bp.gflags = g_dev[dev].flags;
+    bp.sched = g_dev[dev].sched + 2 * (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 128 && block_size == 128) return launch_backward<128, 128>(q, k, v, bp, dev, 0, st);
     if (head_dim == 128 && block_size == 64) return launch_backward<128, 64>(q, k, v, bp, dev, 1, st);
