@@ -30,16 +30,18 @@
 // both) so that no accumulator is shared between CTAs: no atomics, and the
 // results are deterministic.
 //
-// CTA = 12 warps: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer (one
-// thread), warp 2 builds the union list in shared memory (in the dQ kernel:
-// item after item, double-buffered, and loads the item's Q and dO), warps 4..11 the element-wise passes and the epilogue: thread = one
+// CTA = 12 warps: warp 0 TMA producer; warp 1 TMEM owner and MMA issuer (one
+// thread; in the dQ kernel it issues S and dP while one thread of warp 3
+// issues dQ); warp 2 builds the union list in shared memory (in the dQ
+// kernel item after item, double-buffered, and it also loads the item's Q
+// and dO); warps 4..11 the element-wise passes and the epilogue: thread = one
 // tile row = one TMEM lane, warps 4..7 on the first half of the columns and
 // warps 8..11 on the second (two warps per SM sub-partition hide the
 // exponential and TMEM latencies; a single warpgroup was measured to leave
-// the tensor core idle most of the time); warp 3 idles. With B = 64 a 128-row tile holds two
-// blocks and every row masks by its own block's tag. Every wait is bounded;
-// on a timeout the CTA drains its own copies and MMAs, frees TMEM and exits
-// with the device timeout flag set.
+// the tensor core idle most of the time). In the dK/dV kernel warp 3 idles.
+// With B = 64 a 128-row tile holds two blocks and every row masks by its own
+// block's tag. Every wait is bounded; on a timeout the CTA drains its own
+// copies and MMAs, frees TMEM and exits with the device timeout flag set.
 #pragma once
 
 #include <climits>
@@ -170,12 +172,12 @@ struct BwdQCfg {
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
     static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
     // barriers: qd_full, qd_empty, k_full[ST], v_full[ST], kv_empty[ST], s_full, ds_full, acc_done,
-    // drain, dp_full, s_free, list_full[2], list_empty[2]
-    static constexpr int NBAR = 2 + 3 * ST + 6 + 4;
+    // drain, dp_full, s_free, list_full[2], list_empty[2], dq_done, drain of the dQ issuer
+    static constexpr int NBAR = 2 + 3 * ST + 6 + 4 + 2;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
-    static constexpr uint32_t LIST_CONSUMERS = 10;  // producer, MMA issuer, 8 element-wise warps
+    static constexpr uint32_t LIST_CONSUMERS = 11;  // producer, 2 MMA issuers, 8 element-wise warps
     static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_ACC = 2 * BK;
     // Q and dO, the A operands of every S and dP MMA of an item, sit in TMEM
     // (HD/2 columns each): those MMAs read only K or V from shared memory.
@@ -219,6 +221,8 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t bar_sfree = bar_s + 40u;
     auto bar_lf = [&](int b) { return bar_s + 48u + 8u * b; };
     auto bar_le = [&](int b) { return bar_s + 64u + 8u * b; };
+    const uint32_t bar_dqd = bar_s + 80u;  // dQ(G) done: dP's columns (its dS) are free
+    const uint32_t bar_dr2 = bar_s + 88u;
     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
     // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
@@ -245,6 +249,8 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mbar_init(bar_lf(b), 1);
             mbar_init(bar_le(b), C::LIST_CONSUMERS);
         }
+        mbar_init(bar_dqd, 1);
+        mbar_init(bar_dr2, 1);
         *abort_cta = 0;
         fence_mbar_init();
     }
@@ -354,45 +360,17 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ S and dP issuer
+        // Element G (counted over all items) uses stage G % ST. S(G) and dP(G)
+        // are committed separately so that the element-wise warps start on P
+        // while dP is still running. S(G) is issued once the warps have loaded
+        // S(G-1) (they keep P in registers); dP(G) once dQ(G-1), issued by the
+        // other thread, has read dS(G-1) from dP's columns.
         if (lane == 0) {
             constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S = Q K^T, dP = dO V^T
-            constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);  // dQ += dS K (K as MN-major B)
             const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
             const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
             bool issued = false, fail = false;
-            // Element G (counted over all items) uses stage G % ST; S(G) and dP(G)
-            // are committed separately so that the element-wise warps start on P
-            // while dP is still running. Order per element: [S(G) read out]
-            // S(G+1); [dS(G) ready] dQ(G), dP(G+1). The warps keep P in
-            // registers, so S(G+1) may overwrite S(G) as soon as they have
-            // loaded it; dS(G) sits in dP's columns and dP(G+1) is issued after
-            // dQ(G) has read it.
-            auto issue_s = [&](int G) {
-                const int st = G % C::ST;
-                if (!mbar_wait(bar_kf(st), (G / C::ST) & 1, ctl)) return false;
-                tc_fence_after();
-                const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_QA + kk * 8, dk_desc + kstep(kk, BK), idesc_s,
-                                 kk > 0 ? 1u : 0u);
-                umma_commit(bar_s);
-                issued = true;
-                return true;
-            };
-            auto issue_dp = [&](int G) {
-                const int st = G % C::ST;
-                if (!mbar_wait(bar_vf(st), (G / C::ST) & 1, ctl)) return false;
-                tc_fence_after();
-                const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_DOA + kk * 8, dv_desc + kstep(kk, BK),
-                                 idesc_s, kk > 0 ? 1u : 0u);
-                umma_commit(bar_dp);
-                return true;
-            };
             int G = 0;
             for (int k = 0; !fail; ++k) {
                 const int b = k & 1;
@@ -400,8 +378,8 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 if (list_item[b] < 0) break;
                 const int len = list_len[b];
                 if (!mbar_wait(bar_qd, k & 1, ctl)) break;
-                // Q and dO into TMEM (after the previous item's MMAs that read them,
-                // in issue order); the shared-memory buffers are then free.
+                // Q and dO into TMEM (after the previous item's S and dP MMAs, in
+                // issue order); the shared-memory buffers are then free.
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
@@ -410,52 +388,85 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 }
                 umma_commit(bar_qe);
                 issued = true;
-                if (len > 0) {
-                    // S's columns are free once the warps have loaded S of the previous
-                    // element; dP's (its dS) were read by its dQ, issued before.
-                    if (G > 0 && !mbar_wait(bar_sfree, (G - 1) & 1, ctl)) break;
-                    tc_fence_after();
-                    if (!issue_s(G) || !issue_dp(G)) break;
-                    for (int n = 0; n < len; ++n, ++G) {
-                        const int st = G % C::ST;
-                        const bool more = n + 1 < len;
-                        if (more) {
-                            if (!mbar_wait(bar_sfree, G & 1, ctl)) {
-                                fail = true;
-                                break;
-                            }
-                            tc_fence_after();
-                            if (!issue_s(G + 1)) {
-                                fail = true;
-                                break;
-                            }
-                        }
-                        if (!mbar_wait(bar_ds, G & 1, ctl)) {
-                            fail = true;
-                            break;
-                        }
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint64_t bk =
-                                umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
-                            umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
-                                         (n > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(bar_ke(st));
-                        if (more && !issue_dp(G + 1)) {
-                            fail = true;
-                            break;
-                        }
+                for (int n = 0; n < len; ++n, ++G) {
+                    const int st = G % C::ST;
+                    // S(G): S's columns are free once the warps have loaded S(G-1)
+                    // (S(G) is issued only after this wait: the phases cannot alias)
+                    if ((G > 0 && !mbar_wait(bar_sfree, (G - 1) & 1, ctl)) ||
+                        !mbar_wait(bar_kf(st), (G / C::ST) & 1, ctl)) {
+                        fail = true;
+                        break;
                     }
-                    if (fail) break;
-                    umma_commit(bar_acc);  // dQ of this item is complete once its last MMA is
+                    tc_fence_after();
+                    const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_QA + kk * 8, dk_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+                    umma_commit(bar_s);
+                    // dP(G): dP's columns are free once dQ(G-1) has completed
+                    if ((G > 0 && !mbar_wait(bar_dqd, (G - 1) & 1, ctl)) ||
+                        !mbar_wait(bar_vf(st), (G / C::ST) & 1, ctl)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_DOA + kk * 8, dv_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+                    umma_commit(bar_dp);
                 }
+                if (fail) break;
                 mbar_arrive(bar_le(b));
             }
             if (*abort_cta && issued) {
                 umma_commit(bar_dr);
                 mbar_drain(bar_dr, 0, kDrainNs);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ dQ issuer
+        // dQ(G) += dS(G) K once the warps have written dS(G); its commit frees
+        // dP's columns for dP(G+1) and releases the K/V stage (dS(G) needed S(G)
+        // and dP(G) complete, so every read of the stage is done). The S/dP
+        // thread waits for every element's loads in order, so a stage cannot
+        // be refilled before it has passed the stage.
+        if (lane == 0) {
+            constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);  // dQ += dS K (K as MN-major B)
+            bool issued = false, fail = false;
+            int G = 0;
+            for (int k = 0; !fail; ++k) {
+                const int b = k & 1;
+                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                if (list_item[b] < 0) break;
+                const int len = list_len[b];
+                for (int n = 0; n < len; ++n, ++G) {
+                    const int st = G % C::ST;
+                    if (!mbar_wait(bar_ds, G & 1, ctl)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t bk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
+                                     (n > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_dqd);
+                    umma_commit(bar_ke(st));
+                    issued = true;
+                }
+                if (fail) break;
+                if (len > 0) umma_commit(bar_acc);  // dQ of this item is complete once its last MMA is
+                mbar_arrive(bar_le(b));
+            }
+            if (*abort_cta && issued) {
+                umma_commit(bar_dr2);
+                mbar_drain(bar_dr2, 0, kDrainNs);
             }
         }
         __syncwarp();
