@@ -38,7 +38,8 @@
 // tile row = one TMEM lane, warps 4..7 on the first half of the columns and
 // warps 8..11 on the second (two warps per SM sub-partition hide the
 // exponential and TMEM latencies; a single warpgroup was measured to leave
-// the tensor core idle most of the time). In the dK/dV kernel warp 3 idles.
+// the tensor core idle most of the time). In the dK/dV kernel warp 1 issues
+// S^T and dP^T and one thread of warp 3 issues dV and dK.
 // With B = 64 a 128-row tile holds two blocks and every row masks by its own
 // block's tag. Every wait is bounded; on a timeout the CTA drains its own
 // copies and MMAs, frees TMEM and exits with the device timeout flag set.
@@ -177,7 +178,12 @@ struct BwdQCfg {
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
-    static constexpr uint32_t LIST_CONSUMERS = 11;  // producer, 2 MMA issuers, 8 element-wise warps
+    // 64-key blocks: one thread issues S and dP, another dQ (one thread issuing
+    // all 20 MMAs of an element, with their waits and commits, was the limit;
+    // with 128-key blocks one thread keeps up with the tensor core).
+    static constexpr bool SPLIT = BK == 64;
+    // producer, MMA issuer(s), 8 element-wise warps
+    static constexpr uint32_t LIST_CONSUMERS = SPLIT ? 11 : 10;
     static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_ACC = 2 * BK;
     // Q and dO, the A operands of every S and dP MMA of an item, sit in TMEM
     // (HD/2 columns each): those MMAs read only K or V from shared memory.
@@ -359,57 +365,149 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ S and dP issuer
-        // Element G (counted over all items) uses stage G % ST. S(G) and dP(G)
-        // are committed separately so that the element-wise warps start on P
-        // while dP is still running. S(G) is issued once the warps have loaded
-        // S(G-1) (they keep P in registers); dP(G) once dQ(G-1), issued by the
-        // other thread, has read dS(G-1) from dP's columns.
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S = Q K^T, dP = dO V^T
-            const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
-            const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
-            bool issued = false, fail = false;
-            int G = 0;
-            for (int k = 0; !fail; ++k) {
-                const int b = k & 1;
-                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
-                if (list_item[b] < 0) break;
-                const int len = list_len[b];
-                if (!mbar_wait(bar_qd, k & 1, ctl)) break;
-                // Q and dO into TMEM (after the previous item's S and dP MMAs, in
-                // issue order); the shared-memory buffers are then free.
-                tc_fence_after();
+    } else if (warp == 1 || (C::SPLIT && warp == 3)) {
+        if constexpr (C::SPLIT) {
+            if (warp == 1) {
+                // ------------------------------------------------------------ S and dP issuer
+                // Element G (counted over all items) uses stage G % ST. S(G) and dP(G)
+                // are committed separately so that the element-wise warps start on P
+                // while dP is still running. S(G) is issued once the warps have loaded
+                // S(G-1) (they keep P in registers); dP(G) once dQ(G-1), issued by the
+                // other thread, has read dS(G-1) from dP's columns.
+                if (lane == 0) {
+                    constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S = Q K^T, dP = dO V^T
+                    const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
+                    const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
+                    bool issued = false, fail = false;
+                    int G = 0;
+                    for (int k = 0; !fail; ++k) {
+                        const int b = k & 1;
+                        if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                        if (list_item[b] < 0) break;
+                        const int len = list_len[b];
+                        if (!mbar_wait(bar_qd, k & 1, ctl)) break;
+                        // Q and dO into TMEM (after the previous item's S and dP MMAs, in
+                        // issue order); the shared-memory buffers are then free.
+                        tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    tmem_cp_128x256b(tmem + C::COL_QA + kk * 8, dq_desc + kstep(kk, C::M));
-                    tmem_cp_128x256b(tmem + C::COL_DOA + kk * 8, ddo_desc + kstep(kk, C::M));
-                }
-                umma_commit(bar_qe);
-                issued = true;
-                for (int n = 0; n < len; ++n, ++G) {
-                    const int st = G % C::ST;
-                    // S(G): S's columns are free once the warps have loaded S(G-1)
-                    // (S(G) is issued only after this wait: the phases cannot alias)
-                    if ((G > 0 && !mbar_wait(bar_sfree, (G - 1) & 1, ctl)) ||
-                        !mbar_wait(bar_kf(st), (G / C::ST) & 1, ctl)) {
-                        fail = true;
-                        break;
+                        for (int kk = 0; kk < HD / 16; ++kk) {
+                            tmem_cp_128x256b(tmem + C::COL_QA + kk * 8, dq_desc + kstep(kk, C::M));
+                            tmem_cp_128x256b(tmem + C::COL_DOA + kk * 8, ddo_desc + kstep(kk, C::M));
+                        }
+                        umma_commit(bar_qe);
+                        issued = true;
+                        for (int n = 0; n < len; ++n, ++G) {
+                            const int st = G % C::ST;
+                            // S(G): S's columns are free once the warps have loaded S(G-1)
+                            // (S(G) is issued only after this wait: the phases cannot alias)
+                            if ((G > 0 && !mbar_wait(bar_sfree, (G - 1) & 1, ctl)) ||
+                                !mbar_wait(bar_kf(st), (G / C::ST) & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < HD / 16; ++kk)
+                                umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_QA + kk * 8, dk_desc + kstep(kk, BK),
+                                             idesc_s, kk > 0 ? 1u : 0u);
+                            umma_commit(bar_s);
+                            // dP(G): dP's columns are free once dQ(G-1) has completed
+                            if ((G > 0 && !mbar_wait(bar_dqd, (G - 1) & 1, ctl)) ||
+                                !mbar_wait(bar_vf(st), (G / C::ST) & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < HD / 16; ++kk)
+                                umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_DOA + kk * 8, dv_desc + kstep(kk, BK),
+                                             idesc_s, kk > 0 ? 1u : 0u);
+                            umma_commit(bar_dp);
+                        }
+                        if (fail) break;
+                        mbar_arrive(bar_le(b));
                     }
+                    if (*abort_cta && issued) {
+                        umma_commit(bar_dr);
+                        mbar_drain(bar_dr, 0, kDrainNs);
+                    }
+                }
+            } else {
+                // ------------------------------------------------------------ dQ issuer
+                // dQ(G) += dS(G) K once the warps have written dS(G); its commit frees
+                // dP's columns for dP(G+1) and releases the K/V stage (dS(G) needed S(G)
+                // and dP(G) complete, so every read of the stage is done). The S/dP
+                // thread waits for every element's loads in order, so a stage cannot
+                // be refilled before it has passed the stage.
+                if (lane == 0) {
+                    constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);  // dQ += dS K (K as MN-major B)
+                    bool issued = false, fail = false;
+                    int G = 0;
+                    for (int k = 0; !fail; ++k) {
+                        const int b = k & 1;
+                        if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                        if (list_item[b] < 0) break;
+                        const int len = list_len[b];
+                        for (int n = 0; n < len; ++n, ++G) {
+                            const int st = G % C::ST;
+                            if (!mbar_wait(bar_ds, G & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
+                            tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < BK / 16; ++kk) {
+                                const uint64_t bk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
+                                umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
+                                             (n > 0 || kk > 0) ? 1u : 0u);
+                            }
+                            umma_commit(bar_dqd);
+                            umma_commit(bar_ke(st));
+                            issued = true;
+                        }
+                        if (fail) break;
+                        if (len > 0) umma_commit(bar_acc);  // dQ of this item is complete once its last MMA is
+                        mbar_arrive(bar_le(b));
+                    }
+                    if (*abort_cta && issued) {
+                        umma_commit(bar_dr2);
+                        mbar_drain(bar_dr2, 0, kDrainNs);
+                    }
+                }
+            }
+        } else {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S = Q K^T, dP = dO V^T
+                constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);  // dQ += dS K (K as MN-major B)
+                const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
+                const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
+                bool issued = false, fail = false;
+                // Element G (counted over all items) uses stage G % ST; S(G) and dP(G)
+                // are committed separately so that the element-wise warps start on P
+                // while dP is still running. Order per element: [S(G) read out]
+                // S(G+1); [dS(G) ready] dQ(G), dP(G+1). The warps keep P in
+                // registers, so S(G+1) may overwrite S(G) as soon as they have
+                // loaded it; dS(G) sits in dP's columns and dP(G+1) is issued after
+                // dQ(G) has read it.
+                auto issue_s = [&](int G) {
+                    const int st = G % C::ST;
+                    if (!mbar_wait(bar_kf(st), (G / C::ST) & 1, ctl)) return false;
                     tc_fence_after();
                     const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_QA + kk * 8, dk_desc + kstep(kk, BK),
-                                     idesc_s, kk > 0 ? 1u : 0u);
+                        umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_QA + kk * 8, dk_desc + kstep(kk, BK), idesc_s,
+                                     kk > 0 ? 1u : 0u);
                     umma_commit(bar_s);
-                    // dP(G): dP's columns are free once dQ(G-1) has completed
-                    if ((G > 0 && !mbar_wait(bar_dqd, (G - 1) & 1, ctl)) ||
-                        !mbar_wait(bar_vf(st), (G / C::ST) & 1, ctl)) {
-                        fail = true;
-                        break;
-                    }
+                    issued = true;
+                    return true;
+                };
+                auto issue_dp = [&](int G) {
+                    const int st = G % C::ST;
+                    if (!mbar_wait(bar_vf(st), (G / C::ST) & 1, ctl)) return false;
                     tc_fence_after();
                     const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
 #pragma unroll
@@ -417,56 +515,72 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_DOA + kk * 8, dv_desc + kstep(kk, BK),
                                      idesc_s, kk > 0 ? 1u : 0u);
                     umma_commit(bar_dp);
-                }
-                if (fail) break;
-                mbar_arrive(bar_le(b));
-            }
-            if (*abort_cta && issued) {
-                umma_commit(bar_dr);
-                mbar_drain(bar_dr, 0, kDrainNs);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 3) {
-        // ------------------------------------------------------------ dQ issuer
-        // dQ(G) += dS(G) K once the warps have written dS(G); its commit frees
-        // dP's columns for dP(G+1) and releases the K/V stage (dS(G) needed S(G)
-        // and dP(G) complete, so every read of the stage is done). The S/dP
-        // thread waits for every element's loads in order, so a stage cannot
-        // be refilled before it has passed the stage.
-        if (lane == 0) {
-            constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);  // dQ += dS K (K as MN-major B)
-            bool issued = false, fail = false;
-            int G = 0;
-            for (int k = 0; !fail; ++k) {
-                const int b = k & 1;
-                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
-                if (list_item[b] < 0) break;
-                const int len = list_len[b];
-                for (int n = 0; n < len; ++n, ++G) {
-                    const int st = G % C::ST;
-                    if (!mbar_wait(bar_ds, G & 1, ctl)) {
-                        fail = true;
-                        break;
-                    }
+                    return true;
+                };
+                int G = 0;
+                for (int k = 0; !fail; ++k) {
+                    const int b = k & 1;
+                    if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                    if (list_item[b] < 0) break;
+                    const int len = list_len[b];
+                    if (!mbar_wait(bar_qd, k & 1, ctl)) break;
+                    // Q and dO into TMEM (after the previous item's MMAs that read them,
+                    // in issue order); the shared-memory buffers are then free.
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t bk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
-                                     (n > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        tmem_cp_128x256b(tmem + C::COL_QA + kk * 8, dq_desc + kstep(kk, C::M));
+                        tmem_cp_128x256b(tmem + C::COL_DOA + kk * 8, ddo_desc + kstep(kk, C::M));
                     }
-                    umma_commit(bar_dqd);
-                    umma_commit(bar_ke(st));
+                    umma_commit(bar_qe);
                     issued = true;
+                    if (len > 0) {
+                        // S's columns are free once the warps have loaded S of the previous
+                        // element; dP's (its dS) were read by its dQ, issued before.
+                        if (G > 0 && !mbar_wait(bar_sfree, (G - 1) & 1, ctl)) break;
+                        tc_fence_after();
+                        if (!issue_s(G) || !issue_dp(G)) break;
+                        for (int n = 0; n < len; ++n, ++G) {
+                            const int st = G % C::ST;
+                            const bool more = n + 1 < len;
+                            if (more) {
+                                if (!mbar_wait(bar_sfree, G & 1, ctl)) {
+                                    fail = true;
+                                    break;
+                                }
+                                tc_fence_after();
+                                if (!issue_s(G + 1)) {
+                                    fail = true;
+                                    break;
+                                }
+                            }
+                            if (!mbar_wait(bar_ds, G & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
+                            tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < BK / 16; ++kk) {
+                                const uint64_t bk =
+                                    umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
+                                umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
+                                             (n > 0 || kk > 0) ? 1u : 0u);
+                            }
+                            umma_commit(bar_ke(st));
+                            if (more && !issue_dp(G + 1)) {
+                                fail = true;
+                                break;
+                            }
+                        }
+                        if (fail) break;
+                        umma_commit(bar_acc);  // dQ of this item is complete once its last MMA is
+                    }
+                    mbar_arrive(bar_le(b));
                 }
-                if (fail) break;
-                if (len > 0) umma_commit(bar_acc);  // dQ of this item is complete once its last MMA is
-                mbar_arrive(bar_le(b));
-            }
-            if (*abort_cta && issued) {
-                umma_commit(bar_dr2);
-                mbar_drain(bar_dr2, 0, kDrainNs);
+                if (*abort_cta && issued) {
+                    umma_commit(bar_dr);
+                    mbar_drain(bar_dr, 0, kDrainNs);
+                }
             }
         }
         __syncwarp();
@@ -607,8 +721,9 @@ struct BwdKVCfg {
     static constexpr uint32_t OFF_LIST = OFF_STAT + ST * STATBYTES;
     static constexpr uint32_t OFF_SCR = OFF_LIST + LIST_CAP * 4;  // list-merge scratch (ROWS > 1)
     static constexpr uint32_t OFF_BAR = OFF_SCR + (ROWS > 1 ? ROWS * LIST_CAP * 4 : 0);
-    // barriers: kv_full, q_full[ST], q_empty[ST], s_full, p_full, acc_done, drain, dp_full, ds_full
-    static constexpr int NBAR = 1 + 2 * ST + 6;
+    // barriers: kv_full, q_full[ST], q_empty[ST], s_full, p_full, acc_done, drain, dp_full, ds_full,
+    // dv_done, dk_done, drain of the dV/dK issuer
+    static constexpr int NBAR = 1 + 2 * ST + 6 + 3;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
@@ -617,6 +732,11 @@ struct BwdKVCfg {
     // every S^T and dP^T MMA of the CTA, sit in TMEM (HD/2 columns each).
     static constexpr bool A_IN_TMEM = 2 * BK + 3 * HD <= 512;
     static constexpr uint32_t COL_KA = 2 * BK + 2 * HD, COL_VA = 2 * BK + 2 * HD + HD / 2;
+    // 64-key blocks: one thread issues S^T and dP^T, another dV and dK (one
+    // thread issuing all 24 MMAs of an element, with their waits and commits,
+    // was the limit; with 128-key blocks one thread keeps up with the tensor
+    // core, and splitting only added completion waits: measured 3 % slower).
+    static constexpr bool SPLIT = BK == 64;
     static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD + (A_IN_TMEM ? HD : 0)) <= 256 ? 256 : 512;
     static_assert(2 * BK + 2 * HD <= 512, "TMEM budget");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -664,6 +784,9 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const uint32_t bar_dr = bar_s + 24u;
     const uint32_t bar_dp = bar_s + 32u;
     const uint32_t bar_ds = bar_s + 40u;
+    const uint32_t bar_dvd = bar_s + 48u;  // dV(n) done: S^T's columns (its P^T) are free
+    const uint32_t bar_dkd = bar_s + 56u;  // dK(n) done: dP^T's columns (its dS^T) are free
+    const uint32_t bar_dr2 = bar_s + 64u;
     uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2] list length
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
@@ -681,6 +804,9 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         mbar_init(bar_p, 256);
         mbar_init(bar_acc, 1);
         mbar_init(bar_dr, 1);
+        mbar_init(bar_dvd, 1);
+        mbar_init(bar_dkd, 1);
+        mbar_init(bar_dr2, 1);
         *abort_cta = 0;
         fence_mbar_init();
     }
@@ -757,92 +883,194 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && len > 0) {
-            constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
-            constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);   // dV += P^T dO, dK += dS^T Q
-            const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
-            const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
-            bool issued = false;
-            // S^T(n) and dP^T(n) are committed separately so that the element-wise
-            // warps compute P^T while dP^T is still running. Order per element n:
-            // [P^T(n) ready] dV(n), S^T(n+1); [dS^T(n) ready] dK(n), dP^T(n+1).
-            // S^T(n+1) overwrites P^T(n) after dV(n) has read it (MMAs of one
-            // thread run in issue order; the warps keep P in registers for the
-            // dS pass); dP^T(n+1) overwrites dS^T(n) after dK(n).
-            auto issue_st = [&](int n) {
-                const int st = n % C::ST;
-                if (!mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl)) return false;
-                tc_fence_after();
-                const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
+    } else if (warp == 1 || (C::SPLIT && warp == 3)) {
+        if constexpr (C::SPLIT) {
+            if (warp == 1) {
+                // ------------------------------------------------------------ S^T and dP^T issuer
+                // S^T(n) and dP^T(n) are committed separately so that the element-wise
+                // warps compute P^T while dP^T is still running. S^T(n) overwrites
+                // P^T(n-1) and so waits for dV(n-1)'s commit; dP^T(n) overwrites
+                // dS^T(n-1) and waits for dK(n-1)'s (both issued by the other thread;
+                // the warps keep P in registers for the dS pass).
+                if (lane == 0 && len > 0) {
+                    constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
+                    const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
+                    const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
+                    bool issued = false;
+                    const bool kv_ok = mbar_wait(bar_kv, 0, ctl);
+                    if (kv_ok && C::A_IN_TMEM) {  // K and V into TMEM, before every MMA that reads them
+                        tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    if constexpr (C::A_IN_TMEM)
-                        umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_KA + kk * 8, dq_desc + kstep(kk, BK), idesc_s,
-                                     kk > 0 ? 1u : 0u);
-                    else
-                        umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK), idesc_s,
-                                     kk > 0 ? 1u : 0u);
-                }
-                umma_commit(bar_s);
-                issued = true;
-                return true;
-            };
-            auto issue_dpt = [&](int n) {  // stage already waited for by issue_st(n)
-                const int st = n % C::ST;
-                const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
+                        for (int kk = 0; kk < HD / 16; ++kk) {
+                            tmem_cp_128x256b(tmem + C::COL_KA + kk * 8, dk_desc + kstep(kk, C::M));
+                            tmem_cp_128x256b(tmem + C::COL_VA + kk * 8, dv_desc + kstep(kk, C::M));
+                        }
+                        issued = true;
+                    }
+                    for (int n = 0; kv_ok && n < len; ++n) {
+                        const int st = n % C::ST;
+                        if ((n > 0 && !mbar_wait(bar_dvd, (n - 1) & 1, ctl)) ||
+                            !mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl))
+                            break;
+                        tc_fence_after();
+                        const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    if constexpr (C::A_IN_TMEM)
-                        umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_VA + kk * 8, ddo_desc + kstep(kk, BK),
-                                     idesc_s, kk > 0 ? 1u : 0u);
-                    else
-                        umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
-                                     idesc_s, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(bar_dp);
-            };
-            const bool kv_ok = mbar_wait(bar_kv, 0, ctl);
-            if (kv_ok && C::A_IN_TMEM) {  // K and V into TMEM, before every MMA that reads them
-                tc_fence_after();
+                        for (int kk = 0; kk < HD / 16; ++kk) {
+                            if constexpr (C::A_IN_TMEM)
+                                umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_KA + kk * 8, dq_desc + kstep(kk, BK), idesc_s,
+                                             kk > 0 ? 1u : 0u);
+                            else
+                                umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK), idesc_s,
+                                             kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(bar_s);
+                        issued = true;
+                        if (n > 0 && !mbar_wait(bar_dkd, (n - 1) & 1, ctl)) break;
+                        tc_fence_after();
+                        const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    tmem_cp_128x256b(tmem + C::COL_KA + kk * 8, dk_desc + kstep(kk, C::M));
-                    tmem_cp_128x256b(tmem + C::COL_VA + kk * 8, dv_desc + kstep(kk, C::M));
+                        for (int kk = 0; kk < HD / 16; ++kk) {
+                            if constexpr (C::A_IN_TMEM)
+                                umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_VA + kk * 8, ddo_desc + kstep(kk, BK),
+                                             idesc_s, kk > 0 ? 1u : 0u);
+                            else
+                                umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
+                                             idesc_s, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(bar_dp);
+                    }
+                    if (*abort_cta && issued) {
+                        umma_commit(bar_dr);
+                        mbar_drain(bar_dr, 0, kDrainNs);
+                    }
                 }
-                issued = true;
+            } else {
+                // ------------------------------------------------------------ dV and dK issuer
+                // dV(n) += P^T(n) dO once P^T(n) is written; dK(n) += dS^T(n) Q once
+                // dS^T(n) is. The commit after dK(n) releases the Q/dO stage (dS^T(n)
+                // needed S^T(n) and dP^T(n) complete, so every read of it is done);
+                // the other thread waits for every stage's loads in order, so a stage
+                // cannot be refilled before it has passed the stage.
+                if (lane == 0 && len > 0) {
+                    constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);   // dV += P^T dO, dK += dS^T Q
+                    bool issued = false;
+                    for (int n = 0; n < len; ++n) {
+                        const int st = n % C::ST;
+                        if (!mbar_wait(bar_p, n & 1, ctl)) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                            umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
+                                         (n > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(bar_dvd);
+                        issued = true;
+                        if (!mbar_wait(bar_ds, n & 1, ctl)) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                            umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + packed_col<BK>(kk), bq, idesc_a,
+                                         (n > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(bar_dkd);
+                        umma_commit(bar_qe(st));
+                        if (n + 1 == len && !*abort_cta) umma_commit(bar_acc);
+                    }
+                    if (*abort_cta && issued) {
+                        umma_commit(bar_dr2);
+                        mbar_drain(bar_dr2, 0, kDrainNs);
+                    }
+                }
             }
-            if (kv_ok && issue_st(0)) {
-                issue_dpt(0);
-                for (int n = 0; n < len; ++n) {
+        } else {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0 && len > 0) {
+                constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
+                constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);   // dV += P^T dO, dK += dS^T Q
+                const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
+                const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
+                bool issued = false;
+                // S^T(n) and dP^T(n) are committed separately so that the element-wise
+                // warps compute P^T while dP^T is still running. Order per element n:
+                // [P^T(n) ready] dV(n), S^T(n+1); [dS^T(n) ready] dK(n), dP^T(n+1).
+                // S^T(n+1) overwrites P^T(n) after dV(n) has read it (MMAs of one
+                // thread run in issue order; the warps keep P in registers for the
+                // dS pass); dP^T(n+1) overwrites dS^T(n) after dK(n).
+                auto issue_st = [&](int n) {
                     const int st = n % C::ST;
-                    const bool more = n + 1 < len;
-                    if (!mbar_wait(bar_p, n & 1, ctl)) break;
+                    if (!mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl)) return false;
+                    tc_fence_after();
+                    const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        if constexpr (C::A_IN_TMEM)
+                            umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_KA + kk * 8, dq_desc + kstep(kk, BK), idesc_s,
+                                         kk > 0 ? 1u : 0u);
+                        else
+                            umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK), idesc_s,
+                                         kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar_s);
+                    issued = true;
+                    return true;
+                };
+                auto issue_dpt = [&](int n) {  // stage already waited for by issue_st(n)
+                    const int st = n % C::ST;
+                    const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        if constexpr (C::A_IN_TMEM)
+                            umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_VA + kk * 8, ddo_desc + kstep(kk, BK),
+                                         idesc_s, kk > 0 ? 1u : 0u);
+                        else
+                            umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
+                                         idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar_dp);
+                };
+                const bool kv_ok = mbar_wait(bar_kv, 0, ctl);
+                if (kv_ok && C::A_IN_TMEM) {  // K and V into TMEM, before every MMA that reads them
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
-                                     (n > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        tmem_cp_128x256b(tmem + C::COL_KA + kk * 8, dk_desc + kstep(kk, C::M));
+                        tmem_cp_128x256b(tmem + C::COL_VA + kk * 8, dv_desc + kstep(kk, C::M));
                     }
-                    if (more && !issue_st(n + 1)) break;
-                    if (!mbar_wait(bar_ds, n & 1, ctl)) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + packed_col<BK>(kk), bq, idesc_a,
-                                     (n > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    umma_commit(bar_qe(st));
-                    if (more) issue_dpt(n + 1);
+                    issued = true;
                 }
-                if (!*abort_cta) umma_commit(bar_acc);
-            }
-            if (*abort_cta && issued) {
-                umma_commit(bar_dr);
-                mbar_drain(bar_dr, 0, kDrainNs);
+                if (kv_ok && issue_st(0)) {
+                    issue_dpt(0);
+                    for (int n = 0; n < len; ++n) {
+                        const int st = n % C::ST;
+                        const bool more = n + 1 < len;
+                        if (!mbar_wait(bar_p, n & 1, ctl)) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                            umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
+                                         (n > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        if (more && !issue_st(n + 1)) break;
+                        if (!mbar_wait(bar_ds, n & 1, ctl)) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                            umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + packed_col<BK>(kk), bq, idesc_a,
+                                         (n > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(bar_qe(st));
+                        if (more) issue_dpt(n + 1);
+                    }
+                    if (!*abort_cta) umma_commit(bar_acc);
+                }
+                if (*abort_cta && issued) {
+                    umma_commit(bar_dr);
+                    mbar_drain(bar_dr, 0, kDrainNs);
+                }
             }
         }
         __syncwarp();
