@@ -97,6 +97,16 @@ def test_stride_one_matches_autograd_of_causal_sdpa(s2gpu):
         assert (g.float() - r).abs().max().item() <= 2e-2 * max(1.0, r.abs().max().item())
 
 
+@pytest.mark.parametrize("bk,batch,seq", [(64, 8, 2048), (128, 4, 4096)])
+def test_many_items_per_cta(s2gpu, bk, batch, seq):
+    # 1024 query tiles for at most 148 persistent dQ CTAs: each CTA runs several
+    # items (double-buffered lists, barrier phases carried across items)
+    w = synth.PrefillWorkload("t", batch, 8, 64, seq, bk, 4, 1, seed=96)
+    q, k, v = synth.prefill_inputs(w)
+    lay = s2gpu.build_layout(w.heads, bk, 4, 1, w.num_blocks, device="cuda")
+    run_backward(s2gpu, w, lay, q, k, v, upstream(w, 7))
+
+
 def test_backward_is_deterministic(s2gpu):
     w = synth.PrefillWorkload("t", 1, 4, 128, 1024, 64, 4, 2, seed=94)
     q, k, v = (t.cuda() for t in synth.prefill_inputs(w))

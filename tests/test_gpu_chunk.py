@@ -80,6 +80,15 @@ def test_many_sequences_with_empty_chunks(s2gpu):
     case(s2gpu, ctx, qlen, H=2, D=64, B=64, S=3, L=1, seed=21)
 
 
+@pytest.mark.parametrize("B", [64, 128])
+def test_many_items_per_cta(s2gpu, B):
+    # ~400 tile-pair items for at most 148 persistent CTAs
+    rng = np.random.default_rng(22)
+    ctx = [int(c) for c in rng.integers(600, 2600, size=16)]
+    qlen = [min(c, int(rng.integers(300, 700))) for c in ctx]
+    case(s2gpu, ctx, qlen, H=8, D=64, B=B, S=4, L=1, seed=22 + B)
+
+
 def test_grouped_kv_heads(s2gpu):
     case(s2gpu, [700, 260], [300, 260], H=8, hkv=2, seed=5)
 
