@@ -333,20 +333,28 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             const ChunkItem I = items[b];
             const uint32_t* L = list + b * C::LIST_CAP;
             const int len = list_len[b];
-            for (int e = 0; e < len; ++e, ++n) {
-                const int st = n % C::ST;
-                if (!warp_wait(bar_ke(st), ((n / C::ST) & 1) ^ 1, ctl)) {
-                    stop = true;
-                    break;
-                }
+            // the cache plane of this lane's page of element e (the block-table
+            // read of the next element is issued before waiting for its stage)
+            auto page_plane = [&](int e) {
                 const int lp = list_j(L[e]) * C::PPB + lane;  // logical page of this lane
-                int32_t plane = oob_plane;
+                int32_t pl = oob_plane;
                 if (lane < C::PPB && lp * kChunkPage < I.n) {
                     const int32_t phys = __ldg(p.block_table + (int64_t)I.s * p.max_pages + lp);
                     if (phys < 0 || phys >= p.num_pages)
                         atomicOr(p.gflags, kFlagIndex);
                     else
-                        plane = phys * p.heads_kv + I.hkv;
+                        pl = phys * p.heads_kv + I.hkv;
+                }
+                return pl;
+            };
+            int32_t plane_next = len > 0 ? page_plane(0) : oob_plane;
+            for (int e = 0; e < len; ++e, ++n) {
+                const int st = n % C::ST;
+                const int32_t plane = plane_next;
+                if (e + 1 < len) plane_next = page_plane(e + 1);
+                if (!warp_wait(bar_ke(st), ((n / C::ST) & 1) ^ 1, ctl)) {
+                    stop = true;
+                    break;
                 }
                 if (lane == 0) mbar_arrive_expect_tx(bar_kf(st), 2 * C::KVBYTES);
                 __syncwarp();
