@@ -8,7 +8,10 @@ One step = one pass of the whole path over one batch of synthetic input:
   * decode (split-KV paged kernel + combine) over 64 sequences, 32 heads,
     head_dim 128, contexts U[4096, 32768], 16-token pages, permuted block table,
     B 128, S 16, L 4.
-The layouts are built once (host, per layout) before timing.
+The layouts are built once (host, per layout) before timing. After the W
+warm-up steps, untimed steps run for --settle-s seconds: the GPU reaches its
+power cap within ~0.1 s of sustained load, and the timed region is divided
+by the sustained tensor peak, so it is timed in that same state.
 
 Headline: prefill effective TFLOP/s (4 * head_dim per visible (query, key)
 pair; the dense work the pattern skips is not counted), from CUDA events around
@@ -118,6 +121,35 @@ def source_sha(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
+def settle(fn, seconds, dist, device, sync=None):
+    """Run fn (one untimed step) until `seconds` of wall time have passed, in
+    batches with a device sync after each, so that the clocks and power state
+    seen by the timed region are the sustained ones. Ranks agree on the count
+    (max over ranks), so every rank runs the same number of steps. Returns it."""
+    import torch
+
+    if sync is None:
+        def sync():
+            torch.cuda.synchronize(device)
+    if seconds <= 0:
+        return 0
+    n, batch, t0 = 0, 4, time.time()
+    while time.time() - t0 < seconds:
+        for _ in range(batch):
+            fn()
+        n += batch
+        sync()
+        batch = min(batch * 2, 256)
+    if dist is not None:
+        t = torch.tensor([n], dtype=torch.int64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        for _ in range(int(t.item()) - n):
+            fn()
+        n = int(t.item())
+        sync()
+    return n
+
+
 def max_over_ranks(vals, dist, device):
     """Element-wise maximum of per-rank timings (one all-reduce; identity on
     one process). Every rank must call it, with the same number of values."""
@@ -202,10 +234,18 @@ class ClockSampler:
             self._stop.set()
             self.t.join()
 
-    def summary(self):
-        if not self.ok or not self.samples:
+    def summary(self, t_on=None, t_off=None):
+        """Median SM clock and the reasons seen over the samples taken between
+        t_on and t_off (the timed region; the sampler also runs through the
+        warm-up so that NVML's readings are current when the region starts)."""
+        samples = self.samples
+        if t_on is not None:
+            inside = [s for s in samples if t_on <= s[0] <= t_off]
+            # a region shorter than the period: the samples nearest to it
+            samples = inside or sorted(samples, key=lambda s: abs(s[0] - t_on))[:2]
+        if not self.ok or not samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
-        loaded = [s for s in self.samples if not (s[2] & 0x1)] or self.samples
+        loaded = [s for s in samples if not (s[2] & 0x1)] or samples
         reasons = set()
         for _, _, rs, _ in loaded:
             for bit, name in self.REASONS.items():
@@ -273,29 +313,31 @@ def run_ours(args, rank, world, dist):
         if evs:
             evs[2].record(stream)
 
+    sampler = ClockSampler(dev.index)
+    sampler.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    settle_steps = settle(step, args.settle_s, dist, dev)
     rc, flags = s2attn.device_status(reset=True)
     if rc != 0:
         raise RuntimeError(f"device flags {flags:#x} after warm-up")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    sampler = ClockSampler(dev.index)
-    sampler.start()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    t_on = time.time()
     start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     end.record(stream)
     torch.cuda.synchronize()
+    t_off = time.time()
     if dist:
         dist.barrier()
-    sampler.stop()
     total_ms = start.elapsed_time(end)
     pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs) if wd else 0.0
@@ -410,6 +452,7 @@ def run_ours(args, rank, world, dist):
         for _ in range(3):
             bwd()
         torch.cuda.synchronize()
+        settle(bwd, args.settle_s / 3, dist, dev)
         bwd_steps = max(3, min(args.steps, args.bwd_steps))
         bev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         if dist:
@@ -443,6 +486,7 @@ def run_ours(args, rank, world, dist):
         for _ in range(3):
             chunk_call()
         torch.cuda.synchronize()
+        settle(chunk_call, args.settle_s / 3, dist, dev)
         chunk_steps = max(3, min(args.steps, args.bwd_steps))
         cev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         if dist:
@@ -466,7 +510,8 @@ def run_ours(args, rank, world, dist):
     vals = [total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms, chunk_ms]
     vals = max_over_ranks(vals, dist, dev)
     total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms, chunk_ms = vals
-    clocks = sampler.summary()
+    sampler.stop()
+    clocks = sampler.summary(t_on, t_off)
     if rank != 0:
         return None
 
@@ -484,6 +529,10 @@ def run_ours(args, rank, world, dist):
         "n_gpus": world,
         "steps": K,
         "warmup": args.warmup,
+        "settle": {"steps": settle_steps, "seconds": args.settle_s,
+                   "why": "untimed steps after the warm-up until the GPU's power state has "
+                          "settled (sw_power_cap engages within ~0.1 s of sustained load), so "
+                          "the timed region matches the sustained peak it is divided by"},
         "ms_per_step": round(total_ms / K, 4),
         "higher_is_better": True,
         "scaling": "weak",
@@ -675,6 +724,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--settle-s", type=float, default=1.5,
+                    help="untimed steps after the warm-up until this many seconds have passed "
+                         "(the power state settles; the backward and chunk legs take a third each)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--prefill", default="prefill_1p3b",
                     choices=["tiny", "prefill_1p3b", "prefill_7b_hybrid", "prefill_long_131k"])

@@ -30,6 +30,18 @@ def _worker(rank, world, port, out):
 
         if rank != 0:
             out[10 + rank] = bench.run_reference(A, rank)  # no work off rank 0
+
+        # settle: a slow rank and a fast one still run the same number of steps
+        import time
+
+        calls = [0]
+
+        def step():
+            calls[0] += 1
+            time.sleep(0.02 if rank else 0.001)
+
+        n = bench.settle(step, 0.2, tdist, "cpu", sync=lambda: None)
+        out[20 + rank] = (n, calls[0])
     finally:
         tdist.destroy_process_group()
 
@@ -42,6 +54,8 @@ def test_timings_reduce_to_the_max_over_two_gloo_ranks():
         want = [2.0, 10.0, 3.5, 7.0]
         assert out[0] == want and out[1] == want
         assert out[11] is None
+        (n0, c0), (n1, c1) = out[20], out[21]
+        assert n0 == n1 == c0 == c1 and n0 >= 4
 
 
 def test_single_process_is_identity():
@@ -49,3 +63,21 @@ def test_single_process_is_identity():
     import bench
 
     assert bench.max_over_ranks([1.0, 2.0], None, "cpu") == [1.0, 2.0]
+
+
+def test_clock_summary_keeps_only_the_timed_window():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)
+    cs.ok, cs.max_mhz = True, 1965
+    # (time, MHz, reasons, util): cold before the region, power-capped inside it
+    cs.samples = [(0.0, 1965, 0x0, 90), (0.5, 1965, 0x0, 90), (1.0, 1800, 0x4, 99),
+                  (1.1, 1790, 0x4, 99), (1.2, 1810, 0x4, 99), (2.0, 1965, 0x1, 0)]
+    s = cs.summary(0.95, 1.25)
+    assert s["sm_mhz"] == 1800 and s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
+    # a region between two samples reports the nearest ones
+    s = cs.summary(0.6, 0.7)
+    assert s["samples"] == 2 and s["sm_mhz"] in (1965, 1882.5)
+    # no window: every sample that is not idle
+    assert cs.summary()["samples"] == 5
