@@ -25,7 +25,11 @@
 //                        list them): S^T = K Q^T and dP^T = V dO^T into TMEM,
 //                        P^T and dS^T (bf16) written back over them, then
 //                        dV += P^T dO and dK += dS^T Q with the A operands
-//                        read from TMEM.
+//                        read from TMEM. 128-key blocks.
+//   s2_bwd_dkv_persistent_kernel
+//                        the same per key tile for 64-key blocks (two blocks
+//                        per tile), persistent over tiles like the dQ kernel,
+//                        with K and V in TMEM.
 // dQ and dK/dV are computed by separate kernels (S and dP are recomputed by
 // both) so that no accumulator is shared between CTAs: no atomics, and the
 // results are deterministic.
@@ -38,8 +42,9 @@
 // tile row = one TMEM lane, warps 4..7 on the first half of the columns and
 // warps 8..11 on the second (two warps per SM sub-partition hide the
 // exponential and TMEM latencies; a single warpgroup was measured to leave
-// the tensor core idle most of the time). In the dK/dV kernel warp 1 issues
-// S^T and dP^T and one thread of warp 3 issues dV and dK.
+// the tensor core idle most of the time). In the persistent dK/dV kernel warp 2
+// also loads each tile's K and V, warp 1 copies them into TMEM and issues S^T
+// and dP^T, and one thread of warp 3 issues dV and dK.
 // With B = 64 a 128-row tile holds two blocks and every row masks by its own
 // block's tag. Every wait is bounded; on a timeout the CTA drains its own
 // copies and MMAs, frees TMEM and exits with the device timeout flag set.
@@ -74,7 +79,8 @@ struct BackwardParams {
     float scale_log2;  // scale * log2 e
     uint64_t timeout_ns;
     uint32_t* gflags;
-    int* sched;  // dQ kernel work counter {next item, CTAs done}, zero at launch
+    int* sched;     // dQ kernel work counter {next item, CTAs done}, zero at launch
+    int* sched_kv;  // the same for the persistent dK/dV kernel (64-key blocks)
 };
 
 // Descriptor offset (16-byte units) of k-step kk (16 elements) of a K-major
@@ -721,9 +727,8 @@ struct BwdKVCfg {
     static constexpr uint32_t OFF_LIST = OFF_STAT + ST * STATBYTES;
     static constexpr uint32_t OFF_SCR = OFF_LIST + LIST_CAP * 4;  // list-merge scratch (ROWS > 1)
     static constexpr uint32_t OFF_BAR = OFF_SCR + (ROWS > 1 ? ROWS * LIST_CAP * 4 : 0);
-    // barriers: kv_full, q_full[ST], q_empty[ST], s_full, p_full, acc_done, drain, dp_full, ds_full,
-    // dv_done, dk_done, drain of the dV/dK issuer
-    static constexpr int NBAR = 1 + 2 * ST + 6 + 3;
+    // barriers: kv_full, q_full[ST], q_empty[ST], s_full, p_full, acc_done, drain, dp_full, ds_full
+    static constexpr int NBAR = 1 + 2 * ST + 6;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
@@ -732,16 +737,13 @@ struct BwdKVCfg {
     // every S^T and dP^T MMA of the CTA, sit in TMEM (HD/2 columns each).
     static constexpr bool A_IN_TMEM = 2 * BK + 3 * HD <= 512;
     static constexpr uint32_t COL_KA = 2 * BK + 2 * HD, COL_VA = 2 * BK + 2 * HD + HD / 2;
-    // 64-key blocks: one thread issues S^T and dP^T, another dV and dK (one
-    // thread issuing all 24 MMAs of an element, with their waits and commits,
-    // was the limit; with 128-key blocks one thread keeps up with the tensor
-    // core, and splitting only added completion waits: measured 3 % slower).
-    static constexpr bool SPLIT = BK == 64;
     static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD + (A_IN_TMEM ? HD : 0)) <= 256 ? 256 : 512;
     static_assert(2 * BK + 2 * HD <= 512, "TMEM budget");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
+// One key tile per CTA; launched for 128-key blocks (64-key blocks use the
+// persistent kernel below).
 template <int HD, int BK>
 __global__ void __launch_bounds__(384, 1)
 s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
@@ -784,9 +786,6 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const uint32_t bar_dr = bar_s + 24u;
     const uint32_t bar_dp = bar_s + 32u;
     const uint32_t bar_ds = bar_s + 40u;
-    const uint32_t bar_dvd = bar_s + 48u;  // dV(n) done: S^T's columns (its P^T) are free
-    const uint32_t bar_dkd = bar_s + 56u;  // dK(n) done: dP^T's columns (its dS^T) are free
-    const uint32_t bar_dr2 = bar_s + 64u;
     uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] tmem, [1] abort, [2] list length
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
@@ -804,9 +803,6 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         mbar_init(bar_p, 256);
         mbar_init(bar_acc, 1);
         mbar_init(bar_dr, 1);
-        mbar_init(bar_dvd, 1);
-        mbar_init(bar_dkd, 1);
-        mbar_init(bar_dr2, 1);
         *abort_cta = 0;
         fence_mbar_init();
     }
@@ -883,194 +879,92 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             }
         }
         __syncwarp();
-    } else if (warp == 1 || (C::SPLIT && warp == 3)) {
-        if constexpr (C::SPLIT) {
-            if (warp == 1) {
-                // ------------------------------------------------------------ S^T and dP^T issuer
-                // S^T(n) and dP^T(n) are committed separately so that the element-wise
-                // warps compute P^T while dP^T is still running. S^T(n) overwrites
-                // P^T(n-1) and so waits for dV(n-1)'s commit; dP^T(n) overwrites
-                // dS^T(n-1) and waits for dK(n-1)'s (both issued by the other thread;
-                // the warps keep P in registers for the dS pass).
-                if (lane == 0 && len > 0) {
-                    constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
-                    const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
-                    const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
-                    bool issued = false;
-                    const bool kv_ok = mbar_wait(bar_kv, 0, ctl);
-                    if (kv_ok && C::A_IN_TMEM) {  // K and V into TMEM, before every MMA that reads them
-                        tc_fence_after();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && len > 0) {
+            constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
+            constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);   // dV += P^T dO, dK += dS^T Q
+            const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
+            const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
+            bool issued = false;
+            // S^T(n) and dP^T(n) are committed separately so that the element-wise
+            // warps compute P^T while dP^T is still running. Order per element n:
+            // [P^T(n) ready] dV(n), S^T(n+1); [dS^T(n) ready] dK(n), dP^T(n+1).
+            // S^T(n+1) overwrites P^T(n) after dV(n) has read it (MMAs of one
+            // thread run in issue order; the warps keep P in registers for the
+            // dS pass); dP^T(n+1) overwrites dS^T(n) after dK(n).
+            auto issue_st = [&](int n) {
+                const int st = n % C::ST;
+                if (!mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
 #pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk) {
-                            tmem_cp_128x256b(tmem + C::COL_KA + kk * 8, dk_desc + kstep(kk, C::M));
-                            tmem_cp_128x256b(tmem + C::COL_VA + kk * 8, dv_desc + kstep(kk, C::M));
-                        }
-                        issued = true;
-                    }
-                    for (int n = 0; kv_ok && n < len; ++n) {
-                        const int st = n % C::ST;
-                        if ((n > 0 && !mbar_wait(bar_dvd, (n - 1) & 1, ctl)) ||
-                            !mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl))
-                            break;
-                        tc_fence_after();
-                        const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk) {
-                            if constexpr (C::A_IN_TMEM)
-                                umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_KA + kk * 8, dq_desc + kstep(kk, BK), idesc_s,
-                                             kk > 0 ? 1u : 0u);
-                            else
-                                umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK), idesc_s,
-                                             kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(bar_s);
-                        issued = true;
-                        if (n > 0 && !mbar_wait(bar_dkd, (n - 1) & 1, ctl)) break;
-                        tc_fence_after();
-                        const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk) {
-                            if constexpr (C::A_IN_TMEM)
-                                umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_VA + kk * 8, ddo_desc + kstep(kk, BK),
-                                             idesc_s, kk > 0 ? 1u : 0u);
-                            else
-                                umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
-                                             idesc_s, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(bar_dp);
-                    }
-                    if (*abort_cta && issued) {
-                        umma_commit(bar_dr);
-                        mbar_drain(bar_dr, 0, kDrainNs);
-                    }
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    if constexpr (C::A_IN_TMEM)
+                        umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_KA + kk * 8, dq_desc + kstep(kk, BK), idesc_s,
+                                     kk > 0 ? 1u : 0u);
+                    else
+                        umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK), idesc_s,
+                                     kk > 0 ? 1u : 0u);
                 }
-            } else {
-                // ------------------------------------------------------------ dV and dK issuer
-                // dV(n) += P^T(n) dO once P^T(n) is written; dK(n) += dS^T(n) Q once
-                // dS^T(n) is. The commit after dK(n) releases the Q/dO stage (dS^T(n)
-                // needed S^T(n) and dP^T(n) complete, so every read of it is done);
-                // the other thread waits for every stage's loads in order, so a stage
-                // cannot be refilled before it has passed the stage.
-                if (lane == 0 && len > 0) {
-                    constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);   // dV += P^T dO, dK += dS^T Q
-                    bool issued = false;
-                    for (int n = 0; n < len; ++n) {
-                        const int st = n % C::ST;
-                        if (!mbar_wait(bar_p, n & 1, ctl)) break;
-                        tc_fence_after();
+                umma_commit(bar_s);
+                issued = true;
+                return true;
+            };
+            auto issue_dpt = [&](int n) {  // stage already waited for by issue_st(n)
+                const int st = n % C::ST;
+                const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                            umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
-                                         (n > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(bar_dvd);
-                        issued = true;
-                        if (!mbar_wait(bar_ds, n & 1, ctl)) break;
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                            umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + packed_col<BK>(kk), bq, idesc_a,
-                                         (n > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(bar_dkd);
-                        umma_commit(bar_qe(st));
-                        if (n + 1 == len && !*abort_cta) umma_commit(bar_acc);
-                    }
-                    if (*abort_cta && issued) {
-                        umma_commit(bar_dr2);
-                        mbar_drain(bar_dr2, 0, kDrainNs);
-                    }
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    if constexpr (C::A_IN_TMEM)
+                        umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_VA + kk * 8, ddo_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+                    else
+                        umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
+                                     idesc_s, kk > 0 ? 1u : 0u);
                 }
+                umma_commit(bar_dp);
+            };
+            const bool kv_ok = mbar_wait(bar_kv, 0, ctl);
+            if (kv_ok && C::A_IN_TMEM) {  // K and V into TMEM, before every MMA that reads them
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    tmem_cp_128x256b(tmem + C::COL_KA + kk * 8, dk_desc + kstep(kk, C::M));
+                    tmem_cp_128x256b(tmem + C::COL_VA + kk * 8, dv_desc + kstep(kk, C::M));
+                }
+                issued = true;
             }
-        } else {
-            // ------------------------------------------------------------ MMA issuer
-            if (lane == 0 && len > 0) {
-                constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
-                constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);   // dV += P^T dO, dK += dS^T Q
-                const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
-                const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
-                bool issued = false;
-                // S^T(n) and dP^T(n) are committed separately so that the element-wise
-                // warps compute P^T while dP^T is still running. Order per element n:
-                // [P^T(n) ready] dV(n), S^T(n+1); [dS^T(n) ready] dK(n), dP^T(n+1).
-                // S^T(n+1) overwrites P^T(n) after dV(n) has read it (MMAs of one
-                // thread run in issue order; the warps keep P in registers for the
-                // dS pass); dP^T(n+1) overwrites dS^T(n) after dK(n).
-                auto issue_st = [&](int n) {
+            if (kv_ok && issue_st(0)) {
+                issue_dpt(0);
+                for (int n = 0; n < len; ++n) {
                     const int st = n % C::ST;
-                    if (!mbar_wait(bar_qf(st), (n / C::ST) & 1, ctl)) return false;
-                    tc_fence_after();
-                    const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
-                        if constexpr (C::A_IN_TMEM)
-                            umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_KA + kk * 8, dq_desc + kstep(kk, BK), idesc_s,
-                                         kk > 0 ? 1u : 0u);
-                        else
-                            umma_bf16_ss(tmem + C::COL_S, dk_desc + kstep(kk, C::M), dq_desc + kstep(kk, BK), idesc_s,
-                                         kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(bar_s);
-                    issued = true;
-                    return true;
-                };
-                auto issue_dpt = [&](int n) {  // stage already waited for by issue_st(n)
-                    const int st = n % C::ST;
-                    const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
-                        if constexpr (C::A_IN_TMEM)
-                            umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_VA + kk * 8, ddo_desc + kstep(kk, BK),
-                                         idesc_s, kk > 0 ? 1u : 0u);
-                        else
-                            umma_bf16_ss(tmem + C::COL_DP, dv_desc + kstep(kk, C::M), ddo_desc + kstep(kk, BK),
-                                         idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(bar_dp);
-                };
-                const bool kv_ok = mbar_wait(bar_kv, 0, ctl);
-                if (kv_ok && C::A_IN_TMEM) {  // K and V into TMEM, before every MMA that reads them
+                    const bool more = n + 1 < len;
+                    if (!mbar_wait(bar_p, n & 1, ctl)) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
-                        tmem_cp_128x256b(tmem + C::COL_KA + kk * 8, dk_desc + kstep(kk, C::M));
-                        tmem_cp_128x256b(tmem + C::COL_VA + kk * 8, dv_desc + kstep(kk, C::M));
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
+                                     (n > 0 || kk > 0) ? 1u : 0u);
                     }
-                    issued = true;
-                }
-                if (kv_ok && issue_st(0)) {
-                    issue_dpt(0);
-                    for (int n = 0; n < len; ++n) {
-                        const int st = n % C::ST;
-                        const bool more = n + 1 < len;
-                        if (!mbar_wait(bar_p, n & 1, ctl)) break;
-                        tc_fence_after();
+                    if (more && !issue_st(n + 1)) break;
+                    if (!mbar_wait(bar_ds, n & 1, ctl)) break;
+                    tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                            umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
-                                         (n > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        if (more && !issue_st(n + 1)) break;
-                        if (!mbar_wait(bar_ds, n & 1, ctl)) break;
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                            umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + packed_col<BK>(kk), bq, idesc_a,
-                                         (n > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(bar_qe(st));
-                        if (more) issue_dpt(n + 1);
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + packed_col<BK>(kk), bq, idesc_a,
+                                     (n > 0 || kk > 0) ? 1u : 0u);
                     }
-                    if (!*abort_cta) umma_commit(bar_acc);
+                    umma_commit(bar_qe(st));
+                    if (more) issue_dpt(n + 1);
                 }
-                if (*abort_cta && issued) {
-                    umma_commit(bar_dr);
-                    mbar_drain(bar_dr, 0, kDrainNs);
-                }
+                if (!*abort_cta) umma_commit(bar_acc);
+            }
+            if (*abort_cta && issued) {
+                umma_commit(bar_dr);
+                mbar_drain(bar_dr, 0, kDrainNs);
             }
         }
         __syncwarp();
@@ -1179,6 +1073,506 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ dK, dV (persistent, B = 64)
+
+// 64-key blocks: each CTA takes work items (one 128-row key tile = two 64-key
+// blocks of one K/V plane, in the order above: key tiles outermost, so the
+// tiles seen by the most query blocks come first) from a device counter.
+// K and V are only the A operands of S^T and dP^T, and sit in TMEM, so their
+// shared-memory copy is needed only for the tcgen05.cp at the start of an
+// item: one buffer suffices, and the next tile's K and V (and its union list,
+// double-buffered) load while the current tile runs. Element counters run over
+// all items of the CTA, so stages, barrier phases and the S^T/dP^T ->
+// dV/dK hand-offs carry across item boundaries unchanged.
+template <int HD>
+struct BwdKVPCfg {
+    static constexpr int BK = 64;
+    static constexpr int M = 128;
+    static constexpr int ROWS = 2;                     // key blocks per tile
+    static constexpr uint32_t TBYTES = M * HD * 2;     // K or V tile
+    static constexpr uint32_t QBYTES = BK * HD * 2;    // one query block of Q or dO
+    static constexpr uint32_t STATBYTES = BK * 8;      // L2 of the BK queries, then their D
+    static constexpr int ST = 2;
+    static constexpr int LIST_CAP = 4096;  // grouped heads: the lists of every query head of the group
+    static constexpr uint32_t OFF_K = 0;
+    static constexpr uint32_t OFF_V = TBYTES;
+    static constexpr uint32_t OFF_Q = 2 * TBYTES;              // [stage][panel][BK rows x 128 B]
+    static constexpr uint32_t OFF_DO = OFF_Q + ST * QBYTES;
+    static constexpr uint32_t OFF_STAT = OFF_DO + ST * QBYTES;
+    static constexpr uint32_t OFF_LIST = OFF_STAT + ST * STATBYTES;  // two list buffers
+    static constexpr uint32_t OFF_SCR = OFF_LIST + 2 * LIST_CAP * 4;  // list-merge scratch
+    static constexpr uint32_t OFF_BAR = OFF_SCR + ROWS * LIST_CAP * 4;
+    // barriers: kv_full, kv_empty, q_full[ST], q_empty[ST], s_full, p_full, acc_done, dp_full,
+    // ds_full, dv_done, dk_done, drain x 2, list_full[2], list_empty[2]
+    static constexpr int NBAR = 2 + 2 * ST + 9 + 4;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
+    static constexpr uint32_t SMEM = OFF_MISC + 32;
+    static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
+    // Q/dO producer, the two MMA threads, 8 element-wise warps
+    static constexpr uint32_t LIST_CONSUMERS = 11;
+    static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_DV = 2 * BK, COL_DK = 2 * BK + HD;
+    static constexpr uint32_t COL_KA = 2 * BK + 2 * HD, COL_VA = 2 * BK + 2 * HD + HD / 2;
+    static constexpr uint32_t TMEM_COLS = (2 * BK + 3 * HD) <= 256 ? 256 : 512;
+    static_assert(2 * BK + 3 * HD <= 512, "TMEM budget");
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
+
+// Work item w of the dK/dV kernels: key tile kt of K/V plane bkv, the first
+// query head h of its group and that head's (batch, head) plane.
+struct KvItem {
+    int kt, bkv, h, bq0;
+};
+
+__device__ __forceinline__ KvItem kv_item(const BackwardParams& p, int w)
+{
+    const int BHk = p.batch * p.heads_kv, grp = p.heads / p.heads_kv;
+    KvItem it;
+    it.kt = w / BHk;
+    it.bkv = w % BHk;
+    it.h = (it.bkv % p.heads_kv) * grp;
+    it.bq0 = (it.bkv / p.heads_kv) * p.heads + it.h;
+    return it;
+}
+
+// Key block r (0 or 1) of a 64-key tile, -1 if none.
+__device__ __forceinline__ int kv_item_block(const BackwardParams& p, const KvItem& it, int r)
+{
+    const int j = __ldg(p.key_tiles + ((int64_t)it.h * p.ntiles + it.kt) * 2 + r);
+    return j < p.nb ? j : -1;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(384, 1)
+s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                             const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                             const BackwardParams p)
+{
+    using C = BwdKVPCfg<HD>;
+    constexpr int BK = C::BK;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_items = p.ntiles * p.batch * p.heads_kv;
+    const int grp = p.heads / p.heads_kv;
+
+    const uint32_t bar_kv = sb + C::OFF_BAR;
+    const uint32_t bar_kve = bar_kv + 8u;  // K, V copied into TMEM: the buffer may be refilled
+    auto bar_qf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + s); };
+    auto bar_qe = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + C::ST + s); };
+    const uint32_t bar_s = sb + C::OFF_BAR + 8u * (2 + 2 * C::ST);
+    const uint32_t bar_p = bar_s + 8u;
+    const uint32_t bar_acc = bar_s + 16u;
+    const uint32_t bar_dp = bar_s + 24u;
+    const uint32_t bar_ds = bar_s + 32u;
+    const uint32_t bar_dvd = bar_s + 40u;  // dV(G) done: S^T's columns (its P^T) are free
+    const uint32_t bar_dkd = bar_s + 48u;  // dK(G) done: dP^T's columns (its dS^T) are free
+    const uint32_t bar_dr = bar_s + 56u;
+    const uint32_t bar_dr2 = bar_s + 64u;
+    auto bar_lf = [&](int b) { return bar_s + 72u + 8u * b; };
+    auto bar_le = [&](int b) { return bar_s + 88u + 8u * b; };
+    const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
+    // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
+    int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
+    volatile int* abort_cta = misc + 1;
+    volatile int* list_len = misc + 2;
+    volatile int* list_item = misc + 4;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_kv, 1);
+        mbar_init(bar_kve, 1);
+        for (int s = 0; s < C::ST; ++s) {
+            mbar_init(bar_qf(s), 1);
+            mbar_init(bar_qe(s), 1);
+        }
+        mbar_init(bar_s, 1);
+        mbar_init(bar_p, 256);
+        mbar_init(bar_acc, 1);
+        mbar_init(bar_dp, 1);
+        mbar_init(bar_ds, 256);
+        mbar_init(bar_dvd, 1);
+        mbar_init(bar_dkd, 1);
+        mbar_init(bar_dr, 1);
+        mbar_init(bar_dr2, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_lf(b), 1);
+            mbar_init(bar_le(b), C::LIST_CONSUMERS);
+        }
+        *abort_cta = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtl ctl{p.timeout_ns, p.gflags, abort_cta};
+    constexpr uint64_t kDrainNs = 200000000ull;
+
+    if (warp == 2) {
+        // ------------------------------------------------------------ items, union lists, K and V
+        uint32_t* wlist = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
+        int32_t* scratch = reinterpret_cast<int32_t*>(smem + C::OFF_SCR);
+        int w = blockIdx.x;  // first item static, the rest from the work counter
+        int m = 0;           // K/V loads issued (items with a non-empty list)
+        for (int k = 0;; ++k) {
+            const int b = k & 1;
+            // list buffer b is free once item k-2 is consumed
+            if (!warp_wait(bar_le(b), ((k >> 1) & 1) ^ 1, ctl)) break;
+            if (w >= num_items) {  // tell every role there is no more work
+                if (lane == 0) {
+                    list_item[b] = -1;
+                    list_len[b] = 0;
+                    mbar_arrive(bar_lf(b));
+                }
+                break;
+            }
+            int w_next = 0;
+            if (lane == 0) w_next = (int)gridDim.x + atomicAdd(p.sched_kv, 1);
+            w_next = __shfl_sync(0xffffffffu, w_next, 0);
+            const KvItem it = kv_item(p, w);
+            int kb[C::ROWS];
+            int lo = INT_MAX;
+#pragma unroll
+            for (int r = 0; r < C::ROWS; ++r) {
+                kb[r] = kv_item_block(p, it, r);
+                if (kb[r] >= 0 && kb[r] < lo) lo = kb[r];
+            }
+            uint32_t* L = wlist + b * C::LIST_CAP;
+            int total = 0;
+            for (int hh = 0; hh < grp; ++hh) {  // the group's query heads, one list after another
+                const int n = warp_union_list<C::ROWS>(p.col_ptr, p.row_idx, (it.h + hh) * (p.nb + 1), kb, p.nb,
+                                                       p.nnz, lo, p.nb - 1, L + total, C::LIST_CAP - total,
+                                                       scratch, p.gflags);
+                for (int t = lane; t < n; t += 32) L[total + t] |= (uint32_t)hh << 28;
+                __syncwarp();
+                total += n;
+            }
+            if (lane == 0) {
+                list_len[b] = total;
+                list_item[b] = w;
+                mbar_arrive(bar_lf(b));
+            }
+            if (total > 0) {
+                // K and V of the tile, once the previous tile's copies into TMEM are done
+                if (!warp_wait(bar_kve, (m & 1) ^ 1, ctl)) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar_kv, 2 * C::TBYTES);
+                    const int kany = kb[0] >= 0 ? kb[0] : kb[1];  // a missing block loads the other's rows
+#pragma unroll
+                    for (int r = 0; r < C::ROWS; ++r) {
+                        const int32_t krow = (kb[r] >= 0 ? kb[r] : kany) * BK;
+#pragma unroll
+                        for (int pn = 0; pn < HD / 64; ++pn) {
+                            tma_load_3d(sb + C::OFF_K + pn * (C::M * 128) + r * (BK * 128), &tmK, pn * 64, krow,
+                                        it.bkv, bar_kv);
+                            tma_load_3d(sb + C::OFF_V + pn * (C::M * 128) + r * (BK * 128), &tmV, pn * 64, krow,
+                                        it.bkv, bar_kv);
+                        }
+                    }
+                }
+                ++m;
+            }
+            w = w_next;
+        }
+        if (lane == 0 && *abort_cta && m > 0) mbar_drain(bar_kv, (m - 1) & 1, kDrainNs);
+        __syncwarp();
+    } else if (warp == 0) {
+        // ------------------------------------------------------------ Q, dO and statistics producer
+        if (lane == 0) {
+            int n = 0;  // elements over all items; element n uses stage n % ST
+            bool stop = false;
+            for (int k = 0; !stop; ++k) {
+                const int b = k & 1;
+                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                const int w = list_item[b];
+                if (w < 0) break;
+                const int bq0 = kv_item(p, w).bq0;
+                const uint32_t* L = list + b * C::LIST_CAP;
+                const int len = list_len[b];
+                for (int e = 0; e < len; ++e, ++n) {
+                    const int st = n % C::ST;
+                    if (!mbar_wait(bar_qe(st), ((n / C::ST) & 1) ^ 1, ctl)) {
+                        stop = true;
+                        break;
+                    }
+                    const int i = list_j(L[e]);
+                    const int bq = bq0 + (int)(L[e] >> 28);  // query plane of this entry
+                    mbar_arrive_expect_tx(bar_qf(st), 2 * C::QBYTES + C::STATBYTES);
+#pragma unroll
+                    for (int pn = 0; pn < HD / 64; ++pn) {
+                        tma_load_3d(sb + C::OFF_Q + st * C::QBYTES + pn * (BK * 128), &tmQ, pn * 64, i * BK, bq,
+                                    bar_qf(st));
+                        tma_load_3d(sb + C::OFF_DO + st * C::QBYTES + pn * (BK * 128), &tmDO, pn * 64, i * BK, bq,
+                                    bar_qf(st));
+                    }
+                    const float* sx = p.stats + ((int64_t)bq * p.ntiles + (i * BK) / 128) * 256 + (i * BK) % 128;
+                    bulk_load(sb + C::OFF_STAT + st * C::STATBYTES, sx, BK * 4, bar_qf(st));
+                    bulk_load(sb + C::OFF_STAT + st * C::STATBYTES + BK * 4, sx + 128, BK * 4, bar_qf(st));
+                }
+                if (!stop) mbar_arrive(bar_le(b));
+            }
+            if (*abort_cta)  // let this CTA's own loads land before exit
+                for (int m = (n > C::ST ? n - C::ST : 0); m < n; ++m)
+                    mbar_drain(bar_qf(m % C::ST), (m / C::ST) & 1, kDrainNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ K, V into TMEM; S^T and dP^T issuer
+        // S^T(G) overwrites P^T(G-1) and so waits for dV(G-1)'s commit; dP^T(G)
+        // overwrites dS^T(G-1) and waits for dK(G-1)'s (both issued by the other
+        // thread; the element-wise warps keep P in registers for the dS pass).
+        // A tile's K and V are copied into TMEM after the previous tile's MMAs
+        // that read them (one thread: issue order).
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
+            const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
+            const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
+            bool issued = false, fail = false;
+            int G = 0, m = 0;
+            for (int k = 0; !fail; ++k) {
+                const int b = k & 1;
+                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                if (list_item[b] < 0) break;
+                const int len = list_len[b];
+                if (len > 0) {
+                    if (!mbar_wait(bar_kv, m & 1, ctl)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        tmem_cp_128x256b(tmem + C::COL_KA + kk * 8, dk_desc + kstep(kk, C::M));
+                        tmem_cp_128x256b(tmem + C::COL_VA + kk * 8, dv_desc + kstep(kk, C::M));
+                    }
+                    umma_commit(bar_kve);
+                    issued = true;
+                    ++m;
+                }
+                for (int n = 0; n < len; ++n, ++G) {
+                    const int st = G % C::ST;
+                    if ((G > 0 && !mbar_wait(bar_dvd, (G - 1) & 1, ctl)) ||
+                        !mbar_wait(bar_qf(st), (G / C::ST) & 1, ctl)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_KA + kk * 8, dq_desc + kstep(kk, BK), idesc_s,
+                                     kk > 0 ? 1u : 0u);
+                    umma_commit(bar_s);
+                    if (G > 0 && !mbar_wait(bar_dkd, (G - 1) & 1, ctl)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_VA + kk * 8, ddo_desc + kstep(kk, BK), idesc_s,
+                                     kk > 0 ? 1u : 0u);
+                    umma_commit(bar_dp);
+                }
+                if (fail) break;
+                mbar_arrive(bar_le(b));
+            }
+            if (*abort_cta && issued) {
+                umma_commit(bar_dr);
+                mbar_drain(bar_dr, 0, kDrainNs);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ dV and dK issuer
+        // dV(G) += P^T(G) dO once P^T(G) is written; dK(G) += dS^T(G) Q once
+        // dS^T(G) is. The commit after dK(G) releases the Q/dO stage (dS^T(G)
+        // needed S^T(G) and dP^T(G) complete, so every read of it is done). A
+        // tile's first dV and dK overwrite the accumulators: their P^T and dS^T
+        // come from element-wise threads that have already read the previous
+        // tile's accumulators out.
+        if (lane == 0) {
+            constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);  // dV += P^T dO, dK += dS^T Q
+            bool issued = false, fail = false;
+            int G = 0;
+            for (int k = 0; !fail; ++k) {
+                const int b = k & 1;
+                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                if (list_item[b] < 0) break;
+                const int len = list_len[b];
+                for (int n = 0; n < len; ++n, ++G) {
+                    const int st = G % C::ST;
+                    if (!mbar_wait(bar_p, G & 1, ctl)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
+                                     (n > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_dvd);
+                    issued = true;
+                    if (!mbar_wait(bar_ds, G & 1, ctl)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                        umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + packed_col<BK>(kk), bq, idesc_a,
+                                     (n > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_dkd);
+                    umma_commit(bar_qe(st));
+                    if (n + 1 == len) umma_commit(bar_acc);  // the tile's dK, dV are complete with it
+                }
+                if (fail) break;
+                mbar_arrive(bar_le(b));
+            }
+            if (*abort_cta && issued) {
+                umma_commit(bar_dr2);
+                mbar_drain(bar_dr2, 0, kDrainNs);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ element-wise passes + epilogue
+        constexpr int HALF = BK / 2;  // query columns per warpgroup
+        const int quad = warp & 3, g = (warp - 4) >> 2;
+        const int r = quad * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const int kbit = r >> 6;  // key block of this row within the tile
+        const float sc = p.scale_log2;
+        bool fail = false;
+        int G = 0, n_acc = 0;  // elements, and tiles with an accumulation, so far
+        for (int k = 0; !fail; ++k) {
+            const int b = k & 1;
+            if (!warp_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+            const int w = list_item[b];
+            if (w < 0) break;
+            const KvItem it = kv_item(p, w);
+            const int kbr = kv_item_block(p, it, kbit);
+            const int kpos = kbr * BK + (r % BK);
+            const bool row_valid = kbr >= 0 && kpos < p.seq;
+            const uint32_t* L = list + b * C::LIST_CAP;
+            const int len = list_len[b];
+            for (int n = 0; n < len; ++n, ++G) {
+                const int st = G % C::ST;
+                const uint32_t ent = L[n];
+                // the stage's query statistics came by bulk copy: observe its barrier
+                // too (already complete: the MMAs of this element waited for it)
+                if (!warp_wait(bar_qf(st), (G / C::ST) & 1, ctl) || !warp_wait(bar_s, G & 1, ctl)) {
+                    fail = true;
+                    break;
+                }
+                tc_fence_after();
+                const float* sx = reinterpret_cast<const float*>(smem + C::OFF_STAT + st * C::STATBYTES) + g * HALF;
+                const float* sy = sx + BK;
+                const bool vis = row_valid && ((list_bits(ent) >> kbit) & 1);
+                const int lim = kpos - list_j(ent) * BK - g * HALF;  // column c of this half visible iff c >= lim
+                // P pass (needs S^T only): P^T as bf16 pairs, kept in registers too
+                uint32_t sr[HALF], pk[HALF / 2];
+                tmem_ld_cols<HALF>(tl + C::COL_S + g * HALF, sr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < HALF; c += 4) {
+                    const float4 x = *reinterpret_cast<const float4*>(sx + c);
+                    const float p0 = (vis && c >= lim) ? ex2(fmaf(__uint_as_float(sr[c]), sc, -x.x)) : 0.f;
+                    const float p1 = (vis && c + 1 >= lim) ? ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -x.y)) : 0.f;
+                    const float p2 = (vis && c + 2 >= lim) ? ex2(fmaf(__uint_as_float(sr[c + 2]), sc, -x.z)) : 0.f;
+                    const float p3 = (vis && c + 3 >= lim) ? ex2(fmaf(__uint_as_float(sr[c + 3]), sc, -x.w)) : 0.f;
+                    pk[c / 2] = pack_bf16x2(p0, p1);
+                    pk[c / 2 + 1] = pack_bf16x2(p2, p3);
+                }
+                tmem_st_cols<HALF / 2>(tl + C::COL_S + g * HALF, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_p);
+                if (!warp_wait(bar_dp, G & 1, ctl)) {
+                    fail = true;
+                    break;
+                }
+                tc_fence_after();
+                // dS pass: dS^T = P^T (dP^T - D)
+                tmem_ld_cols<HALF>(tl + C::COL_DP + g * HALF, sr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < HALF; c += 4) {
+                    const float4 y = *reinterpret_cast<const float4*>(sy + c);
+                    const float d0 = bf16lo(pk[c / 2]) * (__uint_as_float(sr[c]) - y.x);
+                    const float d1 = bf16hi(pk[c / 2]) * (__uint_as_float(sr[c + 1]) - y.y);
+                    const float d2 = bf16lo(pk[c / 2 + 1]) * (__uint_as_float(sr[c + 2]) - y.z);
+                    const float d3 = bf16hi(pk[c / 2 + 1]) * (__uint_as_float(sr[c + 3]) - y.w);
+                    pk[c / 2] = pack_bf16x2(d0, d1);
+                    pk[c / 2 + 1] = pack_bf16x2(d2, d3);
+                }
+                tmem_st_cols<HALF / 2>(tl + C::COL_DP + g * HALF, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_ds);
+            }
+            if (fail) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_le(b));
+            // warpgroup 0 stores dV, warpgroup 1 stores dK (times the scale); the
+            // next tile's first dV/dK MMA waits for this thread's next P^T/dS^T,
+            // so it follows these loads
+            const int64_t row = (int64_t)it.bkv * p.seq + kpos;
+            uint16_t* grow = (g == 0 ? p.dv : p.dk) + row * HD;
+            if (len > 0) {
+                if (!warp_wait(bar_acc, (n_acc++) & 1, ctl)) break;
+                tc_fence_after();
+                const float f = g == 0 ? 1.0f : p.scale;
+                const uint32_t col = g == 0 ? C::COL_DV : C::COL_DK;
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tl + col + 32 * c, o);
+                    tmem_wait_ld();
+                    if (row_valid) {
+#pragma unroll
+                        for (int e2 = 0; e2 < 32; e2 += 8) {
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * f, __uint_as_float(o[e2 + 1]) * f);
+                            v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * f, __uint_as_float(o[e2 + 3]) * f);
+                            v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * f, __uint_as_float(o[e2 + 5]) * f);
+                            v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * f, __uint_as_float(o[e2 + 7]) * f);
+                            *reinterpret_cast<uint4*>(grow + 32 * c + e2) = v;
+                        }
+                    }
+                }
+            } else if (row_valid) {  // no query block lists this tile's key blocks
+                for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(grow + d) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    if (threadIdx.x == 0) {
+        // The last CTA to finish resets the counter for the next launch on this slot
+        // (every CTA has stopped taking items by now).
+        __threadfence();
+        if (atomicAdd(p.sched_kv + 1, 1) == (int)gridDim.x - 1) {
+            atomicExch(p.sched_kv, 0);
+            atomicExch(p.sched_kv + 1, 0);
+            __threadfence();
+        }
     }
 }
 

@@ -156,14 +156,16 @@ int launch_prefill(const void* q, const void* k, const void* v, s2::PrefillParam
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
-// Backward: row statistics, then the dQ kernel and the dK/dV kernel (one CTA
-// per 128-row tile each; neither writes what the other reads).
+// Backward: row statistics, then the dQ kernel and the dK/dV kernel (neither
+// writes what the other reads). The dQ kernel is persistent; so is the dK/dV
+// kernel for 64-key blocks (one CTA per 128-row key tile for 128-key blocks).
 template <int HD, int BK>
 int launch_backward(const void* q, const void* k, const void* v, s2::BackwardParams& bp, int dev,
                     int attr_slot, cudaStream_t stream)
 {
     using CQ = s2::BwdQCfg<HD, BK>;
     using CK = s2::BwdKVCfg<HD, BK>;
+    using CKP = s2::BwdKVPCfg<HD>;
     const uint64_t planes = (uint64_t)bp.batch * bp.heads, kvplanes = (uint64_t)bp.batch * bp.heads_kv;
     CUtensorMap q128, do128, kbk, vbk, qbk, dobk;
     if (make_map(&q128, q, planes, bp.seq, HD, 128) || make_map(&do128, bp.dout, planes, bp.seq, HD, 128) ||
@@ -171,15 +173,19 @@ int launch_backward(const void* q, const void* k, const void* v, s2::BackwardPar
         make_map(&qbk, q, planes, bp.seq, HD, BK) || make_map(&dobk, bp.dout, planes, bp.seq, HD, BK))
         return S2_ERR_CUDA;
     auto kq = s2::s2_bwd_dq_kernel<HD, BK>;
-    auto kkv = s2::s2_bwd_dkv_kernel<HD, BK>;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!g_dev[dev].backward_attr_done[attr_slot]) {
-            if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::SMEM_ALLOC) !=
-                    cudaSuccess ||
-                cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, CK::SMEM_ALLOC) !=
-                    cudaSuccess)
-                return S2_ERR_CUDA;
+            cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::SMEM_ALLOC);
+            if constexpr (BK == 64)
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(s2::s2_bwd_dkv_persistent_kernel<HD>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, CKP::SMEM_ALLOC);
+            if constexpr (BK != 64)
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(s2::s2_bwd_dkv_kernel<HD, BK>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, CK::SMEM_ALLOC);
+            if (e != cudaSuccess) return S2_ERR_CUDA;
             g_dev[dev].backward_attr_done[attr_slot] = true;
         }
     }
@@ -194,7 +200,14 @@ int launch_backward(const void* q, const void* k, const void* v, s2::BackwardPar
     const uint64_t qgrid = qitems < (uint64_t)g_dev[dev].num_sms ? qitems : (uint64_t)g_dev[dev].num_sms;
     kq<<<(unsigned)qgrid, 384, CQ::SMEM_ALLOC, stream>>>(q128, do128, kbk, vbk, bp);
     if (cudaGetLastError() != cudaSuccess) return S2_ERR_CUDA;
-    kkv<<<(unsigned)(kvplanes * bp.ntiles), 384, CK::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
+    const uint64_t kvitems = kvplanes * (uint64_t)bp.ntiles;
+    if constexpr (BK == 64) {  // persistent, at most one CTA per SM (work counter slot in bp.sched_kv)
+        const uint64_t kvgrid = kvitems < (uint64_t)g_dev[dev].num_sms ? kvitems : (uint64_t)g_dev[dev].num_sms;
+        s2::s2_bwd_dkv_persistent_kernel<HD>
+            <<<(unsigned)kvgrid, 384, CKP::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
+    } else {
+        s2::s2_bwd_dkv_kernel<HD, BK><<<(unsigned)kvitems, 384, CK::SMEM_ALLOC, stream>>>(qbk, dobk, kbk, vbk, bp);
+    }
     return cudaGetLastError() == cudaSuccess ? S2_OK : S2_ERR_CUDA;
 }
 
@@ -421,6 +434,7 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
     bp.timeout_ns = g_timeout_ns.load();
     bp.gflags = g_dev[dev].flags;
     bp.sched = g_dev[dev].sched + 2 * (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
+    bp.sched_kv = g_dev[dev].sched + 2 * (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 128 && block_size == 128) return launch_backward<128, 128>(q, k, v, bp, dev, 0, st);
     if (head_dim == 128 && block_size == 64) return launch_backward<128, 64>(q, k, v, bp, dev, 1, st);

@@ -102,10 +102,11 @@ def test_bad_context_length_is_flagged(s2gpu):
     assert torch.isfinite(out.float()).all()
 
 
-def test_backward_wait_timeout_is_reported_and_recoverable(s2gpu):
-    w = synth.PrefillWorkload("t", 1, 4, 128, 2048, 128, 1, 1, seed=31)  # dense: long lists
+@pytest.mark.parametrize("bk", [128, 64])
+def test_backward_wait_timeout_is_reported_and_recoverable(s2gpu, bk):
+    w = synth.PrefillWorkload("t", 1, 4, 128, 2048, bk, 1, 1, seed=31)  # dense: long lists
     q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
-    lay = s2gpu.build_layout(4, 128, 1, 1, 16, device="cuda")
+    lay = s2gpu.build_layout(4, bk, 1, 1, 2048 // bk, device="cuda")
     o, lse = s2gpu.prefill(q, k, v, lay, scale=w.scale, want_lse=True)
     do = torch.randn_like(q, dtype=torch.float32).to(torch.bfloat16)
     s2gpu.set_wait_timeout_ns(0)
@@ -143,10 +144,11 @@ def test_chunk_wait_timeout_is_reported_and_recoverable(s2gpu):
     parity(out.reshape(-1, 128), ref.reshape(-1, 128))
 
 
-def test_malformed_transposed_layout_is_flagged_not_faulted(s2gpu):
-    w = synth.PrefillWorkload("t", 1, 2, 128, 512, 128, 2, 1, seed=33)
+@pytest.mark.parametrize("bk", [128, 64])
+def test_malformed_transposed_layout_is_flagged_not_faulted(s2gpu, bk):
+    w = synth.PrefillWorkload("t", 1, 2, 128, 512, bk, 2, 1, seed=33)
     q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
-    lay = s2gpu.build_layout(2, 128, 2, 1, 4, device="cuda").transposed("cuda")
+    lay = s2gpu.build_layout(2, bk, 2, 1, 512 // bk, device="cuda").transposed("cuda")
     o, lse = s2gpu.prefill(q, k, v, lay, scale=w.scale, want_lse=True)
     lay.d_t_row_idx[1] = 1 << 20  # a query block far outside the layout
     s2gpu.backward(q, k, v, o, lse, torch.ones_like(q), lay, scale=w.scale)
