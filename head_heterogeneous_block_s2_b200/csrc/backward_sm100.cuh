@@ -1106,8 +1106,8 @@ struct BwdKVPCfg {
     static constexpr uint32_t OFF_SCR = OFF_LIST + 2 * LIST_CAP * 4;  // list-merge scratch
     static constexpr uint32_t OFF_BAR = OFF_SCR + ROWS * LIST_CAP * 4;
     // barriers: kv_full, kv_empty, q_full[ST], q_empty[ST], s_full, p_full, acc_done, dp_full,
-    // ds_full, dv_done, dk_done, drain x 2, list_full[2], list_empty[2]
-    static constexpr int NBAR = 2 + 2 * ST + 9 + 4;
+    // ds_full, drain x 2, list_full[2], list_empty[2]
+    static constexpr int NBAR = 2 + 2 * ST + 7 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
@@ -1161,7 +1161,7 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
     const int grp = p.heads / p.heads_kv;
 
     const uint32_t bar_kv = sb + C::OFF_BAR;
-    const uint32_t bar_kve = bar_kv + 8u;  // K, V copied into TMEM: the buffer may be refilled
+    const uint32_t bar_kve = bar_kv + 8u;  // K and V copied into TMEM (one commit each): refill
     auto bar_qf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + s); };
     auto bar_qe = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + C::ST + s); };
     const uint32_t bar_s = sb + C::OFF_BAR + 8u * (2 + 2 * C::ST);
@@ -1169,12 +1169,10 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
     const uint32_t bar_acc = bar_s + 16u;
     const uint32_t bar_dp = bar_s + 24u;
     const uint32_t bar_ds = bar_s + 32u;
-    const uint32_t bar_dvd = bar_s + 40u;  // dV(G) done: S^T's columns (its P^T) are free
-    const uint32_t bar_dkd = bar_s + 48u;  // dK(G) done: dP^T's columns (its dS^T) are free
-    const uint32_t bar_dr = bar_s + 56u;
-    const uint32_t bar_dr2 = bar_s + 64u;
-    auto bar_lf = [&](int b) { return bar_s + 72u + 8u * b; };
-    auto bar_le = [&](int b) { return bar_s + 88u + 8u * b; };
+    const uint32_t bar_dr = bar_s + 40u;
+    const uint32_t bar_dr2 = bar_s + 48u;
+    auto bar_lf = [&](int b) { return bar_s + 56u + 8u * b; };
+    auto bar_le = [&](int b) { return bar_s + 72u + 8u * b; };
     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
     // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
@@ -1185,18 +1183,16 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        mbar_init(bar_kve, 1);
+        mbar_init(bar_kve, 2);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_qf(s), 1);
-            mbar_init(bar_qe(s), 1);
+            mbar_init(bar_qe(s), 2);  // one commit from each MMA thread
         }
         mbar_init(bar_s, 1);
         mbar_init(bar_p, 256);
-        mbar_init(bar_acc, 1);
+        mbar_init(bar_acc, 2);
         mbar_init(bar_dp, 1);
         mbar_init(bar_ds, 256);
-        mbar_init(bar_dvd, 1);
-        mbar_init(bar_dkd, 1);
         mbar_init(bar_dr, 1);
         mbar_init(bar_dr2, 1);
         for (int b = 0; b < 2; ++b) {
@@ -1325,19 +1321,46 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
                     mbar_drain(bar_qf(m % C::ST), (m / C::ST) & 1, kDrainNs);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ K, V into TMEM; S^T and dP^T issuer
-        // S^T(G) overwrites P^T(G-1) and so waits for dV(G-1)'s commit; dP^T(G)
-        // overwrites dS^T(G-1) and waits for dK(G-1)'s (both issued by the other
-        // thread; the element-wise warps keep P in registers for the dS pass).
-        // A tile's K and V are copied into TMEM after the previous tile's MMAs
-        // that read them (one thread: issue order).
+    } else if (warp == 1 || warp == 3) {
+        // ------------------------------------------------------------ MMA issuers
+        // Thread A (warp 1): K into TMEM, then per element dV(G) += P^T(G) dO
+        // followed by S^T(G+1) = K Q^T. Thread B (warp 3): V into TMEM, then
+        // dK(G) += dS^T(G) Q followed by dP^T(G+1) = V dO^T. S^T(G+1) overwrites
+        // P^T(G) and dP^T(G+1) overwrites dS^T(G), each after the MMA of the same
+        // thread that reads it (one thread: issue order), and after the
+        // element-wise threads have read S^T(G) / dP^T(G) (they wrote P^T(G) /
+        // dS^T(G) before arriving). Both threads read every stage, so a stage is
+        // released by one commit from each (after dV(G) and after dK(G)); so are
+        // the tile's accumulators (after its last dV and dK) and the shared-memory
+        // K/V buffer (after each thread's copy into TMEM). A tile's first dV and
+        // dK overwrite the accumulators: their P^T and dS^T come from
+        // element-wise threads that have already read the previous tile's out.
         if (lane == 0) {
+            const bool tA = warp == 1;
             constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
-            const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K, 16, 1024);
-            const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V, 16, 1024);
+            constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);  // dV += P^T dO, dK += dS^T Q
+            const uint64_t a_desc = umma_sdesc(sb + (tA ? C::OFF_K : C::OFF_V), 16, 1024);
+            const uint32_t col_a = tA ? C::COL_KA : C::COL_VA;      // K or V in TMEM
+            const uint32_t col_x = tA ? C::COL_S : C::COL_DP;       // S^T / P^T or dP^T / dS^T
+            const uint32_t col_acc = tA ? C::COL_DV : C::COL_DK;
+            const uint32_t off_b = tA ? C::OFF_Q : C::OFF_DO;       // B of S^T / dP^T
+            const uint32_t off_b2 = tA ? C::OFF_DO : C::OFF_Q;      // B of dV / dK
+            const uint32_t bar_x = tA ? bar_s : bar_dp;             // S^T / dP^T written
+            const uint32_t bar_y = tA ? bar_p : bar_ds;             // P^T / dS^T written
             bool issued = false, fail = false;
             int G = 0, m = 0;
+            auto issue_x = [&](int g) {  // S^T(g) or dP^T(g)
+                const int st = g % C::ST;
+                if (!mbar_wait(bar_qf(st), (g / C::ST) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint64_t b_desc = umma_sdesc(sb + off_b + st * C::QBYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_bf16_ts(tmem + col_x, tmem + col_a + kk * 8, b_desc + kstep(kk, BK), idesc_s,
+                                 kk > 0 ? 1u : 0u);
+                umma_commit(bar_x);
+                return true;
+            };
             for (int k = 0; !fail; ++k) {
                 const int b = k & 1;
                 if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
@@ -1347,102 +1370,41 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
                     if (!mbar_wait(bar_kv, m & 1, ctl)) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
-                        tmem_cp_128x256b(tmem + C::COL_KA + kk * 8, dk_desc + kstep(kk, C::M));
-                        tmem_cp_128x256b(tmem + C::COL_VA + kk * 8, dv_desc + kstep(kk, C::M));
-                    }
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        tmem_cp_128x256b(tmem + col_a + kk * 8, a_desc + kstep(kk, C::M));
                     umma_commit(bar_kve);
                     issued = true;
                     ++m;
+                    if (!issue_x(G)) break;
                 }
                 for (int n = 0; n < len; ++n, ++G) {
                     const int st = G % C::ST;
-                    if ((G > 0 && !mbar_wait(bar_dvd, (G - 1) & 1, ctl)) ||
-                        !mbar_wait(bar_qf(st), (G / C::ST) & 1, ctl)) {
-                        fail = true;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_KA + kk * 8, dq_desc + kstep(kk, BK), idesc_s,
-                                     kk > 0 ? 1u : 0u);
-                    umma_commit(bar_s);
-                    if (G > 0 && !mbar_wait(bar_dkd, (G - 1) & 1, ctl)) {
-                        fail = true;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_VA + kk * 8, ddo_desc + kstep(kk, BK), idesc_s,
-                                     kk > 0 ? 1u : 0u);
-                    umma_commit(bar_dp);
-                }
-                if (fail) break;
-                mbar_arrive(bar_le(b));
-            }
-            if (*abort_cta && issued) {
-                umma_commit(bar_dr);
-                mbar_drain(bar_dr, 0, kDrainNs);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 3) {
-        // ------------------------------------------------------------ dV and dK issuer
-        // dV(G) += P^T(G) dO once P^T(G) is written; dK(G) += dS^T(G) Q once
-        // dS^T(G) is. The commit after dK(G) releases the Q/dO stage (dS^T(G)
-        // needed S^T(G) and dP^T(G) complete, so every read of it is done). A
-        // tile's first dV and dK overwrite the accumulators: their P^T and dS^T
-        // come from element-wise threads that have already read the previous
-        // tile's accumulators out.
-        if (lane == 0) {
-            constexpr uint32_t idesc_a = umma_idesc(128, HD, 0, 1);  // dV += P^T dO, dK += dS^T Q
-            bool issued = false, fail = false;
-            int G = 0;
-            for (int k = 0; !fail; ++k) {
-                const int b = k & 1;
-                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
-                if (list_item[b] < 0) break;
-                const int len = list_len[b];
-                for (int n = 0; n < len; ++n, ++G) {
-                    const int st = G % C::ST;
-                    if (!mbar_wait(bar_p, G & 1, ctl)) {
+                    if (!mbar_wait(bar_y, G & 1, ctl)) {
                         fail = true;
                         break;
                     }
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t bdo = umma_sdesc(sb + C::OFF_DO + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_DV, tmem + C::COL_S + packed_col<BK>(kk), bdo, idesc_a,
+                        const uint64_t bb = umma_sdesc(sb + off_b2 + st * C::QBYTES + kk * 2048, BK * 128, 1024);
+                        umma_bf16_ts(tmem + col_acc, tmem + col_x + packed_col<BK>(kk), bb, idesc_a,
                                      (n > 0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit(bar_dvd);
-                    issued = true;
-                    if (!mbar_wait(bar_ds, G & 1, ctl)) {
-                        fail = true;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t bq = umma_sdesc(sb + C::OFF_Q + st * C::QBYTES + kk * 2048, BK * 128, 1024);
-                        umma_bf16_ts(tmem + C::COL_DK, tmem + C::COL_DP + packed_col<BK>(kk), bq, idesc_a,
-                                     (n > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    umma_commit(bar_dkd);
                     umma_commit(bar_qe(st));
-                    if (n + 1 == len) umma_commit(bar_acc);  // the tile's dK, dV are complete with it
+                    if (n + 1 == len) {
+                        umma_commit(bar_acc);  // the tile's dV (dK) is complete with it
+                    } else if (!issue_x(G + 1)) {
+                        fail = true;
+                        break;
+                    }
                 }
                 if (fail) break;
                 mbar_arrive(bar_le(b));
             }
             if (*abort_cta && issued) {
-                umma_commit(bar_dr2);
-                mbar_drain(bar_dr2, 0, kDrainNs);
+                const uint32_t dr = tA ? bar_dr : bar_dr2;
+                umma_commit(dr);
+                mbar_drain(dr, 0, kDrainNs);
             }
         }
         __syncwarp();
