@@ -19,7 +19,8 @@
 //                        lists (the forward's lists): S = Q K^T and dP = dO V^T
 //                        into TMEM, dS (bf16) written back over dP, dQ += dS K
 //                        with dS read from TMEM and K from shared memory as an
-//                        MN-major B.
+//                        MN-major B. An element is 128 keys: one 128-key
+//                        block, or two list entries with 64-key blocks.
 //   s2_bwd_dkv_kernel    one 128-row key tile per CTA, walking the union of
 //                        its key blocks' transposed lists (query blocks that
 //                        list them): S^T = K Q^T and dP^T = V dO^T into TMEM,
@@ -35,16 +36,16 @@
 // results are deterministic.
 //
 // CTA = 12 warps: warp 0 TMA producer; warp 1 TMEM owner and MMA issuer (one
-// thread; in the dQ kernel it issues S and dP while one thread of warp 3
-// issues dQ); warp 2 builds the union list in shared memory (in the dQ
-// kernel item after item, double-buffered, and it also loads the item's Q
-// and dO); warps 4..11 the element-wise passes and the epilogue: thread = one
-// tile row = one TMEM lane, warps 4..7 on the first half of the columns and
-// warps 8..11 on the second (two warps per SM sub-partition hide the
-// exponential and TMEM latencies; a single warpgroup was measured to leave
-// the tensor core idle most of the time). In the persistent dK/dV kernel warp 2
-// also loads each tile's K and V, warp 1 copies them into TMEM and issues S^T
-// and dP^T, and one thread of warp 3 issues dV and dK.
+// thread); warp 2 builds the union list in shared memory (in the persistent
+// kernels item after item, double-buffered, and it also loads the item's Q
+// and dO, or K and V); warps 4..11 the element-wise passes and the epilogue:
+// thread = one tile row = one TMEM lane, warps 4..7 on the first half of the
+// columns and warps 8..11 on the second (two warps per SM sub-partition hide
+// the exponential and TMEM latencies; a single warpgroup was measured to leave
+// the tensor core idle most of the time). In the persistent dK/dV kernel
+// (N = 64 products, which one thread issues at half the tensor core's rate) a
+// thread of warp 3 issues too: dV(G) then S^T(G+1) from warp 1, dK(G) then
+// dP^T(G+1) from warp 3.
 // With B = 64 a 128-row tile holds two blocks and every row masks by its own
 // block's tag. Every wait is bounded; on a timeout the CTA drains its own
 // copies and MMAs, frees TMEM and exits with the device timeout flag set.
@@ -167,35 +168,41 @@ template <int HD, int BK>
 struct BwdQCfg {
     static constexpr int M = 128;
     static constexpr int ROWS = (BK == 128) ? 1 : 2;  // query blocks per tile
+    // One element = NK = 128 keys: one 128-key block, or two consecutive
+    // entries of the union list with 64-key blocks (an odd last entry is
+    // paired with a fully masked pad). The two entries of a pair need not be
+    // adjacent blocks: each element-wise warpgroup masks its own 64 columns
+    // by its own entry, and every row of the tile computes every element of
+    // the union anyway, so pairing adds no masked work beyond the pad. S, dP
+    // and dQ are then N = 128 / K = 128 products, which one thread issues at
+    // the tensor core's rate.
+    static constexpr int NK = 128;
+    static constexpr int KPE = NK / BK;               // list entries per element
     static constexpr uint32_t TBYTES = M * HD * 2;    // Q or dO tile
-    static constexpr uint32_t KVBYTES = BK * HD * 2;  // one K or V block
+    static constexpr uint32_t KVBYTES = NK * HD * 2;  // K or V of one element
     static constexpr int ST = 2;
     static constexpr int LIST_CAP = 2048;
     static constexpr uint32_t LIST_BYTES = 2 * LIST_CAP * 4;  // double-buffered
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_DO = TBYTES;
-    static constexpr uint32_t OFF_K = 2 * TBYTES;              // [stage][panel][BK rows x 128 B]
+    static constexpr uint32_t OFF_K = 2 * TBYTES;              // [stage][panel][NK rows x 128 B]
     static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
     static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
     // barriers: qd_full, qd_empty, k_full[ST], v_full[ST], kv_empty[ST], s_full, ds_full, acc_done,
-    // drain, dp_full, s_free, list_full[2], list_empty[2], dq_done, drain of the dQ issuer
-    static constexpr int NBAR = 2 + 3 * ST + 6 + 4 + 2;
+    // drain, dp_full, s_free, list_full[2], list_empty[2]
+    static constexpr int NBAR = 2 + 3 * ST + 6 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
-    // 64-key blocks: one thread issues S and dP, another dQ (one thread issuing
-    // all 20 MMAs of an element, with their waits and commits, was the limit;
-    // with 128-key blocks one thread keeps up with the tensor core).
-    static constexpr bool SPLIT = BK == 64;
-    // producer, MMA issuer(s), 8 element-wise warps
-    static constexpr uint32_t LIST_CONSUMERS = SPLIT ? 11 : 10;
-    static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_ACC = 2 * BK;
+    // producer, MMA issuer, 8 element-wise warps
+    static constexpr uint32_t LIST_CONSUMERS = 10;
+    static constexpr uint32_t COL_S = 0, COL_DP = NK, COL_ACC = 2 * NK;
     // Q and dO, the A operands of every S and dP MMA of an item, sit in TMEM
     // (HD/2 columns each): those MMAs read only K or V from shared memory.
-    static constexpr uint32_t COL_QA = 2 * BK + HD, COL_DOA = 2 * BK + HD + HD / 2;
-    static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD) <= 256 ? 256 : 512;
-    static_assert(2 * BK + 2 * HD <= 512, "TMEM budget");
+    static constexpr uint32_t COL_QA = 2 * NK + HD, COL_DOA = 2 * NK + HD + HD / 2;
+    static constexpr uint32_t TMEM_COLS = (2 * NK + 2 * HD) <= 256 ? 256 : 512;
+    static_assert(2 * NK + 2 * HD <= 512, "TMEM budget");
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
@@ -233,8 +240,6 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t bar_sfree = bar_s + 40u;
     auto bar_lf = [&](int b) { return bar_s + 48u + 8u * b; };
     auto bar_le = [&](int b) { return bar_s + 64u + 8u * b; };
-    const uint32_t bar_dqd = bar_s + 80u;  // dQ(G) done: dP's columns (its dS) are free
-    const uint32_t bar_dr2 = bar_s + 88u;
     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
     // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
@@ -261,8 +266,6 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mbar_init(bar_lf(b), 1);
             mbar_init(bar_le(b), C::LIST_CONSUMERS);
         }
-        mbar_init(bar_dqd, 1);
-        mbar_init(bar_dr2, 1);
         *abort_cta = 0;
         fence_mbar_init();
     }
@@ -344,23 +347,35 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const int bkv = (bh / p.heads) * p.heads_kv + (bh % p.heads) / (p.heads / p.heads_kv);
                 const uint32_t* L = list + b * C::LIST_CAP;
                 const int len = list_len[b];
-                for (int e = 0; e < len; ++e, ++n) {
+                const int nel = (len + C::KPE - 1) / C::KPE;
+                for (int e = 0; e < nel; ++e, ++n) {
                     const int st = n % C::ST;
                     if (!mbar_wait(bar_ke(st), ((n / C::ST) & 1) ^ 1, ctl)) {
                         stop = true;
                         break;
                     }
-                    const int32_t krow = list_j(L[e]) * BK;
+                    // entry h of the element into rows h*BK.. of the stage (a pad loads
+                    // the first entry's block again: finite data, masked)
                     mbar_arrive_expect_tx(bar_kf(st), C::KVBYTES);
 #pragma unroll
-                    for (int pn = 0; pn < HD / 64; ++pn)
-                        tma_load_3d(sb + C::OFF_K + st * C::KVBYTES + pn * (BK * 128), &tmK, pn * 64, krow,
-                                    bkv, bar_kf(st));
+                    for (int h = 0; h < C::KPE; ++h) {
+                        const int ei = e * C::KPE + h;
+                        const int32_t krow = list_j(L[ei < len ? ei : e * C::KPE]) * BK;
+#pragma unroll
+                        for (int pn = 0; pn < HD / 64; ++pn)
+                            tma_load_3d(sb + C::OFF_K + st * C::KVBYTES + pn * (C::NK * 128) + h * (BK * 128), &tmK,
+                                        pn * 64, krow, bkv, bar_kf(st));
+                    }
                     mbar_arrive_expect_tx(bar_vf(st), C::KVBYTES);
 #pragma unroll
-                    for (int pn = 0; pn < HD / 64; ++pn)
-                        tma_load_3d(sb + C::OFF_V + st * C::KVBYTES + pn * (BK * 128), &tmV, pn * 64, krow,
-                                    bkv, bar_vf(st));
+                    for (int h = 0; h < C::KPE; ++h) {
+                        const int ei = e * C::KPE + h;
+                        const int32_t krow = list_j(L[ei < len ? ei : e * C::KPE]) * BK;
+#pragma unroll
+                        for (int pn = 0; pn < HD / 64; ++pn)
+                            tma_load_3d(sb + C::OFF_V + st * C::KVBYTES + pn * (C::NK * 128) + h * (BK * 128), &tmV,
+                                        pn * 64, krow, bkv, bar_vf(st));
+                    }
                 }
                 if (!stop) mbar_arrive(bar_le(b));
             }
@@ -371,228 +386,115 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 }
         }
         __syncwarp();
-    } else if (warp == 1 || (C::SPLIT && warp == 3)) {
-        if constexpr (C::SPLIT) {
-            if (warp == 1) {
-                // ------------------------------------------------------------ S and dP issuer
-                // Element G (counted over all items) uses stage G % ST. S(G) and dP(G)
-                // are committed separately so that the element-wise warps start on P
-                // while dP is still running. S(G) is issued once the warps have loaded
-                // S(G-1) (they keep P in registers); dP(G) once dQ(G-1), issued by the
-                // other thread, has read dS(G-1) from dP's columns.
-                if (lane == 0) {
-                    constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S = Q K^T, dP = dO V^T
-                    const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
-                    const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
-                    bool issued = false, fail = false;
-                    int G = 0;
-                    for (int k = 0; !fail; ++k) {
-                        const int b = k & 1;
-                        if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
-                        if (list_item[b] < 0) break;
-                        const int len = list_len[b];
-                        if (!mbar_wait(bar_qd, k & 1, ctl)) break;
-                        // Q and dO into TMEM (after the previous item's S and dP MMAs, in
-                        // issue order); the shared-memory buffers are then free.
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = umma_idesc(128, C::NK, 0, 0);  // S = Q K^T, dP = dO V^T
+            constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);     // dQ += dS K (K as MN-major B)
+            const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
+            const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
+            bool issued = false, fail = false;
+            // Element G (counted over all items) uses stage G % ST; S(G) and dP(G)
+            // are committed separately so that the element-wise warps start on P
+            // while dP is still running. Order per element: [S(G) read out]
+            // S(G+1); [dS(G) ready] dQ(G), dP(G+1). The warps keep P in
+            // registers, so S(G+1) may overwrite S(G) as soon as they have
+            // loaded it; dS(G) sits in dP's columns and dP(G+1) is issued after
+            // dQ(G) has read it.
+            auto issue_s = [&](int G) {
+                const int st = G % C::ST;
+                if (!mbar_wait(bar_kf(st), (G / C::ST) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_QA + kk * 8, dk_desc + kstep(kk, C::NK), idesc_s,
+                                 kk > 0 ? 1u : 0u);
+                umma_commit(bar_s);
+                issued = true;
+                return true;
+            };
+            auto issue_dp = [&](int G) {
+                const int st = G % C::ST;
+                if (!mbar_wait(bar_vf(st), (G / C::ST) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_DOA + kk * 8, dv_desc + kstep(kk, C::NK),
+                                 idesc_s, kk > 0 ? 1u : 0u);
+                umma_commit(bar_dp);
+                return true;
+            };
+            int G = 0;
+            for (int k = 0; !fail; ++k) {
+                const int b = k & 1;
+                if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
+                if (list_item[b] < 0) break;
+                const int len = (list_len[b] + C::KPE - 1) / C::KPE;  // elements
+                if (!mbar_wait(bar_qd, k & 1, ctl)) break;
+                // Q and dO into TMEM (after the previous item's MMAs that read them,
+                // in issue order); the shared-memory buffers are then free.
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    tmem_cp_128x256b(tmem + C::COL_QA + kk * 8, dq_desc + kstep(kk, C::M));
+                    tmem_cp_128x256b(tmem + C::COL_DOA + kk * 8, ddo_desc + kstep(kk, C::M));
+                }
+                umma_commit(bar_qe);
+                issued = true;
+                if (len > 0) {
+                    // S's columns are free once the warps have loaded S of the previous
+                    // element; dP's (its dS) were read by its dQ, issued before.
+                    if (G > 0 && !mbar_wait(bar_sfree, (G - 1) & 1, ctl)) break;
+                    tc_fence_after();
+                    if (!issue_s(G) || !issue_dp(G)) break;
+                    for (int n = 0; n < len; ++n, ++G) {
+                        const int st = G % C::ST;
+                        const bool more = n + 1 < len;
+                        if (more) {
+                            if (!mbar_wait(bar_sfree, G & 1, ctl)) {
+                                fail = true;
+                                break;
+                            }
+                            tc_fence_after();
+                            if (!issue_s(G + 1)) {
+                                fail = true;
+                                break;
+                            }
+                        }
+                        if (!mbar_wait(bar_ds, G & 1, ctl)) {
+                            fail = true;
+                            break;
+                        }
                         tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk) {
-                            tmem_cp_128x256b(tmem + C::COL_QA + kk * 8, dq_desc + kstep(kk, C::M));
-                            tmem_cp_128x256b(tmem + C::COL_DOA + kk * 8, ddo_desc + kstep(kk, C::M));
+                        for (int kk = 0; kk < C::NK / 16; ++kk) {
+                            const uint64_t bk =
+                                umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, C::NK * 128, 1024);
+                            umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<C::NK>(kk), bk, idesc_q,
+                                         (n > 0 || kk > 0) ? 1u : 0u);
                         }
-                        umma_commit(bar_qe);
-                        issued = true;
-                        for (int n = 0; n < len; ++n, ++G) {
-                            const int st = G % C::ST;
-                            // S(G): S's columns are free once the warps have loaded S(G-1)
-                            // (S(G) is issued only after this wait: the phases cannot alias)
-                            if ((G > 0 && !mbar_wait(bar_sfree, (G - 1) & 1, ctl)) ||
-                                !mbar_wait(bar_kf(st), (G / C::ST) & 1, ctl)) {
-                                fail = true;
-                                break;
-                            }
-                            tc_fence_after();
-                            const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
-#pragma unroll
-                            for (int kk = 0; kk < HD / 16; ++kk)
-                                umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_QA + kk * 8, dk_desc + kstep(kk, BK),
-                                             idesc_s, kk > 0 ? 1u : 0u);
-                            umma_commit(bar_s);
-                            // dP(G): dP's columns are free once dQ(G-1) has completed
-                            if ((G > 0 && !mbar_wait(bar_dqd, (G - 1) & 1, ctl)) ||
-                                !mbar_wait(bar_vf(st), (G / C::ST) & 1, ctl)) {
-                                fail = true;
-                                break;
-                            }
-                            tc_fence_after();
-                            const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
-#pragma unroll
-                            for (int kk = 0; kk < HD / 16; ++kk)
-                                umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_DOA + kk * 8, dv_desc + kstep(kk, BK),
-                                             idesc_s, kk > 0 ? 1u : 0u);
-                            umma_commit(bar_dp);
+                        umma_commit(bar_ke(st));
+                        if (more && !issue_dp(G + 1)) {
+                            fail = true;
+                            break;
                         }
-                        if (fail) break;
-                        mbar_arrive(bar_le(b));
                     }
-                    if (*abort_cta && issued) {
-                        umma_commit(bar_dr);
-                        mbar_drain(bar_dr, 0, kDrainNs);
-                    }
+                    if (fail) break;
+                    umma_commit(bar_acc);  // dQ of this item is complete once its last MMA is
                 }
-            } else {
-                // ------------------------------------------------------------ dQ issuer
-                // dQ(G) += dS(G) K once the warps have written dS(G); its commit frees
-                // dP's columns for dP(G+1) and releases the K/V stage (dS(G) needed S(G)
-                // and dP(G) complete, so every read of the stage is done). The S/dP
-                // thread waits for every element's loads in order, so a stage cannot
-                // be refilled before it has passed the stage.
-                if (lane == 0) {
-                    constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);  // dQ += dS K (K as MN-major B)
-                    bool issued = false, fail = false;
-                    int G = 0;
-                    for (int k = 0; !fail; ++k) {
-                        const int b = k & 1;
-                        if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
-                        if (list_item[b] < 0) break;
-                        const int len = list_len[b];
-                        for (int n = 0; n < len; ++n, ++G) {
-                            const int st = G % C::ST;
-                            if (!mbar_wait(bar_ds, G & 1, ctl)) {
-                                fail = true;
-                                break;
-                            }
-                            tc_fence_after();
-#pragma unroll
-                            for (int kk = 0; kk < BK / 16; ++kk) {
-                                const uint64_t bk = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
-                                umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
-                                             (n > 0 || kk > 0) ? 1u : 0u);
-                            }
-                            umma_commit(bar_dqd);
-                            umma_commit(bar_ke(st));
-                            issued = true;
-                        }
-                        if (fail) break;
-                        if (len > 0) umma_commit(bar_acc);  // dQ of this item is complete once its last MMA is
-                        mbar_arrive(bar_le(b));
-                    }
-                    if (*abort_cta && issued) {
-                        umma_commit(bar_dr2);
-                        mbar_drain(bar_dr2, 0, kDrainNs);
-                    }
-                }
+                mbar_arrive(bar_le(b));
             }
-        } else {
-            // ------------------------------------------------------------ MMA issuer
-            if (lane == 0) {
-                constexpr uint32_t idesc_s = umma_idesc(128, BK, 0, 0);  // S = Q K^T, dP = dO V^T
-                constexpr uint32_t idesc_q = umma_idesc(128, HD, 0, 1);  // dQ += dS K (K as MN-major B)
-                const uint64_t dq_desc = umma_sdesc(sb + C::OFF_Q, 16, 1024);
-                const uint64_t ddo_desc = umma_sdesc(sb + C::OFF_DO, 16, 1024);
-                bool issued = false, fail = false;
-                // Element G (counted over all items) uses stage G % ST; S(G) and dP(G)
-                // are committed separately so that the element-wise warps start on P
-                // while dP is still running. Order per element: [S(G) read out]
-                // S(G+1); [dS(G) ready] dQ(G), dP(G+1). The warps keep P in
-                // registers, so S(G+1) may overwrite S(G) as soon as they have
-                // loaded it; dS(G) sits in dP's columns and dP(G+1) is issued after
-                // dQ(G) has read it.
-                auto issue_s = [&](int G) {
-                    const int st = G % C::ST;
-                    if (!mbar_wait(bar_kf(st), (G / C::ST) & 1, ctl)) return false;
-                    tc_fence_after();
-                    const uint64_t dk_desc = umma_sdesc(sb + C::OFF_K + st * C::KVBYTES, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ts(tmem + C::COL_S, tmem + C::COL_QA + kk * 8, dk_desc + kstep(kk, BK), idesc_s,
-                                     kk > 0 ? 1u : 0u);
-                    umma_commit(bar_s);
-                    issued = true;
-                    return true;
-                };
-                auto issue_dp = [&](int G) {
-                    const int st = G % C::ST;
-                    if (!mbar_wait(bar_vf(st), (G / C::ST) & 1, ctl)) return false;
-                    tc_fence_after();
-                    const uint64_t dv_desc = umma_sdesc(sb + C::OFF_V + st * C::KVBYTES, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16_ts(tmem + C::COL_DP, tmem + C::COL_DOA + kk * 8, dv_desc + kstep(kk, BK),
-                                     idesc_s, kk > 0 ? 1u : 0u);
-                    umma_commit(bar_dp);
-                    return true;
-                };
-                int G = 0;
-                for (int k = 0; !fail; ++k) {
-                    const int b = k & 1;
-                    if (!mbar_wait(bar_lf(b), (k >> 1) & 1, ctl)) break;
-                    if (list_item[b] < 0) break;
-                    const int len = list_len[b];
-                    if (!mbar_wait(bar_qd, k & 1, ctl)) break;
-                    // Q and dO into TMEM (after the previous item's MMAs that read them,
-                    // in issue order); the shared-memory buffers are then free.
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
-                        tmem_cp_128x256b(tmem + C::COL_QA + kk * 8, dq_desc + kstep(kk, C::M));
-                        tmem_cp_128x256b(tmem + C::COL_DOA + kk * 8, ddo_desc + kstep(kk, C::M));
-                    }
-                    umma_commit(bar_qe);
-                    issued = true;
-                    if (len > 0) {
-                        // S's columns are free once the warps have loaded S of the previous
-                        // element; dP's (its dS) were read by its dQ, issued before.
-                        if (G > 0 && !mbar_wait(bar_sfree, (G - 1) & 1, ctl)) break;
-                        tc_fence_after();
-                        if (!issue_s(G) || !issue_dp(G)) break;
-                        for (int n = 0; n < len; ++n, ++G) {
-                            const int st = G % C::ST;
-                            const bool more = n + 1 < len;
-                            if (more) {
-                                if (!mbar_wait(bar_sfree, G & 1, ctl)) {
-                                    fail = true;
-                                    break;
-                                }
-                                tc_fence_after();
-                                if (!issue_s(G + 1)) {
-                                    fail = true;
-                                    break;
-                                }
-                            }
-                            if (!mbar_wait(bar_ds, G & 1, ctl)) {
-                                fail = true;
-                                break;
-                            }
-                            tc_fence_after();
-#pragma unroll
-                            for (int kk = 0; kk < BK / 16; ++kk) {
-                                const uint64_t bk =
-                                    umma_sdesc(sb + C::OFF_K + st * C::KVBYTES + kk * 2048, BK * 128, 1024);
-                                umma_bf16_ts(tmem + C::COL_ACC, tmem + C::COL_DP + packed_col<BK>(kk), bk, idesc_q,
-                                             (n > 0 || kk > 0) ? 1u : 0u);
-                            }
-                            umma_commit(bar_ke(st));
-                            if (more && !issue_dp(G + 1)) {
-                                fail = true;
-                                break;
-                            }
-                        }
-                        if (fail) break;
-                        umma_commit(bar_acc);  // dQ of this item is complete once its last MMA is
-                    }
-                    mbar_arrive(bar_le(b));
-                }
-                if (*abort_cta && issued) {
-                    umma_commit(bar_dr);
-                    mbar_drain(bar_dr, 0, kDrainNs);
-                }
+            if (*abort_cta && issued) {
+                umma_commit(bar_dr);
+                mbar_drain(bar_dr, 0, kDrainNs);
             }
         }
         __syncwarp();
     } else if (warp >= 4) {
         // ------------------------------------------------------------ element-wise passes + epilogue
-        constexpr int HALF = BK / 2;  // key columns per warpgroup
+        constexpr int HALF = C::NK / 2;  // key columns per warpgroup (one entry's block when paired)
         const int quad = warp & 3, g = (warp - 4) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
@@ -615,16 +517,21 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 dy = sp[128];
             }
             const uint32_t* L = list + b * C::LIST_CAP;
-            const int len = list_len[b];
+            const int nent = list_len[b];
+            const int len = (nent + C::KPE - 1) / C::KPE;  // elements
             for (int n = 0; n < len; ++n, ++G) {
-                const uint32_t ent = L[n];
+                // this warpgroup's entry: the element's block (128-key blocks), or
+                // entry g of the pair (64-key blocks; past the list: a masked pad)
+                const int ei = n * C::KPE + (C::KPE == 2 ? g : 0);
+                const uint32_t ent = ei < nent ? L[ei] : 0u;
                 if (!warp_wait(bar_s, G & 1, ctl)) {
                     fail = true;
                     break;
                 }
                 tc_fence_after();
                 const bool vis = row_valid && ((list_bits(ent) >> rowbit) & 1);
-                const int lim = qpos - list_j(ent) * BK - g * HALF;  // column c of this half visible iff c <= lim
+                // column c of this half visible iff c <= lim
+                const int lim = qpos - list_j(ent) * BK - (C::KPE == 2 ? 0 : g * HALF);
                 // P pass (needs S only; dP may still be running): P as bf16 pairs in registers
                 uint32_t sr[HALF], pk[HALF / 2];
                 tmem_ld_cols<HALF>(tl + C::COL_S + g * HALF, sr);
