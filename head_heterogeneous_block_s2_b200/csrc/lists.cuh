@@ -15,13 +15,10 @@
 namespace s2 {
 
 // Warp-wide bounded wait (every lane polls: measured faster than one lane
-// polling and broadcasting), backing off 128 ns between failed polls: the
-// element-wise warps wait on every MMA, and their polling slowed the MMA
-// issuers on the same SM sub-partitions (the back-off measured +2-3 % on the
-// prefill and chunked prefill, +1 % on the backward; 64-512 ns alike).
+// polling and broadcasting).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl)
 {
-    const bool ok = mbar_wait(bar, parity, ctl, 128u);
+    const bool ok = mbar_wait(bar, parity, ctl);
     return __all_sync(0xffffffffu, ok);
 }
 

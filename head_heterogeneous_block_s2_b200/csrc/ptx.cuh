@@ -84,12 +84,8 @@ struct WaitCtl {
 
 // Wait until the phase with the given parity of `bar` has completed. Gives up
 // (returns false) when the CTA is aborting or after ctl.timeout_ns; a timeout
-// sets the device timeout flag and the CTA abort flag. A nonzero backoff_ns
-// sleeps that long between failed polls (for whole warps that wait: their
-// polling otherwise takes issue slots from the MMA-issuing threads that share
-// their SM sub-partition).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl,
-                                          uint32_t backoff_ns = 0)
+// sets the device timeout flag and the CTA abort flag.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl)
 {
     if (ctl.timeout_ns == 0) {  // a zero limit: succeed only if the phase is already complete
         if (mbar_test_wait(bar, parity)) return true;
@@ -100,7 +96,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0;; ++it) {
-        if (backoff_ns) __nanosleep(backoff_ns);
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 15u) == 0u) {
             // Stop at once when this CTA is aborting or any CTA has timed out
