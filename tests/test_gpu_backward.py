@@ -83,6 +83,29 @@ def test_mask_layout_with_empty_rows(s2gpu, bk):
     assert (dk[0, 1, 3 * bk:4 * bk] == 0).all() and (dv[0, 1, 3 * bk:4 * bk] == 0).all()
 
 
+def test_odd_union_lists_and_empty_key_tiles(s2gpu):
+    """64-key blocks: query tiles (two query blocks) whose union list has an
+    odd length (the dQ kernel pairs entries into 128-key elements, so the last
+    pair is a masked pad) and key tiles that no query lists (the persistent
+    dK/dV kernel must write zeros for them)."""
+    nb, H, bk = 10, 2, 64
+    m = np.zeros((H, nb, nb), dtype=np.uint8)
+    for t in range(nb // 2):
+        m[0, 2 * t, 0] = 1            # head 0: unions {0, 1}, then {0, 2t, 2t+1} (odd)
+        m[0, 2 * t, 2 * t] = 1
+        m[0, 2 * t + 1, 2 * t + 1] = 1
+        m[1, 2 * t + 1, 2 * t + 1] = 1  # head 1: union {2t+1} (one entry); even blocks unlisted
+    w = synth.PrefillWorkload("t", 2, H, 128, nb * bk, bk, 1, 1, seed=95)
+    q, k, v = synth.prefill_inputs(w)
+    lay = s2gpu.build_layout_mask(m, bk, device="cuda")
+    dq, dk, dv = run_backward(s2gpu, w, lay, q, k, v, upstream(w, 6), bmask=m)
+    for j in range(0, nb, 2):  # head 1's even key blocks: no query lists them
+        assert (dk[:, 1, j * bk:(j + 1) * bk] == 0).all() and (dv[:, 1, j * bk:(j + 1) * bk] == 0).all()
+    # head 1's even query blocks list no key: zero dQ
+    for i in range(0, nb, 2):
+        assert (dq[:, 1, i * bk:(i + 1) * bk] == 0).all()
+
+
 def test_stride_one_matches_autograd_of_causal_sdpa(s2gpu):
     w = synth.PrefillWorkload("t", 1, 2, 128, 512, 128, 1, 1, seed=93)
     q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
