@@ -619,8 +619,8 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
 template <int HD, int BK>
 struct BwdKVCfg {
-    static constexpr int M = 128;
-    static constexpr int ROWS = (BK == 128) ? 1 : 2;   // key blocks per tile
+    static_assert(BK == 128, "64-key blocks use s2_bwd_dkv_persistent_kernel");
+    static constexpr int M = 128;                      // one key block per tile
     static constexpr uint32_t TBYTES = M * HD * 2;     // K or V tile
     static constexpr uint32_t QBYTES = BK * HD * 2;    // one query block of Q or dO
     static constexpr uint32_t STATBYTES = BK * 8;      // L2 of the BK queries, then their D
@@ -632,16 +632,15 @@ struct BwdKVCfg {
     static constexpr uint32_t OFF_DO = OFF_Q + ST * QBYTES;
     static constexpr uint32_t OFF_STAT = OFF_DO + ST * QBYTES;
     static constexpr uint32_t OFF_LIST = OFF_STAT + ST * STATBYTES;
-    static constexpr uint32_t OFF_SCR = OFF_LIST + LIST_CAP * 4;  // list-merge scratch (ROWS > 1)
-    static constexpr uint32_t OFF_BAR = OFF_SCR + (ROWS > 1 ? ROWS * LIST_CAP * 4 : 0);
+    static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_CAP * 4;
     // barriers: kv_full, q_full[ST], q_empty[ST], s_full, p_full, acc_done, drain, dp_full, ds_full
     static constexpr int NBAR = 1 + 2 * ST + 6;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     static constexpr uint32_t SMEM = OFF_MISC + 32;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
     static constexpr uint32_t COL_S = 0, COL_DP = BK, COL_DV = 2 * BK, COL_DK = 2 * BK + HD;
-    // When TMEM has room (B = 64, or head_dim 64), K and V, the A operands of
-    // every S^T and dP^T MMA of the CTA, sit in TMEM (HD/2 columns each).
+    // When TMEM has room (head_dim 64), K and V, the A operands of every S^T
+    // and dP^T MMA of the CTA, sit in TMEM (HD/2 columns each).
     static constexpr bool A_IN_TMEM = 2 * BK + 3 * HD <= 512;
     static constexpr uint32_t COL_KA = 2 * BK + 2 * HD, COL_VA = 2 * BK + 2 * HD + HD / 2;
     static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * HD + (A_IN_TMEM ? HD : 0)) <= 256 ? 256 : 512;
@@ -671,18 +670,7 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const int grp = p.heads / p.heads_kv;
     const int h = (bkv % p.heads_kv) * grp;         // first query head of the group
     const int bq0 = (bkv / p.heads_kv) * p.heads + h;  // its (batch, head) plane
-    // Key blocks of this tile: one 128-row block, or two 64-row blocks chosen on
-    // the host so that their transposed lists overlap (see s2_build_key_tiles).
-    int kb[C::ROWS];
-    if (C::ROWS == 1) {
-        kb[0] = kt;
-    } else {
-#pragma unroll
-        for (int r = 0; r < C::ROWS; ++r) {
-            kb[r] = __ldg(p.key_tiles + ((int64_t)h * p.ntiles + kt) * C::ROWS + r);
-            if (kb[r] >= p.nb) kb[r] = -1;
-        }
-    }
+    int kb[1] = {kt};  // the tile's key block
 
     const uint32_t bar_kv = sb + C::OFF_BAR;
     auto bar_qf = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
@@ -719,30 +707,18 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
     if (threadIdx.x == 0) {  // K and V of the tile do not depend on the list: load them now
         mbar_arrive_expect_tx(bar_kv, 2 * C::TBYTES);
-        int kany = 0;  // a missing block loads a present one's rows (finite data, masked)
+        const int32_t krow = kt * BK;
 #pragma unroll
-        for (int r = 0; r < C::ROWS; ++r)
-            if (kb[r] >= 0) kany = kb[r];
-#pragma unroll
-        for (int r = 0; r < C::ROWS; ++r) {
-            const int32_t krow = (kb[r] >= 0 ? kb[r] : kany) * BK;
-#pragma unroll
-            for (int pn = 0; pn < HD / 64; ++pn) {
-                tma_load_3d(sb + C::OFF_K + pn * (C::M * 128) + r * (BK * 128), &tmK, pn * 64, krow, bkv, bar_kv);
-                tma_load_3d(sb + C::OFF_V + pn * (C::M * 128) + r * (BK * 128), &tmV, pn * 64, krow, bkv, bar_kv);
-            }
+        for (int pn = 0; pn < HD / 64; ++pn) {
+            tma_load_3d(sb + C::OFF_K + pn * (C::M * 128), &tmK, pn * 64, krow, bkv, bar_kv);
+            tma_load_3d(sb + C::OFF_V + pn * (C::M * 128), &tmV, pn * 64, krow, bkv, bar_kv);
         }
     }
-    if (warp == 2) {  // union of the tile's key blocks' query-block lists
-        int lo = INT_MAX;
-#pragma unroll
-        for (int r = 0; r < C::ROWS; ++r)
-            if (kb[r] >= 0 && kb[r] < lo) lo = kb[r];
+    if (warp == 2) {  // the tile's key block's query-block lists
         int total = 0;
         for (int hh = 0; hh < grp; ++hh) {  // the group's query heads, one list after another
-            const int n = warp_union_list<C::ROWS>(p.col_ptr, p.row_idx, (h + hh) * (p.nb + 1), kb, p.nb, p.nnz,
-                                                   lo, p.nb - 1, list + total, C::LIST_CAP - total,
-                                                   reinterpret_cast<int32_t*>(smem + C::OFF_SCR), p.gflags);
+            const int n = warp_union_list<1>(p.col_ptr, p.row_idx, (h + hh) * (p.nb + 1), kb, p.nb, p.nnz, kt,
+                                             p.nb - 1, list + total, C::LIST_CAP - total, nullptr, p.gflags);
             for (int t = lane; t < n; t += 32) list[total + t] |= (uint32_t)hh << 28;
             __syncwarp();
             total += n;
@@ -881,9 +857,9 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const int quad = warp & 3, g = (warp - 4) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        const int kbit = (BK == 128) ? 0 : (r >> 6);
-        const int kpos = kb[kbit] * BK + (r % BK);
-        const bool row_valid = kb[kbit] >= 0 && kpos < p.seq;
+        const int kbit = 0;  // the list entries' row tag of the tile's one key block
+        const int kpos = kt * BK + r;
+        const bool row_valid = kpos < p.seq;
         const float sc = p.scale_log2;
         bool fail = false;
         for (int n = 0; n < len; ++n) {
