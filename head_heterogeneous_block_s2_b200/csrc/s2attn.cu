@@ -24,9 +24,10 @@ namespace {
 
 __device__ uint32_t g_s2_flags;
 
-// Work counters of the persistent prefill kernel: {next item, CTAs done} per
-// slot. Each launch takes the next slot in turn; the kernel's last CTA resets
-// its slot, so a slot is free again once its launch has finished.
+// Work counters of the persistent kernels (prefill, chunked prefill, and the
+// backward's dQ and 64-key dK/dV kernels): {next item, CTAs done} per slot.
+// Each launch takes the next slot in turn; the kernel's last CTA resets its
+// slot, so a slot is free again once its launch has finished.
 constexpr int kSchedSlots = 64;
 __device__ int g_s2_sched[2 * kSchedSlots];
 std::atomic<uint32_t> g_launch_seq{0};
