@@ -60,7 +60,27 @@ def prefill_flops(lay, w) -> int:
 
 
 def prefill_issued_flops(lay, w) -> int:
+    """FLOPs of the layout's whole blocks (nnz * B * B pairs)."""
     return 4 * w.head_dim * w.block * w.block * int(lay.col_idx.size) * w.batch
+
+
+def prefill_mma_flops(lay, w) -> int:
+    """FLOPs the prefill kernel's MMAs compute. A 128-row tile visits every
+    key block that any of its query blocks lists: with B = 128 that is its one
+    row's list (= the whole-block count); with B = 64 it is the union of two
+    consecutive rows' lists, computed for all 128 rows."""
+    if w.block == 128:
+        return prefill_issued_flops(lay, w)
+    rp, ci, nb = lay.row_ptr, lay.col_idx, lay.num_blocks
+    per = 128 // w.block
+    visits = 0
+    for h in range(lay.heads):
+        for i0 in range(0, nb, per):
+            u = set()
+            for i in range(i0, min(i0 + per, nb)):
+                u.update(ci[rp[h * (nb + 1) + i]: rp[h * (nb + 1) + i + 1]].tolist())
+            visits += len(u)
+    return 4 * w.head_dim * 128 * w.block * visits * w.batch
 
 
 def decode_counts(lay, w, ctx_lens):
@@ -282,6 +302,7 @@ def run_ours(args, rank, world, dist):
     out = torch.empty_like(q)
     flops = prefill_flops(lay_p, wp)
     issued = prefill_issued_flops(lay_p, wp)
+    mma = prefill_mma_flops(lay_p, wp)
     if wd is not None:
         d = synth.decode_inputs(wd, device=dev)
         nb_d = -(-wd.ctx_max // wd.block)
@@ -546,6 +567,7 @@ def run_ours(args, rank, world, dist):
                         "local": wp.local, "dense_heads": list(wp.dense_heads),
                         "algorithmic_gflop_per_step": round(flops / 1e9, 3),
                         "issued_gflop_per_step": round(issued / 1e9, 3),
+                        "mma_gflop_per_step": round(mma / 1e9, 3),
                         "ms_per_step": round(pre_ms / K, 4)},
             "layout_build_ms_host": round(layout_ms, 3),
             "l2": "inputs larger than L2 (prefill Q+K+V 403 MB; decode active KV > 1.7 GB)",
