@@ -60,6 +60,9 @@ def _load():
     lib.s2o_backward.restype = i32
     lib.s2o_backward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, vp, i64,
                                  vp, dbl, vp, vp, vp, i32]
+    lib.s2o_backward_sampled.restype = i32
+    lib.s2o_backward_sampled.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, vp,
+                                         i64, vp, dbl, i64, vp, i64, vp, i64, vp, vp, vp, vp, i32]
     lib.s2o_range_block_active.restype = i32
     lib.s2o_range_block_active.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp]
     lib.s2o_range_block_mask.restype = None
@@ -280,6 +283,42 @@ def backward(q, k, v, dout, B, scale, S=None, L=None, dense_heads=None, bmask=No
                               _ptr(dv), int(nthreads))
     if rc != 0:
         raise ValueError("oracle backward rejected its arguments")
+    return dq, dk, dv
+
+
+def backward_sampled(q, k, v, dout, B, scale, planes, qrows, krows, S=None, L=None,
+                     dense_heads=None, bmask=None, nthreads=0):
+    """Oracle gradients of ``backward`` for chosen rows only.
+
+    planes: K/V plane ids b * Hkv + g. qrows: query rows hh * seq + t of each
+    plane's group (query head g * (H / Hkv) + hh, position t). krows: key
+    positions. Returns dq [n_planes, len(qrows), D] and dk, dv
+    [n_planes, len(krows), D] (fp64): the same numbers as the full backward's
+    rows, at the cost of the sampled planes' rows from the smallest sampled
+    position on.
+    """
+    q, k, v, do = _bits(q), _bits(k), _bits(v), _bits(dout)
+    batch, H, seq, D = q.shape
+    Hkv = k.shape[1]
+    assert k.shape == (batch, Hkv, seq, D) and v.shape == k.shape and do.shape == q.shape
+    if bmask is not None:
+        bm = np.ascontiguousarray(np.asarray(bmask, dtype=np.uint8))
+        assert bm.ndim == 3 and bm.shape[0] == H and bm.shape[1] == bm.shape[2]
+        nbm, S_, L_, d = bm.shape[1], 0, 0, None
+    else:
+        bm, nbm, S_, L_, d = None, 0, int(S), int(L), _dense(H, dense_heads)
+    a = lambda x: np.ascontiguousarray(np.asarray(x, dtype=np.int64).reshape(-1))
+    pl, qr, kr = a(planes), a(qrows), a(krows)
+    dq = np.zeros((pl.size, qr.size, D), dtype=np.float64)
+    dk = np.zeros((pl.size, kr.size, D), dtype=np.float64)
+    dv = np.zeros_like(dk)
+    rc = _load().s2o_backward_sampled(_ptr(q), _ptr(k), _ptr(v), _ptr(do), batch, H, Hkv, seq, D, B,
+                                      S_, L_, _ptr(d), nbm, _ptr(bm), float(scale), pl.size,
+                                      _ptr(pl), qr.size, _ptr(qr) if qr.size else None, kr.size,
+                                      _ptr(kr) if kr.size else None, _ptr(dq), _ptr(dk), _ptr(dv),
+                                      int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle backward_sampled rejected its arguments")
     return dq, dk, dv
 
 

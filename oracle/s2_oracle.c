@@ -136,7 +136,8 @@ void s2o_range_block_mask(int64_t H, int64_t nb, const int64_t* range_ptr, const
 /* ------------------------------------------------------------------------- */
 
 typedef struct {
-    int kind; /* 0 = prefill rows, 1 = decode items, 2 = backward planes, 3 = chunk rows */
+    int kind; /* 0 = prefill rows, 1 = decode items, 2 = backward planes, 3 = chunk rows,
+                 4 = row statistics of sampled planes, 5 = sampled gradient rows */
     const uint16_t *q, *k, *v, *dout;
     double *dq, *dk, *dv; /* backward outputs */
     const int32_t *block_table, *ctx_lens, *q_start;
@@ -148,6 +149,11 @@ typedef struct {
     int64_t n_items;
     const int64_t* items;
     double *out, *lse;
+    /* sampled backward: K/V planes b * Hkv + g, query rows hh * seq + q of the
+     * group's heads, key positions; row statistics from q_lo on */
+    int64_t n_planes, nq, nk, q_lo;
+    const int64_t *planes, *qrows, *krows;
+    double *st_lse, *st_D;
     int64_t next;
     int failed;
     pthread_mutex_t lock;
@@ -345,6 +351,130 @@ static void backward_plane(const job_t* J, int64_t e, double* s, double* p, doub
     }
 }
 
+/* Sampled backward, pass 1. Item t names (sampled plane p, query head hh of
+ * its group, row q >= q_lo). The row's statistics by their definitions:
+ * LSE = log sum_k exp(s_k) and D = sum_k P_k dP_k over the visible keys, with
+ * s_k = scale Q.K_k, P_k = exp(s_k - LSE) and dP_k = dO.V_k. A row with no
+ * visible key gets LSE = -inf and D = 0. */
+static void row_stats(const job_t* J, int64_t t, double* s, double* qd, double* dod)
+{
+    const int64_t D = J->D, seq = J->seq, H = J->H, grp = H / J->Hkv, per = seq - J->q_lo;
+    const int64_t p = t / (grp * per), hh = (t / per) % grp, q = J->q_lo + t % per;
+    const int64_t e = J->planes[p], b = e / J->Hkv, h = (e % J->Hkv) * grp + hh;
+    const int dense = J->dense ? J->dense[h] != 0 : 0;
+    const int64_t i = q / J->B;
+    const uint16_t* K = J->k + e * seq * D;
+    const uint16_t* V = J->v + e * seq * D;
+    const uint16_t* Q = J->q + ((b * H + h) * seq + q) * D;
+    const uint16_t* dO = J->dout + ((b * H + h) * seq + q) * D;
+    double* lse = J->st_lse + (p * grp + hh) * seq + q;
+    double* Dq = J->st_D + (p * grp + hh) * seq + q;
+    for (int64_t d = 0; d < D; ++d) {
+        qd[d] = bf16_bits_to_double(Q[d]);
+        dod[d] = bf16_bits_to_double(dO[d]);
+    }
+    double m = -INFINITY;
+    for (int64_t k = 0; k <= q; ++k) {
+        if (!visible(J, h, i, k / J->B, dense)) continue;
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qd[d] * bf16_bits_to_double(K[k * D + d]);
+        s[k] = J->scale * dot;
+        if (s[k] > m) m = s[k];
+    }
+    if (m == -INFINITY) {
+        *lse = -INFINITY;
+        *Dq = 0.0;
+        return;
+    }
+    double den = 0.0;
+    for (int64_t k = 0; k <= q; ++k)
+        if (visible(J, h, i, k / J->B, dense)) den += exp(s[k] - m);
+    *lse = m + log(den);
+    double acc = 0.0;
+    for (int64_t k = 0; k <= q; ++k) {
+        if (!visible(J, h, i, k / J->B, dense)) continue;
+        double dpk = 0.0;
+        for (int64_t d = 0; d < D; ++d) dpk += dod[d] * bf16_bits_to_double(V[k * D + d]);
+        acc += exp(s[k] - *lse) * dpk;
+    }
+    *Dq = acc;
+}
+
+/* Sampled backward, pass 2. Item t names (sampled plane p, entry r): for
+ * r < nq the dQ row of query row qrows[r] (head hh = qrows[r] / seq of the
+ * group), dQ = scale sum_k dS_k K_k; otherwise the dK and dV rows of key
+ * position krows[r - nq], summed over the group's query heads and the rows
+ * q >= k that see it: dV = sum_q P dO_q, dK = scale sum_q dS Q_q, with
+ * dS = P (dP - D_q). */
+static void sampled_grad(const job_t* J, int64_t t, double* qd, double* dod)
+{
+    const int64_t D = J->D, seq = J->seq, H = J->H, grp = H / J->Hkv, n = J->nq + J->nk;
+    const int64_t p = t / n, r = t % n;
+    const int64_t e = J->planes[p], b = e / J->Hkv, g = e % J->Hkv;
+    const uint16_t* K = J->k + e * seq * D;
+    const uint16_t* V = J->v + e * seq * D;
+    if (r < J->nq) {
+        const int64_t hh = J->qrows[r] / seq, q = J->qrows[r] % seq, h = g * grp + hh;
+        const int dense = J->dense ? J->dense[h] != 0 : 0;
+        const int64_t i = q / J->B;
+        const uint16_t* Q = J->q + ((b * H + h) * seq + q) * D;
+        const uint16_t* dO = J->dout + ((b * H + h) * seq + q) * D;
+        const double lse = J->st_lse[(p * grp + hh) * seq + q];
+        const double Dq = J->st_D[(p * grp + hh) * seq + q];
+        double* dQ = J->dq + (p * J->nq + r) * D;
+        for (int64_t d = 0; d < D; ++d) {
+            qd[d] = bf16_bits_to_double(Q[d]);
+            dod[d] = bf16_bits_to_double(dO[d]);
+            dQ[d] = 0.0;
+        }
+        if (lse == -INFINITY) return; /* no visible key: no gradient */
+        for (int64_t k = 0; k <= q; ++k) {
+            if (!visible(J, h, i, k / J->B, dense)) continue;
+            double dot = 0.0, dpk = 0.0;
+            for (int64_t d = 0; d < D; ++d) {
+                dot += qd[d] * bf16_bits_to_double(K[k * D + d]);
+                dpk += dod[d] * bf16_bits_to_double(V[k * D + d]);
+            }
+            const double pk = exp(J->scale * dot - lse);
+            const double ds = pk * (dpk - Dq);
+            for (int64_t d = 0; d < D; ++d) dQ[d] += J->scale * ds * bf16_bits_to_double(K[k * D + d]);
+        }
+        return;
+    }
+    const int64_t kpos = J->krows[r - J->nq], j = kpos / J->B;
+    double* dK = J->dk + (p * J->nk + r - J->nq) * D;
+    double* dV = J->dv + (p * J->nk + r - J->nq) * D;
+    double* kd = qd; /* K and V of the key row */
+    double* vd = dod;
+    for (int64_t d = 0; d < D; ++d) {
+        kd[d] = bf16_bits_to_double(K[kpos * D + d]);
+        vd[d] = bf16_bits_to_double(V[kpos * D + d]);
+        dK[d] = dV[d] = 0.0;
+    }
+    for (int64_t hh = 0; hh < grp; ++hh) {
+        const int64_t h = g * grp + hh;
+        const int dense = J->dense ? J->dense[h] != 0 : 0;
+        for (int64_t q = kpos; q < seq; ++q) {
+            if (!visible(J, h, q / J->B, j, dense)) continue;
+            const uint16_t* Q = J->q + ((b * H + h) * seq + q) * D;
+            const uint16_t* dO = J->dout + ((b * H + h) * seq + q) * D;
+            const double lse = J->st_lse[(p * grp + hh) * seq + q];
+            const double Dq = J->st_D[(p * grp + hh) * seq + q];
+            double dot = 0.0, dpk = 0.0;
+            for (int64_t d = 0; d < D; ++d) {
+                dot += bf16_bits_to_double(Q[d]) * kd[d];
+                dpk += bf16_bits_to_double(dO[d]) * vd[d];
+            }
+            const double pk = exp(J->scale * dot - lse);
+            const double ds = pk * (dpk - Dq);
+            for (int64_t d = 0; d < D; ++d) {
+                dV[d] += pk * bf16_bits_to_double(dO[d]);
+                dK[d] += J->scale * ds * bf16_bits_to_double(Q[d]);
+            }
+        }
+    }
+}
+
 static void* worker(void* arg)
 {
     job_t* J = (job_t*)arg;
@@ -369,6 +499,14 @@ static void* worker(void* arg)
         const int64_t id = J->items ? J->items[t] : t;
         if (J->kind == 2) {
             backward_plane(J, id, s, p, qd, dod);
+            continue;
+        }
+        if (J->kind == 4) {
+            row_stats(J, id, s, qd, dod);
+            continue;
+        }
+        if (J->kind == 5) {
+            sampled_grad(J, id, qd, dod);
             continue;
         }
         double* out = J->out + t * J->D;
@@ -562,6 +700,67 @@ int s2o_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const 
     J.S = S; J.L = L; J.dense = dense; J.bmask = bmask; J.nbm = nbm; J.scale = scale;
     J.n_items = batch * Hkv; J.items = NULL;
     return run_job(&J, nthreads);
+}
+
+/* Backward oracle on a sample: the gradients of s2o_backward for chosen rows.
+ * planes[n_planes]: K/V planes b * Hkv + g. qrows[nq]: query rows of each
+ * sampled plane's group, hh * seq + q (query head g * (H / Hkv) + hh).
+ * krows[nk]: key positions. Outputs dq [n_planes][nq][D], dk and dv
+ * [n_planes][nk][D], fp64. Each row's softmax statistics are computed by
+ * their definitions from q_lo = the smallest sampled position on (a key is
+ * seen only by rows at or after it), then each sampled gradient row sums its
+ * terms one by one. Returns 0 or -1. */
+int s2o_backward_sampled(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         const uint16_t* dout, int64_t batch, int64_t H, int64_t Hkv, int64_t seq,
+                         int64_t D, int64_t B, int64_t S, int64_t L, const uint8_t* dense,
+                         int64_t nbm, const uint8_t* bmask, double scale, int64_t n_planes,
+                         const int64_t* planes, int64_t nq, const int64_t* qrows, int64_t nk,
+                         const int64_t* krows, double* dq, double* dk, double* dv, int nthreads)
+{
+    if (!q || !k || !v || !dout || batch < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || seq < 1 ||
+        D < 1 || B < 1 || n_planes < 1 || !planes || nq < 0 || nk < 0 || nq + nk < 1 ||
+        (nq && (!qrows || !dq)) || (nk && (!krows || !dk || !dv)))
+        return -1;
+    if (bmask ? nbm < (seq + B - 1) / B : (S < 1 || L < 1)) return -1;
+    const int64_t grp = H / Hkv;
+    int64_t q_lo = seq;
+    for (int64_t p = 0; p < n_planes; ++p)
+        if (planes[p] < 0 || planes[p] >= batch * Hkv) return -1;
+    for (int64_t r = 0; r < nq; ++r) {
+        if (qrows[r] < 0 || qrows[r] >= grp * seq) return -1;
+        if (qrows[r] % seq < q_lo) q_lo = qrows[r] % seq;
+    }
+    for (int64_t r = 0; r < nk; ++r) {
+        if (krows[r] < 0 || krows[r] >= seq) return -1;
+        if (krows[r] < q_lo) q_lo = krows[r];
+    }
+    const size_t nst = (size_t)(n_planes * grp * seq);
+    double* st_lse = (double*)malloc(sizeof(double) * nst);
+    double* st_D = (double*)malloc(sizeof(double) * nst);
+    if (!st_lse || !st_D) {
+        free(st_lse);
+        free(st_D);
+        return -1;
+    }
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.k = k; J.v = v; J.dout = dout;
+    J.dq = dq; J.dk = dk; J.dv = dv;
+    J.batch = batch; J.H = H; J.Hkv = Hkv; J.seq = seq; J.D = D; J.B = B;
+    J.S = S; J.L = L; J.dense = dense; J.bmask = bmask; J.nbm = nbm; J.scale = scale;
+    J.n_planes = n_planes; J.planes = planes; J.nq = nq; J.qrows = qrows; J.nk = nk;
+    J.krows = krows; J.q_lo = q_lo; J.st_lse = st_lse; J.st_D = st_D;
+    J.kind = 4;
+    J.n_items = n_planes * grp * (seq - q_lo);
+    int rc = run_job(&J, nthreads);
+    if (rc == 0) {
+        J.kind = 5;
+        J.n_items = n_planes * (nq + nk);
+        rc = run_job(&J, nthreads);
+    }
+    free(st_lse);
+    free(st_D);
+    return rc;
 }
 
 /* Chunked-prefill oracle: each sequence s appends a chunk of

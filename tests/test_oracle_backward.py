@@ -118,3 +118,68 @@ def test_grouped_heads_sum_over_the_group(hkv):
     assert np.abs(dq - rq).max() < 1e-12
     assert np.abs(dk - rk.reshape(2, hkv, g, 24, 16).sum(2)).max() < 1e-12
     assert np.abs(dv - rv.reshape(2, hkv, g, 24, 16).sum(2)).max() < 1e-12
+
+
+def _sample(rng, grp, seq, nq, nk):
+    qr = rng.choice(grp * seq, nq, replace=False)
+    kr = rng.choice(seq, nk, replace=False)
+    return qr, kr
+
+
+@pytest.mark.parametrize("B,S,L,dense,seq,hkv,use_mask", [
+    (4, 4, 1, (), 32, 3, False), (8, 2, 2, (1,), 40, 3, False), (4, 3, 1, (), 30, 1, False),
+    (8, 3, 1, (), 48, 3, True)])
+def test_sampled_backward_equals_autograd_rows(B, S, L, dense, seq, hkv, use_mask):
+    """The sampled entry's rows against torch autograd of fp64 SDPA (grouped
+    heads by repeating K/V; a random block mask with an empty row)."""
+    H = 3
+    w, q, k, v, do = inputs(2, H, 16, seq, B, S, L, dense, seed=B + seq)
+    k, v = k[:, :hkv].contiguous(), v[:, :hkv].contiguous()
+    grp = H // hkv
+    nb = -(-seq // B)
+    if use_mask:
+        rng = np.random.default_rng(1)
+        bm = np.tril(rng.random((H, nb, nb)) < 0.5).astype(np.uint8)
+        for h in range(H):
+            bm[h, np.arange(nb), np.arange(nb)] = 1
+        tm = np.repeat(np.repeat(bm.astype(bool), B, 1), B, 2)[:, :seq, :seq] & np.tril(
+            np.ones((seq, seq), dtype=bool))[None]
+        kw = dict(bmask=bm)
+    else:
+        tm = token_mask_hhst(H, seq, B, S, L, dense)
+        kw = dict(S=S, L=L, dense_heads=dense)
+    rq, rk, rv = sdpa_grads(q, k.repeat_interleave(grp, 1), v.repeat_interleave(grp, 1), do, tm[None],
+                            w.scale)
+    rk = rk.reshape(2, hkv, grp, seq, 16).sum(2)
+    rv = rv.reshape(2, hkv, grp, seq, 16).sum(2)
+    rng = np.random.default_rng(seq)
+    planes = [0, 2 * hkv - 1] if hkv > 1 else [1]
+    qr, kr = _sample(rng, grp, seq, 7, 6)
+    kr[0] = 0  # the first key (seen by every later row that lists its block)
+    dq, dk, dv = oracle.backward_sampled(q, k, v, do, B, w.scale, planes, qr, kr, **kw)
+    for n, e in enumerate(planes):
+        b, g = divmod(e, hkv)
+        for r, row in enumerate(qr):
+            hh, t = divmod(int(row), seq)
+            assert np.abs(dq[n, r] - rq[b, g * grp + hh, t]).max() < 1e-11
+        assert np.abs(dk[n] - rk[b, g, kr]).max() < 1e-11
+        assert np.abs(dv[n] - rv[b, g, kr]).max() < 1e-11
+
+
+def test_sampled_backward_equals_full_backward_rows():
+    """Same numbers as the full backward's rows (one head per group: query rows
+    are positions of the plane's own head)."""
+    w, q, k, v, do = inputs(2, 4, 32, 64, 8, 4, 2, (2,), seed=9)
+    full = oracle.backward(q, k, v, do, 8, w.scale, S=4, L=2, dense_heads=(2,))
+    planes = [1, 2, 4, 7]
+    qr = np.array([0, 17, 40, 63])
+    kr = np.array([5, 31, 63])
+    dq, dk, dv = oracle.backward_sampled(q, k, v, do, 8, w.scale, planes, qr, kr, S=4, L=2,
+                                         dense_heads=(2,))
+    for n, e in enumerate(planes):
+        b, h = divmod(e, 4)
+        assert np.abs(dq[n] - full[0][b, h, qr]).max() < 1e-12
+        assert np.abs(dk[n] - full[1][b, h, kr]).max() < 1e-12
+        assert np.abs(dv[n] - full[2][b, h, kr]).max() < 1e-12
+    with pytest.raises(ValueError):  # a query row outside the group's heads
+        oracle.backward_sampled(q, k, v, do, 8, w.scale, planes, [64], kr, S=4, L=2)
