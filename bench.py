@@ -2,23 +2,25 @@
 """Benchmark of the HHST sparse-attention hot path on B200.
 
 One step = one pass of the whole path over one batch of synthetic input:
-  * prefill (block-sparse attention, tcgen05 kernel) over the 1.3B-shaped
-    layer batch: batch 4, 16 heads, head_dim 128, seq 8192, B 64, S 8, L 2,
-    per-head K scale U(0.5, 2);
-  * decode (split-KV paged kernel + combine) over 64 sequences, 32 heads,
-    head_dim 128, contexts U[4096, 32768], 16-token pages, permuted block table,
-    B 128, S 16, L 4.
-The layouts are built once (host, per layout) before timing. After the W
-warm-up steps, untimed steps run for --settle-s seconds: the GPU reaches its
-power cap within ~0.1 s of sustained load, and the timed region is divided
-by the sustained tensor peak, so it is timed in that same state.
+  * prefill (block-sparse attention, tcgen05 kernel) over the long-context
+    workload: batch 1, 32 heads, head_dim 128, seq 131072, B 128, S 16, L 4,
+    one planted key row per head (the largest single-GPU prefill);
+  * decode (split-KV paged kernel, plus the combine when it splits) over 64
+    sequences, 32 heads, head_dim 128, contexts U[4096, 32768], 16-token pages,
+    permuted block table, B 128, S 16, L 4.
+The layouts are built once (host, per layout) before timing.
 
 Headline: prefill effective TFLOP/s (4 * head_dim per visible (query, key)
 pair; the dense work the pattern skips is not counted), from CUDA events around
 the prefill launches inside the timed steps. The decode part reports active
-K+V GB/s and tokens/s in "decode". Multi-GPU: one process per GPU, each
-processing its own batch (weak scaling, no collective on the data path);
-time = max over ranks.
+K+V GB/s and tokens/s in "decode". The other prefill workloads (1.3B-shaped,
+7B hybrid), the backward and the chunked prefill are timed as separate legs,
+each with its own roofline. Tensor-bound fractions divide by the measured
+burst bf16 peak (cuBLAS, MEASURED_PEAKS.json "bf16_tflops"); the sampled SM
+clocks of each timed region are reported beside it.
+
+Multi-GPU: one process per GPU, each processing its own batch (weak scaling,
+no collective on the data path); time = max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -27,7 +29,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import sys
@@ -41,6 +42,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "HHST sparse attn fwd effective TFLOP/s & % bf16 TC peak; decode KV GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HEADLINE = "prefill_long_131k"
 
 
 def log(*a):
@@ -122,6 +124,20 @@ def chunk_flops(lay, w, ctx_lens, qlens) -> int:
     return 4 * w.head_dim * pairs
 
 
+def plant_positions(w, last_row_blocks, seed=7):
+    """For every head, a token of a key block j <= nb/2 that the last query
+    block lists (a strided block: the local window sits at the end), seeded.
+    ``last_row_blocks[h]`` is the key-block list of (head h, last query block)."""
+    rng = np.random.default_rng(seed)
+    nb = w.num_blocks
+    pos = {}
+    for h in range(w.heads):
+        cands = [int(j) for j in last_row_blocks[h] if int(j) <= nb // 2]
+        j = int(rng.choice(cands))
+        pos[h] = j * w.block + int(rng.integers(w.block))
+    return pos
+
+
 # Sources each kernel is compiled from (its ncu traffic figure stays valid while
 # these files are unchanged).
 KERNEL_SOURCES = {
@@ -139,35 +155,6 @@ def source_sha(kernel: str) -> str:
         h.update(fn.encode())
         h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
-
-
-def settle(fn, seconds, dist, device, sync=None):
-    """Run fn (one untimed step) until `seconds` of wall time have passed, in
-    batches with a device sync after each, so that the clocks and power state
-    seen by the timed region are the sustained ones. Ranks agree on the count
-    (max over ranks), so every rank runs the same number of steps. Returns it."""
-    import torch
-
-    if sync is None:
-        def sync():
-            torch.cuda.synchronize(device)
-    if seconds <= 0:
-        return 0
-    n, batch, t0 = 0, 4, time.time()
-    while time.time() - t0 < seconds:
-        for _ in range(batch):
-            fn()
-        n += batch
-        sync()
-        batch = min(batch * 2, 256)
-    if dist is not None:
-        t = torch.tensor([n], dtype=torch.int64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        for _ in range(int(t.item()) - n):
-            fn()
-        n = int(t.item())
-        sync()
-    return n
 
 
 def max_over_ranks(vals, dist, device):
@@ -201,6 +188,12 @@ def load_traffic(kernel: str, workload: str):
     if not e or e.get("source_sha") != source_sha(kernel):
         return None
     return e.get("dram_bytes_per_launch")
+
+
+def roofline(kernel, bound, achieved, peak, unit, traffic, peak_source):
+    return {"kernel": kernel, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+            "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": peak_source}
 
 
 # ---------------------------------------------------------------- clocks
@@ -277,6 +270,62 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 
+class Timer:
+    """CUDA events on the launching stream around a block of calls, between
+    a barrier (multi-rank) and device synchronisations; wall-clock bounds for
+    the clock samples."""
+
+    def __init__(self, stream, dist):
+        self.stream, self.dist = stream, dist
+
+    def run(self, fn, n):
+        import torch
+
+        if self.dist:
+            self.dist.barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_on = time.time()
+        a.record(self.stream)
+        for _ in range(n):
+            fn()
+        b.record(self.stream)
+        torch.cuda.synchronize()
+        t_off = time.time()
+        if self.dist:
+            self.dist.barrier()
+        return a.elapsed_time(b), (t_on, t_off)
+
+
+def check_flags(s2attn, what):
+    rc, flags = s2attn.device_status(reset=True)
+    if rc != 0:
+        raise RuntimeError(f"device flags {flags:#x} after {what}")
+
+
+def make_prefill(wp, dev, s2attn, synth):
+    """Inputs (resident), layout and work counts of one prefill workload."""
+    lay = s2attn.build_layout(wp.heads, wp.block, wp.stride, wp.local, wp.num_blocks,
+                              wp.dense_heads, device=dev)
+    plant = None
+    if wp.planted:
+        plant = plant_positions(wp, [lay.row(h, wp.num_blocks - 1) for h in range(wp.heads)])
+    q, k, v = synth.prefill_inputs(wp, device=dev, plant_positions=plant)
+    return dict(w=wp, q=q, k=k, v=v, lay=lay, flops=prefill_flops(lay, wp),
+                issued=prefill_issued_flops(lay, wp), mma=prefill_mma_flops(lay, wp), plant=plant)
+
+
+def prefill_config(P, ms_per_call):
+    wp = P["w"]
+    return {"batch": wp.batch, "heads": wp.heads, "head_dim": wp.head_dim, "seq": wp.seq,
+            "block": wp.block, "stride": wp.stride, "local": wp.local,
+            "dense_heads": list(wp.dense_heads), "planted_keys": P["plant"] is not None,
+            "algorithmic_gflop_per_call": round(P["flops"] / 1e9, 3),
+            "issued_gflop_per_call": round(P["issued"] / 1e9, 3),
+            "mma_gflop_per_call": round(P["mma"] / 1e9, 3),
+            "ms_per_call": round(ms_per_call, 4)}
+
+
 def run_ours(args, rank, world, dist):
     import torch
 
@@ -285,24 +334,29 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     s2attn.load()
-    wp = synth.PREFILL_WORKLOADS[args.prefill]
-    wd = synth.DECODE_WORKLOADS[args.decode] if args.decode != "none" else None
-    if wd is not None and args.decode_batch > 0:
-        wd = wd.with_(batch=args.decode_batch)
+    peaks, peak_src = load_peaks()
+    tc_peak = float(peaks["bf16_tflops"])
+    tc_src = f"{peak_src} bf16_tflops (burst cuBLAS bf16 GEMM)"
+    hbm = float(peaks["hbm_gbs"])
+    stream = torch.cuda.current_stream(dev)
+    timer = Timer(stream, dist)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
 
     # setup (untimed): inputs resident in HBM, layouts built once per layout
     t0 = time.time()
-    q, k, v = synth.prefill_inputs(wp, device=dev)
-    lay_p = s2attn.build_layout(wp.heads, wp.block, wp.stride, wp.local, wp.num_blocks,
-                                wp.dense_heads, device=dev)
-    layout_ms = None
+    wp = synth.PREFILL_WORKLOADS[args.prefill]
+    P = make_prefill(wp, dev, s2attn, synth)
+    q, k, v, lay_p = P["q"], P["k"], P["v"], P["lay"]
     t1 = time.time()
-    _ = s2attn.build_layout(wp.heads, wp.block, wp.stride, wp.local, wp.num_blocks, wp.dense_heads)
+    s2attn.build_layout(wp.heads, wp.block, wp.stride, wp.local, wp.num_blocks, wp.dense_heads)
     layout_ms = (time.time() - t1) * 1e3
     out = torch.empty_like(q)
-    flops = prefill_flops(lay_p, wp)
-    issued = prefill_issued_flops(lay_p, wp)
-    mma = prefill_mma_flops(lay_p, wp)
+    flops = P["flops"]
+    wd = synth.DECODE_WORKLOADS[args.decode] if args.decode != "none" else None
+    if wd is not None and args.decode_batch > 0:
+        wd = wd.with_(batch=args.decode_batch)
+    splits = 0
     if wd is not None:
         d = synth.decode_inputs(wd, device=dev)
         nb_d = -(-wd.ctx_max // wd.block)
@@ -320,8 +374,6 @@ def run_ours(args, rank, world, dist):
     log(f"[rank {rank}] setup {time.time() - t0:.1f}s; prefill {flops / 1e9:.1f} GFLOP/step"
         + (f"; decode {kv_bytes / 1e9:.3f} GB active KV, splits {splits}" if wd else ""))
 
-    stream = torch.cuda.current_stream(dev)
-
     def step(evs=None):
         if evs:
             evs[0].record(stream)
@@ -334,164 +386,144 @@ def run_ours(args, rank, world, dist):
         if evs:
             evs[2].record(stream)
 
-    sampler = ClockSampler(dev.index)
-    sampler.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    settle_steps = settle(step, args.settle_s, dist, dev)
-    rc, flags = s2attn.device_status(reset=True)
-    if rc != 0:
-        raise RuntimeError(f"device flags {flags:#x} after warm-up")
+    check_flags(s2attn, "warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    t_on = time.time()
-    start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    end.record(stream)
-    torch.cuda.synchronize()
-    t_off = time.time()
-    if dist:
-        dist.barrier()
-    total_ms = start.elapsed_time(end)
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    it = iter(evs)
+    total_ms, (t_on, t_off) = timer.run(lambda: step(next(it)), K)
     pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs) if wd else 0.0
-    rc, flags = s2attn.device_status(reset=True)
-    if rc != 0:
-        raise RuntimeError(f"device flags {flags:#x} after timing")
+    check_flags(s2attn, "timing")
+    clocks = sampler.summary(t_on, t_off)
 
     # ---------------- end to end through the public API with host buffers
     # Prefill leg, pipelined like a serving loop: every step copies its Q, K, V
     # from pinned host memory and reads its output back, on two copy streams
     # with double-buffered device tensors, so step i+1's uploads overlap step
     # i's prefill and download. Decode leg: one stream, step after step.
-    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, args.e2e_steps))
-    hq = q.cpu().pin_memory()
-    hk = k.cpu().pin_memory()
-    hv = v.cpu().pin_memory()
-    hout = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
-    gq = [torch.empty_like(q) for _ in range(2)]
-    gk = [torch.empty_like(k) for _ in range(2)]
-    gv = [torch.empty_like(v) for _ in range(2)]
-    gout = [torch.empty_like(out) for _ in range(2)]
+    e2e_steps = 0 if args.no_e2e else max(1, min(K, args.e2e_steps))
+    e2e_pre_ms = e2e_dec_ms = 0.0
     h2d_pre = 3 * q.numel() * q.element_size()
     d2h_pre = out.numel() * out.element_size()
-    s_up, s_down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    ev_up = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_free = [torch.cuda.Event() for _ in range(2)]  # the slot's D2H (so also its prefill) is done
-    if wd is not None:
-        hdq = d.q.cpu().pin_memory()
-        hbt = d.block_table.cpu().pin_memory()
-        hcl = d.ctx_lens.cpu().pin_memory()
-        hdout = torch.empty(d.q.shape, dtype=d.q.dtype).pin_memory()
-        gdq, gbt, gcl = torch.empty_like(d.q), torch.empty_like(d.block_table), torch.empty_like(d.ctx_lens)
-        h2d_dec = sum(t.numel() * t.element_size() for t in (hdq, hbt, hcl))
-        d2h_dec = hdout.numel() * hdout.element_size()
-
-    def e2e_prefill(i):
-        b = i & 1
-        with torch.cuda.stream(s_up):
-            if i >= 2:
-                s_up.wait_event(ev_free[b])
-            gq[b].copy_(hq, non_blocking=True)
-            gk[b].copy_(hk, non_blocking=True)
-            gv[b].copy_(hv, non_blocking=True)
-            ev_up[b].record(s_up)
-        stream.wait_event(ev_up[b])
-        s2attn.prefill(gq[b], gk[b], gv[b], lay_p, scale=wp.scale, out=gout[b])
-        ev_done[b].record(stream)
-        with torch.cuda.stream(s_down):
-            s_down.wait_event(ev_done[b])
-            hout[b].copy_(gout[b], non_blocking=True)
-            ev_free[b].record(s_down)
-
-    def e2e_decode(ev):
-        ev[0].record(stream)
-        gdq.copy_(hdq, non_blocking=True)
-        gbt.copy_(hbt, non_blocking=True)
-        gcl.copy_(hcl, non_blocking=True)
-        s2attn.decode(gdq, d.k_cache, d.v_cache, gbt, gcl, lay_d, scale=wd.scale,
-                      num_splits=splits, out=dout, workspace=ws)
-        hdout.copy_(dout, non_blocking=True)
-        ev[1].record(stream)
-
-    e2e_pre_ms = e2e_dec_ms = 0.0
+    hq = hk = hv = None
+    if e2e_steps or (world == 1 and not args.no_cpu_baseline):
+        hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
     if e2e_steps:
+        hout = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
+        gq = [q, torch.empty_like(q)]
+        gk = [k, torch.empty_like(k)]
+        gv = [v, torch.empty_like(v)]
+        gout = [torch.empty_like(out) for _ in range(2)]
+        s_up, s_down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_up = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_free = [torch.cuda.Event() for _ in range(2)]  # the slot's D2H (so also its prefill) is done
+
+        def e2e_prefill(i):
+            b = i & 1
+            with torch.cuda.stream(s_up):
+                if i >= 2:
+                    s_up.wait_event(ev_free[b])
+                gq[b].copy_(hq, non_blocking=True)
+                gk[b].copy_(hk, non_blocking=True)
+                gv[b].copy_(hv, non_blocking=True)
+                ev_up[b].record(s_up)
+            stream.wait_event(ev_up[b])
+            s2attn.prefill(gq[b], gk[b], gv[b], lay_p, scale=wp.scale, out=gout[b])
+            ev_done[b].record(stream)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(ev_done[b])
+                hout[b].copy_(gout[b], non_blocking=True)
+                ev_free[b].record(s_down)
+
         for i in range(2):  # warm-up: both slots once
             e2e_prefill(i)
         torch.cuda.synchronize()
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ta, tb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if dist:
             dist.barrier()
-        t0.record(s_up)
+        ta.record(s_up)
         for i in range(e2e_steps):
             e2e_prefill(i)
-        t1.record(s_down)
+        tb.record(s_down)
         torch.cuda.synchronize()
-        e2e_pre_ms = t0.elapsed_time(t1)
+        e2e_pre_ms = ta.elapsed_time(tb)
         assert torch.equal(hout[(e2e_steps - 1) & 1], out.cpu()), "e2e output differs from the device output"
+        del hout, gout, gq[1], gk[1], gv[1]
         if wd is not None:
-            e2e_decode([torch.cuda.Event(enable_timing=True) for _ in range(2)])
-            torch.cuda.synchronize()
-            eevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
-            if dist:
-                dist.barrier()
-            for i in range(e2e_steps):
-                e2e_decode(eevs[i])
-            torch.cuda.synchronize()
-            e2e_dec_ms = sum(e[0].elapsed_time(e[1]) for e in eevs)
+            hdq = d.q.cpu().pin_memory()
+            hbt = d.block_table.cpu().pin_memory()
+            hcl = d.ctx_lens.cpu().pin_memory()
+            hdout = torch.empty(d.q.shape, dtype=d.q.dtype).pin_memory()
+            gdq, gbt, gcl = torch.empty_like(d.q), torch.empty_like(d.block_table), torch.empty_like(d.ctx_lens)
+            h2d_dec = sum(t.numel() * t.element_size() for t in (hdq, hbt, hcl))
+            d2h_dec = hdout.numel() * hdout.element_size()
 
-    # ---------------- backward (dQ, dK, dV) of a prefill workload, timed on its own
-    bwd_ms, bwd_steps, bwd_info = 0.0, 0, None
-    if args.backward != "none":
-        wb = wp if args.backward == "same" else synth.PREFILL_WORKLOADS[args.backward]
-        if wb is wp:
-            bq, bk_, bv, lay_b = q, k, v, lay_p
-        else:
-            bq, bk_, bv = synth.prefill_inputs(wb, device=dev)
-            lay_b = s2attn.build_layout(wb.heads, wb.block, wb.stride, wb.local, wb.num_blocks,
-                                        wb.dense_heads, device=dev)
+            def e2e_decode():
+                gdq.copy_(hdq, non_blocking=True)
+                gbt.copy_(hbt, non_blocking=True)
+                gcl.copy_(hcl, non_blocking=True)
+                s2attn.decode(gdq, d.k_cache, d.v_cache, gbt, gcl, lay_d, scale=wd.scale,
+                              num_splits=splits, out=dout, workspace=ws)
+                hdout.copy_(dout, non_blocking=True)
+
+            e2e_decode()
+            e2e_dec_ms, _ = timer.run(e2e_decode, e2e_steps)
+    if wd is not None:
+        del d, ws  # free the 21 GB cache before the legs
+    torch.cuda.empty_cache()
+
+    # ---------------- other prefill workloads, each timed on its own
+    legs = []
+    for name in [x for x in args.legs.split(",") if x and x != "none" and x != args.prefill]:
+        L = make_prefill(synth.PREFILL_WORKLOADS[name], dev, s2attn, synth)
+        lout = torch.empty_like(L["q"])
+
+        def call(L=L, lout=lout):
+            s2attn.prefill(L["q"], L["k"], L["v"], L["lay"], scale=L["w"].scale, out=lout)
+
+        for _ in range(3):
+            call()
+        n = max(3, int(args.leg_ms / max(1e-3, L["flops"] / 1e12)))  # ~leg_ms at 1 PFLOP/s
+        ms, win = timer.run(call, n)
+        check_flags(s2attn, f"the {name} leg")
+        legs.append((L, n, ms, sampler.summary(*win)))
+        del L, lout
+        torch.cuda.empty_cache()
+
+    # ---------------- backward (dQ, dK, dV), each workload timed on its own
+    bwds = []
+    for name in [x for x in args.backward.split(",") if x and x != "none"]:
+        wb = synth.PREFILL_WORKLOADS[name]
+        Bk = make_prefill(wb, dev, s2attn, synth) if name != args.prefill else P
+        lay_b = Bk["lay"]
         lay_b.transposed(dev)
-        bo, blse = s2attn.prefill(bq, bk_, bv, lay_b, scale=wb.scale, want_lse=True)
+        bo, blse = s2attn.prefill(Bk["q"], Bk["k"], Bk["v"], lay_b, scale=wb.scale, want_lse=True)
         gen = torch.Generator(device=dev).manual_seed(77)
-        bdo = torch.randn(bq.shape, generator=gen, device=dev).to(torch.bfloat16)
-        bdq, bdk, bdv = torch.empty_like(bq), torch.empty_like(bk_), torch.empty_like(bv)
+        bdo = torch.randn(Bk["q"].shape, generator=gen, device=dev).to(torch.bfloat16)
+        bdq, bdk, bdv = torch.empty_like(Bk["q"]), torch.empty_like(Bk["k"]), torch.empty_like(Bk["v"])
         bws = torch.empty(s2attn.backward_workspace_size(wb.batch, wb.heads, wb.seq),
                           dtype=torch.uint8, device=dev)
 
-        def bwd():
-            s2attn.backward(bq, bk_, bv, bo, blse, bdo, lay_b, scale=wb.scale, dq=bdq, dk=bdk,
-                            dv=bdv, workspace=bws)
+        def bwd(Bk=Bk, bo=bo, blse=blse, bdo=bdo, bdq=bdq, bdk=bdk, bdv=bdv, bws=bws, wb=wb):
+            s2attn.backward(Bk["q"], Bk["k"], Bk["v"], bo, blse, bdo, Bk["lay"], scale=wb.scale,
+                            dq=bdq, dk=bdk, dv=bdv, workspace=bws)
 
         for _ in range(3):
             bwd()
-        torch.cuda.synchronize()
-        settle(bwd, args.settle_s / 3, dist, dev)
-        bwd_steps = max(3, min(args.steps, args.bwd_steps))
-        bev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        if dist:
-            dist.barrier()
-        bev[0].record(stream)
-        for _ in range(bwd_steps):
-            bwd()
-        bev[1].record(stream)
-        torch.cuda.synchronize()
-        bwd_ms = bev[0].elapsed_time(bev[1])
-        rc, flags = s2attn.device_status(reset=True)
-        if rc != 0:
-            raise RuntimeError(f"device flags {flags:#x} after the backward")
-        bflops = prefill_flops(lay_b, wb)
-        bwd_info = (wb, bflops, prefill_issued_flops(lay_b, wb))
+        n = max(3, int(args.leg_ms / max(1e-3, 2.5 * Bk["flops"] / 0.5e12)))  # at 0.5 PFLOP/s
+        ms, win = timer.run(bwd, n)
+        check_flags(s2attn, f"the {name} backward")
+        bwds.append((Bk, n, ms, sampler.summary(*win)))
+        del bo, blse, bdo, bdq, bdk, bdv, bws, Bk
+        torch.cuda.empty_cache()
 
     # ---------------- chunked prefill over the paged cache, timed on its own
-    chunk_ms, chunk_steps, chunk_info = 0.0, 0, None
+    chunk = None
     if args.chunk != "none":
         wc = synth.CHUNK_WORKLOADS[args.chunk]
         ci = synth.chunk_inputs(wc, synth.CHUNK_LEN[wc.name], device=dev)
@@ -506,83 +538,58 @@ def run_ours(args, rank, world, dist):
 
         for _ in range(3):
             chunk_call()
-        torch.cuda.synchronize()
-        settle(chunk_call, args.settle_s / 3, dist, dev)
-        chunk_steps = max(3, min(args.steps, args.bwd_steps))
-        cev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        if dist:
-            dist.barrier()
-        cev[0].record(stream)
-        for _ in range(chunk_steps):
-            chunk_call()
-        cev[1].record(stream)
-        torch.cuda.synchronize()
-        chunk_ms = cev[0].elapsed_time(cev[1])
-        rc, flags = s2attn.device_status(reset=True)
-        if rc != 0:
-            raise RuntimeError(f"device flags {flags:#x} after the chunked prefill")
         ctx_h = ci.ctx_lens.cpu().tolist()
         qs = ci.q_start.cpu().tolist()
         qlens = [qs[i + 1] - qs[i] for i in range(len(ctx_h))]
-        chunk_info = (wc, chunk_flops(lay_c, wc, ctx_h, qlens), sum(qlens))
+        cflops = chunk_flops(lay_c, wc, ctx_h, qlens)
+        n = max(3, int(args.leg_ms / max(1e-3, cflops / 0.7e12)))  # at 0.7 PFLOP/s
+        ms, win = timer.run(chunk_call, n)
+        check_flags(s2attn, "the chunked prefill")
+        chunk = (wc, cflops, sum(qlens), n, ms, sampler.summary(*win))
         del ci, cout
 
     # ---------------- max over ranks
-    vals = [total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms, chunk_ms]
+    vals = [total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms] + [x[2] for x in legs] + \
+        [x[2] for x in bwds] + ([chunk[4]] if chunk else [])
     vals = max_over_ranks(vals, dist, dev)
-    total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms, bwd_ms, chunk_ms = vals
+    total_ms, pre_ms, dec_ms, e2e_pre_ms, e2e_dec_ms = vals[:5]
+    rest = vals[5:]
+    legs = [(L, n, rest.pop(0), c) for (L, n, _, c) in legs]
+    bwds = [(B_, n, rest.pop(0), c) for (B_, n, _, c) in bwds]
+    if chunk:
+        chunk = chunk[:4] + (rest.pop(0), chunk[5])
     sampler.stop()
-    clocks = sampler.summary(t_on, t_off)
     if rank != 0:
         return None
 
-    peaks, peak_src = load_peaks()
-    K = args.steps
-    tc_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-    pre_tflops = world * flops * K / (pre_ms * 1e-3) / 1e12
-    per_launch_tflops = flops / (pre_ms / K * 1e-3) / 1e12
+    per_launch = flops / (pre_ms / K * 1e-3) / 1e12
     launches = K * (1 + ((1 + (1 if splits > 1 else 0)) if wd else 0))
-    splits = splits if wd else 0
     line = {
         "metric": METRIC,
-        "value": round(pre_tflops, 2),
+        "value": round(world * flops * K / (pre_ms * 1e-3) / 1e12, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": K,
         "warmup": args.warmup,
-        "settle": {"steps": settle_steps, "seconds": args.settle_s,
-                   "why": "untimed steps after the warm-up until the GPU's power state has "
-                          "settled (sw_power_cap engages within ~0.1 s of sustained load), so "
-                          "the timed region matches the sustained peak it is divided by"},
         "ms_per_step": round(total_ms / K, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16, torch generator on device)",
+        "data": "synthetic (seeded N(0,1) bf16, torch generator on device; planted keys chosen "
+                "from the layout)",
         "config": {
-            "workload": f"{wp.name}+{wd.name}" if wd else wp.name,
-            "prefill": {"batch": wp.batch, "heads": wp.heads, "head_dim": wp.head_dim,
-                        "seq": wp.seq, "block": wp.block, "stride": wp.stride,
-                        "local": wp.local, "dense_heads": list(wp.dense_heads),
-                        "algorithmic_gflop_per_step": round(flops / 1e9, 3),
-                        "issued_gflop_per_step": round(issued / 1e9, 3),
-                        "mma_gflop_per_step": round(mma / 1e9, 3),
-                        "ms_per_step": round(pre_ms / K, 4)},
+            "workload": wp.name,
+            "step": f"{wp.name} prefill + {wd.name} decode" if wd else f"{wp.name} prefill",
+            "prefill": prefill_config(P, pre_ms / K),
             "layout_build_ms_host": round(layout_ms, 3),
-            "l2": "inputs larger than L2 (prefill Q+K+V 403 MB; decode active KV > 1.7 GB)",
+            "l2": "inputs larger than L2 (prefill Q+K+V 3.2 GB; decode active KV 1.7 GB of a "
+                  "21 GB cache)",
             "parallelism": f"replicas x{world} (no data-path collective)",
         },
-        "roofline": {
-            "kernel": f"s2_prefill_pair_kernel<{wp.head_dim},{wp.block}>",
-            "bound": "tensor",
-            "achieved": round(per_launch_tflops, 2),
-            "peak": tc_peak,
-            "unit": "TFLOP/s",
-            "frac": round(per_launch_tflops / tc_peak, 4),
-            "traffic": load_traffic("s2_prefill_pair_kernel", wp.name),
-            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long loop)",
-        },
+        "roofline": roofline(f"s2_prefill_pair_kernel<{wp.head_dim},{wp.block}>", "tensor", per_launch,
+                             tc_peak, "TFLOP/s", load_traffic("s2_prefill_pair_kernel", wp.name),
+                             tc_src),
         "e2e": None if not e2e_steps else {
             "value": round(world * flops * e2e_steps / (e2e_pre_ms * 1e-3) / 1e12, 3),
             "unit": "TFLOP/s",
@@ -598,11 +605,10 @@ def run_ours(args, rank, world, dist):
         "clocks": clocks,
     }
     if wd is not None:
-        dec_gbs = world * kv_bytes * K / (dec_ms * 1e-3) / 1e9
-        per_launch_gbs = kv_bytes / (dec_ms / K * 1e-3) / 1e9
-        hbm = float(peaks["hbm_gbs"])
+        per_gbs = kv_bytes / (dec_ms / K * 1e-3) / 1e9
         line["decode"] = {
-            "value": round(dec_gbs, 1), "unit": "GB/s",
+            "workload": wd.name,
+            "value": round(world * kv_bytes * K / (dec_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
             "tokens_per_s": round(world * wd.batch * K / (dec_ms * 1e-3), 1),
             "ms_per_step": round(dec_ms / K, 4),
             "active_kv_bytes_per_step": kv_bytes,
@@ -611,102 +617,116 @@ def run_ours(args, rank, world, dist):
             "config": {"batch": wd.batch, "heads": wd.heads, "head_dim": wd.head_dim,
                        "ctx": [wd.ctx_min, wd.ctx_max], "page": wd.page_size,
                        "block": wd.block, "stride": wd.stride, "local": wd.local},
-            "roofline": {"kernel": "s2_decode_split_kernel<128>" + (" + combine" if splits > 1 else ""),
-                         "bound": "hbm", "achieved": round(per_launch_gbs, 1), "peak": hbm,
-                         "unit": "GB/s", "frac": round(per_launch_gbs / hbm, 4),
-                         "traffic": load_traffic("s2_decode_split_kernel", wd.name),
-                         "peak_source": f"{peak_src} hbm_gbs"},
+            "roofline": roofline("s2_decode_split_kernel<128>" + (" + combine" if splits > 1 else ""),
+                                 "hbm", per_gbs, hbm, "GB/s",
+                                 load_traffic("s2_decode_split_kernel", wd.name), f"{peak_src} hbm_gbs"),
             "e2e": None if not e2e_steps else {
                 "value": round(world * kv_bytes * e2e_steps / (e2e_dec_ms * 1e-3) / 1e9, 1),
                 "unit": "GB/s", "h2d_bytes_per_step": h2d_dec, "d2h_bytes_per_step": d2h_dec},
         }
-    if bwd_info is not None:
-        wb, bflops, bissued = bwd_info
+    line["prefill_legs"] = []
+    for L, n, ms, c in legs:
+        w_ = L["w"]
+        per = L["flops"] / (ms / n * 1e-3) / 1e12
+        line["prefill_legs"].append({
+            "workload": w_.name, "value": round(world * per, 2), "unit": "TFLOP/s", "calls": n,
+            "config": prefill_config(L, ms / n),
+            "roofline": roofline(f"s2_prefill_pair_kernel<{w_.head_dim},{w_.block}>", "tensor", per,
+                                 tc_peak, "TFLOP/s", load_traffic("s2_prefill_pair_kernel", w_.name),
+                                 tc_src),
+            "clocks": c})
+    line["gpu_launches_legs"] = sum(n for _, n, _, _ in legs)
+    line["backward"] = []
+    for Bk, n, ms, c in bwds:
+        wb = Bk["w"]
         # dS needs S (recomputed), dP, and then dV, dK, dQ: 5 products of the
         # forward's 2, so 2.5x its FLOPs; S and dP are computed by both backward
         # kernels here, so 7 products are issued.
-        alg = 2.5 * bflops
-        per = alg / (bwd_ms / bwd_steps * 1e-3) / 1e12
-        line["backward"] = {
-            "value": round(world * alg * bwd_steps / (bwd_ms * 1e-3) / 1e12, 2),
-            "unit": "TFLOP/s",
-            "workload": wb.name,
-            "ms_per_call": round(bwd_ms / bwd_steps, 4),
-            "steps": bwd_steps,
+        alg = 2.5 * Bk["flops"]
+        per = alg / (ms / n * 1e-3) / 1e12
+        line["backward"].append({
+            "workload": wb.name, "value": round(world * per, 2), "unit": "TFLOP/s",
+            "ms_per_call": round(ms / n, 4), "calls": n,
             "algorithmic_gflop_per_call": round(alg / 1e9, 3),
-            "issued_gflop_per_call": round(3.5 * bissued / 1e9, 3),
+            "issued_gflop_per_call": round(3.5 * Bk["issued"] / 1e9, 3),
             "kernels": "s2_bwd_stats_kernel + s2_bwd_dq_kernel + s2_bwd_dkv_kernel",
-            "roofline": {"bound": "tensor", "achieved": round(per, 2), "peak": tc_peak,
-                         "unit": "TFLOP/s", "frac": round(per / tc_peak, 4),
-                         "traffic": load_traffic("s2_bwd", wb.name),
-                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
-        }
-        line["gpu_launches_backward"] = 3 * bwd_steps
-    if chunk_info is not None:
-        wc, cflops, total_q = chunk_info
-        per = cflops / (chunk_ms / chunk_steps * 1e-3) / 1e12
+            "roofline": roofline("backward (3 kernels)", "tensor", per, tc_peak, "TFLOP/s",
+                                 load_traffic("s2_bwd", wb.name), tc_src),
+            "clocks": c})
+    line["gpu_launches_backward"] = sum(3 * n for _, n, _, _ in bwds)
+    if chunk is not None:
+        wc, cflops, total_q, n, ms, c = chunk
+        per = cflops / (ms / n * 1e-3) / 1e12
         line["chunk"] = {
-            "value": round(world * cflops * chunk_steps / (chunk_ms * 1e-3) / 1e12, 2),
-            "unit": "TFLOP/s",
-            "workload": wc.name,
-            "ms_per_call": round(chunk_ms / chunk_steps, 4),
-            "steps": chunk_steps,
-            "chunk_rows": total_q,
+            "workload": wc.name, "value": round(world * per, 2), "unit": "TFLOP/s",
+            "ms_per_call": round(ms / n, 4), "calls": n, "chunk_rows": total_q,
             "algorithmic_gflop_per_call": round(cflops / 1e9, 3),
             "config": {"batch": wc.batch, "heads": wc.heads, "head_dim": wc.head_dim,
                        "ctx": [wc.ctx_min, wc.ctx_max], "chunk": synth.CHUNK_LEN[wc.name],
                        "page": wc.page_size, "block": wc.block, "stride": wc.stride,
                        "local": wc.local},
             "kernels": "s2_chunk_prefill_kernel",
-            "roofline": {"bound": "tensor", "achieved": round(per, 2), "peak": tc_peak,
-                         "unit": "TFLOP/s", "frac": round(per / tc_peak, 4),
-                         "traffic": load_traffic("s2_chunk_prefill_kernel", wc.name),
-                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
-        }
-        line["gpu_launches_chunk"] = chunk_steps
+            "roofline": roofline("s2_chunk_prefill_kernel<128,128>", "tensor", per, tc_peak, "TFLOP/s",
+                                 load_traffic("s2_chunk_prefill_kernel", wc.name), tc_src),
+            "clocks": c}
+        line["gpu_launches_chunk"] = n
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wp, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(wp, args.cpu_seconds, (hq, hk, hv), P["plant"], flops)
     return line
 
 
 # ---------------------------------------------------------------- oracle arm
 
-def oracle_sample(wp, n_rows, seed, q=None, k=None, v=None):
+def oracle_sample(wp, n_rows, seed, qkv):
     """Time the fp64 oracle on n_rows seeded random rows of the prefill workload.
     Returns (seconds, algorithmic flops of those rows, threads)."""
     import oracle
-    from head_heterogeneous_block_s2_b200 import synth
 
-    if q is None:
-        q, k, v = synth.prefill_inputs(wp)
+    q, k, v = qkv
     rng = np.random.default_rng(seed)
     total = wp.batch * wp.heads * wp.seq
     rows = np.sort(rng.choice(total, n_rows, replace=False)).astype(np.int64)
     # visible keys of each sampled row (the work the definition does)
-    mask = oracle.block_mask(wp.heads, wp.num_blocks, wp.stride, wp.local, wp.dense_heads)
+    cnt = oracle.block_mask(wp.heads, wp.num_blocks, wp.stride, wp.local,
+                            wp.dense_heads).sum(axis=2, dtype=np.int64)  # active blocks per row
     t = rows % wp.seq
     h = (rows // wp.seq) % wp.heads
     i = t // wp.block
-    full = mask[h, i, :].astype(np.int64)  # active blocks of each row
-    nfull = full.sum(1) - 1  # blocks before the diagonal
+    nfull = cnt[h, i] - 1  # active blocks before the diagonal
     keys = nfull * wp.block + (t % wp.block) + 1
     flops = int(4 * wp.head_dim * keys.sum())
     t0 = time.perf_counter()
     oracle.prefill(q, k, v, wp.block, wp.stride, wp.local, wp.scale, wp.dense_heads, rows=rows)
     dt = time.perf_counter() - t0
-    return dt, flops, oracle.default_threads(), (q, k, v)
+    return dt, flops, oracle.default_threads()
 
 
-def cpu_baseline(wp, seconds):
+def oracle_inputs(wp):
+    """The workload's inputs on the host (planted keys chosen with the oracle's
+    own block mask, which equals the layout's lists)."""
+    import oracle
+    from head_heterogeneous_block_s2_b200 import synth
+
+    plant = None
+    if wp.planted:
+        m = oracle.block_mask(wp.heads, wp.num_blocks, wp.stride, wp.local, wp.dense_heads)
+        plant = plant_positions(wp, [np.nonzero(m[h, wp.num_blocks - 1])[0] for h in range(wp.heads)])
+    return synth.prefill_inputs(wp, plant_positions=plant), plant
+
+
+def cpu_baseline(wp, seconds, qkv, plant, full):
     """The oracle as it stands, on the host cores, over a bounded row sample
-    calibrated to take about `seconds`."""
-    dt, fl, th, qkv = oracle_sample(wp, 512, 1)
-    n = int(min(wp.batch * wp.heads * wp.seq, max(512, 512 * seconds / max(dt, 1e-3))))
-    dt, fl, th, _ = oracle_sample(wp, n, 2, *qkv)
-    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": th, "kind": "oracle",
+    calibrated to take about `seconds`; the full workload's time is
+    extrapolated from the sample's rate (labelled as such)."""
+    dt, fl, th = oracle_sample(wp, 256, 1, qkv)
+    n = int(min(wp.batch * wp.heads * wp.seq, max(256, 256 * seconds / max(dt, 1e-3))))
+    dt, fl, th = oracle_sample(wp, n, 2, qkv)
+    rate = fl / dt
+    return {"value": round(rate / 1e12, 6), "unit": "TFLOP/s", "cores": th, "kind": "oracle",
             "sample": f"{n} seeded random query rows of {wp.name} "
-                      f"({n / (wp.batch * wp.heads * wp.seq):.2%} of the batch), fp64, "
-                      f"{dt:.1f} s on {th} threads"}
+                      f"({n / (wp.batch * wp.heads * wp.seq):.2%} of the batch"
+                      f"{', planted keys' if plant else ''}), fp64, {dt:.1f} s on {th} threads",
+            "full_workload_s_extrapolated": round(full / rate, 1)}
 
 
 def run_reference(args, rank):
@@ -715,15 +735,16 @@ def run_reference(args, rank):
     from head_heterogeneous_block_s2_b200 import synth
 
     wp = synth.PREFILL_WORKLOADS[args.prefill]
+    qkv, plant = oracle_inputs(wp)
     # calibrate rows per step so the whole run takes about args.ref_seconds
-    dt, fl, th, qkv = oracle_sample(wp, 256, 1)
+    dt, fl, th = oracle_sample(wp, 128, 1, qkv)
     per_step_s = args.ref_seconds / max(1, args.steps + args.warmup)
-    n = int(max(16, min(wp.batch * wp.heads * wp.seq, 256 * per_step_s / max(dt, 1e-4))))
+    n = int(max(16, min(wp.batch * wp.heads * wp.seq, 128 * per_step_s / max(dt, 1e-4))))
     for i in range(args.warmup):
-        oracle_sample(wp, n, 100 + i, *qkv)
+        oracle_sample(wp, n, 100 + i, qkv)
     tot_t = tot_f = 0.0
     for i in range(args.steps):
-        dt, fl, th, _ = oracle_sample(wp, n, 1000 + i, *qkv)
+        dt, fl, th = oracle_sample(wp, n, 1000 + i, qkv)
         tot_t += dt
         tot_f += fl
     val = tot_f / tot_t / 1e12
@@ -735,7 +756,8 @@ def run_reference(args, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wp.name, "rows_per_step": n},
         "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": th, "kind": "oracle",
-                         "sample": f"{n} seeded random query rows of {wp.name} per step"},
+                         "sample": f"{n} seeded random query rows of {wp.name} per step"
+                                   f"{' (planted keys)' if plant else ''}"},
         "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -744,27 +766,27 @@ def run_reference(args, rank):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--settle-s", type=float, default=1.5,
-                    help="untimed steps after the warm-up until this many seconds have passed "
-                         "(the power state settles; the backward and chunk legs take a third each)")
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--prefill", default="prefill_1p3b",
-                    choices=["tiny", "prefill_1p3b", "prefill_7b_hybrid", "prefill_long_131k"])
+    ap.add_argument("--prefill", default=HEADLINE,
+                    choices=["tiny", "prefill_1p3b", "prefill_7b_hybrid", "prefill_long_131k"],
+                    help="the step's prefill workload (the headline)")
     ap.add_argument("--decode", default="decode_paged", choices=["decode_paged", "none"])
     ap.add_argument("--splits", type=int, default=0, help="decode splits (0 = automatic)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="override the decode batch (small cases for profiling only)")
+    ap.add_argument("--legs", default="prefill_1p3b,prefill_7b_hybrid",
+                    help="other prefill workloads, each timed on its own ('none' = skip)")
+    ap.add_argument("--leg-ms", type=float, default=150.0,
+                    help="approximate GPU time of each separately timed leg")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling only)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--backward", default="same",
-                    help="prefill workload whose backward is timed separately ('same' = the "
-                         "prefill workload, 'none' = skip)")
-    ap.add_argument("--bwd-steps", type=int, default=20)
+    ap.add_argument("--backward", default="prefill_1p3b,prefill_7b_hybrid",
+                    help="prefill workloads whose backward is timed separately ('none' = skip)")
     ap.add_argument("--chunk", default="chunk_paged", choices=["chunk_paged", "none"],
                     help="chunked prefill over the paged cache, timed separately")
     args = ap.parse_args()

@@ -80,8 +80,9 @@ struct BackwardParams {
     float scale_log2;  // scale * log2 e
     uint64_t timeout_ns;
     uint32_t* gflags;
-    int* sched;     // dQ kernel work counter {next item, CTAs done}, zero at launch
+    int* sched;     // dQ kernel work-counter slot (sched_claim / sched_take / sched_leave)
     int* sched_kv;  // the same for the persistent dK/dV kernel (64-key blocks)
+    int sched_id, sched_kv_id;  // the two launches' nonzero ids
 };
 
 // Descriptor offset (16-byte units) of k-step kk (16 elements) of a K-major
@@ -267,6 +268,7 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mbar_init(bar_le(b), C::LIST_CONSUMERS);
         }
         *abort_cta = 0;
+        misc[6] = sched_claim(p.sched, p.sched_id, WaitCtl{p.timeout_ns, p.gflags, abort_cta});
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -296,7 +298,7 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     mbar_arrive(bar_lf(b));
                     break;
                 }
-                const int w_next = (int)gridDim.x + atomicAdd(p.sched, 1);
+                const int w_next = misc[6] ? (int)gridDim.x + sched_take(p.sched) : num_items;
                 const int qt = item_qt(w), bh = item_bh(w), h = bh % p.heads;
                 UnionWalk<C::ROWS> it;
                 int len = 0;
@@ -603,16 +605,8 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    if (threadIdx.x == 0) {
-        // The last CTA to finish resets the counter for the next launch on this slot
-        // (every CTA has stopped taking items by now).
-        __threadfence();
-        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
-            atomicExch(p.sched, 0);
-            atomicExch(p.sched + 1, 0);
-            __threadfence();
-        }
-    }
+    // every CTA has stopped taking items by now; the last one frees the slot
+    if (threadIdx.x == 0 && misc[6]) sched_leave(p.sched);
 }
 
 // ------------------------------------------------------------------ dK, dV
@@ -1083,6 +1077,7 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
             mbar_init(bar_le(b), C::LIST_CONSUMERS);
         }
         *abort_cta = 0;
+        misc[6] = sched_claim(p.sched_kv, p.sched_kv_id, WaitCtl{p.timeout_ns, p.gflags, abort_cta});
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -1115,7 +1110,7 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
                 break;
             }
             int w_next = 0;
-            if (lane == 0) w_next = (int)gridDim.x + atomicAdd(p.sched_kv, 1);
+            if (lane == 0) w_next = misc[6] ? (int)gridDim.x + sched_take(p.sched_kv) : num_items;
             w_next = __shfl_sync(0xffffffffu, w_next, 0);
             const KvItem it = kv_item(p, w);
             int kb[C::ROWS];
@@ -1409,16 +1404,8 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    if (threadIdx.x == 0) {
-        // The last CTA to finish resets the counter for the next launch on this slot
-        // (every CTA has stopped taking items by now).
-        __threadfence();
-        if (atomicAdd(p.sched_kv + 1, 1) == (int)gridDim.x - 1) {
-            atomicExch(p.sched_kv, 0);
-            atomicExch(p.sched_kv + 1, 0);
-            __threadfence();
-        }
-    }
+    // every CTA has stopped taking items by now; the last one frees the slot
+    if (threadIdx.x == 0 && misc[6]) sched_leave(p.sched_kv);
 }
 
 }  // namespace s2

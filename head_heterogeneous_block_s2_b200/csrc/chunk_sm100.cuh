@@ -59,7 +59,8 @@ struct ChunkParams {
     float scale_log2;
     uint64_t timeout_ns;
     uint32_t* gflags;
-    int* sched;                  // work counter {next item, CTAs done}, zero at launch
+    int* sched;                  // work-counter slot (sched_claim / sched_take / sched_leave)
+    int sched_id;                // this launch's nonzero id
 };
 
 constexpr int kChunkPage = 16;  // tokens per cache page
@@ -221,6 +222,7 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         }
         mbar_init(bar_dr, 1);
         *abort_cta = 0;
+        misc[6] = sched_claim(p.sched, p.sched_id, WaitCtl{p.timeout_ns, p.gflags, abort_cta});
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -264,7 +266,7 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 break;
             }
             int64_t w_next = 0;
-            if (lane == 0) w_next = (int64_t)gridDim.x + atomicAdd(p.sched, 1);
+            if (lane == 0) w_next = misc[6] ? (int64_t)gridDim.x + sched_take(p.sched) : num_items;
             w_next = __shfl_sync(0xffffffffu, w_next, 0);
             if (lane == 0) {
                 // the item's query blocks, without those wholly before the chunk or
@@ -653,16 +655,8 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    if (threadIdx.x == 0) {
-        // The last CTA to finish resets the counter for the next launch on this slot
-        // (every CTA has stopped taking items by now).
-        __threadfence();
-        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
-            atomicExch(p.sched, 0);
-            atomicExch(p.sched + 1, 0);
-            __threadfence();
-        }
-    }
+    // every CTA has stopped taking items by now; the last one frees the slot
+    if (threadIdx.x == 0 && misc[6]) sched_leave(p.sched);
 }
 
 }  // namespace s2

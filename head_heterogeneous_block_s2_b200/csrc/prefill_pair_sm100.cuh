@@ -244,6 +244,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
         for (int i = 0; i < 4; ++i) mbar_init(bar_dr + 8u * i, 1);
         *abort_cta = 0;
+        misc[6] = sched_claim(p.sched, p.sched_id, WaitCtl{p.timeout_ns, p.gflags, abort_cta});
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -273,7 +274,7 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     mbar_arrive(bar_lf(b));
                     break;
                 }
-                const int w_next = (int)gridDim.x + atomicAdd(p.sched, 1);
+                const int w_next = misc[6] ? (int)gridDim.x + sched_take(p.sched) : num_items;
                 const PairItem I = pair_item<BK>(p, w);
                 UnionWalk<C::ROWS> it;
                 int len = 0;
@@ -805,16 +806,8 @@ s2_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    if (threadIdx.x == 0) {
-        // The last CTA to finish resets the counter for the next launch on this slot
-        // (every CTA has stopped taking items by now).
-        __threadfence();
-        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
-            atomicExch(p.sched, 0);
-            atomicExch(p.sched + 1, 0);
-            __threadfence();
-        }
-    }
+    // every CTA has stopped taking items by now; the last one frees the slot
+    if (threadIdx.x == 0 && misc[6]) sched_leave(p.sched);
 }
 
 }  // namespace s2

@@ -123,6 +123,52 @@ __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint64
     return true;
 }
 
+// ---------------------------------------------------------------- work counters
+//
+// A persistent launch takes its work items from a counter slot
+// {owner, next item, CTAs done, unused} of a device-wide ring. The host gives
+// every launch a nonzero id and a slot; the launch owns the slot from the
+// first CTA's claim until its last CTA leaves, so two launches in flight at
+// once (on any streams) never share counters: a launch whose slot is still
+// held by an earlier one waits for it (bounded), and on expiry its CTAs take
+// no items beyond their first and the timeout flag reports it.
+constexpr int kSchedWords = 4;
+
+// Claim the slot for launch `id` (one thread per CTA, before any item is taken).
+__device__ __forceinline__ bool sched_claim(int* slot, int id, const WaitCtl& ctl)
+{
+    for (uint64_t t0 = 0;;) {
+        const int old = atomicCAS(slot, 0, id);
+        if (old == 0 || old == id) {
+            __threadfence();  // the counters are read after the owner (the releaser fenced them)
+            return true;
+        }
+        if (ctl.timeout_ns == 0 || (*reinterpret_cast<volatile uint32_t*>(ctl.gflags) & kFlagTimeout)) break;
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        if (now - t0 >= ctl.timeout_ns) break;
+        __nanosleep(1024);
+    }
+    atomicOr(ctl.gflags, kFlagTimeout);
+    return false;
+}
+
+// Next item index of the launch (from 0; the caller adds its static items).
+__device__ __forceinline__ int sched_take(int* slot) { return atomicAdd(slot + 1, 1); }
+
+// One CTA that claimed the slot is done taking items: the last one resets the
+// counters and then frees the slot.
+__device__ __forceinline__ void sched_leave(int* slot)
+{
+    __threadfence();
+    if (atomicAdd(slot + 2, 1) == (int)(gridDim.x * gridDim.y * gridDim.z) - 1) {
+        atomicExch(slot + 1, 0);
+        atomicExch(slot + 2, 0);
+        __threadfence();
+        atomicExch(slot, 0);
+    }
+}
+
 // ---------------------------------------------------------------- copies
 
 __device__ __forceinline__ void fence_proxy_async_smem()

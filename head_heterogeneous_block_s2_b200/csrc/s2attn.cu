@@ -25,12 +25,15 @@ namespace {
 __device__ uint32_t g_s2_flags;
 
 // Work counters of the persistent kernels (prefill, chunked prefill, and the
-// backward's dQ and 64-key dK/dV kernels): {next item, CTAs done} per slot.
-// Each launch takes the next slot in turn; the kernel's last CTA resets its
-// slot, so a slot is free again once its launch has finished.
-constexpr int kSchedSlots = 64;
-__device__ int g_s2_sched[2 * kSchedSlots];
+// backward's dQ and 64-key dK/dV kernels): a ring of slots {owner, next item,
+// CTAs done, unused}. Each launch gets the next slot in turn and a nonzero id;
+// its CTAs claim the slot before taking items and the last one frees it, so a
+// slot reused while an earlier launch still holds it makes the new launch
+// wait for that one (see sched_claim), never share its counters.
+constexpr int kSchedSlots = 1024;
+__device__ int g_s2_sched[s2::kSchedWords * kSchedSlots];
 std::atomic<uint32_t> g_launch_seq{0};
+
 
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 
@@ -47,6 +50,14 @@ struct DevInfo {
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
+
+// The slot and id of the next persistent launch on device `dev`.
+int* next_sched(int dev, int* id)
+{
+    const uint32_t s = g_launch_seq.fetch_add(1);
+    *id = (int)(s % 0x7ffffffeu) + 1;
+    return g_dev[dev].sched + s2::kSchedWords * (int)(s % kSchedSlots);
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -127,6 +138,16 @@ int make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t head
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The logits' multiplier: 0 selects 1/sqrt(head_dim). Returns false for a
+// non-finite value, and for a negative one where `positive` is required (the
+// prefill-type kernels take the row maximum of the unscaled logits).
+bool resolve_scale(float& scale, int32_t head_dim, bool positive)
+{
+    if (!std::isfinite(scale)) return false;
+    if (scale == 0.f) scale = 1.0f / std::sqrt((float)head_dim);
+    return !positive || scale > 0.f;
+}
 
 template <int HD, int BK>
 int launch_prefill(const void* q, const void* k, const void* v, s2::PrefillParams& pp, int dev,
@@ -317,6 +338,12 @@ int s2_device_status(int reset, uint32_t* flags_out)
     if (reset) {
         const uint32_t z = 0;
         if (cudaMemcpyToSymbol(g_s2_flags, &z, sizeof z) != cudaSuccess) return S2_ERR_CUDA;
+        // After a timeout a work-counter slot may still be held by a launch whose
+        // CTAs did not all claim it; with the device idle every slot is free.
+        if ((f & s2::kFlagTimeout) &&
+            (cudaMemset(g_dev[dev].sched, 0, sizeof(int) * s2::kSchedWords * kSchedSlots) != cudaSuccess ||
+             cudaDeviceSynchronize() != cudaSuccess))
+            return S2_ERR_CUDA;
     }
     if (flags_out) *flags_out = f;
     if (f & s2::kFlagTimeout) return S2_ERR_TIMEOUT;
@@ -330,7 +357,7 @@ int s2_attn_prefill_gqa(const void* q, const void* k, const void* v, void* o, fl
                         const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz, void* stream)
 {
     if (!q || !k || !v || !o || !row_ptr || (!col_idx && nnz > 0)) return S2_ERR_INVALID_ARG;
-    if (batch < 1 || heads < 1 || seq < 1 || nnz < 0 || !std::isfinite(scale) || !(scale > 0.f))
+    if (batch < 1 || heads < 1 || seq < 1 || nnz < 0 || !resolve_scale(scale, head_dim, true))
         return S2_ERR_INVALID_ARG;
     if (heads_kv < 1 || heads % heads_kv != 0) return S2_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
@@ -362,7 +389,7 @@ int s2_attn_prefill_gqa(const void* q, const void* k, const void* v, void* o, fl
     pp.scale_log2 = scale * 1.4426950408889634f;
     pp.timeout_ns = g_timeout_ns.load();
     pp.gflags = g_dev[dev].flags;
-    pp.sched = g_dev[dev].sched + 2 * (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
+    pp.sched = next_sched(dev, &pp.sched_id);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 128 && block_size == 128) return launch_prefill<128, 128>(q, k, v, pp, dev, 0, st);
     if (head_dim == 128 && block_size == 64) return launch_prefill<128, 64>(q, k, v, pp, dev, 1, st);
@@ -388,7 +415,7 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !row_ptr || !col_ptr ||
         ((!col_idx || !row_idx) && nnz > 0) || !workspace || (block_size == 64 && !key_tiles))
         return S2_ERR_INVALID_ARG;
-    if (batch < 1 || heads < 1 || seq < 1 || nnz < 0 || !std::isfinite(scale) || !(scale > 0.f))
+    if (batch < 1 || heads < 1 || seq < 1 || nnz < 0 || !resolve_scale(scale, head_dim, true))
         return S2_ERR_INVALID_ARG;
     if (heads_kv < 1 || heads % heads_kv != 0) return S2_ERR_INVALID_ARG;
     // grouped heads: a key tile walks every query head's list of its group (tags of 4 bits)
@@ -434,8 +461,8 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
     bp.scale_log2 = scale * 1.4426950408889634f;
     bp.timeout_ns = g_timeout_ns.load();
     bp.gflags = g_dev[dev].flags;
-    bp.sched = g_dev[dev].sched + 2 * (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
-    bp.sched_kv = g_dev[dev].sched + 2 * (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
+    bp.sched = next_sched(dev, &bp.sched_id);
+    bp.sched_kv = next_sched(dev, &bp.sched_kv_id);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 128 && block_size == 128) return launch_backward<128, 128>(q, k, v, bp, dev, 0, st);
     if (head_dim == 128 && block_size == 64) return launch_backward<128, 64>(q, k, v, bp, dev, 1, st);
@@ -464,7 +491,7 @@ int s2_attn_chunk_prefill(const void* q, const void* k_cache, const void* v_cach
         (!col_idx && nnz > 0) || !out)
         return S2_ERR_INVALID_ARG;
     if (batch < 1 || heads < 1 || max_pages < 1 || num_pages < 1 || num_blocks < 1 || nnz < 0 ||
-        max_q_len < 1 || total_q < 1 || !std::isfinite(scale) || !(scale > 0.f))
+        max_q_len < 1 || total_q < 1 || !resolve_scale(scale, head_dim, true))
         return S2_ERR_INVALID_ARG;
     if (heads_kv < 1 || heads % heads_kv != 0) return S2_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;
@@ -500,7 +527,7 @@ int s2_attn_chunk_prefill(const void* q, const void* k_cache, const void* v_cach
     cp.scale_log2 = scale * 1.4426950408889634f;
     cp.timeout_ns = g_timeout_ns.load();
     cp.gflags = g_dev[dev].flags;
-    cp.sched = g_dev[dev].sched + 2 * (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
+    cp.sched = next_sched(dev, &cp.sched_id);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 128 && block_size == 128) return launch_chunk<128, 128>(q, k_cache, v_cache, cp, dev, 0, st);
     if (head_dim == 128 && block_size == 64) return launch_chunk<128, 64>(q, k_cache, v_cache, cp, dev, 1, st);
@@ -539,7 +566,7 @@ int s2_attn_decode_gqa(const void* q, const void* k_cache, const void* v_cache,
         (!col_idx && nnz > 0) || !out)
         return S2_ERR_INVALID_ARG;
     if (batch < 1 || heads < 1 || max_pages < 1 || num_pages < 1 || num_blocks < 1 || nnz < 0 ||
-        !std::isfinite(scale) || num_splits > kMaxSplits)
+        !resolve_scale(scale, head_dim, false) || num_splits > kMaxSplits)
         return S2_ERR_INVALID_ARG;
     if (heads_kv < 1 || heads % heads_kv != 0) return S2_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return S2_ERR_UNSUPPORTED;

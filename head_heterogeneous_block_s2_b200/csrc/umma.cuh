@@ -20,7 +20,8 @@ struct PrefillParams {
     float scale_log2;  // scale * log2(e)
     uint64_t timeout_ns;
     uint32_t* gflags;
-    int* sched;  // pair kernel work counter {next item, CTAs done}, zero at launch
+    int* sched;    // work-counter slot of this launch (sched_claim / sched_take / sched_leave)
+    int sched_id;  // this launch's nonzero id
 };
 
 // UMMA shared-memory descriptor, SWIZZLE_128B, version 1 (sm_100).

@@ -327,7 +327,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: Layout,
         lse = torch.empty((batch, heads, seq), dtype=torch.float32, device=q.device)
     if lse is not None:
         _need(lse, "lse", torch.float32)
-    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    sc = 0.0 if scale is None else float(scale)  # 0: the library uses 1/sqrt(head_dim)
     if hkv == heads:
         rc = load().s2_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), batch, heads,
                                     seq, hd, sc, layout.block_size, layout.num_blocks,
@@ -382,7 +382,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     ws_len = workspace.numel() * workspace.element_size()
-    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    sc = 0.0 if scale is None else float(scale)  # 0: the library uses 1/sqrt(head_dim)
     rc = load().s2_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
                                  _ptr(dq), _ptr(dk), _ptr(dv), batch, heads, hkv, seq, hd, sc,
                                  layout.block_size, layout.num_blocks, _ptr(layout.d_row_ptr),
@@ -425,7 +425,7 @@ def chunk_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
         lse = torch.empty((total_q, heads), dtype=torch.float32, device=q.device)
     if lse is not None:
         _need(lse, "lse", torch.float32)
-    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    sc = 0.0 if scale is None else float(scale)  # 0: the library uses 1/sqrt(head_dim)
     rc = load().s2_attn_chunk_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                       _ptr(ctx_lens), _ptr(q_start), batch, heads, hkv, hd, page_size,
                                       block_table.shape[1], num_pages, int(max_q_len), total_q,
@@ -475,7 +475,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    sc = 0.0 if scale is None else float(scale)  # 0: the library uses 1/sqrt(head_dim)
     if h2 == heads:
         rc = load().s2_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                    _ptr(ctx_lens), batch, heads, hd, page_size, block_table.shape[1],
@@ -530,7 +530,7 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
         lse = torch.empty((batch, heads), dtype=torch.float32, device=q.device)
     if lse is not None:
         _need(lse, "lse", torch.float32)
-    sc = float(scale) if scale is not None else 1.0 / float(hd) ** 0.5
+    sc = 0.0 if scale is None else float(scale)  # 0: the library uses 1/sqrt(head_dim)
     rc = load().s2_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                        _ptr(ctx_lens), batch, heads, hd, page_size,
                                        block_table.shape[1], num_pages, layout.block_size,

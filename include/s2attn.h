@@ -20,11 +20,26 @@
  * Conventions for every entry point:
  *  - Returns an int status (S2_OK = 0, else one of the S2_ERR_* codes). No C++
  *    exception crosses the ABI. A call that returns an error launches nothing.
- *  - The caller owns every buffer. The library never allocates, frees or
- *    synchronises device memory (s2_device_status is the one synchronous call).
+ *  - The caller owns every buffer. No call allocates, frees or synchronises
+ *    device memory (s2_device_status is the one synchronous call). The library
+ *    does hold three fixed file-scope device arrays on every GPU that loads it,
+ *    until the process exits: the error flags, 1024 work-counter slots (16 KB)
+ *    and the 8 MiB scratch of s2_attn_decode_noalloc (see there).
  *  - Device pointers must stay valid until the work queued on `stream` ends.
  *    `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream). Launches are asynchronous.
+ *  - Launches on different streams may overlap. The persistent kernels
+ *    (prefill, chunked prefill, backward) take their work items from a counter
+ *    slot that each launch owns from start to end; slots are handed out in
+ *    turn, and a launch whose slot is still held by an earlier launch that has
+ *    not finished waits for it (within the wait bound below, after which its
+ *    CTAs stop taking items and S2_ERR_TIMEOUT is reported). So any number of
+ *    launches may be in flight at once without sharing counters. The one
+ *    shared buffer is the scratch of s2_attn_decode_noalloc.
+ *  - The device addresses of those arrays are looked up once per device and
+ *    kept for the life of the process: after cudaDeviceReset, or anything else
+ *    that replaces the device's primary context, unload and reload the library.
+ *  - `scale` (the logits' multiplier) 0 selects 1/sqrt(head_dim).
  *  - Tensors are bf16 (IEEE bfloat16 bit patterns in uint16 storage), dense and
  *    row-major with the innermost dimension last, 16-byte aligned.
  *  - Device waits inside the kernels are bounded. A wait that runs out sets a
@@ -184,6 +199,13 @@ int s2_build_key_tiles(int32_t num_heads, int32_t num_blocks, const int32_t* col
 /*
  * O = HHST-masked softmax(scale * Q K^T) V for every query row.
  *
+ * "S2-Attention: Hardware-aware context sharding among attention heads"
+ * (OpenReview forum page, Abstract): each head attends to its own strided
+ * share of the context plus a local window, the heads together cover it, and
+ * the sparsity turns into wall-clock speed only through a FlashAttention-style
+ * kernel that works at the block granularity of the pattern. This is that
+ * forward pass over whole sequences (training and prefill).
+ *
  *   q, k, v   device bf16 [batch][heads][seq][head_dim] (read).
  *   o         device bf16 [batch][heads][seq][head_dim] (written).
  *   lse       device fp32 [batch][heads][seq] or NULL: natural-log
@@ -196,7 +218,7 @@ int s2_build_key_tiles(int32_t num_heads, int32_t num_blocks, const int32_t* col
  *             (read). Lists must be strictly ascending with j <= i; nnz may be
  *             0 (then col_idx may be NULL). A query row whose list is empty
  *             gets a zero output row and LSE = -inf.
- *   scale     multiplier of the logits (1/sqrt(head_dim) in the usual case).
+ *   scale     multiplier of the logits, > 0; 0 selects 1/sqrt(head_dim).
  * Runs tcgen05 tensor-core tiles of 128 query rows; only the listed key blocks
  * are visited and causality is applied inside the diagonal block only.
  * num_blocks is at most 2046 (union lists are staged in shared memory).
@@ -335,6 +357,14 @@ int32_t s2_attn_decode_auto_splits(int32_t batch, int32_t heads);
  * n-1 (n = ctx_lens[s]) attends to keys 0..n-1 of its own context under the
  * same block rule (query block i = (n-1) / block_size).
  *
+ * The inference side of "S2-Attention: Hardware-aware context sharding among
+ * attention heads" (arXiv abstract on the mlsanity index page: a 7B HHST model
+ * served through vLLM runs 4.5x faster than its dense counterpart;
+ * PagedAttention is in its reference list): one new token per sequence over a
+ * paged KV cache, reading only the active blocks. The splits of a context are
+ * merged by the log-sum-exp rule (online softmax as an associative reduction,
+ * the LeanAttention summary on the SampleAttention page).
+ *
  *   q            device bf16 [batch][heads][head_dim] (read).
  *   k_cache,     device bf16 [num_pages][heads][page_size][head_dim] (read):
  *   v_cache      token t of sequence s is row t % page_size of physical page
@@ -347,6 +377,8 @@ int32_t s2_attn_decode_auto_splits(int32_t batch, int32_t heads);
  *   row_ptr, col_idx, nnz: device layout for (heads, num_blocks) from one of
  *                the s2_build_layout* builders; an empty list gives a zero
  *                output and LSE = -inf.
+ *   scale        multiplier of the logits, any finite value; 0 selects
+ *                1/sqrt(head_dim).
  *   out          device bf16 [batch][heads][head_dim] (written).
  *   lse          device fp32 [batch][heads] or NULL (written).
  *   workspace    device, >= s2_attn_decode_workspace_size(...) bytes, 256-byte
@@ -421,7 +453,10 @@ int s2_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cac
  * Synchronise the current device and report the kernels' error flags:
  * S2_OK, S2_ERR_TIMEOUT (a bounded wait ran out) or S2_ERR_DEVICE_INDEX (an
  * index was out of range and skipped). *flags_out (may be NULL) receives the
- * raw bit set (1 = timeout, 2 = index). reset != 0 clears the flags.
+ * raw bit set (1 = timeout, 2 = index). reset != 0 clears the flags and, when
+ * a timeout was flagged, also frees every work-counter slot (a launch that
+ * timed out may not have released its own); call it while no other thread is
+ * launching this library's kernels on the device.
  */
 int s2_device_status(int reset, uint32_t* flags_out);
 

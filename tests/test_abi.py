@@ -1,15 +1,23 @@
 """The C-ABI library loads without a GPU and exports every declared entry point.
 
 Also checks host-side argument validation: calls with bad arguments return
-an error status before touching any device.
+an error status before touching any device. Those calls pass made-up device
+addresses, so they run only on a machine without a GPU: there a call that got
+past validation could not launch anything (it fails at the device check with
+S2_ERR_CUDA), while on a GPU a validation slip would launch a kernel on a wild
+address.
 """
 import ctypes
 import os
 import re
 
 import pytest
+import torch
 
 from head_heterogeneous_block_s2_b200 import s2attn
+
+no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(),
+                                 reason="passes made-up device addresses: CPU-only machines")
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -52,13 +60,25 @@ def _prefill(**over):
                                          vp(a["col_idx"]), a["nnz"], None)
 
 
+@no_gpu_only
 @pytest.mark.parametrize("over,code", [
     (dict(q=None), 1), (dict(row_ptr=None), 1), (dict(batch=0), 1), (dict(seq=600), 1),
     (dict(nb=7), 1), (dict(hd=96), 2), (dict(bs=32), 2), (dict(q=(1 << 20) + 8), 1),
     (dict(scale=float("nan")), 1), (dict(nnz=-1), 1), (dict(col_idx=None), 1),
+    (dict(scale=-0.125), 1),
 ])
 def test_prefill_rejects_bad_arguments_before_launch(over, code):
     assert _prefill(**over) == code
+
+
+@no_gpu_only
+def test_zero_scale_selects_the_default_and_passes_validation():
+    # 0 means 1/sqrt(head_dim): validation accepts it and the call reaches the
+    # device check, which fails here for want of a GPU (S2_ERR_CUDA).
+    assert _prefill(scale=0.0) == 4
+    assert _decode(scale=0.0) == 4
+    assert _decode(scale=-0.1) == 4  # decode takes any finite multiplier
+    assert _decode(scale=float("inf")) == 1
 
 
 def _decode(**over):
@@ -74,6 +94,7 @@ def _decode(**over):
                                         vp(a["lse"]), vp(a["ws"]), a["ws_bytes"], a["splits"], None)
 
 
+@no_gpu_only
 @pytest.mark.parametrize("over,code", [
     (dict(q=None), 1), (dict(bt=None), 1), (dict(page=32), 2), (dict(hd=80), 2),
     (dict(bs=24), 2), (dict(splits=2, ws=None), 1), (dict(splits=2, ws=1 << 20, ws_bytes=16), 3),
@@ -93,6 +114,7 @@ def test_decode_workspace_size():
     assert s2attn.decode_workspace_size(4, 8, 128, 0) == s2attn.decode_workspace_size(4, 8, 128, auto)
 
 
+@no_gpu_only
 def test_grouped_head_entry_points_reject_bad_head_counts():
     lib = s2attn.load()
     vp = ctypes.c_void_p

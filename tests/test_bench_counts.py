@@ -61,3 +61,20 @@ def test_prefill_mma_flops_of_the_bench_workloads():
         assert mma >= bench.prefill_issued_flops(lay, w) >= bench.prefill_flops(lay, w)
         if name == "prefill_1p3b":
             assert mma == 4 * w.head_dim * 128 * w.block * 10994 * w.batch
+
+
+def test_planted_positions_from_the_layout_equal_those_from_the_oracle_mask():
+    """bench.py plants the 131K workload's keys from the library's layout on
+    the GPU arm and from the oracle's block mask on the reference arm: both
+    pick the same tokens, each in a strided key block (beyond the local
+    window) of the first half that the last query block sees."""
+    w = synth.PREFILL_LONG_131K
+    nb = w.num_blocks
+    lay = s2attn.build_layout(w.heads, w.block, w.stride, w.local, nb)
+    m = oracle.block_mask(w.heads, nb, w.stride, w.local)
+    a = bench.plant_positions(w, [lay.row(h, nb - 1) for h in range(w.heads)])
+    b = bench.plant_positions(w, [np.nonzero(m[h, nb - 1])[0] for h in range(w.heads)])
+    assert a == b and len(a) == w.heads
+    for h, t in a.items():
+        j = t // w.block
+        assert m[h, nb - 1, j] and j <= nb // 2 and nb - 1 - j >= w.local

@@ -159,3 +159,43 @@ def test_grouped_kv_heads(s2gpu, hkv, bk):
     ref = oracle.backward(q, k, v, do, bk, w.scale, S=3, L=1, dense_heads=(1,))
     for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
         grad_parity(name, g, r)
+
+
+def _rows(rng, lo, hi, n, block):
+    """n seeded positions in [lo, hi) plus the block edges at both ends."""
+    pos = {lo, hi - 1, lo + block - 1 if hi - lo > block else lo}
+    pos |= set(int(x) for x in rng.integers(lo, hi, n))
+    return np.array(sorted(pos), dtype=np.int64)
+
+
+@pytest.mark.parametrize("name,picks", [
+    # (batch, head, first sampled position): sparse heads over the whole
+    # sequence; a dense head (7B hybrid) over its last blocks only, since every
+    # earlier key of a dense head is seen by all later rows
+    ("prefill_1p3b", [(0, 3, 0), (3, 12, 0), (2, 7, 0)]),
+    ("prefill_7b_hybrid", [(0, 5, 0), (0, 30, 0), (0, 1, 32768 - 4 * 128)]),
+])
+def test_full_size_workload_sampled_gradients(s2gpu, name, picks):
+    """dQ rows and dK/dV key rows of the full-size workloads, sampled per head,
+    against the oracle's gradients of the same rows; the kernels run in the
+    launch configuration of the benchmark's backward leg."""
+    w = synth.PREFILL_WORKLOADS[name]
+    q, k, v = synth.prefill_inputs(w, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(77)
+    do = torch.randn(q.shape, generator=gen, device="cuda").to(torch.bfloat16)
+    lay = s2gpu.build_layout(w.heads, w.block, w.stride, w.local, w.num_blocks, w.dense_heads,
+                             device="cuda")
+    o, lse = s2gpu.prefill(q, k, v, lay, scale=w.scale, want_lse=True)
+    dq, dk, dv = s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale)
+    torch.cuda.synchronize()
+    qh, kh, vh, doh = (t.cpu() for t in (q, k, v, do))
+    rng = np.random.default_rng(w.seed + 300)
+    for b, h, lo in picks:
+        qr = _rows(rng, lo, w.seq, 24, w.block)
+        kr = _rows(rng, lo, w.seq, 24, w.block)
+        rq, rk, rv = oracle.backward_sampled(qh, kh, vh, doh, w.block, w.scale, [b * w.heads + h],
+                                             qr, kr, S=w.stride, L=w.local,
+                                             dense_heads=w.dense_heads)
+        grad_parity(f"{name} dq b{b} h{h}", dq[b, h, torch.from_numpy(qr).cuda()], rq[0])
+        grad_parity(f"{name} dk b{b} h{h}", dk[b, h, torch.from_numpy(kr).cuda()], rk[0])
+        grad_parity(f"{name} dv b{b} h{h}", dv[b, h, torch.from_numpy(kr).cuda()], rv[0])

@@ -30,18 +30,6 @@ def _worker(rank, world, port, out):
 
         if rank != 0:
             out[10 + rank] = bench.run_reference(A, rank)  # no work off rank 0
-
-        # settle: a slow rank and a fast one still run the same number of steps
-        import time
-
-        calls = [0]
-
-        def step():
-            calls[0] += 1
-            time.sleep(0.02 if rank else 0.001)
-
-        n = bench.settle(step, 0.2, tdist, "cpu", sync=lambda: None)
-        out[20 + rank] = (n, calls[0])
     finally:
         tdist.destroy_process_group()
 
@@ -54,8 +42,6 @@ def test_timings_reduce_to_the_max_over_two_gloo_ranks():
         want = [2.0, 10.0, 3.5, 7.0]
         assert out[0] == want and out[1] == want
         assert out[11] is None
-        (n0, c0), (n1, c1) = out[20], out[21]
-        assert n0 == n1 == c0 == c1 and n0 >= 4
 
 
 def test_single_process_is_identity():

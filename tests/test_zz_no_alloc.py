@@ -4,10 +4,14 @@ Some callers of this library cannot call cudaMalloc: plug-ins whose host
 framework owns all device memory, C programs without a device allocator of
 their own, and latency-critical loops that must not allocate (cudaMalloc and
 cudaFree can synchronise the device). For them the library keeps the decode
-split partials in its own built-in scratch array. These tests call that entry
-point through the C ABI and check it against s2_attn_decode with a caller
-workspace, twice in a row on different inputs (the scratch keeps the previous
-call's contents), and check that a shape too large for the scratch is refused.
+split partials in its own built-in scratch array.
+
+These tests call that entry point through the C ABI and check each result
+against the fp64 oracle and against s2_attn_decode with a caller workspace,
+over calls in a row on different inputs that share the scratch: a call with
+more splits leaves partials at offsets a later call with fewer splits does
+not write, and that later call must not read them. A shape too large for the
+scratch is refused before anything runs.
 
 This file is named to be collected last.
 """
@@ -16,6 +20,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from conftest import parity
 from head_heterogeneous_block_s2_b200 import s2attn, synth
 
@@ -30,15 +35,23 @@ def _case(seed, ctx):
     return w, d, lay
 
 
-@pytest.mark.parametrize("splits", [7, 3])
-def test_noalloc_decode_matches_workspace_decode_twice(s2gpu, splits):
-    cases = [_case(31, [1, 16, 17, 128, 129, 3000]), _case(32, [3000, 2999, 640, 5, 1000, 77])]
-    for w, d, lay in cases:  # two calls in a row through the shared scratch
+def test_noalloc_decode_matches_oracle_and_workspace_decode_over_calls(s2gpu):
+    # 7 splits, then 3 on other inputs (the scratch still holds the 7-split
+    # partials), then 7 again: every call is checked on its own
+    cases = [(_case(31, [1, 16, 17, 128, 129, 3000]), 7),
+             (_case(32, [3000, 2999, 640, 5, 1000, 77]), 3),
+             (_case(33, [2048, 1, 2900, 300, 129, 1500]), 7)]
+    for (w, d, lay), splits in cases:
         args = (d.q.cuda(), d.k_cache.cuda(), d.v_cache.cuda(), d.block_table.cuda(),
                 d.ctx_lens.cuda(), lay)
-        ref, ref_lse = s2attn.decode(*args, scale=w.scale, num_splits=splits, want_lse=True)
         got, got_lse = s2attn.decode_noalloc(*args, scale=w.scale, num_splits=splits,
                                              want_lse=True)
+        torch.cuda.synchronize()
+        want, want_lse = oracle.decode(d.q, d.k_cache, d.v_cache, d.block_table.numpy(),
+                                       d.ctx_lens.numpy(), w.block, w.stride, w.local, w.scale)
+        parity(got.reshape(-1, w.head_dim), want)
+        parity(got_lse.reshape(-1), want_lse, max_tol=1e-3, mean_tol=1e-4)
+        ref, ref_lse = s2attn.decode(*args, scale=w.scale, num_splits=splits, want_lse=True)
         torch.cuda.synchronize()
         parity(got.reshape(-1, w.head_dim), ref.double().cpu().numpy().reshape(-1, w.head_dim))
         parity(got_lse.reshape(-1), ref_lse.double().cpu().numpy().reshape(-1),
@@ -47,10 +60,10 @@ def test_noalloc_decode_matches_workspace_decode_twice(s2gpu, splits):
 
 def test_noalloc_decode_rejects_shapes_beyond_the_scratch(s2gpu):
     lib = s2attn.load()
-    vp = ctypes.c_void_p
-    # 64 sequences x 32 heads x 64 splits of fp32 partials need ~68 MB > 8 MiB
+    # 64 sequences x 32 heads x 64 splits of fp32 partials need ~68 MB > 8 MiB.
+    # All pointers are NULL: the size check must refuse the call first, and if
+    # it did not, the pointer check behind it would (nothing can launch).
     assert s2attn.decode_workspace_size(64, 32, 128, 64) > s2attn.NOALLOC_SCRATCH_BYTES
-    rc = lib.s2_attn_decode_noalloc(vp(1 << 20), vp(1 << 20), vp(1 << 20), vp(1 << 20),
-                                    vp(1 << 20), 64, 32, 128, 16, 2048, 100, 128, 256,
-                                    vp(1 << 20), vp(1 << 20), 10, 0.1, vp(1 << 20), None, 64, None)
-    assert rc == 3  # S2_ERR_CAPACITY, nothing launched
+    rc = lib.s2_attn_decode_noalloc(None, None, None, None, None, 64, 32, 128, 16, 2048, 100, 128,
+                                    256, None, None, 10, 0.1, None, None, 64, None)
+    assert rc == 3  # S2_ERR_CAPACITY
