@@ -154,3 +154,53 @@ def test_malformed_transposed_layout_is_flagged_not_faulted(s2gpu, bk):
     s2gpu.backward(q, k, v, o, lse, torch.ones_like(q), lay, scale=w.scale)
     rc, flags = s2gpu.device_status(reset=True)
     assert rc == S2_ERR_DEVICE_INDEX and flags == 2
+
+
+def tiny128():
+    # 128-key blocks: the prefill runs one 128-row tile per item (split kernel)
+    w = synth.PrefillWorkload("t128", 1, 4, 128, 640, 128, 2, 1, seed=12)
+    q, k, v = synth.prefill_inputs(w)
+    lay = s2attn.build_layout(w.heads, w.block, w.stride, w.local, w.num_blocks, device="cuda")
+    return w, q, k, v, lay
+
+
+def test_prefill_128_key_wait_timeout_is_reported_and_recoverable(s2gpu):
+    w, q, k, v, lay = tiny128()
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    s2gpu.set_wait_timeout_ns(0)
+    try:
+        s2gpu.prefill(qc, kc, vc, lay, scale=w.scale)
+        rc, flags = s2gpu.device_status(reset=True)
+    finally:
+        s2gpu.set_wait_timeout_ns(500_000_000)
+    assert rc == S2_ERR_TIMEOUT and flags & 1
+    out, lse = s2gpu.prefill(qc, kc, vc, lay, scale=w.scale, want_lse=True)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.prefill(q, k, v, w.block, w.stride, w.local, w.scale)
+    parity(out.reshape(-1, w.head_dim), ref)
+    parity(lse.reshape(-1), ref_lse, max_tol=1e-3, mean_tol=1e-4)
+
+
+@pytest.mark.parametrize("corrupt", ["future_block", "huge_block", "negative_block", "row_past_nnz"])
+def test_malformed_128_key_layout_is_flagged_not_faulted(s2gpu, corrupt):
+    w, q, k, v, lay = tiny128()
+    row_ptr, col_idx = lay.row_ptr.copy(), lay.col_idx.copy()
+    nb = w.num_blocks
+    if corrupt == "future_block":
+        col_idx[row_ptr[2]] = 4  # head 0, query block 2 lists key block 4 > 2
+    elif corrupt == "huge_block":
+        col_idx[5] = 1 << 20
+    elif corrupt == "negative_block":
+        col_idx[3] = -4
+    else:
+        row_ptr[(nb + 1) + 3] = col_idx.size + 7  # head 1, block 3 ends past the lists
+    bad = s2attn.Layout(lay.heads, lay.block_size, lay.stride, lay.local, lay.num_blocks, (),
+                        row_ptr, col_idx).to("cuda")
+    out = s2gpu.prefill(q.cuda(), k.cuda(), v.cuda(), bad, scale=w.scale)
+    rc, flags = s2gpu.device_status(reset=True)
+    assert rc == S2_ERR_DEVICE_INDEX and flags == 2
+    assert torch.isfinite(out.float()).all()
+    good = s2gpu.prefill(q.cuda(), k.cuda(), v.cuda(), lay, scale=w.scale)
+    torch.cuda.synchronize()
+    ref, _ = oracle.prefill(q, k, v, w.block, w.stride, w.local, w.scale)
+    parity(good.reshape(-1, w.head_dim), ref)
