@@ -54,7 +54,7 @@ class PrefillWorkload:
 
     @property
     def num_blocks(self) -> int:
-        return self.seq // self.block
+        return -(-self.seq // self.block)  # a ragged last block counts
 
     @property
     def scale(self) -> float:
