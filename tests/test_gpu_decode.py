@@ -56,6 +56,19 @@ def test_dense_head_and_many_splits(s2gpu):
         parity(out.reshape(-1, 128), ref)
 
 
+@pytest.mark.parametrize("S,L", [(4, 1000), (1000, 1), (1000, 3)])
+def test_degenerate_strides_and_windows(s2gpu, S, L):
+    # a window past the block count (dense causal) and a stride past it
+    # (the local window plus at most one strided block per head)
+    w = synth.DecodeWorkload("t", 6, 8, 128, 1, 3000, 16, 128, S, L, seed=14)
+    d = synth.decode_inputs(w, ctx_lens=[1, 16, 17, 128, 129, 3000])
+    for splits in (1, 3):
+        out, lse = run(s2gpu, w, d, splits)
+        ref, ref_lse = oracle_decode(w, d)
+        parity(out.reshape(-1, 128), ref)
+        parity(lse.reshape(-1), ref_lse, max_tol=1e-3, mean_tol=1e-4)
+
+
 def test_decode_equals_last_prefill_row(s2gpu):
     # Dense-packed prefill of n tokens vs paged decode of the same tokens.
     H, D, B, S, L, n = 4, 128, 128, 4, 2, 1024

@@ -55,6 +55,22 @@ def test_stride_one_matches_causal_sdpa(s2gpu):
     assert (out.float() - ref).abs().max().item() < 2e-2
 
 
+@pytest.mark.parametrize("bk", [64, 128])
+@pytest.mark.parametrize("S,L", [(4, 1000), (1000, 1), (1000, 3)])
+def test_degenerate_strides_and_windows(s2gpu, bk, S, L):
+    # L past the block count: every block is local (dense causal); S past the
+    # block count: the local window plus, per head h, the one block with
+    # (j + h) mod S == 0 if it lies before the query block
+    w = synth.PrefillWorkload("t", 2, 3, 128, 9 * bk - 7, bk, S, L, seed=23)
+    check_all_rows(s2gpu, w)
+    if L >= w.num_blocks:
+        q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
+        out, _ = run_prefill(s2gpu, w, q, k, v)
+        ref = torch.nn.functional.scaled_dot_product_attention(q.float(), k.float(), v.float(),
+                                                               is_causal=True)
+        assert (out.float() - ref).abs().max().item() < 2e-2
+
+
 def test_scaled_keys_and_large_logits(s2gpu):
     # per-head K scales as in the 1.3B-shaped workload, at a small size
     w = synth.PREFILL_1P3B.with_(batch=1, heads=4, seq=2048)
