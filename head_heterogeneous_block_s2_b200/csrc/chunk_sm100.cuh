@@ -26,7 +26,12 @@
 //    there, so the softmax threads zero them in the V stage before their
 //    tile's P V product reads it (their P is 0 anyway, but 0 times a NaN would
 //    not be);
-//  * the output and the LSE go to the packed chunk rows.
+//  * the output and the LSE go to the packed chunk rows;
+//  * each tile has its own Q buffer barriers: the tile's last S MMA of an item
+//    releases its Q and the next item's Q of that tile loads at once (the
+//    first tile usually sees its last key block one element before the second,
+//    whose diagonal block ends the list), and the tile's O is complete with its
+//    last PV, so its epilogue runs while the other tile finishes the item.
 // Roles: warp 2 maps items (a warp-parallel prefix over the sequences),
 // builds the union list of the item's query blocks and loads Q; warp 0
 // streams K and V; warp 1 owns TMEM and issues tcgen05.mma (S_t = Q_t K^T,
@@ -83,9 +88,9 @@ struct ChunkCfg {
     static constexpr uint32_t OFF_V = OFF_K + ST * KVBYTES;  // [stage][panel][BK rows x 128 B]
     static constexpr uint32_t OFF_LIST = OFF_V + ST * KVBYTES;
     static constexpr uint32_t OFF_BAR = OFF_LIST + LIST_BYTES;
-    // barriers: q_full, q_empty, kv_full[ST], kv_empty[ST], s_full[2], p_full[2],
-    // pv_done[2], drain, list_full[2], list_empty[2]
-    static constexpr int NBAR = 2 + 2 * ST + 6 + 1 + 4;
+    // barriers: q_full[0], q_empty[0], kv_full[ST], kv_empty[ST], s_full[2], p_full[2],
+    // pv_done[2], drain, list_full[2], list_empty[2], q_full[1], q_empty[1]
+    static constexpr int NBAR = 2 + 2 * ST + 6 + 1 + 4 + 2;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
     // misc ints: [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each
     // list buffer (-1: no more), [8..15] and [16..23] the buffers' item fields
@@ -188,8 +193,9 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     const uint32_t sb = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const uint32_t bar_q = sb + C::OFF_BAR;
-    const uint32_t bar_qe = sb + C::OFF_BAR + 8u;
+    // Q of tile t: loaded (q_full) and released by the tile's last S MMA of an item (q_empty)
+    auto bar_q = [&](int t) { return sb + C::OFF_BAR + 8u * (t == 0 ? 0 : 13 + 2 * C::ST); };
+    auto bar_qe = [&](int t) { return sb + C::OFF_BAR + 8u * (t == 0 ? 1 : 14 + 2 * C::ST); };
     auto bar_kf = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + s); };  // K and V of a stage
     auto bar_ke = [&](int s) { return sb + C::OFF_BAR + 8u * (2 + C::ST + s); };
     auto bar_sf = [&](int t) { return sb + C::OFF_BAR + 8u * (2 + 2 * C::ST + t); };
@@ -207,8 +213,10 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     ChunkItem* items = reinterpret_cast<ChunkItem*>(misc + 8);  // [2]: one per list buffer
 
     if (threadIdx.x == 0) {
-        mbar_init(bar_q, 1);
-        mbar_init(bar_qe, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar_q(t), 1);
+            mbar_init(bar_qe(t), 1);
+        }
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(bar_kf(s), 1);
             mbar_init(bar_ke(s), 1);
@@ -252,6 +260,7 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         uint32_t* wlist = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
         int64_t w = blockIdx.x;  // first item static, the rest from the work counter
         int k = 0;
+        int qn[2] = {0, 0};  // Q phases started per tile
         for (;; ++k) {
             const int b = k & 1;
             // union list of this item into buffer b (free once item k-2 is consumed)
@@ -303,24 +312,36 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 list_item[b] = (int)(w & 0x7fffffff);
                 mbar_arrive(bar_lf(b));
             }
-            // Q of the item's tiles, once the previous item's S MMAs are done with
-            // the buffer; tile row r is chunk row q0 + 128 (qt0 + t) - c0 + r
+            // Q of each tile, once the previous item's last S MMA of that tile is done
+            // with its buffer (tile 0 usually sees its last key block one element
+            // before tile 1, so its Q reloads earlier); tile row r is chunk row
+            // q0 + 128 (qt0 + t) - c0 + r. An absent second tile only completes its
+            // barrier phase.
             int q_ok = 1;
             if (lane == 0) {
-                q_ok = mbar_wait(bar_qe, (k & 1) ^ 1, ctl) ? 1 : 0;
-                if (q_ok) {
-                    mbar_arrive_expect_tx(bar_q, (I.tile1 ? 2 : 1) * C::QBYTES);
-                    for (int t = 0; t < (I.tile1 ? 2 : 1); ++t)
+                for (int t = 0; t < 2; ++t) {
+                    if (!mbar_wait(bar_qe(t), (k & 1) ^ 1, ctl)) {
+                        q_ok = 0;
+                        break;
+                    }
+                    if (t == 0 || I.tile1) {
+                        mbar_arrive_expect_tx(bar_q(t), C::QBYTES);
 #pragma unroll
                         for (int pn = 0; pn < HD / 64; ++pn)
                             tma_load_3d(sb + C::OFF_Q + t * C::QBYTES + pn * (C::M * 128), &tmQ, pn * 64, I.h,
-                                        I.q0 + (I.qt0 + t) * C::M - I.c0, bar_q);
+                                        I.q0 + (I.qt0 + t) * C::M - I.c0, bar_q(t));
+                    } else {
+                        mbar_arrive(bar_q(t));
+                    }
+                    ++qn[t];
                 }
             }
-            if (!__shfl_sync(0xffffffffu, q_ok, 0)) break;  // Q of item k was not issued
+            if (!__shfl_sync(0xffffffffu, q_ok, 0)) break;  // Q of item k was not (wholly) issued
             w = w_next;
         }
-        if (lane == 0 && *abort_cta && k > 0) mbar_drain(bar_q, (k - 1) & 1, kDrainNs);
+        if (lane == 0 && *abort_cta)  // let this CTA's own Q loads land before exit
+            for (int t = 0; t < 2; ++t)
+                if (qn[t] > 0) mbar_drain(bar_q(t), (qn[t] - 1) & 1, kDrainNs);
         __syncwarp();
     } else if (warp == 0) {
         // ------------------------------------------------------------ K/V producer
@@ -423,37 +444,76 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 const bool two = items[b].tile1 != 0;
                 const uint32_t* L = list + b * C::LIST_CAP;
                 const int len = list_len[b];
-                if (!mbar_wait(bar_q, k & 1, ctl)) break;
+                // The last element each tile sees (-1: none): its S MMA is the tile's
+                // last read of its Q buffer, its PV completes the tile's O.
+                int lastS[2] = {-1, -1};
+                for (int g = len - 1; g >= 0 && (lastS[0] < 0 || (two && lastS[1] < 0)); --g) {
+                    const int gb = list_bits(L[g]);
+#pragma unroll
+                    for (int t = 0; t < 2; ++t)
+                        if (lastS[t] < 0 && tile_sees_chunk<BK>(gb, t)) lastS[t] = g;
+                }
+                bool q_in[2] = {false, false};  // this item's phase of the tile's Q barrier observed
+                auto take_q = [&](int t) {
+                    if (!q_in[t]) {
+                        if (!mbar_wait(bar_q(t), k & 1, ctl)) return false;
+                        q_in[t] = true;
+                        tc_fence_after();
+                    }
+                    return true;
+                };
                 if (len == 0) {
-                    umma_commit(bar_qe);
+                    if (!take_q(0) || !take_q(1)) break;
+                    umma_commit(bar_qe(0));
+                    umma_commit(bar_qe(1));
                     mbar_arrive(bar_le(b));
                     continue;
                 }
-                if constexpr (C::Q_IN_TMEM) {
-                    // Q of both tiles into TMEM (after the previous item's S MMAs, in
-                    // issue order), then the shared-memory Q buffer is free at once.
-                    tc_fence_after();
-                    for (int t = 0; t < (two ? 2 : 1); ++t) {
-                        const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
+                for (int t = 0; t < 2 && !fail; ++t) {
+                    if constexpr (C::Q_IN_TMEM) {
+                        // Q of the tile into TMEM (after the previous item's S MMAs, in
+                        // issue order), then its shared-memory buffer is free at once.
+                        if (!take_q(t)) {
+                            fail = true;
+                            break;
+                        }
+                        if (t == 0 || two) {
+                            const uint64_t dq = umma_sdesc(sb + C::OFF_Q + t * C::QBYTES, 16, 1024);
 #pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk)
-                            tmem_cp_128x256b(tmem + C::colQ(t) + kk * 8,
-                                             dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4));
+                            for (int kk = 0; kk < HD / 16; ++kk)
+                                tmem_cp_128x256b(tmem + C::colQ(t) + kk * 8,
+                                                 dq + (((kk >> 2) * (C::M * 128) + (kk & 3) * 32) >> 4));
+                        }
+                        umma_commit(bar_qe(t));
+                    } else if (lastS[t] < 0) {  // the tile reads no Q in this item
+                        if (!take_q(t)) {
+                            fail = true;
+                            break;
+                        }
+                        umma_commit(bar_qe(t));
                     }
-                    umma_commit(bar_qe);
                 }
+                if (fail) break;
+                // S_t of element e (in stage st), once the tile's Q has landed; the
+                // tile's last one releases the Q buffer
+                auto s_tile = [&](int t, int e, int st) {
+                    if (!C::Q_IN_TMEM && !take_q(t)) return false;
+                    issue_s(t, st);
+                    if (!C::Q_IN_TMEM && e == lastS[t]) umma_commit(bar_qe(t));
+                    return true;
+                };
                 first_pv[0] = first_pv[1] = true;
                 int bits = list_bits(L[0]);
                 if (!wait_k(n)) break;
                 tc_fence_after();
-                for (int t = 0; t < 2; ++t)
-                    if (tile_sees_chunk<BK>(bits, t)) issue_s(t, n % C::ST);
+                for (int t = 0; t < 2 && !fail; ++t)
+                    if (tile_sees_chunk<BK>(bits, t) && !s_tile(t, 0, n % C::ST)) fail = true;
+                if (fail) break;
                 for (int g = 0;; ++g, ++n) {
                     const bool last = g + 1 == len;
                     const int nbits = last ? 0 : list_bits(L[g + 1]);
                     const int st = n % C::ST;
                     const int st1 = (n + 1) % C::ST;
-                    if (last && !C::Q_IN_TMEM) umma_commit(bar_qe);  // no more S MMAs of this item read Q
                     bool k_next_ready = false;
                     if (bits == 0) {  // malformed element no tile sees: let its loads land first
                         if (!wait_k(n)) {
@@ -467,6 +527,9 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                             if (!mbar_wait(bar_pf(t), pvc[t] & 1, ctl)) { fail = true; break; }
                             tc_fence_after();
                             issue_pv(t, st);
+                            // O_t of the item is complete with the tile's last PV: its
+                            // softmax warps start the epilogue while the other tile runs on
+                            if (g == lastS[t]) umma_commit(bar_pv(t));
                         }
                         if (t == last_t) umma_commit(bar_ke(st));
                         if (!last && tile_sees_chunk<BK>(nbits, t)) {
@@ -475,7 +538,7 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                                 k_next_ready = true;
                                 tc_fence_after();
                             }
-                            issue_s(t, st1);
+                            if (!s_tile(t, g + 1, st1)) { fail = true; break; }
                         }
                     }
                     if (fail) break;
@@ -485,13 +548,7 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     }
                     bits = nbits;
                 }
-                if (!fail) {
-                    // O_t of this item is complete once its last PV is: one commit per
-                    // tile and item (the softmax reads O only in the epilogue)
-                    for (int t = 0; t < 2; ++t)
-                        if (!first_pv[t]) umma_commit(bar_pv(t));
-                    mbar_arrive(bar_le(b));
-                }
+                if (!fail) mbar_arrive(bar_le(b));
             }
             if (*abort_cta && issued) {
                 umma_commit(bar_dr);
@@ -623,6 +680,10 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.0f / l : 0.f;
                 uint16_t* og = p.out + orow * HD;
+                // 32-byte stores (whole L2 sectors, half the store instructions) when
+                // the output is 32-byte aligned: output rows of a tile are heads * HD
+                // elements apart, so every store of the tile touches its own sectors
+                const bool st32 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
 #pragma unroll
                 for (int c = 0; c < HD / 32; ++c) {
                     uint32_t o[32];
@@ -630,13 +691,19 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     tmem_wait_ld();
                     if (row_valid) {
 #pragma unroll
-                        for (int e2 = 0; e2 < 32; e2 += 8) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * inv, __uint_as_float(o[e2 + 1]) * inv);
-                            v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * inv, __uint_as_float(o[e2 + 3]) * inv);
-                            v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * inv, __uint_as_float(o[e2 + 5]) * inv);
-                            v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * inv, __uint_as_float(o[e2 + 7]) * inv);
-                            *reinterpret_cast<uint4*>(og + 32 * c + e2) = v;
+                        for (int e2 = 0; e2 < 32; e2 += 16) {
+                            uint32_t w8[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                w8[i] = pack_bf16x2(__uint_as_float(o[e2 + 2 * i]) * inv,
+                                                    __uint_as_float(o[e2 + 2 * i + 1]) * inv);
+                            if (st32) {
+                                st_global_v8(og + 32 * c + e2, w8);
+                            } else {
+                                *reinterpret_cast<uint4*>(og + 32 * c + e2) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                                *reinterpret_cast<uint4*>(og + 32 * c + e2 + 8) =
+                                    make_uint4(w8[4], w8[5], w8[6], w8[7]);
+                            }
                         }
                     }
                 }

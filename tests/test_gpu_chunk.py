@@ -111,6 +111,32 @@ def test_long_chunk_sampled(s2gpu):
     case(s2gpu, ctx, qlen, H=16, S=16, L=4, seed=8)
 
 
+@pytest.mark.parametrize("B", [64, 128])
+def test_output_only_16_byte_aligned(s2gpu, B):
+    # The epilogue stores whole 32-byte sectors when the output is 32-byte
+    # aligned and falls back to 16-byte stores otherwise: both write the same
+    # bytes, and nothing outside the output.
+    ctx, qlen, H, D = [700, 300], [300, 300], 4, 128
+    w = synth.PrefillWorkload("t", 2, H, D, max(ctx), B, 3, 1, seed=31)
+    qd, kd, vd = synth.prefill_inputs(w)
+    q_start = np.concatenate([[0], np.cumsum(qlen)]).astype(np.int32)
+    q = torch.cat([qd[s, :, ctx[s] - qlen[s]:ctx[s]].transpose(0, 1) for s in range(2)], 0).contiguous()
+    kc, vc, bt = paged(kd, vd, ctx, 31)
+    lay = s2gpu.build_layout(H, B, 3, 1, -(-max(ctx) // B), device="cuda")
+    args = (q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(bt).cuda(),
+            torch.tensor(ctx, dtype=torch.int32).cuda(), torch.from_numpy(q_start).cuda(), lay, max(qlen))
+    ref = s2gpu.chunk_prefill(*args, scale=w.scale)
+    n = ref.numel()
+    buf = torch.full((n + 24,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    base = buf.data_ptr()
+    off = next(e for e in range(0, 24, 8) if (base + 2 * e) % 32 == 16)  # 16- but not 32-byte aligned
+    out = buf[off:off + n].view(ref.shape)
+    s2gpu.chunk_prefill(*args, scale=w.scale, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    assert torch.isnan(buf[:off].float()).all() and torch.isnan(buf[off + n:].float()).all()
+
+
 def test_bad_chunk_length_is_flagged(s2gpu):
     H, D, B = 2, 128, 128
     q = torch.zeros(8, H, D, dtype=torch.bfloat16, device="cuda")
