@@ -576,23 +576,14 @@ s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             if (len > 0) {
                 if (!warp_wait(bar_acc, (n_acc++) & 1, ctl)) break;
                 tc_fence_after();
+                // HD/2 columns per warpgroup, 32 per TMEM load, one wait
+                const bool st32 = (reinterpret_cast<uintptr_t>(p.dq) & 31u) == 0;
+                uint32_t o[HD / 2];
 #pragma unroll
-                for (int c = 0; c < HD / 64; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tl + C::COL_ACC + g * (HD / 2) + 32 * c, o);
-                    tmem_wait_ld();
-                    if (row_valid) {
-#pragma unroll
-                        for (int e2 = 0; e2 < 32; e2 += 8) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * p.scale, __uint_as_float(o[e2 + 1]) * p.scale);
-                            v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * p.scale, __uint_as_float(o[e2 + 3]) * p.scale);
-                            v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * p.scale, __uint_as_float(o[e2 + 5]) * p.scale);
-                            v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * p.scale, __uint_as_float(o[e2 + 7]) * p.scale);
-                            *reinterpret_cast<uint4*>(drow + 32 * c + e2) = v;
-                        }
-                    }
-                }
+                for (int c = 0; c < HD / 64; ++c)
+                    tmem_ld32(tl + C::COL_ACC + g * (HD / 2) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&o[32 * c]));
+                tmem_wait_ld();
+                if (row_valid) store_bf16_row<HD / 2>(drow, o, p.scale, st32);
             } else if (row_valid) {  // no key block listed for this tile
                 for (int d = 0; d < HD / 2; d += 8) *reinterpret_cast<uint4*>(drow + d) = make_uint4(0, 0, 0, 0);
             }
@@ -921,22 +912,13 @@ s2_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     tc_fence_after();
                     const float f = g == 0 ? 1.0f : p.scale;
                     const uint32_t col = g == 0 ? C::COL_DV : C::COL_DK;
+                    const bool st32 = (reinterpret_cast<uintptr_t>(g == 0 ? p.dv : p.dk) & 31u) == 0;
 #pragma unroll
                     for (int c = 0; c < HD / 32; ++c) {
                         uint32_t o[32];
                         tmem_ld32(tl + col + 32 * c, o);
                         tmem_wait_ld();
-                        if (row_valid) {
-#pragma unroll
-                            for (int e2 = 0; e2 < 32; e2 += 8) {
-                                uint4 v;
-                                v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * f, __uint_as_float(o[e2 + 1]) * f);
-                                v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * f, __uint_as_float(o[e2 + 3]) * f);
-                                v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * f, __uint_as_float(o[e2 + 5]) * f);
-                                v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * f, __uint_as_float(o[e2 + 7]) * f);
-                                *reinterpret_cast<uint4*>(grow + 32 * c + e2) = v;
-                            }
-                        }
+                        if (row_valid) store_bf16_row<32>(grow + 32 * c, o, f, st32);
                     }
                 }
             } else if (row_valid) {  // no query block lists this tile's key blocks
@@ -986,7 +968,7 @@ struct BwdKVPCfg {
     // ds_full, drain x 2, list_full[2], list_empty[2]
     static constexpr int NBAR = 2 + 2 * ST + 7 + 4;
     static constexpr uint32_t OFF_MISC = OFF_BAR + ((NBAR * 8 + 15) / 16) * 16;
-    static constexpr uint32_t SMEM = OFF_MISC + 32;
+    static constexpr uint32_t SMEM = OFF_MISC + 48;
     static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;
     // Q/dO producer, the two MMA threads, 8 element-wise warps
     static constexpr uint32_t LIST_CONSUMERS = 11;
@@ -1051,12 +1033,14 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
     auto bar_lf = [&](int b) { return bar_s + 56u + 8u * b; };
     auto bar_le = [&](int b) { return bar_s + 72u + 8u * b; };
     const uint32_t* list = reinterpret_cast<const uint32_t*>(smem + C::OFF_LIST);
-    // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more)
+    // [0] tmem, [1] abort, [2..3] list lengths, [4..5] item of each list buffer (-1: no more),
+    // [6] this CTA holds the work-counter slot, [8..11] the key blocks of each buffer's tile
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
     volatile int* abort_cta = misc + 1;
     volatile int* list_len = misc + 2;
     volatile int* list_item = misc + 4;
+    volatile int* list_kb = misc + 8;  // [buffer][key block r of the tile] (-1: none)
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
@@ -1133,6 +1117,8 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
             if (lane == 0) {
                 list_len[b] = total;
                 list_item[b] = w;
+#pragma unroll
+                for (int r = 0; r < C::ROWS; ++r) list_kb[2 * b + r] = kb[r];
                 mbar_arrive(bar_lf(b));
             }
             if (total > 0) {
@@ -1302,7 +1288,7 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
             const int w = list_item[b];
             if (w < 0) break;
             const KvItem it = kv_item(p, w);
-            const int kbr = kv_item_block(p, it, kbit);
+            const int kbr = list_kb[2 * b + kbit];  // kv_item_block(p, it, kbit), read by the scheduler
             const int kpos = kbr * BK + (r % BK);
             const bool row_valid = kbr >= 0 && kpos < p.seq;
             const uint32_t* L = list + b * C::LIST_CAP;
@@ -1375,22 +1361,16 @@ s2_bwd_dkv_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __gr
                 tc_fence_after();
                 const float f = g == 0 ? 1.0f : p.scale;
                 const uint32_t col = g == 0 ? C::COL_DV : C::COL_DK;
+                // 64 columns per TMEM wait, and 32-byte stores (whole L2 sectors) when
+                // the gradient is 32-byte aligned
+                const bool st32 = (reinterpret_cast<uintptr_t>(g == 0 ? p.dv : p.dk) & 31u) == 0;
 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tl + col + 32 * c, o);
+                for (int c = 0; c < HD / 64; ++c) {
+                    uint32_t o[64];
+                    tmem_ld32(tl + col + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                    tmem_ld32(tl + col + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
                     tmem_wait_ld();
-                    if (row_valid) {
-#pragma unroll
-                        for (int e2 = 0; e2 < 32; e2 += 8) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(o[e2 + 0]) * f, __uint_as_float(o[e2 + 1]) * f);
-                            v.y = pack_bf16x2(__uint_as_float(o[e2 + 2]) * f, __uint_as_float(o[e2 + 3]) * f);
-                            v.z = pack_bf16x2(__uint_as_float(o[e2 + 4]) * f, __uint_as_float(o[e2 + 5]) * f);
-                            v.w = pack_bf16x2(__uint_as_float(o[e2 + 6]) * f, __uint_as_float(o[e2 + 7]) * f);
-                            *reinterpret_cast<uint4*>(grow + 32 * c + e2) = v;
-                        }
-                    }
+                    if (row_valid) store_bf16_row<64>(grow + 64 * c, o, f, st32);
                 }
             } else if (row_valid) {  // no query block lists this tile's key blocks
                 for (int d = 0; d < HD; d += 8) *reinterpret_cast<uint4*>(grow + d) = make_uint4(0, 0, 0, 0);

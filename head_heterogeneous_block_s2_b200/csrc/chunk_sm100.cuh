@@ -689,23 +689,7 @@ s2_chunk_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     uint32_t o[32];
                     tmem_ld32(tl + C::colO(t) + 32 * c, o);
                     tmem_wait_ld();
-                    if (row_valid) {
-#pragma unroll
-                        for (int e2 = 0; e2 < 32; e2 += 16) {
-                            uint32_t w8[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                w8[i] = pack_bf16x2(__uint_as_float(o[e2 + 2 * i]) * inv,
-                                                    __uint_as_float(o[e2 + 2 * i + 1]) * inv);
-                            if (st32) {
-                                st_global_v8(og + 32 * c + e2, w8);
-                            } else {
-                                *reinterpret_cast<uint4*>(og + 32 * c + e2) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-                                *reinterpret_cast<uint4*>(og + 32 * c + e2 + 8) =
-                                    make_uint4(w8[4], w8[5], w8[6], w8[7]);
-                            }
-                        }
-                    }
+                    if (row_valid) store_bf16_row<32>(og + 32 * c, o, inv, st32);
                 }
                 if (row_valid && p.lse) p.lse[orow] = l > 0.f ? (m_used + lg2(l)) * 0.69314718055994531f : -INFINITY;
             } else if (row_valid) {  // no row of this tile lists a key block: zero output

@@ -83,6 +83,31 @@ def test_mask_layout_with_empty_rows(s2gpu, bk):
     assert (dk[0, 1, 3 * bk:4 * bk] == 0).all() and (dv[0, 1, 3 * bk:4 * bk] == 0).all()
 
 
+@pytest.mark.parametrize("bk", [64, 128])
+def test_gradients_only_16_byte_aligned(s2gpu, bk):
+    # The epilogues store whole 32-byte sectors when a gradient array is
+    # 32-byte aligned and fall back to 16-byte stores otherwise: both write the
+    # same bytes, and nothing outside the arrays.
+    w = synth.PrefillWorkload("t", 1, 3, 128, 5 * 128, bk, 3, 1, seed=96)
+    q, k, v = (t.cuda() for t in synth.prefill_inputs(w))
+    do = upstream(w, 4).cuda()
+    lay = s2gpu.build_layout(w.heads, bk, w.stride, w.local, w.num_blocks, device="cuda")
+    o, lse = s2gpu.prefill(q, k, v, lay, scale=w.scale, want_lse=True)
+    ref = s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale)
+    n = q.numel()
+    bufs, outs = [], []
+    for _ in range(3):
+        buf = torch.full((n + 24,), float("nan"), dtype=torch.bfloat16, device="cuda")
+        off = next(e for e in range(0, 24, 8) if (buf.data_ptr() + 2 * e) % 32 == 16)
+        bufs.append((buf, off))
+        outs.append(buf[off:off + n].view(q.shape))
+    s2gpu.backward(q, k, v, o, lse, do, lay, scale=w.scale, dq=outs[0], dk=outs[1], dv=outs[2])
+    torch.cuda.synchronize()
+    for got, want, (buf, off) in zip(outs, ref, bufs):
+        assert torch.equal(got, want)
+        assert torch.isnan(buf[:off].float()).all() and torch.isnan(buf[off + n:].float()).all()
+
+
 def test_odd_union_lists_and_empty_key_tiles(s2gpu):
     """64-key blocks: query tiles (two query blocks) whose union list has an
     odd length (the dQ kernel pairs entries into 128-key elements, so the last
