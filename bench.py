@@ -143,8 +143,8 @@ def plant_positions(w, last_row_blocks, seed=7):
 KERNEL_SOURCES = {
     "s2_prefill_pair_kernel": ("prefill_pair_sm100.cuh", "lists.cuh", "ptx.cuh", "umma.cuh"),
     "s2_decode_split_kernel": ("decode.cuh", "ptx.cuh"),
-    "s2_bwd": ("backward_sm100.cuh", "lists.cuh", "ptx.cuh", "umma.cuh"),
-    "s2_chunk_prefill_kernel": ("chunk_sm100.cuh", "lists.cuh", "ptx.cuh", "umma.cuh"),
+    "s2_bwd": ("backward_sm100.cuh", "lists.cuh", "ptx.cuh", "store.cuh", "umma.cuh"),
+    "s2_chunk_prefill_kernel": ("chunk_sm100.cuh", "lists.cuh", "ptx.cuh", "store.cuh", "umma.cuh"),
 }
 
 

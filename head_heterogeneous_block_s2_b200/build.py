@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libs2attn.so")
 
 SOURCES = [os.path.join(CSRC, "s2attn.cu"), os.path.join(CSRC, "layout.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "umma.cuh", "lists.cuh", "prefill_pair_sm100.cuh", "backward_sm100.cuh", "chunk_sm100.cuh", "decode.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "store.cuh", "umma.cuh", "lists.cuh", "prefill_pair_sm100.cuh", "backward_sm100.cuh", "chunk_sm100.cuh", "decode.cuh")] + [
     os.path.join(INCLUDE, "s2attn.h")]
 
 NVCC_FLAGS = [

@@ -46,6 +46,7 @@
 
 #include "lists.cuh"
 #include "ptx.cuh"
+#include "store.cuh"  // store_bf16_row
 #include "umma.cuh"
 
 namespace s2 {
