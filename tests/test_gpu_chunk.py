@@ -99,6 +99,21 @@ def test_range_layout(s2gpu):
     case(s2gpu, [1000, 333], [400, 333], layout=lay, bmask=oracle.range_block_mask(8, ranges), seed=6)
 
 
+@pytest.mark.parametrize("B", [64, 128])
+def test_mask_layout_with_empty_rows(s2gpu, B):
+    # Random per-head block masks with empty query-block rows: some items have
+    # a tile that sees no key block (its Q is released at once and its rows
+    # get zeros and an LSE of -inf) beside a tile that does.
+    H, n = 3, 1100
+    nb = -(-n // B)
+    rng = np.random.default_rng(40 + B)
+    m = np.tril(rng.random((H, nb, nb)) < 0.35).astype(np.uint8)
+    for h in range(H):
+        m[h, rng.choice(nb, 3, replace=False)] = 0  # empty query-block rows
+    lay = s2gpu.build_layout_mask(m, B, device="cuda")
+    case(s2gpu, [n, 700], [600, 700], H=H, B=B, layout=lay, bmask=m, seed=41 + B)
+
+
 def test_one_token_chunks_match_decode(s2gpu):
     ctx = [1, 17, 500, 1024]
     out = case(s2gpu, ctx, [1, 1, 1, 1], seed=7)
