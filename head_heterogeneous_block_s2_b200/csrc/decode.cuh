@@ -56,7 +56,10 @@ struct DecodeCfg {
     static constexpr uint32_t OFF_META = OFF_BAR + 2 * NS * 8;
     static constexpr uint32_t OFF_MERGE = OFF_META + NS * 8;  // 4 warps x (HD + 2) floats
     static constexpr uint32_t OFF_MISC = OFF_MERGE + 4 * (HD + 2) * 4;
-    static constexpr uint32_t SMEM = OFF_MISC + 32;
+    // batches of up to LPT_MAX sequences start their longest contexts first
+    static constexpr int LPT_MAX = 256;
+    static constexpr uint32_t OFF_CTX = OFF_MISC + 32;  // [LPT_MAX] context lengths
+    static constexpr uint32_t SMEM = OFF_CTX + LPT_MAX * 4;
     static constexpr int DPL = HD / 32;  // output dims per lane
 };
 
@@ -76,7 +79,7 @@ s2_decode_split_kernel(const DecodeParams p)
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t sb = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int sp = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int sp = blockIdx.x, h = blockIdx.y;
     const int H = p.heads;
     const int hkv = h / (H / p.heads_kv);
 
@@ -85,6 +88,29 @@ s2_decode_split_kernel(const DecodeParams p)
     int2* meta = reinterpret_cast<int2*>(smem + C::OFF_META);
     int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
     volatile int* abort_cta = reinterpret_cast<volatile int*>(misc + 7);
+
+    // Sequence of this CTA. CTAs start in grid order, so with up to LPT_MAX
+    // sequences the z-th grid slice takes the sequence with the z-th longest
+    // context (ties by index; the ranks are a permutation): the longest
+    // page lists start first and short ones fill the last wave. Larger
+    // batches keep the index order.
+    int s = blockIdx.z;
+    if (p.batch <= C::LPT_MAX) {
+        int* ctxs = reinterpret_cast<int*>(smem + C::OFF_CTX);
+        for (int i = threadIdx.x; i < p.batch; i += blockDim.x) ctxs[i] = p.ctx_lens[i];
+        __syncthreads();
+        for (int c = threadIdx.x; c < p.batch; c += blockDim.x) {
+            const int nc = ctxs[c];
+            int rank = 0;
+            for (int j = 0; j < p.batch; ++j) {
+                const int nj = ctxs[j];
+                rank += (nj > nc || (nj == nc && j < c)) ? 1 : 0;
+            }
+            if (rank == (int)blockIdx.z) misc[5] = c;
+        }
+        __syncthreads();
+        s = misc[5];
+    }
 
     // Work of this CTA: pages [pg0, pg1) of the (s, h) page list.
     if (threadIdx.x == 0) {

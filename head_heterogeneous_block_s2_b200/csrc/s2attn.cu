@@ -538,15 +538,15 @@ int s2_attn_chunk_prefill(const void* q, const void* k_cache, const void* v_cach
 int32_t s2_attn_decode_auto_splits(int32_t batch, int32_t heads)
 {
     if (batch < 1 || heads < 1) return 1;
-    // Aim for about 4 waves of 3 resident CTAs on each of 148 SMs, but with at
-    // least 256 (sequence, head) pairs no more than 4 splits: measured on
-    // 32 heads, contexts U[4096, 32768] (active K+V GB/s, one launch after an
-    // L2 flush), the best counts were 4 at batch 8 (7 was 7% slower), 4 at 16,
-    // 2 at 32 and 1 (or 2, equal) at 64.
+    // About one wave of resident CTAs (148 SMs x ~2.5): the split kernel starts
+    // the longest contexts first, so the short ones even out the last wave and
+    // more splits only add partials to merge. Measured on 32 heads, contexts
+    // U[4096, 32768] (active K+V GB/s, one launch after an L2 flush), the best
+    // counts were 3 at batch 4, 2 at batch 8 and 1 at batches 16, 32 and 64;
+    // this rule gives exactly those.
     const int64_t bh = (int64_t)batch * heads;
-    const int64_t target = 148 * 3 * 4;
+    const int64_t target = 370;
     int64_t sp = (target + bh - 1) / bh;
-    if (bh >= 256 && sp > 4) sp = 4;
     if (sp < 1) sp = 1;
     if (sp > 16) sp = 16;
     return (int32_t)sp;

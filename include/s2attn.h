@@ -349,7 +349,10 @@ int s2_attn_backward(const void* q, const void* k, const void* v, const void* o,
 size_t s2_attn_decode_workspace_size(int32_t batch, int32_t heads, int32_t head_dim,
                                      int32_t num_splits);
 
-/* The split count s2_attn_decode uses when given num_splits <= 0. */
+/* The split count s2_attn_decode uses when given num_splits <= 0: about one
+ * wave of resident CTAs on a B200, ceil(370 / (batch * heads)), at most 16.
+ * (With up to 256 sequences the split kernel starts the sequences with the
+ * longest contexts first, which evens out the last wave.) */
 int32_t s2_attn_decode_auto_splits(int32_t batch, int32_t heads);
 
 /*
