@@ -114,6 +114,16 @@ def test_decode_workspace_size():
     assert s2attn.decode_workspace_size(4, 8, 128, 0) == s2attn.decode_workspace_size(4, 8, 128, auto)
 
 
+def test_decode_auto_splits_is_about_one_resident_wave():
+    # ceil(370 / (batch * heads)), clamped to [1, 16]: the measured best split
+    # counts on 32 heads were 3, 2, 1, 1, 1 at batches 4, 8, 16, 32, 64
+    assert [s2attn.decode_auto_splits(b, 32) for b in (4, 8, 16, 32, 64)] == [3, 2, 1, 1, 1]
+    for b, h in ((1, 1), (1, 8), (2, 32), (3, 7), (300, 32), (65535, 64)):
+        want = min(16, max(1, -(-370 // (b * h))))
+        assert s2attn.decode_auto_splits(b, h) == want, (b, h)
+    assert s2attn.decode_auto_splits(0, 32) == 1 and s2attn.decode_auto_splits(4, 0) == 1
+
+
 @no_gpu_only
 def test_grouped_head_entry_points_reject_bad_head_counts():
     lib = s2attn.load()

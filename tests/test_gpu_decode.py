@@ -69,6 +69,22 @@ def test_degenerate_strides_and_windows(s2gpu, S, L):
         parity(lse.reshape(-1), ref_lse, max_tol=1e-3, mean_tol=1e-4)
 
 
+@pytest.mark.parametrize("batch", [40, 300])
+def test_equal_contexts_and_batches_past_the_reordering(s2gpu, batch):
+    # Up to 256 sequences start in order of decreasing context length (ties by
+    # index): groups of equal lengths must still map one CTA slice to each
+    # sequence. Past 256 the index order is kept. Every item is checked.
+    rng = np.random.default_rng(batch)
+    ctx = [int(c) for c in rng.choice([1, 17, 300, 1000], size=batch)]
+    w = synth.DecodeWorkload("t", batch, 4, 128, 1, 1000, 16, 128, 4, 2, seed=batch)
+    d = synth.decode_inputs(w, ctx_lens=ctx)
+    for splits in (1, 3):
+        out, lse = run(s2gpu, w, d, splits)
+        ref, ref_lse = oracle_decode(w, d)
+        parity(out.reshape(-1, 128), ref)
+        parity(lse.reshape(-1), ref_lse, max_tol=1e-3, mean_tol=1e-4)
+
+
 def test_decode_equals_last_prefill_row(s2gpu):
     # Dense-packed prefill of n tokens vs paged decode of the same tokens.
     H, D, B, S, L, n = 4, 128, 128, 4, 2, 1024
